@@ -1,0 +1,437 @@
+"""Throughput benchmark of the scaled low-precision GEMM hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one call of the operation on one batch of synthetic inputs that are
+already resident in HBM.  The default workload is the FP8 block-scaled GEMM
+M=16640, N=5120, K=8192 (bf16 out).  Rank 0 prints one JSON line.
+
+With N > 1 (launched by torch.distributed.run) every rank runs an independent
+replica of the workload on its own GPU -- the operation has no exchange step --
+and ``value`` is the total work of all ranks over the slowest rank's time
+("scaling": "weak").
+
+``--impl reference`` times the CPU oracle on the host cores instead (bounded
+row sample per step); it is a reported baseline, not an optimisation target.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "FP8 blockwise GEMM TFLOP/s at 16640x5120x8192; % of B200 dense FP8 peak"
+DEFAULT_WORKLOAD = "fp8_16640x5120x8192"
+L2_BYTES = 126 * 1024 * 1024
+FP8_PER_BF16 = 2.0  # nominal dense fp8 : bf16 tensor throughput on B200 (4.5 : 2.25 PFLOP/s)
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ---------------------------------------------------------------------------
+# helpers that need no GPU (covered by tests/test_bench_host.py)
+# ---------------------------------------------------------------------------
+def load_peaks(path=os.path.join(ROOT, "MEASURED_PEAKS.json")):
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        p["source"] = "measured"
+        return p
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS)
+
+
+def source_digest() -> str:
+    """Hash of the CUDA sources: a stored ncu traffic figure is only valid for the kernel it was taken on."""
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "int8_gemm_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()[:16]
+
+
+def stored_traffic(workload: str):
+    """dram read+write bytes per launch from the committed ncu summary, or None if stale/absent."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            t = json.load(f)
+    except (OSError, ValueError):
+        return None
+    e = t.get(workload)
+    if not e or e.get("source_digest") != source_digest():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+def aggregate(local_ms: float, units_per_rank: float, world: int, reduce_max=None):
+    """Whole-job throughput: all ranks' units over the slowest rank's time."""
+    t = reduce_max(local_ms) if reduce_max else local_ms
+    return t, units_per_rank * world / (t / 1e3)
+
+
+def parse_clock_csv(text: str):
+    rows = []
+    for line in text.strip().splitlines():
+        if not line or line.startswith("index") or "clocks" in line:
+            continue
+        parts = [p.strip() for p in line.split(",")]
+        if len(parts) < 9:
+            continue
+        try:
+            sm = float(parts[1].split()[0])
+            smax = float(parts[2].split()[0])
+            pw = float(parts[3].split()[0]) if parts[3].split()[0] not in ("[N/A]", "N/A") else float("nan")
+        except ValueError:
+            continue
+        rows.append({"sm": sm, "max": smax, "power": pw, "active": parts[4], "hw_slowdown": parts[5],
+                     "hw_thermal": parts[6], "sw_thermal": parts[7], "sw_power_cap": parts[8]})
+    if not rows:
+        return None
+    loaded = [r for r in rows if r["power"] != r["power"] or r["power"] > 300.0] or rows
+    reasons = []
+    for key, name in (("hw_slowdown", "hw_slowdown"), ("hw_thermal", "hw_thermal_slowdown"),
+                      ("sw_thermal", "sw_thermal_slowdown"), ("sw_power_cap", "sw_power_cap")):
+        if any(r[key].lower() == "active" for r in rows):
+            reasons.append(name)
+    return {"sm_mhz": statistics.median(r["sm"] for r in loaded), "sm_max_mhz": max(r["max"] for r in rows),
+            "reasons": reasons, "samples": len(rows), "samples_under_load": len(loaded)}
+
+
+# ---------------------------------------------------------------------------
+# workloads
+# ---------------------------------------------------------------------------
+def describe(w):
+    import workloads as wl
+    if w.op == "fp8_blockwise":
+        flops = 2.0 * w.M * w.N * w.K
+        byts = w.M * w.K + w.N * w.K + 2 * w.M * w.N + 4 * w.M * (w.K // 128) + 4 * (w.K // 128) * (-(-w.N // 128))
+        dtype = "e4m3 (fp32 accumulate)"
+    elif w.op == "int_scaled_mm":
+        flops = 2.0 * w.M * w.N * w.K
+        byts = w.M * w.K + w.N * w.K + 4 * w.M * w.N + 4 * (w.M + w.N)
+        dtype = "s8 (s32 accumulate)"
+    else:
+        flops = 2.0 * w.M * w.G * w.N * w.K
+        kb, nb = w.K // 128, -(-w.N // 128)
+        byts = w.M * w.G * w.K + w.G * w.N * w.K + 2 * w.M * w.G * w.N + w.M * w.G * kb + w.G * nb * kb
+        dtype = "e4m3 (fp32 accumulate)"
+    return flops, float(byts), dtype
+
+
+def build_step(w, device, copies):
+    """Device-resident inputs (`copies` independent sets, rotated per step) and the step closure."""
+    import torch
+
+    import int8_gemm_b200 as bs
+    import workloads as wl
+
+    d = wl.workload_inputs(w)
+    sets = []
+    for _ in range(copies):
+        if w.op == "fp8_blockwise":
+            A, B = d["A"].to(device), d["B_t"].to(device).t()
+            sa, sb = d["scale_a"].to(device), d["scale_b"].to(device)
+            out = torch.empty(w.M, w.N, dtype=torch.bfloat16, device=device)
+            sets.append(lambda A=A, B=B, sa=sa, sb=sb, out=out: bs.bs_gemm_fp8_blockwise(A, B, sa, sb, out=out))
+        elif w.op == "int_scaled_mm":
+            A, B = d["A"].to(device), d["B_t"].to(device).t()
+            sa, sb = d["s_a"].to(device), d["s_b"].to(device)
+            out = torch.empty(w.M, w.N, dtype=torch.float32, device=device)
+            sets.append(lambda A=A, B=B, sa=sa, sb=sb, out=out: bs.int_scaled_mm(A, B, sa, sb, out=out))
+        else:
+            x, wt = d["x"].to(device), d["w"].to(device)
+            xs, ws = d["x_scale"].to(device), d["w_scale"].to(device)
+            out = torch.empty(w.M, w.G, w.N, dtype=torch.bfloat16, device=device)
+            sets.append(lambda x=x, wt=wt, xs=xs, ws=ws, out=out: bs.bmm_a8w8_blockscale(x, wt, xs, ws, out=out))
+    return d, sets
+
+
+def e2e_step_fn(w, d, device):
+    """One end-to-end call: pinned host inputs -> device, GEMM through the public API, result -> host."""
+    import torch
+
+    import int8_gemm_b200 as bs
+
+    pin = {k: v.contiguous().pin_memory() for k, v in d.items()}
+    if w.op == "fp8_blockwise":
+        host_out = torch.empty(w.M, w.N, dtype=torch.bfloat16).pin_memory()
+    elif w.op == "int_scaled_mm":
+        host_out = torch.empty(w.M, w.N, dtype=torch.float32).pin_memory()
+    else:
+        host_out = torch.empty(w.M, w.G, w.N, dtype=torch.bfloat16).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in pin.values())
+    d2h = host_out.numel() * host_out.element_size()
+
+    def step():
+        dev = {k: v.to(device, non_blocking=True) for k, v in pin.items()}
+        if w.op == "fp8_blockwise":
+            out = bs.bs_gemm_fp8_blockwise(dev["A"], dev["B_t"].t(), dev["scale_a"], dev["scale_b"])
+        elif w.op == "int_scaled_mm":
+            out = bs.int_scaled_mm(dev["A"], dev["B_t"].t(), dev["s_a"], dev["s_b"])
+        else:
+            out = bs.bmm_a8w8_blockscale(dev["x"], dev["w"], dev["x_scale"], dev["w_scale"])
+        host_out.copy_(out, non_blocking=True)
+
+    return step, h2d, d2h
+
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.file = None
+
+    def __enter__(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.file, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def result(self):
+        if self.file is None:
+            return None
+        try:
+            with open(self.file.name) as f:
+                txt = f.read()
+            os.unlink(self.file.name)
+        except OSError:
+            return None
+        return parse_clock_csv(txt)
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (reported baseline; never tuned)
+# ---------------------------------------------------------------------------
+def oracle_rows_run(w, d, rows):
+    import oracle
+    if w.op == "fp8_blockwise":
+        oracle.fp8_blockwise(d["A"], d["B_t"], d["scale_a"], d["scale_b"], rows=rows)
+    elif w.op == "int_scaled_mm":
+        oracle.int_scaled_mm(d["A"], d["B_t"], d["s_a"], d["s_b"], rows=rows)
+    else:
+        oracle.bmm_blockscale(d["x"], d["w"], d["x_scale"], d["w_scale"], rows=rows)
+
+
+def cpu_oracle_baseline(w, d, budget_s: float = 12.0):
+    """Times the oracle on a bounded row sample sized to about `budget_s` seconds."""
+    import oracle
+    threads = oracle.num_threads()
+    flops_per_row = describe(w)[0] / w.M
+    n = max(1, min(w.M, threads))
+    t0 = time.perf_counter()
+    oracle_rows_run(w, d, list(range(n)))
+    dt = time.perf_counter() - t0
+    rows = max(n, min(w.M, int(n * budget_s / max(dt, 1e-3) / threads) * threads))
+    t0 = time.perf_counter()
+    oracle_rows_run(w, d, list(range(rows)))
+    dt = time.perf_counter() - t0
+    return {"value": flops_per_row * rows / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "sample": f"{rows} of {w.M} output rows of {w.name} (all columns), fp64 oracle, {dt:.1f} s"}
+
+
+# ---------------------------------------------------------------------------
+# main
+# ---------------------------------------------------------------------------
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    import workloads as wl
+    w = wl.WORKLOADS[args.workload]
+    flops, byts, dtype = describe(w)
+
+    if args.impl == "reference":
+        run_reference(args, w, rank, world, flops)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    import int8_gemm_b200 as bs
+
+    assert torch.cuda.is_available(), "bench.py needs a CUDA device"
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=device)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def reduce_max(v):
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    copies = max(1, math.ceil(3 * L2_BYTES / byts)) if byts < 3 * L2_BYTES else 1
+    d, sets = build_step(w, device, copies)
+    op = {"fp8_blockwise": 1, "int_scaled_mm": 2, "bmm_a8w8_blockscale": 3}[w.op]
+    plan = bs.plan_for(op, w.M, w.G, w.N, w.K, torch.cuda.get_device_properties(device).multi_processor_count)
+
+    for i in range(max(3, args.warmup)):
+        sets[i % copies]()
+    torch.cuda.synchronize()
+    assert bs.device_error() == 0
+
+    K = args.steps
+    stream = torch.cuda.current_stream(device)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    total0, total1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        total0.record(stream)
+        for i in range(K):
+            ev[i][0].record(stream)
+            sets[i % copies]()
+            ev[i][1].record(stream)
+        total1.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    local_ms = total0.elapsed_time(total1)
+    per_launch_ms = sum(a.elapsed_time(b) for a, b in ev) / K
+    err = bs.device_error()
+    assert err == 0, f"device error word 0x{err:x}"
+    step_ms, value = aggregate(local_ms / K, flops, world, reduce_max)
+    value /= 1e12
+
+    # end to end through the public API with pinned host buffers
+    e2e_fn, h2d, d2h = e2e_step_fn(w, d, device)
+    for _ in range(2):
+        e2e_fn()
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = reduce_max(e0.elapsed_time(e1) / args.e2e_steps)
+    e2e_value = flops * world / (e2e_ms / 1e3) / 1e12
+
+    peaks = load_peaks()
+    if w.op in ("fp8_blockwise", "bmm_a8w8_blockscale") and flops / byts > 690 or w.op == "int_scaled_mm":
+        bound, unit = "tensor", "TFLOP/s"
+        peak = peaks["bf16_tflops"] * FP8_PER_BF16
+        achieved = flops / (per_launch_ms / 1e3) / 1e12
+    else:
+        bound, unit = "hbm", "GB/s"
+        peak = peaks["hbm_gbs"]
+        achieved = byts / (per_launch_ms / 1e3) / 1e9
+    traffic = stored_traffic(w.name)
+
+    result = {
+        "metric": METRIC if w.name == DEFAULT_WORKLOAD else f"{w.name} TFLOP/s",
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": round(step_ms, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": dtype,
+        "data": "synthetic (seeded N(0,1) with 1% x20 outliers, quantised per the workload recipe)",
+        "config": {"workload": w.name, "op": w.op, "M": w.M, "N": w.N, "K": w.K, "G": w.G,
+                   "out_dtype": "float32" if w.op == "int_scaled_mm" else "bfloat16",
+                   "l2": (f"inputs larger than L2 ({byts / 1e6:.0f} MB per step)" if copies == 1 else
+                          f"{copies} rotating input copies ({copies * byts / 1e6:.0f} MB) to defeat L2"),
+                   "parallelism": f"replicas x{world}", "plan": plan},
+        "roofline": {"bound": bound, "achieved": round(achieved, 2), "peak": round(peak, 1), "unit": unit,
+                     "frac": round(achieved / peak, 4), "traffic": traffic,
+                     "kernel": "wide_gemm_kernel" if plan["kernel"] == 1 else "skinny_gemm_kernel",
+                     "peak_source": f"{peaks.get('source')}: " + (
+                         "bf16 burst x 2 (fp8:bf16 nominal ratio)" if bound == "tensor" else "HBM copy")},
+        "e2e": {"value": round(e2e_value, 3), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": K * plan["launches"],
+    }
+    clocks = clk.result()
+    if clocks:
+        result["clocks"] = clocks
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_oracle_baseline(w, d)
+    if world > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+
+
+def run_reference(args, w, rank, world, flops):
+    """The oracle on the host cores, per step a bounded row sample of the workload."""
+    if rank != 0:
+        return
+    import oracle
+    import workloads as wl
+    d = wl.workload_inputs(w)
+    threads = oracle.num_threads()
+    rows_per_step = max(1, min(w.M, threads))
+    sample = list(range(rows_per_step))
+    for _ in range(max(1, args.warmup if args.warmup < 3 else 3)):
+        oracle_rows_run(w, d, sample)
+    steps = max(1, min(args.steps, 20))
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        oracle_rows_run(w, d, sample)
+    dt = (time.perf_counter() - t0) / steps
+    value = flops / w.M * rows_per_step / dt / 1e12
+    out = {
+        "impl": "reference", "metric": METRIC if w.name == DEFAULT_WORKLOAD else f"{w.name} TFLOP/s",
+        "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": steps, "warmup": args.warmup,
+        "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64 (oracle)", "data": "synthetic", "config": {"workload": w.name, "M": w.M, "N": w.N, "K": w.K},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": f"{rows_per_step} of {w.M} output rows per step (all columns)"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

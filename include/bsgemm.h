@@ -1,0 +1,199 @@
+/*
+ * bsgemm -- scaled low-precision GEMMs with the dequantisation fused in,
+ * hand-written for NVIDIA B200 (sm_100a: TMA, tcgen05 tensor cores, TMEM).
+ *
+ * C ABI.  Every pointer argument is a DEVICE pointer unless stated otherwise,
+ * owned by the caller; the library keeps no reference after the call returns
+ * and allocates no device memory.  All GEMM calls are asynchronous on the
+ * given stream (a cudaStream_t passed as void*; NULL = legacy default stream).
+ * Argument checks run synchronously on the host before anything is launched;
+ * a call that returns an error status has launched nothing.  There is no CPU
+ * fallback: on a device other than compute capability 10.0 the calls return
+ * BS_ERR_DEVICE.
+ *
+ * Conventions shared by the three operations
+ *   - Sizes are in elements, strides ("ld", "s_*") in elements of the tensor
+ *     they describe.
+ *   - FP8 operands are OCP e4m3 ("float8_e4m3fn") bytes; INT8 operands are
+ *     signed bytes.
+ *   - A is row-major [M, K]; B is the logical [K, N] matrix stored
+ *     column-major, i.e. as N rows of K contiguous bytes (the layout contract
+ *     of check_supported_striding in pytorch/torch/_inductor/kernel/mm.py:
+ *     mat_a row-major, mat_b column-major).
+ *   - Base pointers of A, B and the output must be 16-byte aligned and their
+ *     row strides multiples of 16 bytes (the tensor-memory-accelerator rule).
+ *   - M == 0 or N == 0 is a no-op returning BS_OK (the early exit of
+ *     mm_template in the same file); K == 0 writes zeros.
+ *   - The scale tensors multiply: the dequantised value is code * scale (the
+ *     scaling of the accumulator in apply_scaling, same file).
+ */
+#ifndef BSGEMM_H
+#define BSGEMM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  BS_OK = 0,
+  BS_ERR_NULL = 1,      /* a required pointer is NULL */
+  BS_ERR_SHAPE = 2,     /* negative / unsupported size, or scale shape mismatch */
+  BS_ERR_LAYOUT = 3,    /* stride smaller than the row it describes, bad unit stride */
+  BS_ERR_ALIGNMENT = 4, /* pointer or stride breaks the 16-byte rule */
+  BS_ERR_DTYPE = 5,     /* output dtype not supported by this operation */
+  BS_ERR_DEVICE = 6,    /* current device is not an sm_100 (B200-class) GPU */
+  BS_ERR_CUDA = 7,      /* a CUDA runtime call failed (launch, encode, ...) */
+  BS_ERR_TIMEOUT = 8    /* a kernel gave up on a bounded wait (bs_get_device_error) */
+} bs_status;
+
+typedef enum {
+  BS_OUT_BF16 = 0, /* bfloat16, round-to-nearest-even from the fp32 result */
+  BS_OUT_F32 = 1,  /* float32 */
+  BS_OUT_I32 = 2   /* raw int32 accumulator (int_scaled_mm only) */
+} bs_out_dtype;
+
+/*
+ * Operation 1 -- FP8 block-scaled GEMM.
+ *
+ *   out[m, n] = sum_kb  scale_a[m, kb] * scale_b[kb, n / 128]
+ *                       * sum_{k in block kb} A[m, k] * B[k, n]
+ *
+ * i.e. (A . expand(scale_a)) @ (B . expand(scale_b)) with 1x128 activation
+ * groups and 128x128 weight blocks.  Source: pytorch issue "torch._scaled_mm
+ * with blockwise scaling doesn't work with torch.compile" -- the error text
+ * gives scale_a (16640, 64) and scale_b (64, 40) for M = 16640, K = 8192,
+ * N = 5120, that is scale_a [M, K/128] and scale_b [K/128, N/128].
+ * Accumulation is fp32 inside each 128-deep block and across blocks.
+ *
+ *   A        e4m3 [M, K], row m at A + m*lda                (lda >= K)
+ *   B        e4m3 [K, N] column-major, column n at B + n*ldb (ldb >= K)
+ *   scale_a  fp32 [M, K/128], element (m, kb) at scale_a[m*sa_sm + kb*sa_sk]
+ *   scale_b  fp32 [K/128, ceil(N/128)], element (kb, nb) at
+ *            scale_b[kb*sb_sk + nb*sb_sn]
+ *   out      [M, N] row-major, row stride ldo (>= N), BS_OUT_BF16 or BS_OUT_F32
+ *   K must be a multiple of 128 (one scale per 128-deep group).
+ */
+bs_status bs_gemm_fp8_blockwise(const void* A, int64_t lda, const void* B, int64_t ldb,
+                                const float* scale_a, int64_t sa_sm, int64_t sa_sk,
+                                const float* scale_b, int64_t sb_sk, int64_t sb_sn,
+                                void* out, int64_t ldo, bs_out_dtype out_dtype,
+                                int64_t M, int64_t N, int64_t K, void* stream);
+
+/*
+ * Operation 2 -- INT8 GEMM with a fused, fixed-order fp32 dequantisation.
+ *
+ *   acc[m, n] = sum_k A[m, k] * B[k, n]              (exact, int32)
+ *   out[m, n] = (float(acc) * s_a[m]) * s_b[n]       (two fp32 RNE multiplies)
+ *
+ * Sources: pytorch/ao PR "Remove int_scaled_mm's dependency on triton for
+ * cpu" (the CPU definition: _int_mm, then cast to the scale dtype and
+ * multiply); pytorch/ao issue "Unify scaled INT8 matmul" (both scales fused,
+ * the int32 accumulator cast to fp32 before scaling).  s_b == NULL gives the
+ * row-scale-only form of that CPU definition; s_a == NULL skips the row
+ * multiply.  BS_OUT_BF16 rounds the fp32 result to nearest-even;
+ * BS_OUT_I32 writes acc and ignores the scales (the int32 output layout of
+ * tuned_int_mm, pytorch/torch/_inductor/kernel/mm.py).
+ *
+ *   A    int8 [M, K] row-major (lda >= K);  B int8 [K, N] column-major (ldb >= K)
+ *   s_a  fp32 [M] or NULL;  s_b fp32 [N] or NULL
+ *   out  [M, N] row-major, row stride ldo (>= N)
+ *   K <= 131071, which keeps every int32 accumulator exact.
+ */
+bs_status int_scaled_mm(const int8_t* A, int64_t lda, const int8_t* B, int64_t ldb,
+                        const float* s_a, const float* s_b,
+                        void* out, int64_t ldo, bs_out_dtype out_dtype,
+                        int64_t M, int64_t N, int64_t K, void* stream);
+
+/*
+ * Operation 3 -- batched FP8 GEMM with e8m0 (power-of-two) block scales.
+ *
+ *   out[m, g, n] = sum_kb 2^(x_scale[m, g, kb] - 127) * 2^(w_scale[g, n/128, kb] - 127)
+ *                         * sum_{k in block kb} x[m, g, k] * w[g, n, k]
+ *
+ * Source: ROCm/aiter PR "Add opus fp8 mxscale BMM kernels for gfx950"
+ * (Motivation: the m-major layout x [M, G, K], w [G, N, K] batch-major,
+ * x_scale [M, G, K/128], w_scale [G, N/128, K/128], optional out [M, G, N],
+ * bf16 output; Test Plan: m-major and batch-first layouts of x).
+ *
+ *   x        e4m3, element (m, g, k) at x[m*x_sm + g*x_sg + k].  m-major:
+ *            (x_sm, x_sg) = (G*K, K); batch-first storage [G, M, K]: (K, M*K).
+ *   w        e4m3, element (g, n, k) at w[g*w_sg + n*w_sn + k]  (w_sn >= K)
+ *   x_scale  e8m0 bytes [M, G, K/128], contiguous
+ *   w_scale  e8m0 bytes [G, ceil(N/128), K/128], contiguous
+ *   out      element (m, g, n) at out[m*o_sm + g*o_sg + n]; BS_OUT_BF16 or BS_OUT_F32
+ *   K must be a multiple of 128.  Scale byte 255 encodes NaN and is not checked.
+ */
+bs_status bmm_a8w8_blockscale(const void* x, int64_t x_sm, int64_t x_sg,
+                              const void* w, int64_t w_sg, int64_t w_sn,
+                              const uint8_t* x_scale, const uint8_t* w_scale,
+                              void* out, int64_t o_sm, int64_t o_sg, bs_out_dtype out_dtype,
+                              int64_t M, int64_t G, int64_t N, int64_t K, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* host-side helpers (no device work unless stated)                          */
+/* ------------------------------------------------------------------------ */
+
+/* Static name of a status code ("BS_OK", ...).  Never NULL. */
+const char* bs_status_string(bs_status status);
+
+/* Human-readable detail of the last error returned on the calling host
+ * thread (empty string after a successful call).  Never NULL. */
+const char* bs_last_error_message(void);
+
+/*
+ * Shape rule of operation 1 (the blockwise case of the scale-shape check in
+ * the pytorch issue above): BS_OK iff scale_a is [M, ceil(K/128)] and scale_b
+ * is [ceil(K/128), ceil(N/128)].  The rowwise shapes (M, 1) / (1, N) are
+ * rejected here.  Pure host logic.
+ */
+bs_status bs_check_blockwise_scale_shapes(int64_t M, int64_t N, int64_t K,
+                                          int64_t sa_rows, int64_t sa_cols,
+                                          int64_t sb_rows, int64_t sb_cols);
+
+/* Which kernel a call would launch, for tests and benchmarks. */
+typedef struct {
+  int32_t kernel;  /* 0: none (empty problem), 1: persistent wide, 2: skinny split-K, 3: zero fill */
+  int32_t tile_m;  /* rows of A (M direction) per tile */
+  int32_t tile_n;  /* columns of B (N direction) per tile */
+  int32_t splits;  /* K splits reduced through cluster shared memory (1 = none) */
+  int32_t ctas;    /* CTAs launched */
+  int32_t cluster; /* CTAs per thread-block cluster */
+  int32_t launches;/* kernel launches the call makes */
+} bs_plan;
+
+/* Plan of operation `op` (1 = bs_gemm_fp8_blockwise, 2 = int_scaled_mm,
+ * 3 = bmm_a8w8_blockscale; G = 1 for ops 1 and 2) on a GPU with `num_sms`
+ * streaming multiprocessors.  Pure host logic; honours bs_set_path_override. */
+bs_status bs_plan_for(int32_t op, int64_t M, int64_t G, int64_t N, int64_t K, int32_t num_sms, bs_plan* plan);
+
+/* Force the kernel family for subsequent calls in this process (testing):
+ * 0 = automatic (default), 1 = persistent wide kernel, 2 = skinny split-K
+ * kernel where the operation has one.  Returns the previous setting. */
+int32_t bs_set_path_override(int32_t path);
+
+/* The persistent tile order: fills out[3*t .. 3*t+2] = (batch, tile_row,
+ * tile_col) of linear tile t for t < count (host copy of the mapping the
+ * kernels use).  Pure host logic. */
+bs_status bs_tile_order(int32_t grid_m, int32_t grid_n, int32_t batches, int32_t group_m,
+                        int32_t* out, int64_t count);
+
+/*
+ * Synchronises `stream`, then reads and clears this device's error word,
+ * which a kernel sets when one of its bounded waits gives up (instead of
+ * hanging).  Returns BS_ERR_TIMEOUT and stores the code (0x1000 | role<<8 |
+ * wait kind) in *code when it was set, BS_OK and 0 otherwise.  `code` may be
+ * NULL.  Device work: one stream synchronisation and two small copies.
+ */
+bs_status bs_get_device_error(void* stream, uint32_t* code);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+int32_t bs_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BSGEMM_H */

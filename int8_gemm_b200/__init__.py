@@ -1,0 +1,278 @@
+"""bsgemm: scaled low-precision GEMMs with fused dequantisation for NVIDIA B200.
+
+Thin Python binding over ``libbsgemm.so`` (C ABI, ``include/bsgemm.h``).  The
+functions below only check and marshal arguments -- pointers, strides, the
+current CUDA stream -- and allocate ``out`` when it is not given; every
+arithmetic step runs in the library's sm_100a kernels.  There is no CPU
+fallback: if the library is missing or the device is not an sm_100 GPU the
+calls raise.
+
+    bs_gemm_fp8_blockwise(A, B, scale_a, scale_b, out_dtype=torch.bfloat16)
+    int_scaled_mm(A, B, s_a, s_b=None, out_dtype=torch.float32)
+    bmm_a8w8_blockscale(x, w, x_scale, w_scale, out_dtype=torch.bfloat16)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libbsgemm.so")
+
+BS_OK, BS_ERR_NULL, BS_ERR_SHAPE, BS_ERR_LAYOUT, BS_ERR_ALIGNMENT = 0, 1, 2, 3, 4
+BS_ERR_DTYPE, BS_ERR_DEVICE, BS_ERR_CUDA, BS_ERR_TIMEOUT = 5, 6, 7, 8
+BS_OUT_BF16, BS_OUT_F32, BS_OUT_I32 = 0, 1, 2
+
+PATH_AUTO, PATH_WIDE, PATH_SKINNY = 0, 1, 2
+
+_OUT_CODE = {torch.bfloat16: BS_OUT_BF16, torch.float32: BS_OUT_F32, torch.int32: BS_OUT_I32}
+
+
+class BsgemmError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(message)
+        self.status = status
+
+
+class Plan(ctypes.Structure):
+    _fields_ = [("kernel", ctypes.c_int32), ("tile_m", ctypes.c_int32), ("tile_n", ctypes.c_int32),
+                ("splits", ctypes.c_int32), ("ctas", ctypes.c_int32), ("cluster", ctypes.c_int32),
+                ("launches", ctypes.c_int32)]
+
+    def as_dict(self):
+        return {f: getattr(self, f) for f, _ in self._fields_}
+
+
+_lock = threading.Lock()
+_handle = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libbsgemm.so (raises if it has not been built)."""
+    global _handle
+    with _lock:
+        if _handle is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(f"{LIB_PATH} is missing; build it with `python -m int8_gemm_b200.build`")
+            h = ctypes.CDLL(LIB_PATH)
+            i64, p, i32, u32p = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int32, ctypes.POINTER(ctypes.c_uint32)
+            h.bs_gemm_fp8_blockwise.argtypes = [p, i64, p, i64, p, i64, i64, p, i64, i64, p, i64, ctypes.c_int,
+                                                i64, i64, i64, p]
+            h.int_scaled_mm.argtypes = [p, i64, p, i64, p, p, p, i64, ctypes.c_int, i64, i64, i64, p]
+            h.bmm_a8w8_blockscale.argtypes = [p, i64, i64, p, i64, i64, p, p, p, i64, i64, ctypes.c_int,
+                                              i64, i64, i64, i64, p]
+            for f in (h.bs_gemm_fp8_blockwise, h.int_scaled_mm, h.bmm_a8w8_blockscale):
+                f.restype = ctypes.c_int
+            h.bs_status_string.argtypes = [ctypes.c_int]
+            h.bs_status_string.restype = ctypes.c_char_p
+            h.bs_last_error_message.argtypes = []
+            h.bs_last_error_message.restype = ctypes.c_char_p
+            h.bs_check_blockwise_scale_shapes.argtypes = [i64] * 7
+            h.bs_check_blockwise_scale_shapes.restype = ctypes.c_int
+            h.bs_plan_for.argtypes = [i32, i64, i64, i64, i64, i32, ctypes.POINTER(Plan)]
+            h.bs_plan_for.restype = ctypes.c_int
+            h.bs_set_path_override.argtypes = [i32]
+            h.bs_set_path_override.restype = i32
+            h.bs_tile_order.argtypes = [i32, i32, i32, i32, ctypes.POINTER(ctypes.c_int32), i64]
+            h.bs_tile_order.restype = ctypes.c_int
+            h.bs_get_device_error.argtypes = [p, u32p]
+            h.bs_get_device_error.restype = ctypes.c_int
+            h.bs_version.restype = i32
+            _handle = h
+    return _handle
+
+
+def _check(status: int):
+    if status != BS_OK:
+        h = lib()
+        name = h.bs_status_string(status).decode()
+        msg = h.bs_last_error_message().decode()
+        raise BsgemmError(status, f"{name}: {msg}")
+
+
+def status_string(status: int) -> str:
+    return lib().bs_status_string(status).decode()
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _cuda(t, name):
+    if not isinstance(t, torch.Tensor) or t.device.type != "cuda":
+        raise BsgemmError(BS_ERR_DEVICE, f"{name} must be a CUDA tensor (there is no CPU path)")
+
+
+def _bytes8(t: torch.Tensor, name: str) -> torch.Tensor:
+    if t.dtype in (torch.float8_e4m3fn, torch.uint8, torch.int8):
+        return t
+    raise BsgemmError(BS_ERR_DTYPE, f"{name} must be float8_e4m3fn (or its uint8 bytes), got {t.dtype}")
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def bs_gemm_fp8_blockwise(A: torch.Tensor, B: torch.Tensor, scale_a: torch.Tensor, scale_b: torch.Tensor,
+                          out_dtype: torch.dtype = torch.bfloat16, out: torch.Tensor | None = None) -> torch.Tensor:
+    """FP8 block-scaled GEMM: out = (A . expand(scale_a)) @ (B . expand(scale_b)).
+
+    A       e4m3 [M, K] row-major (A.stride(1) == 1)
+    B       e4m3 [K, N] column-major (B.stride(0) == 1), e.g. ``B_t.t()`` for B_t [N, K]
+    scale_a fp32 [M, K/128] (1x128 groups, any strides)
+    scale_b fp32 [K/128, N/128] (128x128 blocks, any strides)
+    """
+    for t, n in ((A, "A"), (B, "B"), (scale_a, "scale_a"), (scale_b, "scale_b")):
+        _cuda(t, n)
+    _bytes8(A, "A"), _bytes8(B, "B")
+    if A.dim() != 2 or B.dim() != 2 or A.shape[1] != B.shape[0]:
+        raise BsgemmError(BS_ERR_SHAPE, f"A [M,K] and B [K,N] expected, got {tuple(A.shape)} and {tuple(B.shape)}")
+    M, K = A.shape
+    N = B.shape[1]
+    if scale_a.dtype != torch.float32 or scale_b.dtype != torch.float32:
+        raise BsgemmError(BS_ERR_DTYPE, "scale_a and scale_b must be float32")
+    if scale_a.dim() != 2 or scale_b.dim() != 2:
+        raise BsgemmError(BS_ERR_SHAPE, "scale_a and scale_b must be 2-D")
+    _check(lib().bs_check_blockwise_scale_shapes(M, N, K, *scale_a.shape, *scale_b.shape))
+    if A.stride(1) != 1 and M > 1:
+        raise BsgemmError(BS_ERR_LAYOUT, f"A must be row-major, got strides {A.stride()}")
+    if B.stride(0) != 1 and N > 1:
+        raise BsgemmError(BS_ERR_LAYOUT, f"B must be column-major, got strides {B.stride()}")
+    if out_dtype not in (torch.bfloat16, torch.float32):
+        raise BsgemmError(BS_ERR_DTYPE, f"out_dtype must be bfloat16 or float32, got {out_dtype}")
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=A.device)
+    elif out.dtype != out_dtype or tuple(out.shape) != (M, N) or out.stride(1) != 1:
+        raise BsgemmError(BS_ERR_LAYOUT, "out must be a row-major [M, N] tensor of out_dtype")
+    with torch.cuda.device(A.device):
+        _check(lib().bs_gemm_fp8_blockwise(
+            _ptr(A), A.stride(0), _ptr(B), B.stride(1), _ptr(scale_a), scale_a.stride(0), scale_a.stride(1),
+            _ptr(scale_b), scale_b.stride(0), scale_b.stride(1), _ptr(out), out.stride(0), _OUT_CODE[out_dtype],
+            M, N, K, _stream(A.device)))
+    return out
+
+
+def int_scaled_mm(A: torch.Tensor, B: torch.Tensor, s_a: torch.Tensor | None, s_b: torch.Tensor | None = None,
+                  out_dtype: torch.dtype = torch.float32, out: torch.Tensor | None = None) -> torch.Tensor:
+    """INT8 GEMM with fused (float(acc) * s_a[m]) * s_b[n].
+
+    A int8 [M, K] row-major; B int8 [K, N] column-major; s_a fp32 [M] / [M, 1] or None;
+    s_b fp32 [N] / [1, N] or None.  out_dtype float32, bfloat16 or int32 (raw accumulator).
+    """
+    _cuda(A, "A"), _cuda(B, "B")
+    if A.dtype != torch.int8 or B.dtype != torch.int8:
+        raise BsgemmError(BS_ERR_DTYPE, "A and B must be int8")
+    if A.dim() != 2 or B.dim() != 2 or A.shape[1] != B.shape[0]:
+        raise BsgemmError(BS_ERR_SHAPE, f"A [M,K] and B [K,N] expected, got {tuple(A.shape)} and {tuple(B.shape)}")
+    M, K = A.shape
+    N = B.shape[1]
+    sa = sb = None
+    if s_a is not None:
+        _cuda(s_a, "s_a")
+        if s_a.dtype != torch.float32 or s_a.numel() != M:
+            raise BsgemmError(BS_ERR_SHAPE, f"s_a must be float32 with M={M} elements")
+        sa = s_a.reshape(M).contiguous()
+    if s_b is not None:
+        _cuda(s_b, "s_b")
+        if s_b.dtype != torch.float32 or s_b.numel() != N:
+            raise BsgemmError(BS_ERR_SHAPE, f"s_b must be float32 with N={N} elements")
+        sb = s_b.reshape(N).contiguous()
+    if A.stride(1) != 1 and M > 1:
+        raise BsgemmError(BS_ERR_LAYOUT, f"A must be row-major, got strides {A.stride()}")
+    if B.stride(0) != 1 and N > 1:
+        raise BsgemmError(BS_ERR_LAYOUT, f"B must be column-major, got strides {B.stride()}")
+    if out_dtype not in _OUT_CODE:
+        raise BsgemmError(BS_ERR_DTYPE, f"out_dtype must be float32, bfloat16 or int32, got {out_dtype}")
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=A.device)
+    elif out.dtype != out_dtype or tuple(out.shape) != (M, N) or out.stride(1) != 1:
+        raise BsgemmError(BS_ERR_LAYOUT, "out must be a row-major [M, N] tensor of out_dtype")
+    with torch.cuda.device(A.device):
+        _check(lib().int_scaled_mm(_ptr(A), A.stride(0), _ptr(B), B.stride(1), _ptr(sa), _ptr(sb), _ptr(out),
+                                   out.stride(0), _OUT_CODE[out_dtype], M, N, K, _stream(A.device)))
+    return out
+
+
+def _e8m0_bytes(t: torch.Tensor, name: str) -> torch.Tensor:
+    if t.dtype == torch.uint8:
+        return t
+    if hasattr(torch, "float8_e8m0fnu") and t.dtype == torch.float8_e8m0fnu:
+        return t.view(torch.uint8)
+    raise BsgemmError(BS_ERR_DTYPE, f"{name} must hold e8m0 bytes (uint8 or float8_e8m0fnu), got {t.dtype}")
+
+
+def bmm_a8w8_blockscale(x: torch.Tensor, w: torch.Tensor, x_scale: torch.Tensor, w_scale: torch.Tensor,
+                        out_dtype: torch.dtype = torch.bfloat16, out: torch.Tensor | None = None) -> torch.Tensor:
+    """Batched FP8 GEMM with e8m0 block scales: out[m, g, :] = x[m, g, :] @ w[g]^T (dequantised).
+
+    x        e4m3 [M, G, K] with x.stride(2) == 1 (m-major or batch-first storage)
+    w        e4m3 [G, N, K] with w.stride(2) == 1
+    x_scale  e8m0 [M, G, K/128] contiguous;  w_scale e8m0 [G, N/128, K/128] contiguous
+    """
+    for t, n in ((x, "x"), (w, "w"), (x_scale, "x_scale"), (w_scale, "w_scale")):
+        _cuda(t, n)
+    _bytes8(x, "x"), _bytes8(w, "w")
+    xs, ws = _e8m0_bytes(x_scale, "x_scale"), _e8m0_bytes(w_scale, "w_scale")
+    if x.dim() != 3 or w.dim() != 3 or x.shape[1] != w.shape[0] or x.shape[2] != w.shape[2]:
+        raise BsgemmError(BS_ERR_SHAPE, f"x [M,G,K] and w [G,N,K] expected, got {tuple(x.shape)}, {tuple(w.shape)}")
+    M, G, K = x.shape
+    N = w.shape[1]
+    KB, NB = -(-K // 128), -(-N // 128)
+    if tuple(xs.shape) != (M, G, KB) or tuple(ws.shape) != (G, NB, KB):
+        raise BsgemmError(BS_ERR_SHAPE, f"x_scale must be [{M},{G},{KB}] and w_scale [{G},{NB},{KB}], got "
+                          f"{tuple(xs.shape)} and {tuple(ws.shape)}")
+    if not xs.is_contiguous() or not ws.is_contiguous():
+        raise BsgemmError(BS_ERR_LAYOUT, "x_scale and w_scale must be contiguous")
+    if x.stride(2) != 1 or w.stride(2) != 1:
+        raise BsgemmError(BS_ERR_LAYOUT, "x and w must have unit stride along K")
+    if out_dtype not in (torch.bfloat16, torch.float32):
+        raise BsgemmError(BS_ERR_DTYPE, f"out_dtype must be bfloat16 or float32, got {out_dtype}")
+    if out is None:
+        out = torch.empty((M, G, N), dtype=out_dtype, device=x.device)
+    elif out.dtype != out_dtype or tuple(out.shape) != (M, G, N) or out.stride(2) != 1:
+        raise BsgemmError(BS_ERR_LAYOUT, "out must be [M, G, N] of out_dtype with unit stride along N")
+    with torch.cuda.device(x.device):
+        _check(lib().bmm_a8w8_blockscale(
+            _ptr(x), x.stride(0), x.stride(1), _ptr(w), w.stride(0), w.stride(1), _ptr(xs), _ptr(ws), _ptr(out),
+            out.stride(0), out.stride(1), _OUT_CODE[out_dtype], M, G, N, K, _stream(x.device)))
+    return out
+
+
+# ---------------------------------------------------------------------------
+# host-side helpers
+# ---------------------------------------------------------------------------
+OP_FP8_BLOCKWISE, OP_INT_SCALED_MM, OP_BMM = 1, 2, 3
+
+
+def plan_for(op: int, M: int, G: int, N: int, K: int, num_sms: int = 148) -> dict:
+    p = Plan()
+    _check(lib().bs_plan_for(op, M, G, N, K, num_sms, ctypes.byref(p)))
+    return p.as_dict()
+
+
+def set_path_override(path: int) -> int:
+    return lib().bs_set_path_override(path)
+
+
+def tile_order(grid_m: int, grid_n: int, batches: int = 1, group_m: int = 16):
+    n = grid_m * grid_n * batches
+    buf = (ctypes.c_int32 * (3 * n))()
+    _check(lib().bs_tile_order(grid_m, grid_n, batches, group_m, buf, n))
+    return [(buf[3 * i], buf[3 * i + 1], buf[3 * i + 2]) for i in range(n)]
+
+
+def device_error(stream: torch.cuda.Stream | None = None) -> int:
+    """Synchronise and read/clear the device error word (0 = no kernel timed out)."""
+    code = ctypes.c_uint32(0)
+    s = ctypes.c_void_p((stream or torch.cuda.current_stream()).cuda_stream)
+    st = lib().bs_get_device_error(s, ctypes.byref(code))
+    if st not in (BS_OK, BS_ERR_TIMEOUT):
+        _check(st)
+    return code.value
+
+
+def version() -> int:
+    return lib().bs_version()

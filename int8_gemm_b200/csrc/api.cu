@@ -1,0 +1,528 @@
+// C-ABI layer: argument validation, kernel planning, tensor-map encoding and
+// launches.  All heavy work happens in the sm_100a kernels; nothing here
+// computes a GEMM result, and there is no fallback path.
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "bsgemm.h"
+#include "launch.h"
+
+using namespace bsg;
+
+// Per-device error word written by kernels whose bounded waits give up.
+__device__ uint32_t g_bs_error_word = 0;
+
+namespace {
+
+// ---------------------------------------------------------------------------
+// error reporting
+// ---------------------------------------------------------------------------
+thread_local char g_msg[512] = {0};
+
+bs_status fail(bs_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+void clear_msg() { g_msg[0] = 0; }
+
+// ---------------------------------------------------------------------------
+// driver entry point for tensor-map encoding (no link-time libcuda dependency)
+// ---------------------------------------------------------------------------
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// ---------------------------------------------------------------------------
+// per-device facts
+// ---------------------------------------------------------------------------
+struct DeviceCtx {
+  int sms = 0;
+  uint32_t* err = nullptr;
+  bool ready = false;
+  bs_status status = BS_OK;
+};
+
+constexpr int kMaxDevices = 64;
+DeviceCtx g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+bs_status device_ctx(DeviceCtx** out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(BS_ERR_DEVICE, "no CUDA device: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= kMaxDevices) return fail(BS_ERR_DEVICE, "device index %d out of range", dev);
+  DeviceCtx& d = g_dev[dev];
+  if (!d.ready) {
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    if (!d.ready) {
+      int major = 0, minor = 0, sms = 0;
+      cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+      if (major != 10 || minor != 0) {
+        d.status = BS_ERR_DEVICE;
+      } else {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_bs_error_word);
+        if (e != cudaSuccess) {
+          d.status = BS_ERR_CUDA;
+        } else {
+          d.err = static_cast<uint32_t*>(p);
+          d.sms = sms;
+          d.status = BS_OK;
+        }
+      }
+      d.ready = true;
+    }
+  }
+  if (d.status == BS_ERR_DEVICE) return fail(BS_ERR_DEVICE, "device %d is not an sm_100 GPU", dev);
+  if (d.status != BS_OK) return fail(d.status, "device %d setup failed", dev);
+  *out = &d;
+  return BS_OK;
+}
+
+// ---------------------------------------------------------------------------
+// planning (pure host logic)
+// ---------------------------------------------------------------------------
+std::atomic<int32_t> g_path_override{0};
+
+constexpr int kSkinnyMaxM = 256;
+constexpr int kGroupM = 16;
+
+struct Plan {
+  bs_plan pub;
+  int bmt = 0;
+  int m_tiles = 0, n_tiles = 0;
+  int grid_m = 0, grid_n = 0, num_tiles = 0;
+};
+
+Plan make_plan(int op, int64_t M, int64_t G, int64_t N, int64_t K, int sms) {
+  Plan x;
+  std::memset(&x.pub, 0, sizeof(x.pub));
+  if (M == 0 || N == 0 || G == 0) return x;  // kernel 0: nothing to do
+  if (K == 0) {
+    x.pub.kernel = 3;
+    x.pub.launches = 1;
+    x.pub.splits = 1;
+    x.pub.cluster = 1;
+    x.pub.ctas = sms > 0 ? 2 * sms : 1;
+    return x;
+  }
+  const int KB = static_cast<int>((K + 127) / 128);
+  const int ov = g_path_override.load();
+  const bool skinny_ok = op != 2;
+  const bool skinny = skinny_ok && (ov == 2 || (ov == 0 && M <= kSkinnyMaxM));
+  if (skinny) {
+    const int bmt = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128;
+    x.bmt = bmt;
+    x.m_tiles = static_cast<int>((M + bmt - 1) / bmt);
+    x.n_tiles = static_cast<int>((N + 127) / 128);
+    const long long units = static_cast<long long>(x.m_tiles) * x.n_tiles * G;
+    int S = 1;
+    while (S < 8 && 2 * S <= KB && units * S < 2LL * (sms > 0 ? sms : 148)) S *= 2;
+    x.pub.kernel = 2;
+    x.pub.tile_m = bmt;
+    x.pub.tile_n = 128;
+    x.pub.splits = S;
+    x.pub.cluster = S;
+    x.pub.ctas = static_cast<int32_t>(units * S);
+    x.pub.launches = 1;
+  } else {
+    x.grid_m = static_cast<int>((M + 127) / 128);
+    x.grid_n = static_cast<int>((N + kWideBN - 1) / kWideBN);
+    const long long tiles = static_cast<long long>(x.grid_m) * x.grid_n * G;
+    x.num_tiles = static_cast<int>(tiles);
+    x.pub.kernel = 1;
+    x.pub.tile_m = 128;
+    x.pub.tile_n = kWideBN;
+    x.pub.splits = 1;
+    x.pub.cluster = 1;
+    x.pub.ctas = static_cast<int32_t>(tiles < sms ? tiles : sms);
+    x.pub.launches = 1;
+  }
+  return x;
+}
+
+// ---------------------------------------------------------------------------
+// tensor maps
+// ---------------------------------------------------------------------------
+bs_status encode_3d(CUtensorMap* map, CUtensorMapDataType dt, int esize, const void* base, uint64_t d0, uint64_t d1,
+                    uint64_t d2, uint64_t s1, uint64_t s2, uint32_t box0, uint32_t box1, const char* what) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return fail(BS_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const cuuint64_t dims[3] = {d0, d1, d2};
+  const cuuint64_t strides[2] = {s1 * static_cast<uint64_t>(esize), s2 * static_cast<uint64_t>(esize)};
+  const cuuint32_t box[3] = {box0, box1, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = enc(map, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(BS_ERR_CUDA, "tensor map encoding failed for %s (CUresult %d)", what, static_cast<int>(r));
+  return BS_OK;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+int out_size(bs_out_dtype t) { return t == BS_OUT_BF16 ? 2 : 4; }
+
+CUtensorMapDataType out_tmap_type(bs_out_dtype t) {
+  return t == BS_OUT_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                          : (t == BS_OUT_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_INT32);
+}
+
+OutKind out_kind(bs_out_dtype t) {
+  return t == BS_OUT_BF16 ? OutKind::kBF16 : (t == BS_OUT_F32 ? OutKind::kF32 : OutKind::kI32);
+}
+
+constexpr int64_t kMaxDim = 0x7FFFFFFF;
+
+bs_status check_launch(cudaError_t e, const char* what) {
+  if (e != cudaSuccess) return fail(BS_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  e = cudaPeekAtLastError();
+  if (e != cudaSuccess) return fail(BS_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  return BS_OK;
+}
+
+// Shared launch of the FP8 paths (operations 1 and 3).  Coordinates of the
+// three-dimensional tensor maps are (k, row, batch) for operands and
+// (n, m, batch) for the output.
+struct Fp8Problem {
+  const void* a;
+  int64_t a_rs, a_bs;  // row and batch strides of A (bytes)
+  const void* b;
+  int64_t b_rs, b_bs;  // row (= output column) and batch strides of B (bytes)
+  void* out;
+  int64_t o_rs, o_bs;  // row and batch strides of out (elements)
+  bs_out_dtype out_dtype;
+  int64_t M, G, N, K;
+  Mode mode;
+};
+
+bs_status run_fp8(const Fp8Problem& q, GemmArgs args, cudaStream_t stream, DeviceCtx* dc) {
+  const Plan pl = make_plan(q.mode == Mode::kFp8E8M0 ? 3 : 1, q.M, q.G, q.N, q.K, dc->sms);
+  if (pl.pub.kernel == 0) return BS_OK;
+  if (pl.pub.kernel == 3)
+    return check_launch(launch_fill_zero(q.out, out_size(q.out_dtype), q.M, q.N, q.o_rs, q.G, q.o_bs, stream),
+                        "zero-fill launch");
+  args.err = dc->err;
+  CUtensorMap ta, tb, td;
+  const uint64_t a_bs = q.G > 1 ? static_cast<uint64_t>(q.a_bs) : static_cast<uint64_t>(q.a_rs) * q.M;
+  const uint64_t b_bs = q.G > 1 ? static_cast<uint64_t>(q.b_bs) : static_cast<uint64_t>(q.b_rs) * q.N;
+  const uint64_t o_bs = q.G > 1 ? static_cast<uint64_t>(q.o_bs) : static_cast<uint64_t>(q.o_rs) * q.M;
+  bs_status st;
+  if (pl.pub.kernel == 1) {
+    args.grid_m = pl.grid_m;
+    args.grid_n = pl.grid_n;
+    args.num_tiles = pl.num_tiles;
+    args.group_m = kGroupM;
+    args.splits = 1;
+    if ((st = encode_3d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, q.a, q.K, q.M, q.G, q.a_rs, a_bs, 128, 128, "A")))
+      return st;
+    if ((st = encode_3d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, q.b, q.K, q.N, q.G, q.b_rs, b_bs, 128, kWideBN, "B")))
+      return st;
+    const int es = out_size(q.out_dtype);
+    if ((st = encode_3d(&td, out_tmap_type(q.out_dtype), es, q.out, q.N, q.M, q.G, q.o_rs, o_bs,
+                        static_cast<uint32_t>(128 / es), 32, "out")))
+      return st;
+    return check_launch(launch_wide(q.mode, out_kind(q.out_dtype), ta, tb, td, args, pl.pub.ctas, stream),
+                        "wide kernel launch");
+  }
+  args.splits = pl.pub.splits;
+  if ((st = encode_3d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, q.a, q.K, q.M, q.G, q.a_rs, a_bs, 128,
+                      static_cast<uint32_t>(pl.bmt), "A")))
+    return st;
+  if ((st = encode_3d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, q.b, q.K, q.N, q.G, q.b_rs, b_bs, 128, 128, "B")))
+    return st;
+  SkinnyOut o;
+  o.out = q.out;
+  o.o_sm = q.o_rs;
+  o.o_sg = q.o_bs;
+  return check_launch(
+      launch_skinny(q.mode, out_kind(q.out_dtype), pl.bmt, ta, tb, args, o, pl.n_tiles, pl.m_tiles, stream),
+      "skinny kernel launch");
+}
+
+}  // namespace
+
+// ===========================================================================
+// C ABI
+// ===========================================================================
+extern "C" {
+
+const char* bs_status_string(bs_status s) {
+  switch (s) {
+    case BS_OK: return "BS_OK";
+    case BS_ERR_NULL: return "BS_ERR_NULL";
+    case BS_ERR_SHAPE: return "BS_ERR_SHAPE";
+    case BS_ERR_LAYOUT: return "BS_ERR_LAYOUT";
+    case BS_ERR_ALIGNMENT: return "BS_ERR_ALIGNMENT";
+    case BS_ERR_DTYPE: return "BS_ERR_DTYPE";
+    case BS_ERR_DEVICE: return "BS_ERR_DEVICE";
+    case BS_ERR_CUDA: return "BS_ERR_CUDA";
+    case BS_ERR_TIMEOUT: return "BS_ERR_TIMEOUT";
+  }
+  return "BS_ERR_UNKNOWN";
+}
+
+const char* bs_last_error_message(void) { return g_msg; }
+
+int32_t bs_version(void) { return 100; }
+
+bs_status bs_check_blockwise_scale_shapes(int64_t M, int64_t N, int64_t K, int64_t sa_rows, int64_t sa_cols,
+                                          int64_t sb_rows, int64_t sb_cols) {
+  clear_msg();
+  const int64_t KB = (K + 127) / 128, NB = (N + 127) / 128;
+  if (sa_rows != M || sa_cols != KB || sb_rows != KB || sb_cols != NB)
+    return fail(BS_ERR_SHAPE,
+                "blockwise scaling needs scale_a of shape (%lld, %lld) [1x128 groups] and scale_b of shape "
+                "(%lld, %lld) [128x128 blocks]; got scale_a (%lld, %lld) and scale_b (%lld, %lld)",
+                (long long)M, (long long)KB, (long long)KB, (long long)NB, (long long)sa_rows, (long long)sa_cols,
+                (long long)sb_rows, (long long)sb_cols);
+  return BS_OK;
+}
+
+int32_t bs_set_path_override(int32_t path) { return g_path_override.exchange(path); }
+
+bs_status bs_plan_for(int32_t op, int64_t M, int64_t G, int64_t N, int64_t K, int32_t num_sms, bs_plan* plan) {
+  clear_msg();
+  if (!plan) return fail(BS_ERR_NULL, "plan is NULL");
+  if (op < 1 || op > 3) return fail(BS_ERR_SHAPE, "op must be 1, 2 or 3");
+  if (M < 0 || N < 0 || K < 0 || G < 0 || num_sms <= 0) return fail(BS_ERR_SHAPE, "negative size");
+  *plan = make_plan(op, M, G, N, K, num_sms).pub;
+  return BS_OK;
+}
+
+bs_status bs_tile_order(int32_t grid_m, int32_t grid_n, int32_t batches, int32_t group_m, int32_t* out,
+                        int64_t count) {
+  clear_msg();
+  if (!out) return fail(BS_ERR_NULL, "out is NULL");
+  if (grid_m <= 0 || grid_n <= 0 || batches <= 0 || group_m <= 0) return fail(BS_ERR_SHAPE, "bad grid");
+  if (count > static_cast<int64_t>(grid_m) * grid_n * batches) return fail(BS_ERR_SHAPE, "count exceeds tiles");
+  for (int64_t t = 0; t < count; ++t) {
+    const TileCoord c = tile_coord(static_cast<int>(t), grid_m, grid_n, group_m);
+    out[3 * t + 0] = c.g;
+    out[3 * t + 1] = c.pm;
+    out[3 * t + 2] = c.pn;
+  }
+  return BS_OK;
+}
+
+bs_status bs_get_device_error(void* stream, uint32_t* code) {
+  clear_msg();
+  if (code) *code = 0;
+  DeviceCtx* dc = nullptr;
+  bs_status st = device_ctx(&dc);
+  if (st != BS_OK) return st;
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(BS_ERR_CUDA, "stream synchronize: %s", cudaGetErrorString(e));
+  uint32_t v = 0;
+  e = cudaMemcpy(&v, dc->err, sizeof(v), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return fail(BS_ERR_CUDA, "read error word: %s", cudaGetErrorString(e));
+  if (v == 0) return BS_OK;
+  const uint32_t zero = 0;
+  e = cudaMemcpy(dc->err, &zero, sizeof(zero), cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) return fail(BS_ERR_CUDA, "clear error word: %s", cudaGetErrorString(e));
+  if (code) *code = v;
+  return fail(BS_ERR_TIMEOUT, "a kernel wait timed out (code 0x%x)", v);
+}
+
+bs_status bs_gemm_fp8_blockwise(const void* A, int64_t lda, const void* B, int64_t ldb, const float* scale_a,
+                                int64_t sa_sm, int64_t sa_sk, const float* scale_b, int64_t sb_sk, int64_t sb_sn,
+                                void* out, int64_t ldo, bs_out_dtype out_dtype, int64_t M, int64_t N, int64_t K,
+                                void* stream) {
+  clear_msg();
+  if (M < 0 || N < 0 || K < 0) return fail(BS_ERR_SHAPE, "negative size M=%lld N=%lld K=%lld", (long long)M,
+                                           (long long)N, (long long)K);
+  if (M > kMaxDim || N > kMaxDim || K > kMaxDim) return fail(BS_ERR_SHAPE, "size exceeds 2^31-1");
+  if (K % 128 != 0) return fail(BS_ERR_SHAPE, "K=%lld is not a multiple of 128 (one scale per 128-deep group)",
+                                (long long)K);
+  if (out_dtype != BS_OUT_BF16 && out_dtype != BS_OUT_F32)
+    return fail(BS_ERR_DTYPE, "bs_gemm_fp8_blockwise writes bf16 or f32 only");
+  if (M == 0 || N == 0) return BS_OK;
+  if (!out) return fail(BS_ERR_NULL, "out is NULL");
+  if (ldo < N) return fail(BS_ERR_LAYOUT, "ldo=%lld < N=%lld", (long long)ldo, (long long)N);
+  if (!aligned16(out) || (ldo * out_size(out_dtype)) % 16 != 0)
+    return fail(BS_ERR_ALIGNMENT, "out must be 16-byte aligned with a row stride that is a multiple of 16 bytes");
+  if (K > 0) {
+    if (!A || !B || !scale_a || !scale_b) return fail(BS_ERR_NULL, "A, B, scale_a and scale_b must be non-NULL");
+    if (lda < K || ldb < K) return fail(BS_ERR_LAYOUT, "lda/ldb must be >= K (A row-major, B column-major)");
+    if (!aligned16(A) || !aligned16(B) || lda % 16 != 0 || ldb % 16 != 0)
+      return fail(BS_ERR_ALIGNMENT, "A and B must be 16-byte aligned with lda, ldb multiples of 16");
+    if (!aligned4(scale_a) || !aligned4(scale_b)) return fail(BS_ERR_ALIGNMENT, "scales must be 4-byte aligned");
+    if (sa_sm < 0 || sa_sk < 0 || sb_sk < 0 || sb_sn < 0) return fail(BS_ERR_LAYOUT, "negative scale stride");
+  }
+  DeviceCtx* dc = nullptr;
+  bs_status st = device_ctx(&dc);
+  if (st != BS_OK) return st;
+
+  GemmArgs args;
+  std::memset(&args, 0, sizeof(args));
+  args.M = static_cast<int>(M);
+  args.N = static_cast<int>(N);
+  args.K = static_cast<int>(K);
+  args.G = 1;
+  args.KB = static_cast<int>(K / 128);
+  args.NB = static_cast<int>((N + 127) / 128);
+  args.sa = scale_a;
+  args.sa_sm = sa_sm;
+  args.sa_sk = sa_sk;
+  args.sb = scale_b;
+  args.sb_sk = sb_sk;
+  args.sb_sn = sb_sn;
+  Fp8Problem q{A, lda, 0, B, ldb, 0, out, ldo, 0, out_dtype, M, 1, N, K, Mode::kFp8F32Scale};
+  return run_fp8(q, args, static_cast<cudaStream_t>(stream), dc);
+}
+
+bs_status bmm_a8w8_blockscale(const void* x, int64_t x_sm, int64_t x_sg, const void* w, int64_t w_sg, int64_t w_sn,
+                              const uint8_t* x_scale, const uint8_t* w_scale, void* out, int64_t o_sm, int64_t o_sg,
+                              bs_out_dtype out_dtype, int64_t M, int64_t G, int64_t N, int64_t K, void* stream) {
+  clear_msg();
+  if (M < 0 || N < 0 || K < 0 || G < 0) return fail(BS_ERR_SHAPE, "negative size");
+  if (M > kMaxDim || N > kMaxDim || K > kMaxDim || G > 65535) return fail(BS_ERR_SHAPE, "size out of range");
+  if (K % 128 != 0) return fail(BS_ERR_SHAPE, "K=%lld is not a multiple of 128", (long long)K);
+  if (out_dtype != BS_OUT_BF16 && out_dtype != BS_OUT_F32)
+    return fail(BS_ERR_DTYPE, "bmm_a8w8_blockscale writes bf16 or f32 only");
+  if (M == 0 || N == 0 || G == 0) return BS_OK;
+  if (!out) return fail(BS_ERR_NULL, "out is NULL");
+  const int es = out_size(out_dtype);
+  if (o_sm < 0 || o_sg < 0) return fail(BS_ERR_LAYOUT, "negative output stride");
+  if (!aligned16(out) || (o_sm * es) % 16 != 0 || (o_sg * es) % 16 != 0)
+    return fail(BS_ERR_ALIGNMENT, "out must be 16-byte aligned with strides that are multiples of 16 bytes");
+  if (K > 0) {
+    if (!x || !w || !x_scale || !w_scale) return fail(BS_ERR_NULL, "x, w, x_scale and w_scale must be non-NULL");
+    if (x_sm < 0 || x_sg < 0 || w_sg < 0 || w_sn < K) return fail(BS_ERR_LAYOUT, "bad x / w strides");
+    if (!aligned16(x) || !aligned16(w) || x_sm % 16 || x_sg % 16 || w_sg % 16 || w_sn % 16)
+      return fail(BS_ERR_ALIGNMENT, "x and w must be 16-byte aligned with strides that are multiples of 16");
+  }
+  DeviceCtx* dc = nullptr;
+  bs_status st = device_ctx(&dc);
+  if (st != BS_OK) return st;
+
+  GemmArgs args;
+  std::memset(&args, 0, sizeof(args));
+  args.M = static_cast<int>(M);
+  args.N = static_cast<int>(N);
+  args.K = static_cast<int>(K);
+  args.G = static_cast<int>(G);
+  args.KB = static_cast<int>(K / 128);
+  args.NB = static_cast<int>((N + 127) / 128);
+  args.xs = x_scale;
+  args.ws = w_scale;
+  Fp8Problem q{x, x_sm, x_sg, w, w_sn, w_sg, out, o_sm, o_sg, out_dtype, M, G, N, K, Mode::kFp8E8M0};
+  return run_fp8(q, args, static_cast<cudaStream_t>(stream), dc);
+}
+
+bs_status int_scaled_mm(const int8_t* A, int64_t lda, const int8_t* B, int64_t ldb, const float* s_a,
+                        const float* s_b, void* out, int64_t ldo, bs_out_dtype out_dtype, int64_t M, int64_t N,
+                        int64_t K, void* stream) {
+  clear_msg();
+  if (M < 0 || N < 0 || K < 0) return fail(BS_ERR_SHAPE, "negative size");
+  if (M > kMaxDim || N > kMaxDim) return fail(BS_ERR_SHAPE, "size exceeds 2^31-1");
+  if (K > 131071) return fail(BS_ERR_SHAPE, "K=%lld > 131071 could overflow the int32 accumulator", (long long)K);
+  if (out_dtype != BS_OUT_BF16 && out_dtype != BS_OUT_F32 && out_dtype != BS_OUT_I32)
+    return fail(BS_ERR_DTYPE, "unknown output dtype");
+  if (M == 0 || N == 0) return BS_OK;
+  if (!out) return fail(BS_ERR_NULL, "out is NULL");
+  if (ldo < N) return fail(BS_ERR_LAYOUT, "ldo < N");
+  if (!aligned16(out) || (ldo * out_size(out_dtype)) % 16 != 0)
+    return fail(BS_ERR_ALIGNMENT, "out must be 16-byte aligned with a row stride that is a multiple of 16 bytes");
+  if (K > 0) {
+    if (!A || !B) return fail(BS_ERR_NULL, "A and B must be non-NULL");
+    if (lda < K || ldb < K) return fail(BS_ERR_LAYOUT, "lda/ldb must be >= K (A row-major, B column-major)");
+    if (!aligned16(A) || !aligned16(B) || lda % 16 != 0 || ldb % 16 != 0)
+      return fail(BS_ERR_ALIGNMENT, "A and B must be 16-byte aligned with lda, ldb multiples of 16");
+    if ((s_a && !aligned4(s_a)) || (s_b && !aligned4(s_b)))
+      return fail(BS_ERR_ALIGNMENT, "scales must be 4-byte aligned");
+  }
+  DeviceCtx* dc = nullptr;
+  bs_status st = device_ctx(&dc);
+  if (st != BS_OK) return st;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  const Plan pl = make_plan(2, M, 1, N, K, dc->sms);
+  if (pl.pub.kernel == 3)
+    return check_launch(launch_fill_zero(out, out_size(out_dtype), M, N, ldo, 1, 0, cs), "zero-fill launch");
+
+  GemmArgs args;
+  std::memset(&args, 0, sizeof(args));
+  args.M = static_cast<int>(M);
+  args.N = static_cast<int>(N);
+  args.K = static_cast<int>(K);
+  args.G = 1;
+  args.KB = static_cast<int>((K + 127) / 128);
+  args.NB = static_cast<int>((N + 127) / 128);
+  args.s_row = s_a;
+  args.s_col = s_b;
+  args.grid_m = pl.grid_m;
+  args.grid_n = pl.grid_n;
+  args.num_tiles = pl.num_tiles;
+  args.group_m = kGroupM;
+  args.splits = 1;
+  args.err = dc->err;
+  CUtensorMap ta, tb, td;
+  if ((st = encode_3d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, A, K, M, 1, lda, lda * M, 128, 128, "A"))) return st;
+  if ((st = encode_3d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, B, K, N, 1, ldb, ldb * N, 128, kWideBN, "B")))
+    return st;
+  const int es = out_size(out_dtype);
+  if ((st = encode_3d(&td, out_tmap_type(out_dtype), es, out, N, M, 1, ldo, ldo * M, static_cast<uint32_t>(128 / es),
+                      32, "out")))
+    return st;
+  return check_launch(launch_wide(Mode::kInt8, out_kind(out_dtype), ta, tb, td, args, pl.pub.ctas, cs),
+                      "int8 kernel launch");
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// zero fill (K == 0)
+// ---------------------------------------------------------------------------
+namespace bsg {
+
+__global__ void fill_zero_kernel(char* out, int es, long long rows, long long cols, long long ld, long long batches,
+                                 long long bstride) {
+  const long long total = rows * cols * batches;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long b = i / (rows * cols);
+    const long long rc = i - b * rows * cols;
+    const long long r = rc / cols, c = rc - r * cols;
+    char* p = out + (b * bstride + r * ld + c) * es;
+    if (es == 2)
+      *reinterpret_cast<uint16_t*>(p) = 0;
+    else
+      *reinterpret_cast<uint32_t*>(p) = 0;
+  }
+}
+
+cudaError_t launch_fill_zero(void* out, int elem_size, long long rows, long long cols, long long ld,
+                             long long batches, long long bstride, cudaStream_t stream) {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  fill_zero_kernel<<<2 * sms, 256, 0, stream>>>(static_cast<char*>(out), elem_size, rows, cols, ld, batches, bstride);
+  return cudaGetLastError();
+}
+
+}  // namespace bsg

@@ -1,0 +1,34 @@
+// Internal interface between the C-ABI layer (api.cu) and the kernel
+// translation units.  Not part of the public header.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "skinny_kernel.cuh"
+#include "wide_kernel.cuh"
+
+namespace bsg {
+
+enum class OutKind : int { kBF16 = 0, kF32 = 1, kI32 = 2 };
+
+constexpr int kWideBN = 256;
+constexpr int kWideStages = 4;
+constexpr int kWideThreads = 384;
+constexpr int kSkinnyStages = 4;
+constexpr int kSkinnyThreads = 224;
+
+// Persistent wide kernel over `grid` CTAs.
+cudaError_t launch_wide(Mode mode, OutKind out, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& d,
+                        const GemmArgs& args, int grid, cudaStream_t stream);
+
+// Skinny split-K kernel: grid (n_tiles * splits, m_tiles, G), cluster (splits, 1, 1).
+cudaError_t launch_skinny(Mode mode, OutKind out, int bmt, const CUtensorMap& a, const CUtensorMap& b,
+                          const GemmArgs& args, const SkinnyOut& o, int n_tiles, int m_tiles, cudaStream_t stream);
+
+// Zero-fill of `batches` matrices [rows, cols] (row stride ld, batch stride
+// bstride, elements of `elem_size` bytes).
+cudaError_t launch_fill_zero(void* out, int elem_size, long long rows, long long cols, long long ld,
+                             long long batches, long long bstride, cudaStream_t stream);
+
+}  // namespace bsg

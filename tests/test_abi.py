@@ -1,0 +1,202 @@
+"""Host-side tests of the C-ABI library (no GPU needed).
+
+The library must load and export every function include/bsgemm.h declares;
+argument validation, planning and the persistent tile order are pure host
+logic and are checked here.  No GEMM is computed without a GPU: a well-formed
+call on a machine without an sm_100 device must fail with BS_ERR_DEVICE.
+"""
+from __future__ import annotations
+
+import ctypes
+import json
+import os
+import re
+import subprocess
+
+import pytest
+import torch
+
+import int8_gemm_b200 as bs
+from int8_gemm_b200 import build as bsbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "bsgemm.h")
+GOLDEN = os.path.join(ROOT, "tests", "golden")
+HAS_GPU = torch.cuda.is_available()
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built_library():
+    bsbuild.build()
+    return bs.lib()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*(bs_\w+|int_scaled_mm|bmm_a8w8_blockscale)\s*\(",
+                                 src, flags=re.M)))
+
+
+def test_header_declares_the_three_entry_points():
+    f = declared_functions()
+    for name in ("bs_gemm_fp8_blockwise", "int_scaled_mm", "bmm_a8w8_blockscale"):
+        assert name in f
+    assert len(f) >= 10
+
+
+def test_library_exports_every_declared_symbol():
+    out = subprocess.run(["nm", "-D", "--defined-only", bs.LIB_PATH], capture_output=True, text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    missing = [f for f in declared_functions() if f not in exported]
+    assert not missing, missing
+    for f in declared_functions():
+        assert getattr(bs.lib(), f) is not None
+
+
+def test_status_strings():
+    names = ["BS_OK", "BS_ERR_NULL", "BS_ERR_SHAPE", "BS_ERR_LAYOUT", "BS_ERR_ALIGNMENT", "BS_ERR_DTYPE",
+             "BS_ERR_DEVICE", "BS_ERR_CUDA", "BS_ERR_TIMEOUT"]
+    for code, name in enumerate(names):
+        assert bs.status_string(code) == name
+    assert bs.status_string(99) == "BS_ERR_UNKNOWN"
+    assert bs.version() == 100
+
+
+def test_blockwise_scale_shape_rule_from_the_issue():
+    g = json.load(open(os.path.join(GOLDEN, "scale_shapes_blockwise.json")))
+    h = bs.lib()
+    assert h.bs_check_blockwise_scale_shapes(g["M"], g["N"], g["K"], *g["scale_a"], *g["scale_b"]) == bs.BS_OK
+    st = h.bs_check_blockwise_scale_shapes(g["M"], g["N"], g["K"], *g["rowwise_scale_a"], *g["rowwise_scale_b"])
+    assert st == bs.BS_ERR_SHAPE
+    msg = h.bs_last_error_message().decode()
+    assert "(16640, 64)" in msg and "(64, 40)" in msg and "(16640, 1)" in msg
+    # transposed scale_b is also rejected
+    assert h.bs_check_blockwise_scale_shapes(g["M"], g["N"], g["K"], 16640, 64, 40, 64) == bs.BS_ERR_SHAPE
+
+
+# ---------------------------------------------------------------------------
+# planning
+# ---------------------------------------------------------------------------
+def test_plan_large_fp8_is_persistent_wide():
+    p = bs.plan_for(bs.OP_FP8_BLOCKWISE, 16640, 1, 5120, 8192, 148)
+    assert p == {"kernel": 1, "tile_m": 128, "tile_n": 256, "splits": 1, "ctas": 148, "cluster": 1, "launches": 1}
+
+
+@pytest.mark.parametrize("M", [1, 8, 16, 17, 32, 127, 128, 129, 255, 256])
+def test_plan_skinny_split_k(M):
+    p = bs.plan_for(bs.OP_FP8_BLOCKWISE, M, 1, 7168, 2048, 148)
+    assert p["kernel"] == 2 and p["launches"] == 1
+    assert p["tile_m"] in (16, 32, 64, 128) and p["tile_m"] >= min(M, 128)
+    assert p["splits"] in (1, 2, 4, 8) and p["splits"] <= 2048 // 128
+    assert p["cluster"] == p["splits"]
+    m_tiles = -(-M // p["tile_m"])
+    assert p["ctas"] == m_tiles * (7168 // 128) * p["splits"]
+
+
+def test_plan_int8_and_edges():
+    assert bs.plan_for(bs.OP_INT_SCALED_MM, 4096, 1, 4096, 4096, 148)["kernel"] == 1
+    assert bs.plan_for(bs.OP_INT_SCALED_MM, 1, 1, 4096, 4096, 148)["kernel"] == 1  # no skinny INT8 kernel
+    assert bs.plan_for(bs.OP_FP8_BLOCKWISE, 0, 1, 5120, 8192, 148)["launches"] == 0
+    assert bs.plan_for(bs.OP_FP8_BLOCKWISE, 16, 1, 0, 8192, 148)["launches"] == 0
+    p = bs.plan_for(bs.OP_FP8_BLOCKWISE, 16, 1, 512, 0, 148)
+    assert p["kernel"] == 3 and p["launches"] == 1
+    b = bs.plan_for(bs.OP_BMM, 16384, 8, 1024, 4096, 148)
+    assert b["kernel"] == 1 and b["ctas"] == 148
+    b = bs.plan_for(bs.OP_BMM, 1, 8, 1024, 4096, 148)
+    assert b["kernel"] == 2 and b["ctas"] == 8 * 8 * b["splits"]
+
+
+def test_path_override_forces_kernels():
+    prev = bs.set_path_override(bs.PATH_WIDE)
+    try:
+        assert bs.plan_for(bs.OP_FP8_BLOCKWISE, 1, 1, 7168, 2048, 148)["kernel"] == 1
+        bs.set_path_override(bs.PATH_SKINNY)
+        p = bs.plan_for(bs.OP_FP8_BLOCKWISE, 1000, 1, 7168, 2048, 148)
+        assert p["kernel"] == 2 and p["tile_m"] == 128
+        assert bs.plan_for(bs.OP_INT_SCALED_MM, 1, 1, 4096, 4096, 148)["kernel"] == 1
+    finally:
+        bs.set_path_override(prev)
+    assert bs.plan_for(bs.OP_FP8_BLOCKWISE, 1, 1, 7168, 2048, 148)["kernel"] == 2
+
+
+# ---------------------------------------------------------------------------
+# persistent tile order
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("gm,gn,G,group", [(130, 20, 1, 16), (7, 3, 2, 4), (33, 28, 1, 16), (1, 5, 3, 16), (17, 1, 1, 8)])
+def test_tile_order_is_a_bijection_with_grouped_sweep(gm, gn, G, group):
+    order = bs.tile_order(gm, gn, G, group)
+    assert sorted(order) == sorted((g, m, n) for g in range(G) for m in range(gm) for n in range(gn))
+    per = gm * gn
+    for t, (g, m, n) in enumerate(order):
+        assert g == t // per
+        # tiles of one group share a band of `group` tile rows
+        local = t % per
+        first = (local // (group * gn)) * group
+        assert first <= m < first + group
+
+
+def test_tile_order_columns_sweep_inside_group():
+    order = bs.tile_order(32, 4, 1, 16)
+    assert order[:17] == [(0, m, 0) for m in range(16)] + [(0, 0, 1)]
+
+
+# ---------------------------------------------------------------------------
+# argument validation (host-only; returns before touching a device)
+# ---------------------------------------------------------------------------
+P16 = 1 << 20  # a fake, 16-byte aligned "device" address: never dereferenced
+
+
+def _fp8(**kw):
+    a = dict(A=P16, lda=256, B=P16, ldb=256, sa=P16, sa_sm=2, sa_sk=1, sb=P16, sb_sk=2, sb_sn=1, out=P16, ldo=256,
+             dt=bs.BS_OUT_BF16, M=64, N=256, K=256)
+    a.update(kw)
+    v = ctypes.c_void_p
+    return bs.lib().bs_gemm_fp8_blockwise(v(a["A"]), a["lda"], v(a["B"]), a["ldb"], v(a["sa"]), a["sa_sm"], a["sa_sk"],
+                                          v(a["sb"]), a["sb_sk"], a["sb_sn"], v(a["out"]), a["ldo"], a["dt"],
+                                          a["M"], a["N"], a["K"], None)
+
+
+def test_fp8_validation_codes():
+    assert _fp8(K=200) == bs.BS_ERR_SHAPE
+    assert _fp8(M=-1) == bs.BS_ERR_SHAPE
+    assert _fp8(dt=bs.BS_OUT_I32) == bs.BS_ERR_DTYPE
+    assert _fp8(out=0) == bs.BS_ERR_NULL
+    assert _fp8(A=0) == bs.BS_ERR_NULL
+    assert _fp8(lda=128) == bs.BS_ERR_LAYOUT
+    assert _fp8(ldo=100) == bs.BS_ERR_LAYOUT
+    assert _fp8(A=P16 + 8) == bs.BS_ERR_ALIGNMENT
+    assert _fp8(lda=264) == bs.BS_ERR_ALIGNMENT
+    assert _fp8(ldo=260) == bs.BS_ERR_ALIGNMENT  # 260 * 2 bytes is not a multiple of 16
+    assert _fp8(M=0) == bs.BS_OK and _fp8(N=0) == bs.BS_OK  # empty problem: no-op, no device needed
+
+
+def test_int8_and_bmm_validation_codes():
+    h, v = bs.lib(), ctypes.c_void_p
+    call = lambda **k: h.int_scaled_mm(v(k.get("A", P16)), k.get("lda", 128), v(k.get("B", P16)), k.get("ldb", 128),
+                                       v(P16), v(P16), v(k.get("out", P16)), k.get("ldo", 64), k.get("dt", bs.BS_OUT_F32),
+                                       k.get("M", 8), 64, k.get("K", 128), None)
+    assert call(K=131072) == bs.BS_ERR_SHAPE
+    assert call(dt=7) == bs.BS_ERR_DTYPE
+    assert call(B=0) == bs.BS_ERR_NULL
+    assert call(ldb=64) == bs.BS_ERR_LAYOUT
+    assert call(lda=136) == bs.BS_ERR_ALIGNMENT
+    assert call(M=0) == bs.BS_OK
+    bmm = lambda **k: h.bmm_a8w8_blockscale(v(P16), k.get("x_sm", 1024), 128, v(P16), 128 * 256, 128, v(P16), v(P16),
+                                            v(P16), 2048, 256, bs.BS_OUT_BF16, 4, 8, 256, k.get("K", 128), None)
+    assert bmm(K=64) == bs.BS_ERR_SHAPE
+    assert bmm(x_sm=1000) == bs.BS_ERR_ALIGNMENT
+
+
+@pytest.mark.skipif(HAS_GPU, reason="checks the no-device path")
+def test_well_formed_call_without_gpu_fails_loudly():
+    assert _fp8() == bs.BS_ERR_DEVICE
+    assert "device" in bs.lib().bs_last_error_message().decode().lower()
+
+
+def test_binding_rejects_cpu_tensors():
+    A = torch.zeros(128, 256, dtype=torch.uint8)
+    with pytest.raises(bs.BsgemmError):
+        bs.bs_gemm_fp8_blockwise(A, A.t(), torch.ones(128, 2), torch.ones(2, 1))
+    with pytest.raises(bs.BsgemmError):
+        bs.int_scaled_mm(A.to(torch.int8), A.to(torch.int8).t(), None)

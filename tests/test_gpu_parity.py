@@ -1,0 +1,208 @@
+"""GPU parity: the CUDA path, called through the C ABI, against the CPU oracle.
+
+Inputs come from the seeded generators in ``workloads``; expected values come
+only from ``oracle``.  FP8 results must meet the bound documented in
+tests/parity.py; INT8 results must be bit-exact.  Small shapes compare every
+element; the full-size shapes compare sampled rows (all columns) that cover
+several tiles and the ragged tail.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import int8_gemm_b200 as bs
+import oracle
+import workloads as wl
+from parity import bf16_bits, f32_bits, fp8_check, oracle_fp8, rows_sample, to_f64
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib(cuda_device):
+    bs.lib()
+    yield
+    assert bs.device_error() == 0, "a kernel reported a timed-out wait"
+
+
+@pytest.fixture
+def path():
+    """Force a kernel family for one test, restoring automatic choice after."""
+    def set_(p):
+        bs.set_path_override(p)
+    yield set_
+    bs.set_path_override(bs.PATH_AUTO)
+
+
+def fp8_run(d, out_dtype=torch.bfloat16, out=None):
+    A = d["A"].to(DEV)
+    B = d["B_t"].to(DEV).t()
+    return bs.bs_gemm_fp8_blockwise(A, B, d["scale_a"].to(DEV), d["scale_b"].to(DEV), out_dtype=out_dtype, out=out)
+
+
+# ---------------------------------------------------------------------------
+# operation 1: FP8 block-scaled
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_fp8_tiny_full_matrix(out_dtype):
+    w = wl.WORKLOADS["fp8_tiny_256x256x512"]
+    d = wl.workload_inputs(w)
+    y, S = oracle_fp8(d)
+    fp8_check(fp8_run(d, out_dtype), y, S, out_dtype, "fp8 256x256x512")
+
+
+@pytest.mark.parametrize("M,N,K", [(128, 256, 128), (129, 384, 256), (300, 520, 640), (1, 256, 128),
+                                   (255, 128, 1024), (640, 1280, 384)])
+@pytest.mark.parametrize("kernel", [bs.PATH_WIDE, bs.PATH_SKINNY])
+def test_fp8_ragged_shapes_both_kernels(M, N, K, kernel, path):
+    path(kernel)
+    d = wl.fp8_blockwise_inputs(M, N, K, seed=50 + M + N + K)
+    y, S = oracle_fp8(d)
+    fp8_check(fp8_run(d), y, S, torch.bfloat16, f"fp8 {M}x{N}x{K} kernel={kernel}")
+
+
+@pytest.mark.parametrize("M", wl.SKINNY_M_SWEEP)
+def test_fp8_skinny_sweep_n7168_k2048(M):
+    w = wl.WORKLOADS[f"fp8_skinny_m{M}"]
+    d = wl.workload_inputs(w, sweep=wl.sweep_index(wl.SKINNY_M_SWEEP, M))
+    out = fp8_run(d)
+    rows = None if M <= 255 else rows_sample(M)
+    y, S = oracle_fp8(d, rows=rows)
+    got = out if rows is None else out[torch.tensor(rows, device=DEV)]
+    fp8_check(got, y, S, torch.bfloat16, f"skinny M={M}")
+
+
+@pytest.mark.slow
+def test_fp8_full_size_16640x5120x8192_sampled_rows():
+    w = wl.WORKLOADS["fp8_16640x5120x8192"]
+    d = wl.workload_inputs(w)
+    out = fp8_run(d)
+    rows = rows_sample(w.M, extra=6)
+    y, S = oracle_fp8(d, rows=rows)
+    fp8_check(out[torch.tensor(rows, device=DEV)], y, S, torch.bfloat16, "fp8 16640x5120x8192")
+
+
+def test_fp8_power_of_two_scale_linearity_on_gpu():
+    d = wl.fp8_blockwise_inputs(256, 512, 512, seed=61)
+    base = fp8_run(d, torch.float32)
+    d2 = dict(d)
+    sa = d["scale_a"].clone()
+    sa[5, :] *= 2.0 ** 4
+    d2["scale_a"] = sa
+    moved = fp8_run(d2, torch.float32)
+    assert torch.equal(moved[5], base[5] * 16.0)
+    keep = torch.ones(256, dtype=torch.bool, device=DEV)
+    keep[5] = False
+    assert torch.equal(moved[keep], base[keep])
+
+
+def test_fp8_deterministic_and_no_out_of_bounds_writes():
+    M, N, K = 300, 512, 1024
+    d = wl.fp8_blockwise_inputs(M, N, K, seed=62)
+    canvas = torch.full((M + 3, N + 64), 7.0, dtype=torch.bfloat16, device=DEV)
+    view = canvas[1:M + 1, 8:N + 8]
+    fp8_run(d, out=view)
+    first = view.clone()
+    fp8_run(d, out=view)
+    assert torch.equal(first, view)
+    assert torch.all(canvas[0] == 7.0) and torch.all(canvas[M + 1:] == 7.0)
+    assert torch.all(canvas[:, :8] == 7.0) and torch.all(canvas[:, N + 8:] == 7.0)
+    y, S = oracle_fp8(d)
+    fp8_check(view, y, S, torch.bfloat16, "fp8 strided out")
+
+
+def test_fp8_empty_and_k0():
+    A = torch.zeros(0, 128, dtype=torch.uint8, device=DEV)
+    B = torch.zeros(256, 128, dtype=torch.uint8, device=DEV).t()
+    out = bs.bs_gemm_fp8_blockwise(A, B, torch.ones(0, 1, device=DEV), torch.ones(1, 2, device=DEV))
+    assert out.shape == (0, 256)
+    A = torch.zeros(5, 0, dtype=torch.uint8, device=DEV)
+    B = torch.zeros(256, 0, dtype=torch.uint8, device=DEV).t()
+    out = torch.full((5, 256), 3.0, dtype=torch.bfloat16, device=DEV)
+    bs.bs_gemm_fp8_blockwise(A, B, torch.ones(5, 0, device=DEV), torch.ones(0, 2, device=DEV), out=out)
+    assert torch.all(out == 0)
+
+
+def test_fp8_transposed_scale_a_layout():
+    d = wl.fp8_blockwise_inputs(256, 256, 512, seed=63)
+    y, S = oracle_fp8(d)
+    sa_colmajor = d["scale_a"].t().contiguous().to(DEV).t()  # [M, KB] with strides (1, M)
+    out = bs.bs_gemm_fp8_blockwise(d["A"].to(DEV), d["B_t"].to(DEV).t(), sa_colmajor, d["scale_b"].to(DEV))
+    fp8_check(out, y, S, torch.bfloat16, "column-major scale_a")
+
+
+# ---------------------------------------------------------------------------
+# operation 2: INT8, bit-exact
+# ---------------------------------------------------------------------------
+def int8_run(d, out_dtype, s_b=True):
+    return bs.int_scaled_mm(d["A"].to(DEV), d["B_t"].to(DEV).t(), d["s_a"].to(DEV),
+                            d["s_b"].to(DEV) if s_b else None, out_dtype=out_dtype)
+
+
+def _int8_assert(d, rows, s_b=True):
+    acc, y, bf = oracle.int_scaled_mm(d["A"], d["B_t"], d["s_a"], d["s_b"] if s_b else None, rows=rows)
+    sel = (lambda t: t) if rows is None else (lambda t: t[torch.tensor(rows, device=DEV)])
+    np.testing.assert_array_equal(sel(int8_run(d, torch.int32, s_b)).cpu().numpy(), acc)
+    np.testing.assert_array_equal(f32_bits(sel(int8_run(d, torch.float32, s_b))), y.view(np.uint32))
+    np.testing.assert_array_equal(bf16_bits(sel(int8_run(d, torch.bfloat16, s_b))), bf)
+
+
+@pytest.mark.parametrize("M,N,K", [(128, 256, 128), (300, 520, 1040), (1, 256, 4096), (257, 264, 48)])
+def test_int8_bit_exact_small(M, N, K):
+    _int8_assert(wl.int8_inputs(M, N, K, seed=70 + M), rows=None)
+
+
+def test_int8_row_scale_only():
+    _int8_assert(wl.int8_inputs(200, 256, 512, seed=71), rows=None, s_b=False)
+
+
+def test_int8_4096_cubed_sampled_rows():
+    w = wl.WORKLOADS["int8_4096x4096x4096"]
+    d = wl.workload_inputs(w)
+    _int8_assert(d, rows=rows_sample(w.M, extra=8))
+
+
+# ---------------------------------------------------------------------------
+# operation 3: batched, e8m0 block scales
+# ---------------------------------------------------------------------------
+def bmm_run(d, out_dtype=torch.bfloat16):
+    return bs.bmm_a8w8_blockscale(d["x"].to(DEV) if d["x"].is_contiguous() else _batch_first_to(d["x"]),
+                                  d["w"].to(DEV), d["x_scale"].to(DEV), d["w_scale"].to(DEV), out_dtype=out_dtype)
+
+
+def _batch_first_to(x):
+    # keep the [G, M, K] storage on the device: copy the storage, then view as [M, G, K]
+    return x.permute(1, 0, 2).contiguous().to(DEV).permute(1, 0, 2)
+
+
+@pytest.mark.parametrize("G", wl.BMM_G)
+@pytest.mark.parametrize("M", wl.BMM_M_SWEEP)
+def test_bmm_sweep(M, G):
+    w = wl.WORKLOADS[f"bmm_g{G}_m{M}"]
+    d = wl.workload_inputs(w, sweep=wl.sweep_index(wl.BMM_M_SWEEP, M) + 10 * (G == 2))
+    out = bmm_run(d)
+    rows = None if M <= 1024 else rows_sample(M, extra=4)
+    y, S = oracle.bmm_blockscale(d["x"], d["w"], d["x_scale"], d["w_scale"], rows=rows)
+    got = out if rows is None else out[torch.tensor(rows, device=DEV)]
+    fp8_check(got, y, S, torch.bfloat16, f"bmm M={M} G={G}")
+
+
+@pytest.mark.parametrize("M", [16, 300])
+def test_bmm_batch_first_layout(M):
+    d = wl.bmm_inputs(M, 2, 512, 1024, seed=80 + M, batch_first=True)
+    assert not d["x"].is_contiguous()
+    out = bmm_run(d, torch.float32)
+    y, S = oracle.bmm_blockscale(d["x"], d["w"], d["x_scale"], d["w_scale"])
+    fp8_check(out, y, S, torch.float32, f"bmm batch-first M={M}")
+
+
+def test_bmm_both_kernels_agree_with_oracle(path):
+    d = wl.bmm_inputs(200, 3, 384, 512, seed=81)
+    y, S = oracle.bmm_blockscale(d["x"], d["w"], d["x_scale"], d["w_scale"])
+    for k in (bs.PATH_WIDE, bs.PATH_SKINNY):
+        path(k)
+        fp8_check(bmm_run(d), y, S, torch.bfloat16, f"bmm kernel={k}")
