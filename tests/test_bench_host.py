@@ -1,0 +1,94 @@
+"""Host logic of bench.py without a GPU: clock parsing, traffic bookkeeping,
+the reference (CPU oracle) arm, and the multi-rank aggregation run as two
+gloo ranks on CPU (the replicas share no data; only the timing is reduced)."""
+from __future__ import annotations
+
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+
+
+def test_parse_clock_csv_reports_median_under_load_and_reasons():
+    txt = "\n".join([
+        "0, 1965, 1965, 120.5, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+        "0, 1400, 1965, 990.1, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "0, 1350, 1965, 1001.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "0, 1380, 1965, 998.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+    ])
+    c = bench.parse_clock_csv(txt)
+    assert c["sm_mhz"] == 1380 and c["sm_max_mhz"] == 1965
+    assert c["reasons"] == ["sw_power_cap"] and c["samples_under_load"] == 3
+    assert bench.parse_clock_csv("") is None
+
+
+def test_stored_traffic_requires_current_kernel_sources(tmp_path, monkeypatch):
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    (prof / "traffic.json").write_text(json.dumps({
+        "w_ok": {"source_digest": bench.source_digest(), "dram_bytes_per_launch": 123},
+        "w_stale": {"source_digest": "0" * 16, "dram_bytes_per_launch": 456}}))
+    csrc = tmp_path / "int8_gemm_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    for name in os.listdir(os.path.join(ROOT, "int8_gemm_b200", "csrc")):
+        (csrc / name).write_bytes(open(os.path.join(ROOT, "int8_gemm_b200", "csrc", name), "rb").read())
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.stored_traffic("w_ok") == 123
+    assert bench.stored_traffic("w_stale") is None
+    assert bench.stored_traffic("absent") is None
+
+
+def test_peaks_fall_back_when_file_missing(tmp_path):
+    p = bench.load_peaks(str(tmp_path / "none.json"))
+    assert p["source"] == "fallback" and p["hbm_gbs"] == 6650.0
+
+
+def _rank(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    local_ms = [2.0, 3.0][rank]
+
+    def reduce_max(v):
+        t = torch.tensor([v], dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    t, value = bench.aggregate(local_ms, 1e12, world, reduce_max)
+    q.put((rank, t, value))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_aggregate_two_gloo_ranks_uses_slowest_rank():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = 29500 + os.getpid() % 1000
+    procs = [ctx.Process(target=_rank, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert [r[1] for r in res] == [3.0, 3.0]
+    assert res[0][2] == res[1][2] == pytest.approx(2e12 / 3e-3)
+
+
+def test_reference_arm_prints_contract_line():
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload",
+                        "fp8_tiny_256x256x512", "--steps", "2", "--warmup", "1"],
+                       capture_output=True, text=True, timeout=300, cwd=ROOT)
+    assert r.returncode == 0, r.stderr
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["value"] > 0 and line["unit"] == "TFLOP/s"
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
