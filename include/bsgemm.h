@@ -160,7 +160,7 @@ typedef struct {
   int32_t tile_n;  /* columns of B (N direction) per tile */
   int32_t splits;  /* K splits reduced through cluster shared memory (1 = none) */
   int32_t ctas;    /* CTAs launched */
-  int32_t cluster; /* CTAs per thread-block cluster */
+  int32_t cluster; /* CTAs per thread-block cluster (2 for the CTA-pair wide kernel) */
   int32_t launches;/* kernel launches the call makes */
 } bs_plan;
 
@@ -170,8 +170,9 @@ typedef struct {
 bs_status bs_plan_for(int32_t op, int64_t M, int64_t G, int64_t N, int64_t K, int32_t num_sms, bs_plan* plan);
 
 /* Force the kernel family for subsequent calls in this process (testing):
- * 0 = automatic (default), 1 = persistent wide kernel, 2 = skinny split-K
- * kernel where the operation has one.  Returns the previous setting. */
+ * 0 = automatic (default), 1 = persistent wide kernel on CTA pairs (256 x 256
+ * tiles), 2 = skinny split-K kernel where the operation has one, 3 = persistent
+ * wide kernel on single CTAs (128 x 256 tiles).  Returns the previous setting. */
 int32_t bs_set_path_override(int32_t path);
 
 /* The persistent tile order: fills out[3*t .. 3*t+2] = (batch, tile_row,

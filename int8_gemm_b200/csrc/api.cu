@@ -112,6 +112,7 @@ constexpr int kGroupM = 16;
 
 struct Plan {
   bs_plan pub;
+  int cg = 2;  // wide kernel: CTAs per tile (2 = CTA pair, 256-row tiles)
   int bmt = 0;
   int m_tiles = 0, n_tiles = 0;
   int grid_m = 0, grid_n = 0, num_tiles = 0;
@@ -149,16 +150,19 @@ Plan make_plan(int op, int64_t M, int64_t G, int64_t N, int64_t K, int sms) {
     x.pub.ctas = static_cast<int32_t>(units * S);
     x.pub.launches = 1;
   } else {
-    x.grid_m = static_cast<int>((M + 127) / 128);
+    x.cg = ov == 3 ? 1 : 2;
+    const int tile_m = 128 * x.cg;
+    x.grid_m = static_cast<int>((M + tile_m - 1) / tile_m);
     x.grid_n = static_cast<int>((N + kWideBN - 1) / kWideBN);
     const long long tiles = static_cast<long long>(x.grid_m) * x.grid_n * G;
+    const long long units = (sms > 0 ? sms : 148) / x.cg;  // persistent CTAs (or CTA pairs)
     x.num_tiles = static_cast<int>(tiles);
     x.pub.kernel = 1;
-    x.pub.tile_m = 128;
+    x.pub.tile_m = tile_m;
     x.pub.tile_n = kWideBN;
     x.pub.splits = 1;
-    x.pub.cluster = 1;
-    x.pub.ctas = static_cast<int32_t>(tiles < sms ? tiles : sms);
+    x.pub.cluster = x.cg;
+    x.pub.ctas = static_cast<int32_t>(x.cg * (tiles < units ? tiles : units));
     x.pub.launches = 1;
   }
   return x;
@@ -168,7 +172,8 @@ Plan make_plan(int op, int64_t M, int64_t G, int64_t N, int64_t K, int sms) {
 // tensor maps
 // ---------------------------------------------------------------------------
 bs_status encode_3d(CUtensorMap* map, CUtensorMapDataType dt, int esize, const void* base, uint64_t d0, uint64_t d1,
-                    uint64_t d2, uint64_t s1, uint64_t s2, uint32_t box0, uint32_t box1, const char* what) {
+                    uint64_t d2, uint64_t s1, uint64_t s2, uint32_t box0, uint32_t box1, const char* what,
+                    CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return fail(BS_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   const cuuint64_t dims[3] = {d0, d1, d2};
@@ -176,12 +181,15 @@ bs_status encode_3d(CUtensorMap* map, CUtensorMapDataType dt, int esize, const v
   const cuuint32_t box[3] = {box0, box1, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   const CUresult r = enc(map, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                         swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS)
     return fail(BS_ERR_CUDA, "tensor map encoding failed for %s (CUresult %d)", what, static_cast<int>(r));
   return BS_OK;
 }
+
+// Rows of one B box of the wide kernel: single CTAs load all 256 tile columns,
+// each CTA of a pair its 128.
+uint32_t wide_b_box_rows(int cg) { return static_cast<uint32_t>(kWideBN / cg); }
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
@@ -241,13 +249,14 @@ bs_status run_fp8(const Fp8Problem& q, GemmArgs args, cudaStream_t stream, Devic
     args.splits = 1;
     if ((st = encode_3d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, q.a, q.K, q.M, q.G, q.a_rs, a_bs, 128, 128, "A")))
       return st;
-    if ((st = encode_3d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, q.b, q.K, q.N, q.G, q.b_rs, b_bs, 128, kWideBN, "B")))
+    if ((st = encode_3d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, q.b, q.K, q.N, q.G, q.b_rs, b_bs, 128,
+                        wide_b_box_rows(pl.cg), "B")))
       return st;
     const int es = out_size(q.out_dtype);
     if ((st = encode_3d(&td, out_tmap_type(q.out_dtype), es, q.out, q.N, q.M, q.G, q.o_rs, o_bs,
-                        static_cast<uint32_t>(128 / es), 32, "out")))
+                        static_cast<uint32_t>(64 / es), 32, "out", CU_TENSOR_MAP_SWIZZLE_64B)))
       return st;
-    return check_launch(launch_wide(q.mode, out_kind(q.out_dtype), ta, tb, td, args, pl.pub.ctas, stream),
+    return check_launch(launch_wide(q.mode, out_kind(q.out_dtype), pl.cg, ta, tb, td, args, pl.pub.ctas, stream),
                         "wide kernel launch");
   }
   args.splits = pl.pub.splits;
@@ -483,13 +492,14 @@ bs_status int_scaled_mm(const int8_t* A, int64_t lda, const int8_t* B, int64_t l
   args.err = dc->err;
   CUtensorMap ta, tb, td;
   if ((st = encode_3d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, A, K, M, 1, lda, lda * M, 128, 128, "A"))) return st;
-  if ((st = encode_3d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, B, K, N, 1, ldb, ldb * N, 128, kWideBN, "B")))
+  if ((st = encode_3d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, B, K, N, 1, ldb, ldb * N, 128, wide_b_box_rows(pl.cg),
+                      "B")))
     return st;
   const int es = out_size(out_dtype);
-  if ((st = encode_3d(&td, out_tmap_type(out_dtype), es, out, N, M, 1, ldo, ldo * M, static_cast<uint32_t>(128 / es),
-                      32, "out")))
+  if ((st = encode_3d(&td, out_tmap_type(out_dtype), es, out, N, M, 1, ldo, ldo * M, static_cast<uint32_t>(64 / es),
+                      32, "out", CU_TENSOR_MAP_SWIZZLE_64B)))
     return st;
-  return check_launch(launch_wide(Mode::kInt8, out_kind(out_dtype), ta, tb, td, args, pl.pub.ctas, cs),
+  return check_launch(launch_wide(Mode::kInt8, out_kind(out_dtype), pl.cg, ta, tb, td, args, pl.pub.ctas, cs),
                       "int8 kernel launch");
 }
 

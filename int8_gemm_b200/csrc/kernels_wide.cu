@@ -10,11 +10,12 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 
-template <Mode MODE, typename OutT>
+template <Mode MODE, int CG, typename OutT>
 cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& d, const GemmArgs& args,
                        int grid, cudaStream_t stream) {
-  auto kernel = wide_gemm_kernel<MODE, kWideBN, kWideStages, OutT>;
-  constexpr size_t smem = sizeof(WideSmem<kWideBN, kWideStages>) + 1024;
+  constexpr int STAGES = CG == 2 ? kWideStagesPair : kWideStages;
+  auto kernel = wide_gemm_kernel<MODE, CG, STAGES, OutT>;
+  constexpr size_t smem = sizeof(WideSmem<kWideBN / CG, STAGES>) + 1024;
   static std::atomic<uint64_t> configured{0};  // one bit per device
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -25,35 +26,48 @@ cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b, const CUtenso
     if (e != cudaSuccess) return e;
     configured.fetch_or(bit, std::memory_order_release);
   }
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CG;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
   cfg.blockDim = dim3(kWideThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cfg.attrs = nullptr;
-  cfg.numAttrs = 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = CG == 2 ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, kernel, a, b, d, args);
+}
+
+template <int CG>
+cudaError_t launch_cg(Mode mode, OutKind out, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& d,
+                      const GemmArgs& args, int grid, cudaStream_t stream) {
+  switch (mode) {
+    case Mode::kFp8F32Scale:
+      if (out == OutKind::kBF16) return launch_one<Mode::kFp8F32Scale, CG, __nv_bfloat16>(a, b, d, args, grid, stream);
+      if (out == OutKind::kF32) return launch_one<Mode::kFp8F32Scale, CG, float>(a, b, d, args, grid, stream);
+      break;
+    case Mode::kFp8E8M0:
+      if (out == OutKind::kBF16) return launch_one<Mode::kFp8E8M0, CG, __nv_bfloat16>(a, b, d, args, grid, stream);
+      if (out == OutKind::kF32) return launch_one<Mode::kFp8E8M0, CG, float>(a, b, d, args, grid, stream);
+      break;
+    case Mode::kInt8:
+      if (out == OutKind::kBF16) return launch_one<Mode::kInt8, CG, __nv_bfloat16>(a, b, d, args, grid, stream);
+      if (out == OutKind::kF32) return launch_one<Mode::kInt8, CG, float>(a, b, d, args, grid, stream);
+      if (out == OutKind::kI32) return launch_one<Mode::kInt8, CG, int32_t>(a, b, d, args, grid, stream);
+      break;
+  }
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace
 
-cudaError_t launch_wide(Mode mode, OutKind out, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& d,
-                        const GemmArgs& args, int grid, cudaStream_t stream) {
-  switch (mode) {
-    case Mode::kFp8F32Scale:
-      if (out == OutKind::kBF16) return launch_one<Mode::kFp8F32Scale, __nv_bfloat16>(a, b, d, args, grid, stream);
-      if (out == OutKind::kF32) return launch_one<Mode::kFp8F32Scale, float>(a, b, d, args, grid, stream);
-      break;
-    case Mode::kFp8E8M0:
-      if (out == OutKind::kBF16) return launch_one<Mode::kFp8E8M0, __nv_bfloat16>(a, b, d, args, grid, stream);
-      if (out == OutKind::kF32) return launch_one<Mode::kFp8E8M0, float>(a, b, d, args, grid, stream);
-      break;
-    case Mode::kInt8:
-      if (out == OutKind::kBF16) return launch_one<Mode::kInt8, __nv_bfloat16>(a, b, d, args, grid, stream);
-      if (out == OutKind::kF32) return launch_one<Mode::kInt8, float>(a, b, d, args, grid, stream);
-      if (out == OutKind::kI32) return launch_one<Mode::kInt8, int32_t>(a, b, d, args, grid, stream);
-      break;
-  }
+cudaError_t launch_wide(Mode mode, OutKind out, int cta_group, const CUtensorMap& a, const CUtensorMap& b,
+                        const CUtensorMap& d, const GemmArgs& args, int grid, cudaStream_t stream) {
+  if (cta_group == 2) return launch_cg<2>(mode, out, a, b, d, args, grid, stream);
+  if (cta_group == 1) return launch_cg<1>(mode, out, a, b, d, args, grid, stream);
   return cudaErrorInvalidValue;
 }
 

@@ -13,14 +13,16 @@ namespace bsg {
 enum class OutKind : int { kBF16 = 0, kF32 = 1, kI32 = 2 };
 
 constexpr int kWideBN = 256;
-constexpr int kWideStages = 4;
+constexpr int kWideStages = 4;      // single-CTA tiles: 48 KB per stage
+constexpr int kWideStagesPair = 6;  // CTA-pair tiles: 32 KB per stage and CTA
 constexpr int kWideThreads = 384;
 constexpr int kSkinnyStages = 4;
 constexpr int kSkinnyThreads = 224;
 
-// Persistent wide kernel over `grid` CTAs.
-cudaError_t launch_wide(Mode mode, OutKind out, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& d,
-                        const GemmArgs& args, int grid, cudaStream_t stream);
+// Persistent wide kernel over `grid` CTAs; cta_group 2 launches clusters of two
+// CTAs computing 256 x 256 tiles, cta_group 1 single CTAs computing 128 x 256.
+cudaError_t launch_wide(Mode mode, OutKind out, int cta_group, const CUtensorMap& a, const CUtensorMap& b,
+                        const CUtensorMap& d, const GemmArgs& args, int grid, cudaStream_t stream);
 
 // Skinny split-K kernel: grid (n_tiles * splits, m_tiles, G), cluster (splits, 1, 1).
 cudaError_t launch_skinny(Mode mode, OutKind out, int bmt, const CUtensorMap& a, const CUtensorMap& b,

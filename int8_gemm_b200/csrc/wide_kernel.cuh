@@ -6,12 +6,13 @@
 //               into a STAGES-deep shared-memory ring (full/empty mbarriers).
 //   warp 1      MMA issuer: four tcgen05.mma (K = 32 bytes each) per K block
 //               into a TMEM accumulator; owns the TMEM allocation.
-//   warps 2, 3  idle (they complete warpgroup 0 for the register split).
+//   warps 2, 3  FP8 modes: scale producer (stages the block scales of the
+//               next K blocks in a shared ring); idle for INT8.
 //   warps 4..11 consumers (warpgroups 1 and 2).  Warp w reads TMEM lanes
 //               32*(w%4).. and one half (128 columns) of the tile.
-// Launched with 384 threads x 168 registers; warpgroup 0 gives registers back
-// (40 each) so the consumer warpgroups can hold 128 fp32 accumulators plus a
-// 32-column TMEM slice (232 each): 128*40 + 256*232 = 384*168.
+// Launched with 384 threads x 168 registers; warpgroup 0 keeps 56 each and the
+// consumer warpgroups take 224 each (128 fp32 accumulators plus two 32-column
+// TMEM slices in flight): 128*56 + 256*224 = 384*168.
 //
 // FP8 modes (block scales vary along K):  every 128-deep K block lands in one
 // of two TMEM buffers; the consumers pull the partial P_kb into registers and
@@ -64,19 +65,57 @@ struct GemmArgs {
   uint32_t* err;
 };
 
-template <int BN, int STAGES>
+// Shared-memory layout of one CTA.  In the pair (cta_group::2) variant both
+// CTAs use the same layout: the leader's MMA descriptors address the same
+// offsets in the peer.
+#ifndef BSG_L2_PREFETCH_DISTANCE
+#define BSG_L2_PREFETCH_DISTANCE 8
+#endif
+// K blocks between the L2 prefetch of an operand box and its load into shared
+// memory.  Loads that miss L2 (first touch of a panel, or a line homed in the
+// other die's L2) otherwise set the latency of a whole stage.
+constexpr int kL2PrefetchDistance = BSG_L2_PREFETCH_DISTANCE;
+constexpr int kScaleRing = 16;  // K blocks of scales staged ahead of the consumers
+constexpr int kScaleBatch = 8;  // K blocks whose scale loads are in flight together
+
+template <int BNL, int STAGES>
 struct WideSmem {
-  uint8_t a[STAGES][128 * 128];
-  uint8_t b[STAGES][BN * 128];
-  uint8_t stage_out[8][32 * 128];
+  uint8_t a[STAGES][128 * 128];  // this CTA's 128 A rows of one K block
+  uint8_t b[STAGES][BNL * 128];  // this CTA's BNL B rows (output columns) of one K block
+  uint8_t stage_out[8][32 * 64];  // per consumer warp: 32 rows x 64 bytes, 64-byte swizzle
+  float sa[kScaleRing][128];     // scale_a of this CTA's rows, per K block
+  float sb[kScaleRing][4];       // scale_b of the tile's two 128-column blocks, per K block
   uint64_t full[STAGES];
   uint64_t empty[STAGES];
-  uint64_t acc_full[2];
-  uint64_t acc_empty[2];
+  uint64_t acc_full[2];   // INT8: tile accumulator complete (FP8 uses the stage barriers)
+  uint64_t acc_empty[2];  // accumulator buffer released by every consumer warp (of both CTAs)
+  uint64_t sc_full[kScaleRing];
+  uint64_t sc_empty[kScaleRing];
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
 };
+
+// Row and column-block factors of the block scale (0 outside the problem; the
+// matching partials are zero-filled anyway).
+template <Mode MODE>
+__device__ __forceinline__ float scale_row(const GemmArgs& p, int g, int m, int kb) {
+  if (m >= p.M) return 0.f;
+  if constexpr (MODE == Mode::kFp8F32Scale) {
+    return __ldg(p.sa + static_cast<long long>(m) * p.sa_sm + static_cast<long long>(kb) * p.sa_sk);
+  } else {
+    return e8m0_to_f32(__ldg(p.xs + (static_cast<long long>(m) * p.G + g) * p.KB + kb));
+  }
+}
+template <Mode MODE>
+__device__ __forceinline__ float scale_col(const GemmArgs& p, int g, int kb, int nb) {
+  if (nb >= p.NB) return 0.f;
+  if constexpr (MODE == Mode::kFp8F32Scale) {
+    return __ldg(p.sb + static_cast<long long>(kb) * p.sb_sk + static_cast<long long>(nb) * p.sb_sn);
+  } else {
+    return e8m0_to_f32(__ldg(p.ws + (static_cast<long long>(g) * p.NB + nb) * p.KB + kb));
+  }
+}
 
 // Block scale for row m, K block kb, scale block nb along N; 0 outside the
 // problem (the matching partials are zero-filled anyway).
@@ -94,15 +133,18 @@ __device__ __forceinline__ float block_scale(const GemmArgs& p, int g, int m, in
   }
 }
 
-// Write 32 output values of this lane's row into the 128B-swizzled staging
-// row (row = lane, 16-byte unit u stored at u ^ (lane & 7)).
-template <typename OutT>
-__device__ __forceinline__ void stage_32(uint8_t* stg, int lane, int unit0, const float (&v)[32]) {
-  uint8_t* row = stg + lane * 128;
-  if constexpr (sizeof(OutT) == 2) {
+// Write one 64-byte staging row (this lane's output row; CPC = 64 / sizeof(OutT)
+// values) with the 64-byte swizzle of the output tensor map: 16-byte unit u of
+// row r lives at unit u ^ ((r >> 1) & 3), which also keeps the 8 rows a
+// quarter-warp writes at once on distinct banks.
+template <typename OutT, int CPC>
+__device__ __forceinline__ void stage_row64(uint8_t* stg, int lane, const float (&v)[CPC]) {
+  uint8_t* row = stg + lane * 64;
+  const int sw = (lane >> 1) & 3;
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      uint4 w;
+  for (int q = 0; q < 4; ++q) {
+    uint4 w;
+    if constexpr (sizeof(OutT) == 2) {
       __nv_bfloat162 h0 = __floats2bfloat162_rn(v[q * 8 + 0], v[q * 8 + 1]);
       __nv_bfloat162 h1 = __floats2bfloat162_rn(v[q * 8 + 2], v[q * 8 + 3]);
       __nv_bfloat162 h2 = __floats2bfloat162_rn(v[q * 8 + 4], v[q * 8 + 5]);
@@ -111,15 +153,11 @@ __device__ __forceinline__ void stage_32(uint8_t* stg, int lane, int unit0, cons
       w.y = *reinterpret_cast<uint32_t*>(&h1);
       w.z = *reinterpret_cast<uint32_t*>(&h2);
       w.w = *reinterpret_cast<uint32_t*>(&h3);
-      *reinterpret_cast<uint4*>(row + (((unit0 + q) ^ (lane & 7)) << 4)) = w;
+    } else {
+      w = make_uint4(__float_as_uint(v[q * 4 + 0]), __float_as_uint(v[q * 4 + 1]), __float_as_uint(v[q * 4 + 2]),
+                     __float_as_uint(v[q * 4 + 3]));
     }
-  } else {
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      uint4 w = make_uint4(__float_as_uint(v[q * 4 + 0]), __float_as_uint(v[q * 4 + 1]),
-                           __float_as_uint(v[q * 4 + 2]), __float_as_uint(v[q * 4 + 3]));
-      *reinterpret_cast<uint4*>(row + (((unit0 + q) ^ (lane & 7)) << 4)) = w;
-    }
+    *reinterpret_cast<uint4*>(row + ((q ^ sw) << 4)) = w;
   }
 }
 
@@ -129,23 +167,32 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
   return __all_sync(0xffffffffu, ok);
 }
 
-constexpr int kWideProducerRegs = 40;
-constexpr int kWideConsumerRegs = 232;
+constexpr int kWideProducerRegs = 56;
+constexpr int kWideConsumerRegs = 224;
 static_assert(128 * kWideProducerRegs + 256 * kWideConsumerRegs <= 384 * 168, "register split exceeds launch budget");
 
-template <Mode MODE, int BN, int STAGES, typename OutT>
+// CG = 1: one CTA computes a 128 x 256 tile.  CG = 2: a cluster of two CTAs
+// (a CTA pair) computes a 256 x 256 tile with tcgen05.mma.cta_group::2 issued
+// by the even ("leader") CTA; each CTA loads its own 128 A rows and 128 of the
+// 256 B rows, so per SM a K block costs 32 KB of shared memory instead of 48 KB
+// and more stages fit.  Both CTAs' TMA loads signal the leader's full barrier;
+// the leader's commits arrive on both CTAs' barriers; the peer's consumers
+// release the leader's accumulator barrier remotely.
+template <Mode MODE, int CG, int STAGES, typename OutT>
 __global__ void __launch_bounds__(384, 1)
     wide_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmD, const GemmArgs p) {
-  constexpr int BM = 128, BK = 128;
-  constexpr uint32_t A_BYTES = BM * BK, B_BYTES = BN * BK;
+  constexpr int BM = 128, BK = 128, BN = 256;
+  constexpr int BNL = BN / CG;  // B rows loaded by one CTA
+  constexpr uint32_t A_BYTES = BM * BK, B_BYTES = BNL * BK;
+  constexpr uint32_t STAGE_TX = CG * (A_BYTES + B_BYTES);  // bytes the leader's full barrier waits for
   constexpr int CONSUMER_WARPS = 8;
   constexpr uint32_t TMEM_COLS = 2 * BN;
   constexpr bool IS_INT8 = MODE == Mode::kInt8;
-  constexpr uint32_t IDESC = IS_INT8 ? idesc_s8_s32<BM, BN>() : idesc_e4m3_f32<BM, BN>();
-  constexpr int CPC = 128 / sizeof(OutT);  // output columns per 128-byte staging row
-  static_assert(BN == 256, "consumer layout assumes two 128-column halves");
-  using Smem = WideSmem<BN, STAGES>;
+  constexpr uint32_t IDESC = IS_INT8 ? idesc_s8_s32<BM * CG, BN>() : idesc_e4m3_f32<BM * CG, BN>();
+  constexpr int CPC = 64 / sizeof(OutT);  // output columns per 64-byte staging row
+  static_assert(CG == 1 || CG == 2, "CTA group is 1 or 2");
+  using Smem = WideSmem<BNL, STAGES>;
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
@@ -153,6 +200,9 @@ __global__ void __launch_bounds__(384, 1)
   volatile int* abort = &sm.abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rank = CG == 2 ? static_cast<int>(cluster_ctarank()) : 0;
+  const bool leader = rank == 0;
+  const int unit = blockIdx.x / CG, units = gridDim.x / CG;  // pair (or CTA) index / count
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -161,122 +211,222 @@ __global__ void __launch_bounds__(384, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sm.acc_full[b], 1);
-      mbar_init(&sm.acc_empty[b], CONSUMER_WARPS);
+      mbar_init(&sm.acc_empty[b], CONSUMER_WARPS * CG);
+    }
+    for (int i = 0; i < kScaleRing; ++i) {
+      mbar_init(&sm.sc_full[i], 64);  // every thread of the two scale warps
+      mbar_init(&sm.sc_empty[i], CONSUMER_WARPS);
     }
     mbar_init(&sm.drain, 1);
     sm.abort = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(&sm.tmem_base, TMEM_COLS);
-    tmem_relinquish();
+    if constexpr (CG == 2) {
+      tmem_alloc_pair(&sm.tmem_base, TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(&sm.tmem_base, TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  if constexpr (CG == 2) {
+    cluster_sync_all();  // barriers of both CTAs initialised before any remote signal
+  } else {
+    __syncthreads();
+  }
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
 
   if (warp < 4) {
     regs_dec<kWideProducerRegs>();
     if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      tma_prefetch_desc(&tmA);
-      tma_prefetch_desc(&tmB);
-      uint32_t issued = 0, issued_phase = 0;
-      int stage = 0;
-      uint32_t phase = 0;
-      bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
-        const TileCoord tc = tile_coord(tile, p.grid_m, p.grid_n, p.group_m);
-        const int m0 = tc.pm * BM, n0 = tc.pn * BN;
-        for (int kb = 0; kb < p.KB; ++kb) {
-          if (!wait_bounded(&sm.empty[stage], phase ^ 1u, abort, p.err,
-                            kErrTimeout | kRoleProducer | kWaitStageEmpty)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(&sm.full[stage], A_BYTES + B_BYTES);
-          tma_load_3d(sm.a[stage], &tmA, &sm.full[stage], kb * BK, m0, tc.g);
-          tma_load_3d(sm.b[stage], &tmB, &sm.full[stage], kb * BK, n0, tc.g);
-          issued |= 1u << stage;
-          issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
-          if (++stage == STAGES) {
-            stage = 0;
-            phase ^= 1u;
-          }
-        }
-      }
-      if (!ok) {  // let copies already in flight land before the CTA retires
-        volatile int never = 0;
-        for (int s = 0; s < STAGES; ++s)
-          if ((issued >> s) & 1u) wait_bounded(&sm.full[s], (issued_phase >> s) & 1u, &never, nullptr, 0);
-      }
-    }
-    __syncwarp();
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      int stage = 0, buf = 0;
-      uint32_t phase = 0, bphase = 0;
-      bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
-        if constexpr (IS_INT8) {
-          if (!wait_bounded(&sm.acc_empty[buf], bphase ^ 1u, abort, p.err, kErrTimeout | kRoleMma | kWaitAccEmpty)) {
-            ok = false;
-            break;
-          }
-        }
-        for (int kb = 0; kb < p.KB; ++kb) {
-          if constexpr (!IS_INT8) {
-            if (!wait_bounded(&sm.acc_empty[buf], bphase ^ 1u, abort, p.err,
-                              kErrTimeout | kRoleMma | kWaitAccEmpty)) {
+      // ---------------------------------------------------------- producer
+      if (lane == 0) {
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+        uint32_t issued = 0, issued_phase = 0;
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        for (int tile = unit; ok && tile < p.num_tiles; tile += units) {
+          const TileCoord tc = tile_coord(tile, p.grid_m, p.grid_n, p.group_m);
+          // the tile after this one, for prefetches that run past its last K block
+          const int next_tile = tile + units;
+          TileCoord tn = tc;
+          if (next_tile < p.num_tiles) tn = tile_coord(next_tile, p.grid_m, p.grid_n, p.group_m);
+          const int m0 = tc.pm * (BM * CG) + rank * BM;
+          const int nb0 = tc.pn * BN + rank * BNL;  // this CTA's B rows (tile columns)
+          for (int kb = 0; kb < p.KB; ++kb) {
+            if (!wait_bounded(&sm.empty[stage], phase ^ 1u, abort, p.err,
+                              kErrTimeout | kRoleProducer | kWaitStageEmpty)) {
               ok = false;
               break;
             }
-          }
-          if (!wait_bounded(&sm.full[stage], phase, abort, p.err, kErrTimeout | kRoleMma | kWaitStageFull)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t d = tmem + static_cast<uint32_t>(buf * BN);
-          const uint64_t ad = sdesc_k_sw128(smem_u32(sm.a[stage]));
-          const uint64_t bd = sdesc_k_sw128(smem_u32(sm.b[stage]));
-#pragma unroll
-          for (int k = 0; k < BK / 32; ++k) {
-            if constexpr (IS_INT8) {
-              mma_i8(d, ad + 2 * k, bd + 2 * k, IDESC, (kb > 0 || k > 0) ? 1u : 0u);
+            if (kL2PrefetchDistance > 0) {
+              int pk = kb + kL2PrefetchDistance;
+              const TileCoord* pt = &tc;
+              if (pk >= p.KB) {
+                pk -= p.KB;
+                pt = &tn;
+              }
+              if (pt == &tc || next_tile < p.num_tiles) {
+                tma_prefetch_l2_3d(&tmA, pk * BK, pt->pm * (BM * CG) + rank * BM, pt->g);
+                tma_prefetch_l2_3d(&tmB, pk * BK, pt->pn * BN + rank * BNL, pt->g);
+              }
+            }
+            if (leader) mbar_arrive_expect_tx(&sm.full[stage], STAGE_TX);
+            if constexpr (CG == 2) {
+              const uint32_t bar = mapa_shared(smem_u32(&sm.full[stage]), 0);
+              tma_load_3d_pair(sm.a[stage], &tmA, bar, kb * BK, m0, tc.g);
+              tma_load_3d_pair(sm.b[stage], &tmB, bar, kb * BK, nb0, tc.g);
             } else {
-              mma_f8f6f4(d, ad + 2 * k, bd + 2 * k, IDESC, k > 0 ? 1u : 0u);
+              tma_load_3d(sm.a[stage], &tmA, &sm.full[stage], kb * BK, m0, tc.g);
+              tma_load_3d(sm.b[stage], &tmB, &sm.full[stage], kb * BK, nb0, tc.g);
+            }
+            issued |= 1u << stage;
+            issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+            if (++stage == STAGES) {
+              stage = 0;
+              phase ^= 1u;
             }
           }
-          mma_commit(&sm.empty[stage]);
-          if constexpr (!IS_INT8) {
-            mma_commit(&sm.acc_full[buf]);
-            buf ^= 1;
-            if (buf == 0) bphase ^= 1u;
-          }
-          if (++stage == STAGES) {
-            stage = 0;
-            phase ^= 1u;
-          }
         }
-        if constexpr (IS_INT8) {
-          if (ok) {
-            mma_commit(&sm.acc_full[buf]);
-            buf ^= 1;
-            if (buf == 0) bphase ^= 1u;
+        if (ok) {
+          // tail: wait until the MMAs have released every filled stage, so no
+          // commit arrives on this CTA's barriers after it has retired
+          for (int i = 0; i < STAGES && ok; ++i) {
+            ok = wait_bounded(&sm.empty[stage], phase ^ 1u, abort, p.err, kErrTimeout | kRoleProducer | kWaitDrain);
+            if (++stage == STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
           }
+        } else if (CG == 1 || leader) {  // let copies already in flight land before the CTA retires
+          volatile int never = 0;
+          for (int s = 0; s < STAGES; ++s)
+            if ((issued >> s) & 1u)
+              wait_bounded(&sm.full[s], (issued_phase >> s) & 1u, &never, nullptr, 0);
+        } else {
+          pause_ns(1000000);  // the peer's copies signal the leader's barriers; give them time to land
         }
       }
-      if (!ok) {  // wait until every MMA already issued has finished with TMEM and smem
-        mma_commit(&sm.drain);
-        volatile int never = 0;
-        wait_bounded(&sm.drain, 0, &never, nullptr, 0);
+      __syncwarp();
+    } else if (warp == 1) {
+      // ---------------------------------------------------------- MMA issuer (leader CTA)
+      if (lane == 0 && leader) {
+        int stage = 0, buf = 0;
+        uint32_t phase = 0, bphase = 0;
+        bool ok = true;
+        for (int tile = unit; ok && tile < p.num_tiles; tile += units) {
+          for (int kb = 0; kb < p.KB; ++kb) {
+            // FP8: every K block starts a fresh partial in the next buffer;
+            // INT8: the tile's accumulator is claimed once, at its first K block
+            if (!IS_INT8 || kb == 0) {
+              if (!wait_bounded(&sm.acc_empty[buf], bphase ^ 1u, abort, p.err, kErrTimeout | kRoleMma | kWaitAccEmpty)) {
+                ok = false;
+                break;
+              }
+            }
+            if (!wait_bounded(&sm.full[stage], phase, abort, p.err, kErrTimeout | kRoleMma | kWaitStageFull)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t d = tmem + static_cast<uint32_t>(buf * BN);
+            const uint64_t ad = sdesc_k_sw128(smem_u32(sm.a[stage]));
+            const uint64_t bd = sdesc_k_sw128(smem_u32(sm.b[stage]));
+#pragma unroll
+            for (int k = 0; k < BK / 32; ++k) {
+              const uint32_t acc = IS_INT8 ? ((kb > 0 || k > 0) ? 1u : 0u) : (k > 0 ? 1u : 0u);
+              if constexpr (CG == 2) {
+                if constexpr (IS_INT8) {
+                  mma_i8_pair(d, ad + 2 * k, bd + 2 * k, IDESC, acc);
+                } else {
+                  mma_f8f6f4_pair(d, ad + 2 * k, bd + 2 * k, IDESC, acc);
+                }
+              } else {
+                if constexpr (IS_INT8) {
+                  mma_i8(d, ad + 2 * k, bd + 2 * k, IDESC, acc);
+                } else {
+                  mma_f8f6f4(d, ad + 2 * k, bd + 2 * k, IDESC, acc);
+                }
+              }
+            }
+            // FP8: one commit per K block both frees the stage for the producers
+            // and tells the consumers that the partial is complete.  INT8: the
+            // tile's last K block also commits the accumulator barrier.
+            if constexpr (CG == 2) {
+              mma_commit_pair_mc(&sm.empty[stage], 0x3);
+              if (IS_INT8 && kb == p.KB - 1) mma_commit_pair_mc(&sm.acc_full[buf], 0x3);
+            } else {
+              mma_commit(&sm.empty[stage]);
+              if (IS_INT8 && kb == p.KB - 1) mma_commit(&sm.acc_full[buf]);
+            }
+            if (!IS_INT8 || kb == p.KB - 1) {
+              buf ^= 1;
+              if (buf == 0) bphase ^= 1u;
+            }
+            if (++stage == STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+        }
+        if (!ok) {  // wait until every MMA already issued has finished with TMEM and smem
+          if constexpr (CG == 2) {
+            mma_commit_pair(&sm.drain);
+          } else {
+            mma_commit(&sm.drain);
+          }
+          volatile int never = 0;
+          wait_bounded(&sm.drain, 0, &never, nullptr, 0);
+        }
       }
-    }
-    __syncwarp();
+      __syncwarp();
+    } else if (!IS_INT8) {
+      // ---------------------------------------------------------- scale producer (warps 2, 3)
+      // Stages scale_a of this CTA's 128 rows and scale_b of the tile's two
+      // 128-column blocks for each K block into a ring kScaleRing blocks deep.
+      // The loads of kScaleBatch consecutive K blocks are issued together, so
+      // one global-load latency is paid per batch rather than per K block.
+      const int t = threadIdx.x - 64;  // 0..63
+      uint32_t cnt = 0;                // K blocks staged so far (ring position)
+      bool ok = true;
+      for (int tile = unit; ok && tile < p.num_tiles; tile += units) {
+        const TileCoord tc = tile_coord(tile, p.grid_m, p.grid_n, p.group_m);
+        const int m0 = tc.pm * (BM * CG) + rank * BM, n0 = tc.pn * BN;
+        for (int kb0 = 0; ok && kb0 < p.KB; kb0 += kScaleBatch) {
+          const int nb = p.KB - kb0 < kScaleBatch ? p.KB - kb0 : kScaleBatch;
+          float va[kScaleBatch], vc[kScaleBatch], vb[kScaleBatch];
+#pragma unroll
+          for (int i = 0; i < kScaleBatch; ++i) {
+            if (i < nb) {
+              va[i] = scale_row<MODE>(p, tc.g, m0 + t, kb0 + i);
+              vc[i] = scale_row<MODE>(p, tc.g, m0 + t + 64, kb0 + i);
+              vb[i] = t < 2 ? scale_col<MODE>(p, tc.g, kb0 + i, (n0 >> 7) + t) : 0.f;
+            }
+          }
+#pragma unroll
+          for (int i = 0; i < kScaleBatch; ++i) {
+            if (i < nb) {
+              const uint32_t c = cnt + static_cast<uint32_t>(i);
+              const int slot = static_cast<int>(c % kScaleRing);
+              const uint32_t ph = (c / kScaleRing) & 1u;
+              if (!warp_wait(&sm.sc_empty[slot], ph ^ 1u, abort, p.err, kErrTimeout | kRoleScale | kWaitScaleEmpty)) {
+                ok = false;
+                break;
+              }
+              sm.sa[slot][t] = va[i];
+              sm.sa[slot][t + 64] = vc[i];
+              if (t < 2) sm.sb[slot][t] = vb[i];
+              mbar_arrive(&sm.sc_full[slot]);
+            }
+          }
+          cnt += static_cast<uint32_t>(nb);
+        }
+      }
     }
   } else {
     regs_inc<kWideConsumerRegs>();
@@ -287,54 +437,78 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t t_lane = static_cast<uint32_t>(lg * 32) << 16;
     const int row = lg * 32 + lane;
     uint8_t* stg = sm.stage_out[cw];
-    int buf = 0;
-    uint32_t bphase = 0;
-    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
+    // release target of the accumulator buffers: the leader's barrier
+    // release target of this warpgroup's accumulator half: the leader's barrier
+    const uint32_t acc_empty0 =
+        CG == 2 ? mapa_shared(smem_u32(&sm.acc_empty[0]), 0) : smem_u32(&sm.acc_empty[0]);
+    int buf = 0, sslot = 0;
+    uint32_t bphase = 0, ssph = 0;
+    uint32_t kbc = 0;  // K blocks of this CTA's tiles seen so far (stage = kbc % STAGES)
+    for (int tile = unit; tile < p.num_tiles; tile += units) {
       const TileCoord tc = tile_coord(tile, p.grid_m, p.grid_n, p.group_m);
-      const int m0 = tc.pm * BM, n0 = tc.pn * BN;
+      const int m0 = tc.pm * (BM * CG) + rank * BM, n0 = tc.pn * BN;
       const int m = m0 + row;
       const int ncol0 = n0 + half * 128;
       bool ok = true;
       if constexpr (!IS_INT8) {
-        const int nb = ncol0 >> 7;
         float acc[128];
 #pragma unroll
         for (int j = 0; j < 128; ++j) acc[j] = 0.f;
-        float s_cur = block_scale<MODE>(p, tc.g, m, 0, nb);
         for (int kb = 0; kb < p.KB; ++kb) {
-          const float s_next = (kb + 1 < p.KB) ? block_scale<MODE>(p, tc.g, m, kb + 1, nb) : 0.f;
-          if (!warp_wait(&sm.acc_full[buf], bphase, abort, p.err, kErrTimeout | kRoleConsumer | kWaitAccFull)) {
+          if (!warp_wait(&sm.sc_full[sslot], ssph, abort, p.err, kErrTimeout | kRoleConsumer | kWaitScaleFull)) {
             ok = false;
             break;
           }
+          const float s_cur = sm.sa[sslot][row] * sm.sb[sslot][half];
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.sc_empty[sslot]);
+          if (++sslot == kScaleRing) {
+            sslot = 0;
+            ssph ^= 1u;
+          }
+          // the MMA's commit on this K block's stage marks the partial complete;
+          // the MMA runs at most two K blocks ahead, so the stage's phase
+          // cannot advance again before this wait observes it
+          if (!warp_wait(&sm.empty[kbc % STAGES], (kbc / STAGES) & 1u, abort, p.err,
+                         kErrTimeout | kRoleConsumer | kWaitAccFull)) {
+            ok = false;
+            break;
+          }
+          ++kbc;
           tc_fence_after();
           const uint32_t tb = tmem + t_lane + static_cast<uint32_t>(buf * BN + half * 128);
+          {
+            uint32_t r0[32], r1[32];
+            tmem_ld32x2(tb, tb + 32, r0, r1);
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t r[32];
-            tmem_ld32(tb + c * 32, r);
+            for (int j = 0; j < 32; ++j) acc[j] = fmaf(s_cur, __uint_as_float(r0[j]), acc[j]);
 #pragma unroll
-            for (int j = 0; j < 32; ++j) acc[c * 32 + j] = fmaf(s_cur, __uint_as_float(r[j]), acc[c * 32 + j]);
+            for (int j = 0; j < 32; ++j) acc[32 + j] = fmaf(s_cur, __uint_as_float(r1[j]), acc[32 + j]);
           }
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&sm.acc_empty[buf]);
+          {
+            uint32_t r0[32], r1[32];
+            tmem_ld32x2(tb + 64, tb + 96, r0, r1);
+            // the partial is in registers: hand the TMEM buffer back before the math
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(acc_empty0 + static_cast<uint32_t>(buf * sizeof(uint64_t)));
+#pragma unroll
+            for (int j = 0; j < 32; ++j) acc[64 + j] = fmaf(s_cur, __uint_as_float(r0[j]), acc[64 + j]);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) acc[96 + j] = fmaf(s_cur, __uint_as_float(r1[j]), acc[96 + j]);
+          }
           buf ^= 1;
           if (buf == 0) bphase ^= 1u;
-          s_cur = s_next;
         }
         if (!ok) break;
 #pragma unroll
         for (int ch = 0; ch < 128 / CPC; ++ch) {
           if (lane == 0) bulk_wait_read_all();
           __syncwarp();
+          float v[CPC];
 #pragma unroll
-          for (int sub = 0; sub < CPC / 32; ++sub) {
-            float v[32];
-#pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = acc[ch * CPC + sub * 32 + j];
-            stage_32<OutT>(stg, lane, sub * (32 * static_cast<int>(sizeof(OutT)) / 16), v);
-          }
+          for (int j = 0; j < CPC; ++j) v[j] = acc[ch * CPC + j];
+          stage_row64<OutT, CPC>(stg, lane, v);
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0 && m0 + lg * 32 < p.M && ncol0 + ch * CPC < p.N) {  // skip boxes wholly outside
@@ -343,7 +517,8 @@ __global__ void __launch_bounds__(384, 1)
           }
         }
       } else {
-        if (!warp_wait(&sm.acc_full[buf], bphase, abort, p.err, kErrTimeout | kRoleConsumer | kWaitAccFull)) break;
+        if (!warp_wait(&sm.acc_full[buf], bphase, abort, p.err, kErrTimeout | kRoleConsumer | kWaitAccFull))
+          break;
         tc_fence_after();
         const bool has_row = p.s_row != nullptr, has_col = p.s_col != nullptr;
         const float sr = (has_row && m < p.M) ? __ldg(p.s_row + m) : 1.f;
@@ -352,40 +527,41 @@ __global__ void __launch_bounds__(384, 1)
         for (int ch = 0; ch < 128 / CPC; ++ch) {
           if (lane == 0) bulk_wait_read_all();
           __syncwarp();
-#pragma unroll
-          for (int sub = 0; sub < CPC / 32; ++sub) {
-            const int c0 = ch * CPC + sub * 32;
-            uint32_t r[32];
+          const int c0 = ch * CPC;
+          uint32_t r[CPC];
+          if constexpr (CPC == 32) {
             tmem_ld32(tb + c0, r);
-            float v[32];
-            if constexpr (sizeof(OutT) == 4 && !std::is_same<OutT, float>::value) {
-#pragma unroll
-              for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);  // raw int32 accumulator
-            } else {
-#pragma unroll
-              for (int j = 0; j < 32; ++j) {
-                float f = __int2float_rn(static_cast<int>(r[j]));
-                if (has_row) f = __fmul_rn(f, sr);
-                if (has_col) {
-                  const int n = ncol0 + c0 + j;
-                  const float sc = n < p.N ? __ldg(p.s_col + n) : 0.f;
-                  f = __fmul_rn(f, sc);
-                }
-                v[j] = f;
-              }
-            }
-            stage_32<OutT>(stg, lane, sub * (32 * static_cast<int>(sizeof(OutT)) / 16), v);
+          } else {
+            tmem_ld16(tb + c0, r);
           }
+          float v[CPC];
+          if constexpr (sizeof(OutT) == 4 && !std::is_same<OutT, float>::value) {
+#pragma unroll
+            for (int j = 0; j < CPC; ++j) v[j] = __uint_as_float(r[j]);  // raw int32 accumulator
+          } else {
+#pragma unroll
+            for (int j = 0; j < CPC; ++j) {
+              float f = __int2float_rn(static_cast<int>(r[j]));
+              if (has_row) f = __fmul_rn(f, sr);
+              if (has_col) {
+                const int n = ncol0 + c0 + j;
+                const float sc = n < p.N ? __ldg(p.s_col + n) : 0.f;
+                f = __fmul_rn(f, sc);
+              }
+              v[j] = f;
+            }
+          }
+          stage_row64<OutT, CPC>(stg, lane, v);
           fence_proxy_async_smem();
           __syncwarp();
-          if (lane == 0 && m0 + lg * 32 < p.M && ncol0 + ch * CPC < p.N) {  // skip boxes wholly outside
+          if (lane == 0 && m0 + lg * 32 < p.M && ncol0 + ch * CPC < p.N) {
             tma_store_3d(&tmD, stg, ncol0 + ch * CPC, m0 + lg * 32, tc.g);
             bulk_commit();
           }
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.acc_empty[buf]);
+        if (lane == 0) mbar_arrive_cluster(acc_empty0 + static_cast<uint32_t>(buf * sizeof(uint64_t)));
         buf ^= 1;
         if (buf == 0) bphase ^= 1u;
       }
@@ -395,10 +571,18 @@ __global__ void __launch_bounds__(384, 1)
   }
 
   tc_fence_before();
-  __syncthreads();
+  if constexpr (CG == 2) {
+    cluster_sync_all();  // no CTA retires while its peer may still signal it
+  } else {
+    __syncthreads();
+  }
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, TMEM_COLS);
+    if constexpr (CG == 2) {
+      tmem_dealloc_pair(tmem, TMEM_COLS);
+    } else {
+      tmem_dealloc(tmem, TMEM_COLS);
+    }
   }
 }
 

@@ -78,9 +78,18 @@ def test_blockwise_scale_shape_rule_from_the_issue():
 # ---------------------------------------------------------------------------
 # planning
 # ---------------------------------------------------------------------------
-def test_plan_large_fp8_is_persistent_wide():
+def test_plan_large_fp8_is_persistent_wide_on_cta_pairs():
     p = bs.plan_for(bs.OP_FP8_BLOCKWISE, 16640, 1, 5120, 8192, 148)
-    assert p == {"kernel": 1, "tile_m": 128, "tile_n": 256, "splits": 1, "ctas": 148, "cluster": 1, "launches": 1}
+    assert p == {"kernel": 1, "tile_m": 256, "tile_n": 256, "splits": 1, "ctas": 148, "cluster": 2, "launches": 1}
+    prev = bs.set_path_override(bs.PATH_WIDE_SINGLE)
+    try:
+        p = bs.plan_for(bs.OP_FP8_BLOCKWISE, 16640, 1, 5120, 8192, 148)
+        assert p == {"kernel": 1, "tile_m": 128, "tile_n": 256, "splits": 1, "ctas": 148, "cluster": 1, "launches": 1}
+    finally:
+        bs.set_path_override(prev)
+    # fewer tiles than CTA pairs: one pair per tile
+    p = bs.plan_for(bs.OP_FP8_BLOCKWISE, 300, 1, 512, 1024, 148)
+    assert p["ctas"] == 2 * 2 * 2 and p["cluster"] == 2
 
 
 @pytest.mark.parametrize("M", [1, 8, 16, 17, 32, 127, 128, 129, 255, 256])
@@ -102,7 +111,7 @@ def test_plan_int8_and_edges():
     p = bs.plan_for(bs.OP_FP8_BLOCKWISE, 16, 1, 512, 0, 148)
     assert p["kernel"] == 3 and p["launches"] == 1
     b = bs.plan_for(bs.OP_BMM, 16384, 8, 1024, 4096, 148)
-    assert b["kernel"] == 1 and b["ctas"] == 148
+    assert b["kernel"] == 1 and b["ctas"] == 148 and b["tile_m"] == 256
     b = bs.plan_for(bs.OP_BMM, 1, 8, 1024, 4096, 148)
     assert b["kernel"] == 2 and b["ctas"] == 8 * 8 * b["splits"]
 

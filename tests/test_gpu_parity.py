@@ -57,8 +57,8 @@ def test_fp8_tiny_full_matrix(out_dtype):
 
 @pytest.mark.parametrize("M,N,K", [(128, 256, 128), (129, 384, 256), (300, 520, 640), (1, 256, 128),
                                    (255, 128, 1024), (640, 1280, 384)])
-@pytest.mark.parametrize("kernel", [bs.PATH_WIDE, bs.PATH_SKINNY])
-def test_fp8_ragged_shapes_both_kernels(M, N, K, kernel, path):
+@pytest.mark.parametrize("kernel", [bs.PATH_WIDE, bs.PATH_WIDE_SINGLE, bs.PATH_SKINNY])
+def test_fp8_ragged_shapes_all_kernels(M, N, K, kernel, path):
     path(kernel)
     d = wl.fp8_blockwise_inputs(M, N, K, seed=50 + M + N + K)
     y, S = oracle_fp8(d)
@@ -151,8 +151,11 @@ def _int8_assert(d, rows, s_b=True):
     np.testing.assert_array_equal(bf16_bits(sel(int8_run(d, torch.bfloat16, s_b))), bf)
 
 
-@pytest.mark.parametrize("M,N,K", [(128, 256, 128), (300, 520, 1040), (1, 256, 4096), (257, 264, 48)])
-def test_int8_bit_exact_small(M, N, K):
+@pytest.mark.parametrize("M,N,K", [(128, 256, 128), (300, 520, 1040), (1, 256, 4096), (257, 264, 48),
+                                   (600, 1024, 2048)])
+@pytest.mark.parametrize("kernel", [bs.PATH_WIDE, bs.PATH_WIDE_SINGLE])
+def test_int8_bit_exact_small(M, N, K, kernel, path):
+    path(kernel)
     _int8_assert(wl.int8_inputs(M, N, K, seed=70 + M), rows=None)
 
 
@@ -203,6 +206,6 @@ def test_bmm_batch_first_layout(M):
 def test_bmm_both_kernels_agree_with_oracle(path):
     d = wl.bmm_inputs(200, 3, 384, 512, seed=81)
     y, S = oracle.bmm_blockscale(d["x"], d["w"], d["x_scale"], d["w_scale"])
-    for k in (bs.PATH_WIDE, bs.PATH_SKINNY):
+    for k in (bs.PATH_WIDE, bs.PATH_WIDE_SINGLE, bs.PATH_SKINNY):
         path(k)
         fp8_check(bmm_run(d), y, S, torch.bfloat16, f"bmm kernel={k}")
