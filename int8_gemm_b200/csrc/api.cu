@@ -108,6 +108,10 @@ bs_status device_ctx(DeviceCtx** out) {
 std::atomic<int32_t> g_path_override{0};
 
 constexpr int kSkinnyMaxM = 256;
+
+// CTAs of the skinny kernel that fit on one SM (shared memory of the operand
+// ring, and registers of the BMT accumulators per consumer thread).
+int skinny_ctas_per_sm(int bmt) { return bmt <= 16 ? 3 : (bmt <= 32 ? 2 : 1); }
 constexpr int kGroupM = 16;
 
 struct Plan {
@@ -140,8 +144,12 @@ Plan make_plan(int op, int64_t M, int64_t G, int64_t N, int64_t K, int sms) {
     x.m_tiles = static_cast<int>((M + bmt - 1) / bmt);
     x.n_tiles = static_cast<int>((N + 127) / 128);
     const long long units = static_cast<long long>(x.m_tiles) * x.n_tiles * G;
+    // Split K over a cluster of S CTAs only as far as every CTA stays resident
+    // at once (a second partial wave would double the time of an HBM-bound
+    // stream), S a power of two <= 8 and <= the number of K blocks.
+    const long long slots = static_cast<long long>(skinny_ctas_per_sm(bmt)) * (sms > 0 ? sms : 148);
     int S = 1;
-    while (S < 8 && 2 * S <= KB && units * S < 2LL * (sms > 0 ? sms : 148)) S *= 2;
+    while (S < 8 && 2 * S <= KB && units * 2 * S <= slots) S *= 2;
     x.pub.kernel = 2;
     x.pub.tile_m = bmt;
     x.pub.tile_n = 128;

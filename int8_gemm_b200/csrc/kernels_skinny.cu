@@ -13,7 +13,7 @@ template <Mode MODE, int BMT, typename OutT>
 cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b, const GemmArgs& args, const SkinnyOut& o,
                        int n_tiles, int m_tiles, cudaStream_t stream) {
   auto kernel = skinny_gemm_kernel<MODE, BMT, kSkinnyStages, OutT>;
-  constexpr size_t smem = sizeof(SkinnySmem<BMT, kSkinnyStages, 4>) + 1024;
+  constexpr size_t smem = sizeof(SkinnySmem<BMT, kSkinnyStages, kSkinnyScaleRing>) + 1024;
   static std::atomic<uint64_t> configured{0};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);

@@ -21,6 +21,9 @@
 
 namespace bsg {
 
+constexpr int kSkinnyScaleRing = 16;  // K blocks of scales staged ahead
+constexpr int kSkinnyScaleBatch = 8;  // K blocks whose scale loads are in flight together
+
 template <int BMT, int STAGES, int SSTAGES>
 struct SkinnySmem {
   uint8_t b[STAGES][128 * 128];  // weight rows  (MMA operand "A", 128 rows)
@@ -61,7 +64,8 @@ __global__ void __launch_bounds__(224, 1)
     skinny_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                        const GemmArgs p, const SkinnyOut o) {
   constexpr int BK = 128;
-  constexpr int SSTAGES = 4;
+  constexpr int SSTAGES = kSkinnyScaleRing;
+  constexpr int SBATCH = kSkinnyScaleBatch;
   constexpr uint32_t A_BYTES = BMT * BK, B_BYTES = 128 * BK;
   constexpr int CONSUMER_WARPS = 4;
   constexpr uint32_t ACC_COLS = BMT < 32 ? 32u : static_cast<uint32_t>(BMT);  // one accumulator buffer
@@ -76,6 +80,10 @@ __global__ void __launch_bounds__(224, 1)
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+  if (pad + sizeof(Smem) > dynamic_smem_bytes()) {  // never touch memory the launch did not provide
+    if (threadIdx.x == 0) record_error(p.err, kErrSmemTooSmall);
+    return;
+  }
   Smem& sm = *reinterpret_cast<Smem*>(smem_raw + pad);
   volatile int* abort = &sm.abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -188,17 +196,44 @@ __global__ void __launch_bounds__(224, 1)
     }
     __syncwarp();
   } else if (warp == 6) {
-    // scale producer: s[j] for the BMT activation rows of this CTA
-    int si = 0;
-    uint32_t sphase = 0;
-    for (int i = 0; i < nkb; ++i) {
-      const int kb = kb_lo + i;
-      if (!warp_wait(&sm.sc_empty[si], sphase ^ 1u, abort, p.err, kErrTimeout | kRoleScale | kWaitScaleEmpty)) break;
-      for (int j = lane; j < BMT; j += 32) sm.scale[si][j] = block_scale<MODE>(p, g, m0 + j, kb, nb);
-      mbar_arrive(&sm.sc_full[si]);
-      if (++si == SSTAGES) {
-        si = 0;
-        sphase ^= 1u;
+    // scale producer: s[j] = scale_a[m0+j, kb] * scale_b[kb, nb] for the BMT
+    // activation rows of this CTA.  The loads of SBATCH K blocks are issued
+    // together, so one global-load latency is paid per batch.
+    constexpr int PER_LANE = (BMT + 31) / 32;
+    bool ok = true;
+    for (int i0 = 0; ok && i0 < nkb; i0 += SBATCH) {
+      const int nb_batch = nkb - i0 < SBATCH ? nkb - i0 : SBATCH;
+      float v[SBATCH][PER_LANE];
+      float c[SBATCH];
+#pragma unroll
+      for (int i = 0; i < SBATCH; ++i) {
+        if (i < nb_batch) {
+          const int kb = kb_lo + i0 + i;
+          c[i] = scale_col<MODE>(p, g, kb, nb);
+#pragma unroll
+          for (int q = 0; q < PER_LANE; ++q) {
+            const int j = lane + 32 * q;
+            v[i][q] = j < BMT ? scale_row<MODE>(p, g, m0 + j, kb) : 0.f;
+          }
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < SBATCH; ++i) {
+        if (i < nb_batch) {
+          const uint32_t cnt = static_cast<uint32_t>(i0 + i);
+          const int si = static_cast<int>(cnt % SSTAGES);
+          const uint32_t ph = (cnt / SSTAGES) & 1u;
+          if (!warp_wait(&sm.sc_empty[si], ph ^ 1u, abort, p.err, kErrTimeout | kRoleScale | kWaitScaleEmpty)) {
+            ok = false;
+            break;
+          }
+#pragma unroll
+          for (int q = 0; q < PER_LANE; ++q) {
+            const int j = lane + 32 * q;
+            if (j < BMT) sm.scale[si][j] = v[i][q] * c[i];
+          }
+          mbar_arrive(&sm.sc_full[si]);
+        }
       }
     }
   } else {

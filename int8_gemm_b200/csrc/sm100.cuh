@@ -18,6 +18,7 @@ namespace bsg {
 // Codes written to the device error word (first writer wins):
 //   0x1000 | role << 8 | wait kind.
 enum : uint32_t {
+  kErrSmemTooSmall = 0x2000,  // launch gave less dynamic shared memory than the layout needs
   kErrTimeout = 0x1000,
   kRoleProducer = 1 << 8,
   kRoleMma = 2 << 8,
@@ -48,6 +49,13 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
+}
+
+// Bytes of dynamic shared memory this launch provides.
+__device__ __forceinline__ uint32_t dynamic_smem_bytes() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%dynamic_smem_size;" : "=r"(r));
+  return r;
 }
 
 __device__ __forceinline__ void fence_proxy_async_smem() {

@@ -68,13 +68,6 @@ struct GemmArgs {
 // Shared-memory layout of one CTA.  In the pair (cta_group::2) variant both
 // CTAs use the same layout: the leader's MMA descriptors address the same
 // offsets in the peer.
-#ifndef BSG_L2_PREFETCH_DISTANCE
-#define BSG_L2_PREFETCH_DISTANCE 8
-#endif
-// K blocks between the L2 prefetch of an operand box and its load into shared
-// memory.  Loads that miss L2 (first touch of a panel, or a line homed in the
-// other die's L2) otherwise set the latency of a whole stage.
-constexpr int kL2PrefetchDistance = BSG_L2_PREFETCH_DISTANCE;
 constexpr int kScaleRing = 16;  // K blocks of scales staged ahead of the consumers
 constexpr int kScaleBatch = 8;  // K blocks whose scale loads are in flight together
 
@@ -196,6 +189,10 @@ __global__ void __launch_bounds__(384, 1)
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+  if (pad + sizeof(Smem) > dynamic_smem_bytes()) {  // never touch memory the launch did not provide
+    if (threadIdx.x == 0) record_error(p.err, kErrSmemTooSmall);
+    return;
+  }
   Smem& sm = *reinterpret_cast<Smem*>(smem_raw + pad);
   volatile int* abort = &sm.abort;
 
@@ -252,10 +249,6 @@ __global__ void __launch_bounds__(384, 1)
         bool ok = true;
         for (int tile = unit; ok && tile < p.num_tiles; tile += units) {
           const TileCoord tc = tile_coord(tile, p.grid_m, p.grid_n, p.group_m);
-          // the tile after this one, for prefetches that run past its last K block
-          const int next_tile = tile + units;
-          TileCoord tn = tc;
-          if (next_tile < p.num_tiles) tn = tile_coord(next_tile, p.grid_m, p.grid_n, p.group_m);
           const int m0 = tc.pm * (BM * CG) + rank * BM;
           const int nb0 = tc.pn * BN + rank * BNL;  // this CTA's B rows (tile columns)
           for (int kb = 0; kb < p.KB; ++kb) {
@@ -263,18 +256,6 @@ __global__ void __launch_bounds__(384, 1)
                               kErrTimeout | kRoleProducer | kWaitStageEmpty)) {
               ok = false;
               break;
-            }
-            if (kL2PrefetchDistance > 0) {
-              int pk = kb + kL2PrefetchDistance;
-              const TileCoord* pt = &tc;
-              if (pk >= p.KB) {
-                pk -= p.KB;
-                pt = &tn;
-              }
-              if (pt == &tc || next_tile < p.num_tiles) {
-                tma_prefetch_l2_3d(&tmA, pk * BK, pt->pm * (BM * CG) + rank * BM, pt->g);
-                tma_prefetch_l2_3d(&tmB, pk * BK, pt->pn * BN + rank * BNL, pt->g);
-              }
             }
             if (leader) mbar_arrive_expect_tx(&sm.full[stage], STAGE_TX);
             if constexpr (CG == 2) {
