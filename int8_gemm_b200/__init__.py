@@ -112,6 +112,14 @@ def _bytes8(t: torch.Tensor, name: str) -> torch.Tensor:
     raise BsgemmError(BS_ERR_DTYPE, f"{name} must be float8_e4m3fn (or its uint8 bytes), got {t.dtype}")
 
 
+def _empty_out(lead: tuple, N: int, dtype: torch.dtype, device) -> torch.Tensor:
+    """Output [*lead, N] whose rows start on 16-byte boundaries (the kernels'
+    store alignment): the last dimension is padded in memory, not in shape."""
+    per16 = 16 // torch.empty((), dtype=dtype).element_size()
+    Np = -(-N // per16) * per16
+    return torch.empty((*lead, Np), dtype=dtype, device=device)[..., :N]
+
+
 def _ptr(t):
     return ctypes.c_void_p(t.data_ptr()) if t is not None else None
 
@@ -144,7 +152,7 @@ def bs_gemm_fp8_blockwise(A: torch.Tensor, B: torch.Tensor, scale_a: torch.Tenso
     if out_dtype not in (torch.bfloat16, torch.float32):
         raise BsgemmError(BS_ERR_DTYPE, f"out_dtype must be bfloat16 or float32, got {out_dtype}")
     if out is None:
-        out = torch.empty((M, N), dtype=out_dtype, device=A.device)
+        out = _empty_out((M,), N, out_dtype, A.device)
     elif out.dtype != out_dtype or tuple(out.shape) != (M, N) or out.stride(1) != 1:
         raise BsgemmError(BS_ERR_LAYOUT, "out must be a row-major [M, N] tensor of out_dtype")
     with torch.cuda.device(A.device):
@@ -187,7 +195,7 @@ def int_scaled_mm(A: torch.Tensor, B: torch.Tensor, s_a: torch.Tensor | None, s_
     if out_dtype not in _OUT_CODE:
         raise BsgemmError(BS_ERR_DTYPE, f"out_dtype must be float32, bfloat16 or int32, got {out_dtype}")
     if out is None:
-        out = torch.empty((M, N), dtype=out_dtype, device=A.device)
+        out = _empty_out((M,), N, out_dtype, A.device)
     elif out.dtype != out_dtype or tuple(out.shape) != (M, N) or out.stride(1) != 1:
         raise BsgemmError(BS_ERR_LAYOUT, "out must be a row-major [M, N] tensor of out_dtype")
     with torch.cuda.device(A.device):
@@ -231,7 +239,7 @@ def bmm_a8w8_blockscale(x: torch.Tensor, w: torch.Tensor, x_scale: torch.Tensor,
     if out_dtype not in (torch.bfloat16, torch.float32):
         raise BsgemmError(BS_ERR_DTYPE, f"out_dtype must be bfloat16 or float32, got {out_dtype}")
     if out is None:
-        out = torch.empty((M, G, N), dtype=out_dtype, device=x.device)
+        out = _empty_out((M, G), N, out_dtype, x.device)
     elif out.dtype != out_dtype or tuple(out.shape) != (M, G, N) or out.stride(2) != 1:
         raise BsgemmError(BS_ERR_LAYOUT, "out must be [M, G, N] of out_dtype with unit stride along N")
     with torch.cuda.device(x.device):

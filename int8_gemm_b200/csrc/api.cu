@@ -111,7 +111,11 @@ constexpr int kSkinnyMaxM = 256;
 
 // CTAs of the skinny kernel that fit on one SM (shared memory of the operand
 // ring, and registers of the BMT accumulators per consumer thread).
-int skinny_ctas_per_sm(int bmt) { return bmt <= 16 ? 3 : (bmt <= 32 ? 2 : 1); }
+int skinny_ctas_per_sm(int bmt) {
+  return bmt <= 16 ? SkinnyCfg<16>::CTAS_PER_SM
+                   : (bmt <= 32 ? SkinnyCfg<32>::CTAS_PER_SM
+                                : (bmt <= 64 ? SkinnyCfg<64>::CTAS_PER_SM : SkinnyCfg<128>::CTAS_PER_SM));
+}
 constexpr int kGroupM = 16;
 
 struct Plan {

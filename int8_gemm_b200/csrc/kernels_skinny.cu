@@ -12,8 +12,8 @@ constexpr int kMaxDevices = 64;
 template <Mode MODE, int BMT, typename OutT>
 cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b, const GemmArgs& args, const SkinnyOut& o,
                        int n_tiles, int m_tiles, cudaStream_t stream) {
-  auto kernel = skinny_gemm_kernel<MODE, BMT, kSkinnyStages, OutT>;
-  constexpr size_t smem = sizeof(SkinnySmem<BMT, kSkinnyStages, kSkinnyScaleRing>) + 1024;
+  auto kernel = skinny_gemm_kernel<MODE, BMT, OutT>;
+  constexpr size_t smem = sizeof(SkinnySmemFor<BMT>) + 1024;
   static std::atomic<uint64_t> configured{0};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -24,19 +24,22 @@ cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b, const GemmArg
     if (e != cudaSuccess) return e;
     configured.fetch_or(bit, std::memory_order_release);
   }
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = static_cast<unsigned>(args.splits);
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  // programmatic dependent launch: the prologue may overlap the previous kernel
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(n_tiles * args.splits), static_cast<unsigned>(m_tiles),
                      static_cast<unsigned>(args.G));
-  cfg.blockDim = dim3(kSkinnyThreads, 1, 1);
+  cfg.blockDim = dim3(SkinnyCfg<BMT>::THREADS, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, kernel, a, b, args, o);
 }
 

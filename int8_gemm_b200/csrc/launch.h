@@ -16,8 +16,6 @@ constexpr int kWideBN = 256;
 constexpr int kWideStages = 4;      // single-CTA tiles: 48 KB per stage
 constexpr int kWideStagesPair = 6;  // CTA-pair tiles: 32 KB per stage and CTA
 constexpr int kWideThreads = 384;
-constexpr int kSkinnyStages = 4;
-constexpr int kSkinnyThreads = 224;
 
 // Persistent wide kernel over `grid` CTAs; cta_group 2 launches clusters of two
 // CTAs computing 256 x 256 tiles, cta_group 1 single CTAs computing 128 x 256.

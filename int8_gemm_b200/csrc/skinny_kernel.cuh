@@ -9,11 +9,18 @@
 // second launch) -- the same fp32 partial-sum-then-cast structure as the
 // split-K decomposition decomposeK in pytorch/torch/_inductor/kernel/mm.py.
 //
-// Roles: warp 0 TMA producer, warp 1 MMA issuer, warps 2..5 consumers (warp w
-// owns TMEM lanes 32*(w%4).., i.e. 32 weight rows, and all BMT columns),
-// warp 6 scale producer: per K block it writes s[j] = scale_a[m0+j, kb] *
-// scale_b[kb, nb] (one value per activation row, shared by the CTA because the
-// 128 weight rows form one 128-wide scale block) into a small shared ring.
+// Roles: warp 0 TMA producer, warp 1 MMA issuer and TMEM owner, warp 2 scale
+// producer, warp 3 idle, warps 4.. consumers.  Consumer warp w reads TMEM lanes
+// 32*(w%4).. (32 weight rows) and, when there are eight consumer warps, one
+// half of the BMT accumulator columns.  The scale producer writes, per K block,
+// s[j] = scale_a[m0+j, kb] * scale_b[kb, nb] (one value per activation row,
+// shared by the CTA because its 128 weight rows form one 128-wide scale block)
+// into a small shared ring.
+//
+// The grid never exceeds one wave (the host picks S accordingly), so every
+// CTA streams its weights from the first microsecond: the producer issues the
+// first ring of loads before the CTA-wide barrier, and with programmatic
+// dependent launch the next kernel's prologue overlaps this one's tail.
 #pragma once
 
 #include "sm100.cuh"
@@ -23,6 +30,22 @@ namespace bsg {
 
 constexpr int kSkinnyScaleRing = 16;  // K blocks of scales staged ahead
 constexpr int kSkinnyScaleBatch = 8;  // K blocks whose scale loads are in flight together
+constexpr int kSkinnyAccBufs = 4;     // TMEM accumulator buffers (MMA runs up to 4 K blocks ahead)
+
+// Shape of the kernel for an activation tile of BMT rows (the MMA N).
+template <int BMT>
+struct SkinnyCfg {
+  static constexpr int CW = BMT >= 64 ? 8 : 4;  // consumer warps (two per TMEM lane group when 8)
+  static constexpr int CPW = BMT * 4 / CW;      // accumulator columns per consumer thread
+  static constexpr int THREADS = 128 + 32 * CW;
+  // Shared memory (operand ring) and registers (CPW accumulators per consumer
+  // thread) decide how many CTAs share an SM; the ring depth fills what is left.
+  static constexpr int CTAS_PER_SM = BMT <= 16 ? 3 : (BMT <= 32 ? 2 : 1);
+  static constexpr int STAGES = BMT <= 16 ? 4 : (BMT <= 32 ? 5 : (BMT <= 64 ? 8 : 6));
+  static constexpr uint32_t ACC_COLS = BMT < 32 ? 32u : static_cast<uint32_t>(BMT);
+  static constexpr uint32_t TMEM_COLS = kSkinnyAccBufs * ACC_COLS;  // a power of two: 128, 256 or 512
+  static_assert(CTAS_PER_SM * TMEM_COLS <= 512, "co-resident CTAs must fit in the SM's 512 TMEM columns");
+};
 
 template <int BMT, int STAGES, int SSTAGES>
 struct SkinnySmem {
@@ -31,8 +54,8 @@ struct SkinnySmem {
   float scale[SSTAGES][BMT];
   uint64_t full[STAGES];
   uint64_t empty[STAGES];
-  uint64_t acc_full[2];
-  uint64_t acc_empty[2];
+  uint64_t acc_full[kSkinnyAccBufs];
+  uint64_t acc_empty[kSkinnyAccBufs];
   uint64_t sc_full[SSTAGES];
   uint64_t sc_empty[SSTAGES];
   uint64_t drain;
@@ -40,9 +63,8 @@ struct SkinnySmem {
   int abort;
 };
 
-__host__ __device__ constexpr uint32_t tmem_cols_for(int cols) {
-  return cols <= 32 ? 32u : cols <= 64 ? 64u : cols <= 128 ? 128u : cols <= 256 ? 256u : 512u;
-}
+template <int BMT>
+using SkinnySmemFor = SkinnySmem<BMT, SkinnyCfg<BMT>::STAGES, kSkinnyScaleRing>;
 
 template <typename OutT>
 __device__ __forceinline__ void store_out(OutT* ptr, float v) {
@@ -53,27 +75,110 @@ __device__ __forceinline__ void store_out(OutT* ptr, float v) {
   }
 }
 
+// Four consecutive outputs; `ptr` is 8-byte (bf16) or 16-byte (f32) aligned.
+template <typename OutT>
+__device__ __forceinline__ void store_out4(OutT* ptr, float4 v) {
+  if constexpr (sizeof(OutT) == 2) {
+    __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y);
+    __nv_bfloat162 hi = __floats2bfloat162_rn(v.z, v.w);
+    uint2 u;
+    u.x = *reinterpret_cast<uint32_t*>(&lo);
+    u.y = *reinterpret_cast<uint32_t*>(&hi);
+    *reinterpret_cast<uint2*>(ptr) = u;
+  } else {
+    *reinterpret_cast<float4*>(ptr) = v;
+  }
+}
+
 // Output element (m, g, n) lives at out + m*o_sm + g*o_sg + n.
 struct SkinnyOut {
   void* out;
   long long o_sm, o_sg;
 };
 
-template <Mode MODE, int BMT, int STAGES, typename OutT>
-__global__ void __launch_bounds__(224, 1)
+// CPW consecutive TMEM columns of this warp's 32 lanes with a single wait.
+template <int CPW>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[CPW]) {
+  if constexpr (CPW == 16) {
+    tmem_ld16(taddr, r);
+  } else if constexpr (CPW == 32) {
+    tmem_ld32(taddr, r);
+  } else {
+    static_assert(CPW == 64, "16, 32 or 64 columns per consumer thread");
+    tmem_ld64(taddr, r);
+  }
+}
+
+// Split-K reduction across the S CTAs of a cluster.  Every CTA has published
+// its fp32 partial as red[j * 128 + row] (j = activation row of the tile, row =
+// weight row).  CTA `rank` owns weight rows [rank*R, rank*R + R), R = 128/S;
+// for each (j, 4 rows) it reads the S partials -- all loads of a thread are in
+// flight together -- sums them in rank order 0..S-1 and stores 4 outputs.
+template <int S, int BMT, int CT, typename OutT>
+__device__ __forceinline__ void skinny_cluster_reduce(const float* red, int rank, int ct, int m0, int n0, int g,
+                                                      const GemmArgs& p, const SkinnyOut& o) {
+  constexpr int R = 128 / S;
+  constexpr int R4 = R / 4;
+  constexpr int T = BMT * R4;           // float4 items owned by this CTA
+  constexpr int U = (T + CT - 1) / CT;  // items per consumer thread
+  const uint32_t red_s = smem_u32(red);
+  float4 v[U][S];
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    const int it = ct + u * CT;
+    if (it < T) {
+      const int j = it / R4, r = rank * R + 4 * (it % R4);
+      const uint32_t off = red_s + static_cast<uint32_t>((j * 128 + r) * 4);
+#pragma unroll
+      for (int q = 0; q < S; ++q) v[u][q] = ld_shared_cluster_f4(mapa_shared(off, static_cast<uint32_t>(q)));
+    }
+  }
+  OutT* out = static_cast<OutT*>(o.out);
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    const int it = ct + u * CT;
+    if (it < T) {
+      const int j = it / R4, r = rank * R + 4 * (it % R4);
+      float4 s = v[u][0];
+#pragma unroll
+      for (int q = 1; q < S; ++q) {
+        s.x += v[u][q].x;
+        s.y += v[u][q].y;
+        s.z += v[u][q].z;
+        s.w += v[u][q].w;
+      }
+      const int m = m0 + j, n = n0 + r;
+      if (m < p.M && n < p.N) {
+        OutT* dst = out + static_cast<long long>(m) * o.o_sm + static_cast<long long>(g) * o.o_sg + n;
+        if (n + 3 < p.N) {
+          store_out4<OutT>(dst, s);
+        } else {
+          const float e[4] = {s.x, s.y, s.z, s.w};
+          for (int c = 0; c < 4 && n + c < p.N; ++c) store_out<OutT>(dst + c, e[c]);
+        }
+      }
+    }
+  }
+}
+
+template <Mode MODE, int BMT, typename OutT>
+__global__ void __launch_bounds__(SkinnyCfg<BMT>::THREADS, SkinnyCfg<BMT>::CTAS_PER_SM)
     skinny_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                        const GemmArgs p, const SkinnyOut o) {
+  using Cfg = SkinnyCfg<BMT>;
   constexpr int BK = 128;
+  constexpr int STAGES = Cfg::STAGES;
   constexpr int SSTAGES = kSkinnyScaleRing;
   constexpr int SBATCH = kSkinnyScaleBatch;
+  constexpr int NBUF = kSkinnyAccBufs;
+  constexpr int CW = Cfg::CW;
+  constexpr int CPW = Cfg::CPW;
+  constexpr int CT = 32 * CW;  // consumer threads
   constexpr uint32_t A_BYTES = BMT * BK, B_BYTES = 128 * BK;
-  constexpr int CONSUMER_WARPS = 4;
-  constexpr uint32_t ACC_COLS = BMT < 32 ? 32u : static_cast<uint32_t>(BMT);  // one accumulator buffer
-  constexpr uint32_t TMEM_COLS = tmem_cols_for(2 * ACC_COLS);
+  constexpr uint32_t ACC_COLS = Cfg::ACC_COLS;
   constexpr uint32_t IDESC = idesc_e4m3_f32<128, BMT>();
   static_assert(MODE != Mode::kInt8, "skinny path is FP8 only");
   static_assert(BMT % 16 == 0 && BMT >= 16 && BMT <= 128, "MMA N must be 16..128 in steps of 16");
-  static_assert(2 * ACC_COLS <= TMEM_COLS, "two accumulator buffers");
   using Smem = SkinnySmem<BMT, STAGES, SSTAGES>;
   static_assert(sizeof(float) * 128 * BMT <= sizeof(uint8_t) * STAGES * (128 + BMT) * 128,
                 "split-K reduction buffer reuses the operand ring");
@@ -82,6 +187,10 @@ __global__ void __launch_bounds__(224, 1)
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   if (pad + sizeof(Smem) > dynamic_smem_bytes()) {  // never touch memory the launch did not provide
     if (threadIdx.x == 0) record_error(p.err, kErrSmemTooSmall);
+    return;
+  }
+  if (p.splits != 1 && p.splits != 2 && p.splits != 4 && p.splits != 8) {  // the reduction handles these
+    if (threadIdx.x == 0) record_error(p.err, kErrBadSplit);
     return;
   }
   Smem& sm = *reinterpret_cast<Smem*>(smem_raw + pad);
@@ -100,62 +209,71 @@ __global__ void __launch_bounds__(224, 1)
   const int kb_hi = static_cast<int>((static_cast<long long>(p.KB) * (rank + 1)) / S);
   const int nkb = kb_hi - kb_lo;
 
+  // Producer state lives in thread 0, which initialises the barriers and
+  // issues the first ring of loads before the CTA-wide barrier.
+  int p_i = 0, p_stage = 0;
+  uint32_t p_phase = 0, issued = 0, issued_phase = 0;
+  bool p_ok = true;
+  auto produce = [&](int upto) {
+    for (; p_i < upto; ++p_i) {
+      const int kb = kb_lo + p_i;
+      if (!wait_bounded(&sm.empty[p_stage], p_phase ^ 1u, abort, p.err, kErrTimeout | kRoleProducer | kWaitStageEmpty)) {
+        p_ok = false;
+        return;
+      }
+      mbar_arrive_expect_tx(&sm.full[p_stage], A_BYTES + B_BYTES);
+      tma_load_3d(sm.b[p_stage], &tmB, &sm.full[p_stage], kb * BK, n0, g);
+      tma_load_3d(sm.a[p_stage], &tmA, &sm.full[p_stage], kb * BK, m0, g);
+      issued |= 1u << p_stage;
+      issued_phase = (issued_phase & ~(1u << p_stage)) | (p_phase << p_stage);
+      if (++p_stage == STAGES) {
+        p_stage = 0;
+        p_phase ^= 1u;
+      }
+    }
+  };
+
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&sm.full[s], 1);
       mbar_init(&sm.empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < NBUF; ++b) {
       mbar_init(&sm.acc_full[b], 1);
-      mbar_init(&sm.acc_empty[b], CONSUMER_WARPS);
+      mbar_init(&sm.acc_empty[b], CW);
     }
     for (int s = 0; s < SSTAGES; ++s) {
       mbar_init(&sm.sc_full[s], 32);
-      mbar_init(&sm.sc_empty[s], CONSUMER_WARPS);
+      mbar_init(&sm.sc_empty[s], CW);
     }
     mbar_init(&sm.drain, 1);
     sm.abort = 0;
     fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+    grid_dependency_wait();  // inputs may come from the previous kernel in the stream
+    produce(nkb < STAGES ? nkb : STAGES);  // a fresh ring: these waits return at once
   }
   if (warp == 1) {
-    tmem_alloc(&sm.tmem_base, TMEM_COLS);
+    tmem_alloc(&sm.tmem_base, Cfg::TMEM_COLS);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (threadIdx.x != 0) grid_dependency_wait();
+  grid_launch_dependents();
   const uint32_t tmem = sm.tmem_base;
 
-  float acc[BMT];
+  float acc[CPW];
 #pragma unroll
-  for (int j = 0; j < BMT; ++j) acc[j] = 0.f;
+  for (int j = 0; j < CPW; ++j) acc[j] = 0.f;
   bool consumer_ok = true;
 
   if (warp == 0) {
     if (lane == 0) {
-      tma_prefetch_desc(&tmA);
-      tma_prefetch_desc(&tmB);
-      uint32_t issued = 0, issued_phase = 0;
-      int stage = 0;
-      uint32_t phase = 0;
-      bool ok = true;
-      for (int i = 0; i < nkb; ++i) {
-        const int kb = kb_lo + i;
-        if (!wait_bounded(&sm.empty[stage], phase ^ 1u, abort, p.err, kErrTimeout | kRoleProducer | kWaitStageEmpty)) {
-          ok = false;
-          break;
-        }
-        mbar_arrive_expect_tx(&sm.full[stage], A_BYTES + B_BYTES);
-        tma_load_3d(sm.b[stage], &tmB, &sm.full[stage], kb * BK, n0, g);
-        tma_load_3d(sm.a[stage], &tmA, &sm.full[stage], kb * BK, m0, g);
-        issued |= 1u << stage;
-        issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
-        if (++stage == STAGES) {
-          stage = 0;
-          phase ^= 1u;
-        }
-      }
-      if (!ok) {
+      if (p_ok) produce(nkb);
+      if (!p_ok) {
         volatile int never = 0;
         for (int s = 0; s < STAGES; ++s)
           if ((issued >> s) & 1u) wait_bounded(&sm.full[s], (issued_phase >> s) & 1u, &never, nullptr, 0);
@@ -181,8 +299,10 @@ __global__ void __launch_bounds__(224, 1)
         for (int k = 0; k < BK / 32; ++k) mma_f8f6f4(d, ad + 2 * k, bd + 2 * k, IDESC, k > 0 ? 1u : 0u);
         mma_commit(&sm.empty[stage]);
         mma_commit(&sm.acc_full[buf]);
-        buf ^= 1;
-        if (buf == 0) bphase ^= 1u;
+        if (++buf == NBUF) {
+          buf = 0;
+          bphase ^= 1u;
+        }
         if (++stage == STAGES) {
           stage = 0;
           phase ^= 1u;
@@ -195,7 +315,7 @@ __global__ void __launch_bounds__(224, 1)
       }
     }
     __syncwarp();
-  } else if (warp == 6) {
+  } else if (warp == 2) {
     // scale producer: s[j] = scale_a[m0+j, kb] * scale_b[kb, nb] for the BMT
     // activation rows of this CTA.  The loads of SBATCH K blocks are issued
     // together, so one global-load latency is paid per batch.
@@ -236,48 +356,40 @@ __global__ void __launch_bounds__(224, 1)
         }
       }
     }
-  } else {
-    // consumers (warps 2..5)
-    const int lg = warp & 3;
-    const uint32_t t_lane = static_cast<uint32_t>(lg * 32) << 16;
+  } else if (warp >= 4) {
+    // consumers: per K block, one TMEM load of CPW columns, release the
+    // accumulator buffer, then acc[j] += s[j] * partial[j] in registers
+    const int c0 = ((warp - 4) >> 2) * CPW;  // first accumulator column of this warp
+    const uint32_t t_lane = static_cast<uint32_t>((warp & 3) * 32) << 16;
     int buf = 0, si = 0;
     uint32_t bphase = 0, sphase = 0;
     for (int i = 0; i < nkb; ++i) {
-      if (!warp_wait(&sm.sc_full[si], sphase, abort, p.err, kErrTimeout | kRoleConsumer | kWaitScaleFull) ||
-          !warp_wait(&sm.acc_full[buf], bphase, abort, p.err, kErrTimeout | kRoleConsumer | kWaitAccFull)) {
+      if (!warp_wait(&sm.acc_full[buf], bphase, abort, p.err, kErrTimeout | kRoleConsumer | kWaitAccFull) ||
+          !warp_wait(&sm.sc_full[si], sphase, abort, p.err, kErrTimeout | kRoleConsumer | kWaitScaleFull)) {
         consumer_ok = false;
         break;
       }
       tc_fence_after();
-      const uint32_t tb = tmem + t_lane + static_cast<uint32_t>(buf) * ACC_COLS;
-      const float4* s4 = reinterpret_cast<const float4*>(sm.scale[si]);
-      constexpr int CH = BMT < 32 ? BMT : 32;  // columns per TMEM load
-#pragma unroll
-      for (int c = 0; c < BMT / CH; ++c) {
-        uint32_t r[CH];
-        if constexpr (CH == 16) {
-          tmem_ld16(tb + c * CH, r);
-        } else {
-          tmem_ld32(tb + c * CH, r);
-        }
-#pragma unroll
-        for (int q = 0; q < CH / 4; ++q) {
-          const float4 s = s4[c * (CH / 4) + q];
-          const int j = c * CH + 4 * q;
-          acc[j + 0] = fmaf(s.x, __uint_as_float(r[4 * q + 0]), acc[j + 0]);
-          acc[j + 1] = fmaf(s.y, __uint_as_float(r[4 * q + 1]), acc[j + 1]);
-          acc[j + 2] = fmaf(s.z, __uint_as_float(r[4 * q + 2]), acc[j + 2]);
-          acc[j + 3] = fmaf(s.w, __uint_as_float(r[4 * q + 3]), acc[j + 3]);
-        }
-      }
+      uint32_t r[CPW];
+      tmem_ld_cols<CPW>(tmem + t_lane + static_cast<uint32_t>(buf) * ACC_COLS + static_cast<uint32_t>(c0), r);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&sm.acc_empty[buf]);
-        mbar_arrive(&sm.sc_empty[si]);
+      if (lane == 0) mbar_arrive(&sm.acc_empty[buf]);
+      const float4* s4 = reinterpret_cast<const float4*>(&sm.scale[si][c0]);
+#pragma unroll
+      for (int q = 0; q < CPW / 4; ++q) {
+        const float4 s = s4[q];
+        acc[4 * q + 0] = fmaf(s.x, __uint_as_float(r[4 * q + 0]), acc[4 * q + 0]);
+        acc[4 * q + 1] = fmaf(s.y, __uint_as_float(r[4 * q + 1]), acc[4 * q + 1]);
+        acc[4 * q + 2] = fmaf(s.z, __uint_as_float(r[4 * q + 2]), acc[4 * q + 2]);
+        acc[4 * q + 3] = fmaf(s.w, __uint_as_float(r[4 * q + 3]), acc[4 * q + 3]);
       }
-      buf ^= 1;
-      if (buf == 0) bphase ^= 1u;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.sc_empty[si]);
+      if (++buf == NBUF) {
+        buf = 0;
+        bphase ^= 1u;
+      }
       if (++si == SSTAGES) {
         si = 0;
         sphase ^= 1u;
@@ -286,21 +398,19 @@ __global__ void __launch_bounds__(224, 1)
   }
 
   // --------------------------------------------------------------- epilogue
-  const bool is_consumer = warp >= 2 && warp <= 5;
-  const int ctid = threadIdx.x - 64;            // 0..127 for consumers (work index)
-  const int wrow = (warp & 3) * 32 + lane;      // consumer's weight row = its TMEM lane
-  char* outb = static_cast<char*>(o.out);
+  const bool is_consumer = warp >= 4;
+  const int ct = static_cast<int>(threadIdx.x) - 128;  // 0..CT-1 for consumers
+  const int wrow = (warp & 3) * 32 + lane;             // consumer's weight row = its TMEM lane
+  const int c0 = ((warp - 4) >> 2) * CPW;
   if (S == 1) {
     if (is_consumer && consumer_ok) {
       const int n = n0 + wrow;
       if (n < p.N) {
+        OutT* out = static_cast<OutT*>(o.out) + static_cast<long long>(g) * o.o_sg + n;
 #pragma unroll
-        for (int j = 0; j < BMT; ++j) {
-          const int m = m0 + j;
-          if (m < p.M)
-            store_out<OutT>(reinterpret_cast<OutT*>(outb) + static_cast<long long>(m) * o.o_sm +
-                                static_cast<long long>(g) * o.o_sg + n,
-                            acc[j]);
+        for (int j = 0; j < CPW; ++j) {
+          const int m = m0 + c0 + j;
+          if (m < p.M) store_out<OutT>(out + static_cast<long long>(m) * o.o_sm, acc[j]);
         }
       }
     }
@@ -309,35 +419,22 @@ __global__ void __launch_bounds__(224, 1)
     float* red = reinterpret_cast<float*>(&sm.b[0][0]);
     if (is_consumer) {
 #pragma unroll
-      for (int j = 0; j < BMT; ++j) red[j * 128 + wrow] = consumer_ok ? acc[j] : 0.f;
+      for (int j = 0; j < CPW; ++j) red[(c0 + j) * 128 + wrow] = consumer_ok ? acc[j] : 0.f;
     }
     cluster_sync_all();
     if (is_consumer) {
-      const int R = 128 / S;  // weight rows reduced by this CTA
-      const int per = (R * BMT) / 128;
-      const uint32_t red_s = smem_u32(red);
-      for (int it = 0; it < per; ++it) {
-        const int idx = ctid + 128 * it;
-        const int r = rank * R + idx % R;
-        const int j = idx / R;
-        const uint32_t off = red_s + static_cast<uint32_t>((j * 128 + r) * 4);
-        float v = ld_shared_cluster_f32(mapa_shared(off, 0));
-        for (int q = 1; q < S; ++q) v += ld_shared_cluster_f32(mapa_shared(off, static_cast<uint32_t>(q)));
-        const int n = n0 + r, m = m0 + j;
-        if (n < p.N && m < p.M)
-          store_out<OutT>(reinterpret_cast<OutT*>(outb) + static_cast<long long>(m) * o.o_sm +
-                              static_cast<long long>(g) * o.o_sg + n,
-                          v);
-      }
+      if (S == 2) skinny_cluster_reduce<2, BMT, CT, OutT>(red, rank, ct, m0, n0, g, p, o);
+      else if (S == 4) skinny_cluster_reduce<4, BMT, CT, OutT>(red, rank, ct, m0, n0, g, p, o);
+      else skinny_cluster_reduce<8, BMT, CT, OutT>(red, rank, ct, m0, n0, g, p, o);
     }
-    cluster_sync_all();
+    cluster_sync_all();  // peers may still be reading this CTA's partial
   }
 
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, TMEM_COLS);
+    tmem_dealloc(tmem, Cfg::TMEM_COLS);
   }
 }
 

@@ -234,6 +234,8 @@ __global__ void __launch_bounds__(384, 1)
     __syncthreads();
   }
   tc_fence_after();
+  grid_dependency_wait();  // inputs may come from the previous kernel in the stream
+  grid_launch_dependents();
   const uint32_t tmem = sm.tmem_base;
 
   if (warp < 4) {

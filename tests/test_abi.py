@@ -209,3 +209,16 @@ def test_binding_rejects_cpu_tensors():
         bs.bs_gemm_fp8_blockwise(A, A.t(), torch.ones(128, 2), torch.ones(2, 1))
     with pytest.raises(bs.BsgemmError):
         bs.int_scaled_mm(A.to(torch.int8), A.to(torch.int8).t(), None)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("N", [1, 7, 8, 130, 259, 4099, 7168])
+def test_default_output_rows_start_on_16_byte_boundaries(N, dtype):
+    """The binding's own output allocation satisfies the 16-byte row-stride rule
+    of the C ABI for any N (padding lives in memory, not in the shape)."""
+    out = bs._empty_out((5,), N, dtype, "cpu")
+    assert out.shape == (5, N) and out.stride(1) == 1
+    assert (out.stride(0) * out.element_size()) % 16 == 0 and out.stride(0) - N < 16 // out.element_size()
+    out3 = bs._empty_out((3, 4), N, dtype, "cpu")
+    assert out3.shape == (3, 4, N)
+    assert all((s * out3.element_size()) % 16 == 0 for s in out3.stride()[:2])

@@ -65,6 +65,20 @@ def test_fp8_ragged_shapes_all_kernels(M, N, K, kernel, path):
     fp8_check(fp8_run(d), y, S, torch.bfloat16, f"fp8 {M}x{N}x{K} kernel={kernel}")
 
 
+@pytest.mark.parametrize("M,N,K", [(5, 259, 512), (200, 131, 256), (70, 1001, 1024), (33, 4099, 256)])
+@pytest.mark.parametrize("kernel", [bs.PATH_WIDE, bs.PATH_WIDE_SINGLE, bs.PATH_SKINNY])
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_fp8_n_not_multiple_of_four(M, N, K, kernel, out_dtype, path):
+    """Output rows padded in memory (16-byte row starts), partial 4-wide and
+    16-byte groups at the end of every row."""
+    path(kernel)
+    d = wl.fp8_blockwise_inputs(M, N, K, seed=90 + M + N + K)
+    y, S = oracle_fp8(d)
+    out = fp8_run(d, out_dtype)
+    assert out.shape == (M, N) and (out.stride(0) * out.element_size()) % 16 == 0
+    fp8_check(out, y, S, out_dtype, f"fp8 {M}x{N}x{K} kernel={kernel}")
+
+
 @pytest.mark.parametrize("M", wl.SKINNY_M_SWEEP)
 def test_fp8_skinny_sweep_n7168_k2048(M):
     w = wl.WORKLOADS[f"fp8_skinny_m{M}"]
@@ -201,6 +215,15 @@ def test_bmm_batch_first_layout(M):
     out = bmm_run(d, torch.float32)
     y, S = oracle.bmm_blockscale(d["x"], d["w"], d["x_scale"], d["w_scale"])
     fp8_check(out, y, S, torch.float32, f"bmm batch-first M={M}")
+
+
+@pytest.mark.parametrize("M,G,N", [(3, 4, 300), (100, 2, 130)])
+def test_bmm_n_not_multiple_of_four(M, G, N, path):
+    d = wl.bmm_inputs(M, G, N, 512, seed=85 + M + N)
+    y, S = oracle.bmm_blockscale(d["x"], d["w"], d["x_scale"], d["w_scale"])
+    for k in (bs.PATH_WIDE, bs.PATH_SKINNY):
+        path(k)
+        fp8_check(bmm_run(d), y, S, torch.bfloat16, f"bmm {M}x{G}x{N} kernel={k}")
 
 
 def test_bmm_both_kernels_agree_with_oracle(path):
