@@ -152,8 +152,11 @@ Plan make_plan(int op, int64_t M, int64_t G, int64_t N, int64_t K, int sms) {
     // at once (a second partial wave would double the time of an HBM-bound
     // stream), S a power of two <= 8 and <= the number of K blocks.
     const long long slots = static_cast<long long>(skinny_ctas_per_sm(bmt)) * (sms > 0 ? sms : 148);
+    // Clusters of 8 CTAs that each fill an SM do not all fit in the GPCs at
+    // once, so those kernels split at most 4 ways.
+    const int max_s = skinny_ctas_per_sm(bmt) > 1 ? 8 : 4;
     int S = 1;
-    while (S < 8 && 2 * S <= KB && units * 2 * S <= slots) S *= 2;
+    while (S < max_s && 2 * S <= KB && units * 2 * S <= slots) S *= 2;
     x.pub.kernel = 2;
     x.pub.tile_m = bmt;
     x.pub.tile_n = 128;

@@ -251,6 +251,12 @@ __global__ void __launch_bounds__(SkinnyCfg<BMT>::THREADS, SkinnyCfg<BMT>::CTAS_
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    // Warm L2 with the first ring of tiles while the previous grid drains;
+    // the copies into shared memory wait for it.
+    for (int i = 0; i < nkb && i < STAGES; ++i) {
+      tma_prefetch_l2_3d(&tmB, (kb_lo + i) * BK, n0, g);
+      tma_prefetch_l2_3d(&tmA, (kb_lo + i) * BK, m0, g);
+    }
     grid_dependency_wait();  // inputs may come from the previous kernel in the stream
     produce(nkb < STAGES ? nkb : STAGES);  // a fresh ring: these waits return at once
   }
@@ -258,10 +264,35 @@ __global__ void __launch_bounds__(SkinnyCfg<BMT>::THREADS, SkinnyCfg<BMT>::CTAS_
     tmem_alloc(&sm.tmem_base, Cfg::TMEM_COLS);
     tmem_relinquish();
   }
+  // Scale producer state: the loads of SBATCH K blocks are issued together
+  // (one global-load latency per batch); the first batch is in flight before
+  // the CTA-wide barrier.
+  constexpr int PER_LANE = (BMT + 31) / 32;
+  float sv[SBATCH][PER_LANE];  // scale_a of the batch, lane j of row j
+  float sc[SBATCH];            // scale_b of the batch
+  auto load_scales = [&](int i0) {
+    const int cnt = nkb - i0 < SBATCH ? nkb - i0 : SBATCH;
+#pragma unroll
+    for (int i = 0; i < SBATCH; ++i) {
+      if (i < cnt) {
+        const int kb = kb_lo + i0 + i;
+        sc[i] = scale_col<MODE>(p, g, kb, nb);
+#pragma unroll
+        for (int q = 0; q < PER_LANE; ++q) {
+          const int j = lane + 32 * q;
+          sv[i][q] = j < BMT ? scale_row<MODE>(p, g, m0 + j, kb) : 0.f;
+        }
+      }
+    }
+  };
+  if (warp == 2) {
+    grid_dependency_wait();
+    load_scales(0);
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (threadIdx.x != 0) grid_dependency_wait();
+  if (threadIdx.x != 0 && warp != 2) grid_dependency_wait();
   grid_launch_dependents();
   const uint32_t tmem = sm.tmem_base;
 
@@ -317,29 +348,14 @@ __global__ void __launch_bounds__(SkinnyCfg<BMT>::THREADS, SkinnyCfg<BMT>::CTAS_
     __syncwarp();
   } else if (warp == 2) {
     // scale producer: s[j] = scale_a[m0+j, kb] * scale_b[kb, nb] for the BMT
-    // activation rows of this CTA.  The loads of SBATCH K blocks are issued
-    // together, so one global-load latency is paid per batch.
-    constexpr int PER_LANE = (BMT + 31) / 32;
+    // activation rows of this CTA, SBATCH K blocks per batch
     bool ok = true;
     for (int i0 = 0; ok && i0 < nkb; i0 += SBATCH) {
-      const int nb_batch = nkb - i0 < SBATCH ? nkb - i0 : SBATCH;
-      float v[SBATCH][PER_LANE];
-      float c[SBATCH];
+      if (i0 > 0) load_scales(i0);
+      const int cnt_batch = nkb - i0 < SBATCH ? nkb - i0 : SBATCH;
 #pragma unroll
       for (int i = 0; i < SBATCH; ++i) {
-        if (i < nb_batch) {
-          const int kb = kb_lo + i0 + i;
-          c[i] = scale_col<MODE>(p, g, kb, nb);
-#pragma unroll
-          for (int q = 0; q < PER_LANE; ++q) {
-            const int j = lane + 32 * q;
-            v[i][q] = j < BMT ? scale_row<MODE>(p, g, m0 + j, kb) : 0.f;
-          }
-        }
-      }
-#pragma unroll
-      for (int i = 0; i < SBATCH; ++i) {
-        if (i < nb_batch) {
+        if (i < cnt_batch) {
           const uint32_t cnt = static_cast<uint32_t>(i0 + i);
           const int si = static_cast<int>(cnt % SSTAGES);
           const uint32_t ph = (cnt / SSTAGES) & 1u;
@@ -350,7 +366,7 @@ __global__ void __launch_bounds__(SkinnyCfg<BMT>::THREADS, SkinnyCfg<BMT>::CTAS_
 #pragma unroll
           for (int q = 0; q < PER_LANE; ++q) {
             const int j = lane + 32 * q;
-            if (j < BMT) sm.scale[si][j] = v[i][q] * c[i];
+            if (j < BMT) sm.scale[si][j] = sv[i][q] * sc[i];
           }
           mbar_arrive(&sm.sc_full[si]);
         }
@@ -403,14 +419,38 @@ __global__ void __launch_bounds__(SkinnyCfg<BMT>::THREADS, SkinnyCfg<BMT>::CTAS_
   const int wrow = (warp & 3) * 32 + lane;             // consumer's weight row = its TMEM lane
   const int c0 = ((warp - 4) >> 2) * CPW;
   if (S == 1) {
-    if (is_consumer && consumer_ok) {
-      const int n = n0 + wrow;
-      if (n < p.N) {
-        OutT* out = static_cast<OutT*>(o.out) + static_cast<long long>(g) * o.o_sg + n;
+    // Stage the tile as output rows [m][n] in the idle operand ring (every MMA
+    // has completed once the last partial was read), then write 16-byte
+    // chunks, consecutive threads covering consecutive bytes of a row.
+    if (is_consumer) {
+      OutT* stg = reinterpret_cast<OutT*>(&sm.b[0][0]);
+      if (consumer_ok) {
 #pragma unroll
         for (int j = 0; j < CPW; ++j) {
-          const int m = m0 + c0 + j;
-          if (m < p.M) store_out<OutT>(out + static_cast<long long>(m) * o.o_sm, acc[j]);
+          if constexpr (sizeof(OutT) == 2) {
+            stg[(c0 + j) * 128 + wrow] = __float2bfloat16_rn(acc[j]);
+          } else {
+            stg[(c0 + j) * 128 + wrow] = acc[j];
+          }
+        }
+      }
+      named_bar_sync(1, CT);
+      constexpr int EPC = 16 / static_cast<int>(sizeof(OutT));  // elements per 16-byte chunk
+      constexpr int CPR = 128 / EPC;                            // chunks per staged row
+      OutT* out = static_cast<OutT*>(o.out) + static_cast<long long>(g) * o.o_sg;
+      if (consumer_ok) {
+        for (int c = ct; c < BMT * CPR; c += CT) {
+          const int row = c / CPR, col = (c % CPR) * EPC;
+          const int m = m0 + row, n = n0 + col;
+          if (m < p.M && n < p.N) {
+            OutT* dst = out + static_cast<long long>(m) * o.o_sm + n;
+            const OutT* src = stg + row * 128 + col;
+            if (n + EPC <= p.N) {
+              *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
+            } else {
+              for (int e = 0; e < EPC && n + e < p.N; ++e) dst[e] = src[e];
+            }
+          }
         }
       }
     }

@@ -191,7 +191,9 @@ __device__ __forceinline__ void tma_load_3d_pair(void* dst, const CUtensorMap* m
 }
 
 // Pull a box of the tensor into L2 ahead of its load (no shared memory, no
-// completion tracking).
+// completion tracking).  L2 is the point of coherence for every later load, so
+// a prefetch may run before the previous grid has finished writing the same
+// memory: it can only warm the cache, never make a stale value visible.
 __device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* map, int c0, int c1, int c2) {
   asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
                    reinterpret_cast<uint64_t>(map)),
@@ -449,6 +451,11 @@ __device__ __forceinline__ float ld_shared_cluster_f32(uint32_t addr) {
   float v;
   asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
   return v;
+}
+// Barrier over the `count` threads (a multiple of 32) that use hardware
+// barrier `id` (1..15; 0 is __syncthreads).
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
