@@ -241,7 +241,7 @@ def oracle_rows_run(w, d, rows):
         oracle.bmm_blockscale(d["x"], d["w"], d["x_scale"], d["w_scale"], rows=rows)
 
 
-def cpu_oracle_baseline(w, d, budget_s: float = 12.0):
+def cpu_oracle_baseline(w, d, budget_s: float = 20.0):
     """Times the oracle on a bounded row sample sized to about `budget_s` seconds."""
     import oracle
     threads = oracle.num_threads()

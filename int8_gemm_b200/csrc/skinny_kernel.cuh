@@ -393,12 +393,18 @@ __global__ void __launch_bounds__(SkinnyCfg<BMT>::THREADS, SkinnyCfg<BMT>::CTAS_
       if (lane == 0) mbar_arrive(&sm.acc_empty[buf]);
       const float4* s4 = reinterpret_cast<const float4*>(&sm.scale[si][c0]);
 #pragma unroll
-      for (int q = 0; q < CPW / 4; ++q) {
+      for (int q = 0; q < CPW / 4; ++q) {  // packed two-wide FMAs
         const float4 s = s4[q];
-        acc[4 * q + 0] = fmaf(s.x, __uint_as_float(r[4 * q + 0]), acc[4 * q + 0]);
-        acc[4 * q + 1] = fmaf(s.y, __uint_as_float(r[4 * q + 1]), acc[4 * q + 1]);
-        acc[4 * q + 2] = fmaf(s.z, __uint_as_float(r[4 * q + 2]), acc[4 * q + 2]);
-        acc[4 * q + 3] = fmaf(s.w, __uint_as_float(r[4 * q + 3]), acc[4 * q + 3]);
+        const float2 lo = __ffma2_rn(make_float2(s.x, s.y),
+                                     make_float2(__uint_as_float(r[4 * q + 0]), __uint_as_float(r[4 * q + 1])),
+                                     make_float2(acc[4 * q + 0], acc[4 * q + 1]));
+        const float2 hi = __ffma2_rn(make_float2(s.z, s.w),
+                                     make_float2(__uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3])),
+                                     make_float2(acc[4 * q + 2], acc[4 * q + 3]));
+        acc[4 * q + 0] = lo.x;
+        acc[4 * q + 1] = lo.y;
+        acc[4 * q + 2] = hi.x;
+        acc[4 * q + 3] = hi.y;
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.sc_empty[si]);

@@ -154,14 +154,25 @@ __device__ __forceinline__ void stage_row64(uint8_t* stg, int lane, const float 
   }
 }
 
+// acc[j] += s * partial[j] for 32 columns, two columns per packed FMA.
+__device__ __forceinline__ void promote32(float* acc, float s, const uint32_t (&r)[32]) {
+#pragma unroll
+  for (int j = 0; j < 32; j += 2) {
+    const float2 t = __ffma2_rn(make_float2(s, s), make_float2(__uint_as_float(r[j]), __uint_as_float(r[j + 1])),
+                                make_float2(acc[j], acc[j + 1]));
+    acc[j] = t.x;
+    acc[j + 1] = t.y;
+  }
+}
+
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort, uint32_t* err,
                                           uint32_t code) {
   const bool ok = wait_bounded(bar, parity, abort, err, code);
   return __all_sync(0xffffffffu, ok);
 }
 
-constexpr int kWideProducerRegs = 56;
-constexpr int kWideConsumerRegs = 224;
+constexpr int kWideProducerRegs = 64;
+constexpr int kWideConsumerRegs = 216;
 static_assert(128 * kWideProducerRegs + 256 * kWideConsumerRegs <= 384 * 168, "register split exceeds launch budget");
 
 // CG = 1: one CTA computes a 128 x 256 tile.  CG = 2: a cluster of two CTAs
@@ -434,6 +445,10 @@ __global__ void __launch_bounds__(384, 1)
       const int ncol0 = n0 + half * 128;
       bool ok = true;
       if constexpr (!IS_INT8) {
+        // fp32 accumulators; the promotion uses the packed two-wide FMA, which
+        // halves the consumers' instruction count (the tensor pipe's issue
+        // rate suffers when the consumer warps sharing its SM sub-partition
+        // issue one FMA per column)
         float acc[128];
 #pragma unroll
         for (int j = 0; j < 128; ++j) acc[j] = 0.f;
@@ -463,10 +478,8 @@ __global__ void __launch_bounds__(384, 1)
           {
             uint32_t r0[32], r1[32];
             tmem_ld32x2(tb, tb + 32, r0, r1);
-#pragma unroll
-            for (int j = 0; j < 32; ++j) acc[j] = fmaf(s_cur, __uint_as_float(r0[j]), acc[j]);
-#pragma unroll
-            for (int j = 0; j < 32; ++j) acc[32 + j] = fmaf(s_cur, __uint_as_float(r1[j]), acc[32 + j]);
+            promote32(acc, s_cur, r0);
+            promote32(acc + 32, s_cur, r1);
           }
           {
             uint32_t r0[32], r1[32];
@@ -475,10 +488,8 @@ __global__ void __launch_bounds__(384, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(acc_empty0 + static_cast<uint32_t>(buf * sizeof(uint64_t)));
-#pragma unroll
-            for (int j = 0; j < 32; ++j) acc[64 + j] = fmaf(s_cur, __uint_as_float(r0[j]), acc[64 + j]);
-#pragma unroll
-            for (int j = 0; j < 32; ++j) acc[96 + j] = fmaf(s_cur, __uint_as_float(r1[j]), acc[96 + j]);
+            promote32(acc + 64, s_cur, r0);
+            promote32(acc + 96, s_cur, r1);
           }
           buf ^= 1;
           if (buf == 0) bphase ^= 1u;
