@@ -68,6 +68,16 @@ def _rank(rank, world, port, q):
     dist.destroy_process_group()
 
 
+def test_tensor_peak_burst_for_short_sustained_for_long_timed_regions():
+    peaks = {"bf16_tflops": 1642.1, "bf16_tflops_sustained": 1397.0, "source": "measured"}
+    p, src = bench.tensor_peak(peaks, 0.05)
+    assert p == 1642.1 * 2 and "burst" in src
+    p, src = bench.tensor_peak(peaks, 1.5)
+    assert p == 1397.0 * 2 and "sustained" in src
+    p, src = bench.tensor_peak({"bf16_tflops": 1590.0, "source": "fallback"}, 1.5)
+    assert p == 1590.0 * 2 and "burst" in src
+
+
 def test_aggregate_two_gloo_ranks_uses_slowest_rank():
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
