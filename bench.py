@@ -169,33 +169,63 @@ def build_step(w, device, copies):
     return d, sets
 
 
-def e2e_step_fn(w, d, device):
-    """One end-to-end call: pinned host inputs -> device, GEMM through the public API, result -> host."""
+def e2e_runner(w, d, device, stream):
+    """End-to-end steps through the public API: each step copies its inputs from pinned host memory to the
+    device, runs the GEMM and copies the result back to pinned host memory.  Consecutive steps are pipelined
+    over three streams with two buffer slots (inputs of step i+1 and the result of step i-1 move while step i
+    computes), as a serving loop would; every step still moves all its bytes."""
     import torch
 
     import int8_gemm_b200 as bs
 
     pin = {k: v.contiguous().pin_memory() for k, v in d.items()}
     if w.op == "fp8_blockwise":
-        host_out = torch.empty(w.M, w.N, dtype=torch.bfloat16).pin_memory()
+        out_shape, out_dtype = (w.M, w.N), torch.bfloat16
     elif w.op == "int_scaled_mm":
-        host_out = torch.empty(w.M, w.N, dtype=torch.float32).pin_memory()
+        out_shape, out_dtype = (w.M, w.N), torch.float32
     else:
-        host_out = torch.empty(w.M, w.G, w.N, dtype=torch.bfloat16).pin_memory()
+        out_shape, out_dtype = (w.M, w.G, w.N), torch.bfloat16
+    host_out = [torch.empty(out_shape, dtype=out_dtype).pin_memory() for _ in range(2)]
+    dev_in = [{k: torch.empty_like(v, device=device) for k, v in pin.items()} for _ in range(2)]
+    dev_out = [torch.empty(out_shape, dtype=out_dtype, device=device) for _ in range(2)]
     h2d = sum(v.numel() * v.element_size() for v in pin.values())
-    d2h = host_out.numel() * host_out.element_size()
+    d2h = host_out[0].numel() * host_out[0].element_size()
+    s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    ev = {name: [torch.cuda.Event() for _ in range(2)] for name in ("in_done", "comp_done", "out_done")}
+    used = [False, False]
 
-    def step():
-        dev = {k: v.to(device, non_blocking=True) for k, v in pin.items()}
+    def compute(x, out):
         if w.op == "fp8_blockwise":
-            out = bs.bs_gemm_fp8_blockwise(dev["A"], dev["B_t"].t(), dev["scale_a"], dev["scale_b"])
+            bs.bs_gemm_fp8_blockwise(x["A"], x["B_t"].t(), x["scale_a"], x["scale_b"], out=out)
         elif w.op == "int_scaled_mm":
-            out = bs.int_scaled_mm(dev["A"], dev["B_t"].t(), dev["s_a"], dev["s_b"])
+            bs.int_scaled_mm(x["A"], x["B_t"].t(), x["s_a"], x["s_b"], out_dtype=torch.float32, out=out)
         else:
-            out = bs.bmm_a8w8_blockscale(dev["x"], dev["w"], dev["x_scale"], dev["w_scale"])
-        host_out.copy_(out, non_blocking=True)
+            bs.bmm_a8w8_blockscale(x["x"], x["w"], x["x_scale"], x["w_scale"], out=out)
 
-    return step, h2d, d2h
+    def run(steps):
+        for i in range(steps):
+            k = i % 2
+            with torch.cuda.stream(s_in):
+                if used[k]:
+                    s_in.wait_event(ev["comp_done"][k])  # the step two back has consumed this input slot
+                for name, v in pin.items():
+                    dev_in[k][name].copy_(v, non_blocking=True)
+                ev["in_done"][k].record(s_in)
+            with torch.cuda.stream(stream):
+                stream.wait_event(ev["in_done"][k])
+                if used[k]:
+                    stream.wait_event(ev["out_done"][k])  # its result slot has been read back
+                compute(dev_in[k], dev_out[k])
+                ev["comp_done"][k].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev["comp_done"][k])
+                host_out[k].copy_(dev_out[k], non_blocking=True)
+                ev["out_done"][k].record(s_out)
+            used[k] = True
+        return s_out
+
+    run.first_stream = s_in
+    return run, h2d, d2h
 
 
 class ClockSampler:
@@ -280,7 +310,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--shape", default=None,
                     help="ad-hoc problem 'M,N,K' (or 'M,G,N,K' for --op bmm) instead of a named workload")
@@ -384,16 +414,14 @@ def main():
     # end to end through the public API with pinned host buffers
     e2e = None
     if args.e2e_steps > 0:
-        e2e_fn, h2d, d2h = e2e_step_fn(w, d, device)
-        for _ in range(2):
-            e2e_fn()
+        e2e_run, h2d, d2h = e2e_runner(w, d, device, stream)
+        e2e_run(2)
         torch.cuda.synchronize()
         barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(args.e2e_steps):
-            e2e_fn()
-        e1.record(stream)
+        e0.record(e2e_run.first_stream)  # every stream is idle here; the first step starts on this one
+        last = e2e_run(args.e2e_steps)
+        e1.record(last)
         torch.cuda.synchronize()
         e2e_ms = reduce_max(e0.elapsed_time(e1) / args.e2e_steps)
         e2e = {"value": round(flops * world / (e2e_ms / 1e3) / 1e12, 3), "unit": "TFLOP/s",
