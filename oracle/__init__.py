@@ -61,7 +61,8 @@ def _load():
             lib.orc_bmm_blockscale.argtypes = [p, i64, i64, p, i64, i64, p, p,
                                                i64, i64, i64, i64, p, i64, p, p]
             lib.orc_int_scaled_mm.argtypes = [p, i64, p, i64, p, p, i64, i64, i64, p, i64, p, p, p]
-            for f in (lib.orc_fp8_blockwise, lib.orc_bmm_blockscale, lib.orc_int_scaled_mm):
+            lib.orc_fp8_rowwise.argtypes = [p, i64, p, i64, p, i64, p, i64, p, i64, i64, i64, p, i64, p, p]
+            for f in (lib.orc_fp8_blockwise, lib.orc_bmm_blockscale, lib.orc_int_scaled_mm, lib.orc_fp8_rowwise):
                 f.restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -195,3 +196,30 @@ def int_scaled_mm(A, B_t, s_a, s_b, rows=None):
     if rc != 0:
         raise ValueError(f"oracle int_scaled_mm failed with code {rc} (2 = int32 overflow)")
     return acc, y, bf
+
+
+def fp8_rowwise(A, B_t, scale_a, scale_b, bias=None, rows=None):
+    """FP8 GEMM with tensorwise or rowwise scales.  A uint8 [M,K] e4m3 codes, B_t uint8 [N,K] codes of
+    B[K,N]; scale_a fp32 scalar (tensorwise) or [M] / [M,1] (rowwise); scale_b fp32 scalar or [N] / [1,N]
+    (the same kind as scale_a); bias fp32 [N] or None.
+
+    Returns (y, S): fp64 [R, N] results and |a*b| magnitude sums times |scale_a*scale_b|."""
+    A, B_t = _row_major_u8(A), _row_major_u8(B_t)
+    M, K = A.shape
+    N = B_t.shape[0]
+    assert B_t.shape[1] == K
+    sa = np.ascontiguousarray(_np(scale_a), dtype=np.float32).reshape(-1)
+    sb = np.ascontiguousarray(_np(scale_b), dtype=np.float32).reshape(-1)
+    assert (sa.size, sb.size) in ((1, 1), (M, N))
+    rowwise = (sa.size, sb.size) == (M, N) and (M, N) != (1, 1)
+    bias_a = None if bias is None else np.ascontiguousarray(_np(bias), dtype=np.float32).reshape(-1)
+    assert bias_a is None or bias_a.size == N
+    r, R = _rows(rows, M)
+    y = np.empty((R, N), dtype=np.float64)
+    S = np.empty((R, N), dtype=np.float64)
+    st = 1 if rowwise else 0
+    rc = _load().orc_fp8_rowwise(_ptr(A), _estride(A, 0), _ptr(B_t), _estride(B_t, 0), _ptr(sa), st, _ptr(sb), st,
+                                 _ptr(bias_a), M, N, K, _ptr(r), R, _ptr(y), _ptr(S))
+    if rc != 0:
+        raise ValueError(f"oracle fp8_rowwise failed with code {rc}")
+    return y, S

@@ -31,6 +31,9 @@
  *       for cpu" (int_scaled_matmul_cpu: _int_mm then .to(scales.dtype) *
  *       scales); pytorch/ao issue "Unify scaled INT8 matmul" (key-differences
  *       table: acc_i32.to(f32) x scale.to(f32), both scales fused).
+ *   - FP8 with tensorwise or rowwise scales (and an optional bias): the exact
+ *     fp64 dot product over all of K times scale_a * scale_b, plus bias[n]
+ *     (see orc_fp8_rowwise for the sources).
  *   - Batched block-scaled GEMM: a loop over g of the FP8 definition with
  *     scale = 2^(byte - 127) decoded exactly from the e8m0 bytes (byte 255 is
  *     NaN).
@@ -218,6 +221,51 @@ int orc_fp8_blockwise(const uint8_t *A, int64_t lda, const uint8_t *B, int64_t l
     free(sa);
     free(sb);
     return rc;
+}
+
+/* FP8 e4m3 A[M,K] x B[K,N] with tensorwise or rowwise fp32 scales and an
+ * optional fp32 bias[N]:
+ *   y[m,n] = (sum_k a[m,k] * b[k,n]) * (scale_a[m * sa_stride] * scale_b[n * sb_stride]) + bias[n]
+ * sa_stride / sb_stride are 0 (one scale for the operand) or 1 (one per row of A
+ * / column of B).  The dot product is exact in fp64 for K < 2^20 (every
+ * product has <= 8 significant bits in [2^-18, 2^17.6]); the scale product is
+ * exact in fp64; the scaling and bias add round once each in fp64.
+ * S[m,n] = |scale_a * scale_b| * sum_k |a * b| for the acceptance bound.
+ *   Sources: pytorch/torch/_inductor/kernel/mm.py, apply_scaling (tensorwise:
+ *   accumulator * (a_scale * b_scale); rowwise: the per-row scale_a times the
+ *   per-column scale_b) and tuned_scaled_mm (bias [N] broadcast over rows);
+ *   the pytorch issue "torch._scaled_mm with blockwise scaling doesn't work
+ *   with torch.compile" (RuntimeError: tensorwise scales are scalars, rowwise
+ *   scale_a is (M, 1) and scale_b is (1, N)). */
+int orc_fp8_rowwise(const uint8_t *A, int64_t lda, const uint8_t *B, int64_t ldb,
+                    const float *scale_a, int64_t sa_stride, const float *scale_b, int64_t sb_stride,
+                    const float *bias, int64_t M, int64_t N, int64_t K,
+                    const int64_t *rows, int64_t nrows, double *y, double *S)
+{
+    if (M < 0 || N < 0 || K < 0 || K >= (1 << 20)) return ORC_ERR_SHAPE;
+    if ((sa_stride != 0 && sa_stride != 1) || (sb_stride != 0 && sb_stride != 1)) return ORC_ERR_SHAPE;
+    build_e4m3_table();
+    if (!rows) nrows = M;
+    for (int64_t i = 0; rows && i < nrows; ++i)
+        if (rows[i] < 0 || rows[i] >= M) return ORC_ERR_SHAPE;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t i = 0; i < nrows; ++i) {
+        const int64_t m = rows ? rows[i] : i;
+        const uint8_t *arow = A + m * lda;
+        for (int64_t n = 0; n < N; ++n) {
+            const uint8_t *bcol = B + n * ldb;
+            double p = 0.0, pabs = 0.0;
+            for (int64_t k = 0; k < K; ++k) {
+                const double t = e4m3_value[arow[k]] * e4m3_value[bcol[k]];
+                p += t;
+                pabs += fabs(t);
+            }
+            const double s = (double)scale_a[m * sa_stride] * (double)scale_b[n * sb_stride];
+            y[i * N + n] = p * s + (bias ? (double)bias[n] : 0.0);
+            S[i * N + n] = fabs(s) * pabs;
+        }
+    }
+    return ORC_OK;
 }
 
 static double e8m0_value(uint8_t byte)

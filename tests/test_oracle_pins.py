@@ -224,6 +224,88 @@ def test_fp8_scale_shapes_from_the_blockwise_issue():
 
 
 # ---------------------------------------------------------------------------
+# FP8 with tensorwise / rowwise scales and bias
+# ---------------------------------------------------------------------------
+def _rowwise_inputs(M, N, K, seed):
+    g = torch.Generator().manual_seed(seed)
+    A = wl.to_e4m3_bytes(torch.randn(M, K, generator=g) * 4)
+    B = wl.to_e4m3_bytes(torch.randn(N, K, generator=g) * 4)
+    sa = (torch.rand(M, generator=g) + 0.5).numpy().astype(np.float32)
+    sb = (torch.rand(N, generator=g) + 0.5).numpy().astype(np.float32)
+    bias = torch.randn(N, generator=g).numpy().astype(np.float32)
+    return A, B, sa, sb, bias
+
+
+@pytest.mark.parametrize("M,N,K", [(3, 5, 48), (2, 129, 128), (4, 7, 300)])
+def test_fp8_rowwise_brute_force_exact_rational(M, N, K):
+    """Exact rational reference (Fraction) of acc * (s_a * s_b) + bias, K not necessarily a multiple of 128."""
+    A, B, sa, sb, bias = _rowwise_inputs(M, N, K, seed=70 + K)
+    y, S = oracle.fp8_rowwise(A, B, sa, sb, bias)
+    ai, bi = _int_codes(A.numpy()), _int_codes(B.numpy())
+    P = ai @ bi.T  # exact integers, scaled by 2^18
+    for m in range(M):
+        for n in range(N):
+            exact = Fraction(int(P[m, n]), 1 << 18) * Fraction(float(sa[m])) * Fraction(float(sb[n])) \
+                + Fraction(float(bias[n]))
+            bound = (abs(exact) + 1) * Fraction(1, 2 ** 51)   # two fp64 roundings (scale, bias add)
+            assert abs(Fraction(float(y[m, n])) - exact) <= bound
+            assert S[m, n] == pytest.approx(float(abs(Fraction(int(np.abs(ai[m] * bi[n]).sum()), 1 << 18))
+                                                  * Fraction(float(sa[m])) * Fraction(float(sb[n]))), rel=1e-15)
+
+
+def test_fp8_rowwise_equals_blockwise_with_broadcast_scales():
+    """A per-row scale_a and a scale_b constant inside each 128-column block is the block-scaled
+    definition with scale_a[m, kb] = s_a[m] and scale_b[kb, nb] = s_b[nb]."""
+    d = wl.fp8_blockwise_inputs(16, 384, 512, seed=71)
+    sa_row = d["scale_a"][:, 0].numpy().copy()
+    sb_blk = d["scale_b"][0, :].numpy().copy()
+    sb_col = np.repeat(sb_blk, 128)[:384]
+    yr, Sr = oracle.fp8_rowwise(d["A"], d["B_t"], sa_row, sb_col)
+    yb, Sb = oracle.fp8_blockwise(d["A"], d["B_t"], np.repeat(sa_row[:, None], 4, 1),
+                                  np.repeat(sb_blk[None, :], 4, 0))
+    assert np.all(np.abs(yr - yb) <= 1e-12 * Sb)
+    np.testing.assert_allclose(Sr, Sb, rtol=1e-12)
+
+
+def test_fp8_tensorwise_is_rowwise_with_constant_vectors():
+    A, B, _, _, bias = _rowwise_inputs(6, 40, 256, seed=72)
+    yt, St = oracle.fp8_rowwise(A, B, np.float32(0.75), np.float32(1.5), bias)
+    yr, Sr = oracle.fp8_rowwise(A, B, np.full(6, 0.75, np.float32), np.full(40, 1.5, np.float32), bias)
+    np.testing.assert_array_equal(yt, yr)
+    np.testing.assert_array_equal(St, Sr)
+
+
+def test_fp8_rowwise_small_integers_unit_scales_and_bias_per_column():
+    rng = np.random.default_rng(13)
+    M, N, K = 4, 24, 200
+    t = oracle.e4m3_table()
+    code_of = {float(v): c for c, v in reversed(list(enumerate(t))) if not np.isnan(v)}
+    ints_a, ints_b = rng.integers(-4, 5, (M, K)), rng.integers(-4, 5, (N, K))
+    enc = np.vectorize(lambda v: code_of[float(v)] if v != 0 else 0)
+    A, B = enc(ints_a).astype(np.uint8), enc(ints_b).astype(np.uint8)
+    bias = np.arange(N, dtype=np.float32) - 10.0
+    y, _ = oracle.fp8_rowwise(A, B, np.ones(M, np.float32), np.ones(N, np.float32), bias)
+    np.testing.assert_array_equal(y, (ints_a @ ints_b.T).astype(np.float64) + bias[None, :])
+    y0, _ = oracle.fp8_rowwise(A, B, np.ones(M, np.float32), np.ones(N, np.float32))
+    np.testing.assert_array_equal(y - y0, np.broadcast_to(bias.astype(np.float64), (M, N)))
+
+
+def test_fp8_rowwise_scale_shapes_from_the_blockwise_issue():
+    """The same compile-error message states the tensorwise (scalar) and rowwise ((16640, 1) and (1, 5120))
+    scale shapes (tests/golden/scale_shapes_blockwise.json); the oracle accepts exactly those kinds."""
+    g = json.load(open(os.path.join(GOLDEN, "scale_shapes_blockwise.json")))
+    M, N = 2, g["N"]
+    A = np.full((M, 256), 0x38, np.uint8)
+    B = np.full((N, 256), 0x38, np.uint8)
+    y, _ = oracle.fp8_rowwise(A, B, np.ones((M, 1), np.float32), np.ones(g["rowwise_scale_b"], np.float32))
+    assert tuple(g["rowwise_scale_a"])[1] == 1 and np.all(y == 256)
+    y, _ = oracle.fp8_rowwise(A, B, np.float32(2.0), np.float32(0.5))
+    assert np.all(y == 256)
+    with pytest.raises(AssertionError):  # blockwise-shaped scales are neither kind
+        oracle.fp8_rowwise(A, B, np.ones((M, 2), np.float32), np.ones((2, 40), np.float32))
+
+
+# ---------------------------------------------------------------------------
 # operation 2: INT8 with fused (float(acc) * s_a) * s_b
 # ---------------------------------------------------------------------------
 @pytest.mark.parametrize("M,N,K", [(17, 33, 64), (64, 128, 4096), (33, 24, 48)])
