@@ -133,6 +133,10 @@ def describe(w):
         flops = 2.0 * w.M * w.N * w.K
         byts = w.M * w.K + w.N * w.K + 4 * w.M * w.N + 4 * (w.M + w.N)
         dtype = "s8 (s32 accumulate)"
+    elif w.op == "fp8_rowwise":
+        flops = 2.0 * w.M * w.N * w.K
+        byts = w.M * w.K + w.N * w.K + 2 * w.M * w.N + 4 * (w.M + 2 * w.N)  # scales and bias
+        dtype = "e4m3 (fp32 accumulate)"
     else:
         flops = 2.0 * w.M * w.G * w.N * w.K
         kb, nb = w.K // 128, -(-w.N // 128)
@@ -161,6 +165,12 @@ def build_step(w, device, copies):
             sa, sb = d["s_a"].to(device), d["s_b"].to(device)
             out = torch.empty(w.M, w.N, dtype=torch.float32, device=device)
             sets.append(lambda A=A, B=B, sa=sa, sb=sb, out=out: bs.int_scaled_mm(A, B, sa, sb, out=out))
+        elif w.op == "fp8_rowwise":
+            A, B = d["A"].to(device), d["B_t"].to(device).t()
+            sa, sb, bias = d["scale_a"].to(device), d["scale_b"].to(device), d["bias"].to(device)
+            out = torch.empty(w.M, w.N, dtype=torch.bfloat16, device=device)
+            sets.append(lambda A=A, B=B, sa=sa, sb=sb, bias=bias, out=out:
+                        bs.bs_gemm_fp8_rowwise(A, B, sa, sb, bias, out=out))
         else:
             x, wt = d["x"].to(device), d["w"].to(device)
             xs, ws = d["x_scale"].to(device), d["w_scale"].to(device)
@@ -178,8 +188,8 @@ def e2e_runner(w, d, device, stream):
 
     import int8_gemm_b200 as bs
 
-    pin = {k: v.contiguous().pin_memory() for k, v in d.items()}
-    if w.op == "fp8_blockwise":
+    pin = {k: v.contiguous().pin_memory() for k, v in d.items() if v is not None}
+    if w.op in ("fp8_blockwise", "fp8_rowwise"):
         out_shape, out_dtype = (w.M, w.N), torch.bfloat16
     elif w.op == "int_scaled_mm":
         out_shape, out_dtype = (w.M, w.N), torch.float32
@@ -199,6 +209,8 @@ def e2e_runner(w, d, device, stream):
             bs.bs_gemm_fp8_blockwise(x["A"], x["B_t"].t(), x["scale_a"], x["scale_b"], out=out)
         elif w.op == "int_scaled_mm":
             bs.int_scaled_mm(x["A"], x["B_t"].t(), x["s_a"], x["s_b"], out_dtype=torch.float32, out=out)
+        elif w.op == "fp8_rowwise":
+            bs.bs_gemm_fp8_rowwise(x["A"], x["B_t"].t(), x["scale_a"], x["scale_b"], x.get("bias"), out=out)
         else:
             bs.bmm_a8w8_blockscale(x["x"], x["w"], x["x_scale"], x["w_scale"], out=out)
 
@@ -279,6 +291,8 @@ def oracle_rows_run(w, d, rows):
         oracle.fp8_blockwise(d["A"], d["B_t"], d["scale_a"], d["scale_b"], rows=rows)
     elif w.op == "int_scaled_mm":
         oracle.int_scaled_mm(d["A"], d["B_t"], d["s_a"], d["s_b"], rows=rows)
+    elif w.op == "fp8_rowwise":
+        oracle.fp8_rowwise(d["A"], d["B_t"], d["scale_a"], d["scale_b"], d["bias"], rows=rows)
     else:
         oracle.bmm_blockscale(d["x"], d["w"], d["x_scale"], d["w_scale"], rows=rows)
 
@@ -367,7 +381,7 @@ def main():
     bs.set_path_override({"auto": 0, "wide": 1, "skinny": 2, "wide1": 3}[args.path])
     copies = max(1, math.ceil(3 * L2_BYTES / byts)) if byts < 3 * L2_BYTES else 1
     d, sets = build_step(w, device, copies)
-    op = {"fp8_blockwise": 1, "int_scaled_mm": 2, "bmm_a8w8_blockscale": 3}[w.op]
+    op = {"fp8_blockwise": 1, "int_scaled_mm": 2, "bmm_a8w8_blockscale": 3, "fp8_rowwise": 4}[w.op]
     plan = bs.plan_for(op, w.M, w.G, w.N, w.K, torch.cuda.get_device_properties(device).multi_processor_count)
 
     for i in range(max(3, args.warmup)):
@@ -428,7 +442,7 @@ def main():
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     peaks = load_peaks()
-    if w.op in ("fp8_blockwise", "bmm_a8w8_blockscale") and flops / byts > 690 or w.op == "int_scaled_mm":
+    if w.op in ("fp8_blockwise", "bmm_a8w8_blockscale", "fp8_rowwise") and flops / byts > 690 or w.op == "int_scaled_mm":
         bound, unit = "tensor", "TFLOP/s"
         peak, peak_source = tensor_peak(peaks, step_ms * K / 1e3)
         achieved = flops / (per_launch_ms / 1e3) / 1e12

@@ -83,6 +83,37 @@ bs_status bs_gemm_fp8_blockwise(const void* A, int64_t lda, const void* B, int64
                                 int64_t M, int64_t N, int64_t K, void* stream);
 
 /*
+ * FP8 GEMM with tensorwise or rowwise scales and an optional bias (the other
+ * scaling modes of torch._scaled_mm).
+ *
+ *   out[m, n] = (sum_k A[m, k] * B[k, n]) * (scale_a[m * sa_stride] * scale_b[n * sb_stride])
+ *               + bias[n]
+ *
+ * Source: pytorch/torch/_inductor/kernel/mm.py -- apply_scaling (tensorwise:
+ * accumulator * (a_scale * b_scale); rowwise: a per-row scale_a times a
+ * per-column scale_b) and tuned_scaled_mm (optional bias [N] added to every
+ * row); the pytorch issue "torch._scaled_mm with blockwise scaling doesn't
+ * work with torch.compile" states the shapes: tensorwise scales are scalars,
+ * rowwise scale_a is (M, 1) and scale_b is (1, N).  The scales are constant
+ * along K, so the fp32 accumulator covers all of K before the scaling.
+ *
+ *   A        e4m3 [M, K], row m at A + m*lda                (lda >= K)
+ *   B        e4m3 [K, N] column-major, column n at B + n*ldb (ldb >= K)
+ *   scale_a  fp32; sa_stride = 0: one scale (tensorwise), 1: [M] (rowwise)
+ *   scale_b  fp32; sb_stride = 0: one scale (tensorwise), 1: [N] (rowwise)
+ *            (both strides equal: the two operands use the same mode)
+ *   bias     fp32 [N] or NULL
+ *   out      [M, N] row-major, row stride ldo (>= N), BS_OUT_BF16 or BS_OUT_F32
+ *   K is free (lda and ldb multiples of 16); K == 0 writes bias (or zeros).
+ * Not a block-scaled operation: it has no counterpart in the block-scaled
+ * statement of the problem above and follows the mm.py scaling modes.
+ */
+bs_status bs_gemm_fp8_rowwise(const void* A, int64_t lda, const void* B, int64_t ldb,
+                              const float* scale_a, int64_t sa_stride, const float* scale_b, int64_t sb_stride,
+                              const float* bias, void* out, int64_t ldo, bs_out_dtype out_dtype,
+                              int64_t M, int64_t N, int64_t K, void* stream);
+
+/*
  * Operation 2 -- INT8 GEMM with a fused, fixed-order fp32 dequantisation.
  *
  *   acc[m, n] = sum_k A[m, k] * B[k, n]              (exact, int32)
@@ -165,7 +196,8 @@ typedef struct {
 } bs_plan;
 
 /* Plan of operation `op` (1 = bs_gemm_fp8_blockwise, 2 = int_scaled_mm,
- * 3 = bmm_a8w8_blockscale; G = 1 for ops 1 and 2) on a GPU with `num_sms`
+ * 3 = bmm_a8w8_blockscale, 4 = bs_gemm_fp8_rowwise; G = 1 for ops 1, 2 and 4)
+ * on a GPU with `num_sms`
  * streaming multiprocessors.  Pure host logic; honours bs_set_path_override. */
 bs_status bs_plan_for(int32_t op, int64_t M, int64_t G, int64_t N, int64_t K, int32_t num_sms, bs_plan* plan);
 

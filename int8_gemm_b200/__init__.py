@@ -62,9 +62,11 @@ def lib() -> ctypes.CDLL:
             h.bs_gemm_fp8_blockwise.argtypes = [p, i64, p, i64, p, i64, i64, p, i64, i64, p, i64, ctypes.c_int,
                                                 i64, i64, i64, p]
             h.int_scaled_mm.argtypes = [p, i64, p, i64, p, p, p, i64, ctypes.c_int, i64, i64, i64, p]
+            h.bs_gemm_fp8_rowwise.argtypes = [p, i64, p, i64, p, i64, p, i64, p, p, i64, ctypes.c_int,
+                                              i64, i64, i64, p]
             h.bmm_a8w8_blockscale.argtypes = [p, i64, i64, p, i64, i64, p, p, p, i64, i64, ctypes.c_int,
                                               i64, i64, i64, i64, p]
-            for f in (h.bs_gemm_fp8_blockwise, h.int_scaled_mm, h.bmm_a8w8_blockscale):
+            for f in (h.bs_gemm_fp8_blockwise, h.int_scaled_mm, h.bmm_a8w8_blockscale, h.bs_gemm_fp8_rowwise):
                 f.restype = ctypes.c_int
             h.bs_status_string.argtypes = [ctypes.c_int]
             h.bs_status_string.restype = ctypes.c_char_p
@@ -163,6 +165,55 @@ def bs_gemm_fp8_blockwise(A: torch.Tensor, B: torch.Tensor, scale_a: torch.Tenso
     return out
 
 
+def bs_gemm_fp8_rowwise(A: torch.Tensor, B: torch.Tensor, scale_a: torch.Tensor, scale_b: torch.Tensor,
+                        bias: torch.Tensor | None = None, out_dtype: torch.dtype = torch.bfloat16,
+                        out: torch.Tensor | None = None) -> torch.Tensor:
+    """FP8 GEMM with tensorwise or rowwise scales: out = (A @ B) * (scale_a * scale_b) + bias.
+
+    A       e4m3 [M, K] row-major;  B e4m3 [K, N] column-major (``B_t.t()`` for B_t [N, K])
+    scale_a fp32 scalar (tensorwise) or [M] / [M, 1] (rowwise)
+    scale_b fp32 scalar (tensorwise) or [N] / [1, N] (rowwise), the same kind as scale_a
+    bias    fp32 [N] or None
+    """
+    for t, n in ((A, "A"), (B, "B"), (scale_a, "scale_a"), (scale_b, "scale_b")):
+        _cuda(t, n)
+    _bytes8(A, "A"), _bytes8(B, "B")
+    if A.dim() != 2 or B.dim() != 2 or A.shape[1] != B.shape[0]:
+        raise BsgemmError(BS_ERR_SHAPE, f"A [M,K] and B [K,N] expected, got {tuple(A.shape)} and {tuple(B.shape)}")
+    M, K = A.shape
+    N = B.shape[1]
+    if scale_a.dtype != torch.float32 or scale_b.dtype != torch.float32:
+        raise BsgemmError(BS_ERR_DTYPE, "scale_a and scale_b must be float32")
+    tensorwise = scale_a.numel() == 1 and scale_b.numel() == 1 and scale_a.dim() in (0, 1) and scale_b.dim() in (0, 1)
+    rowwise = tuple(scale_a.shape) in ((M,), (M, 1)) and tuple(scale_b.shape) in ((N,), (1, N))
+    if not (tensorwise or rowwise):
+        raise BsgemmError(BS_ERR_SHAPE, "tensorwise scales are scalars; rowwise scale_a is (M, 1) and scale_b (1, N); "
+                                        f"got {tuple(scale_a.shape)} and {tuple(scale_b.shape)}")
+    stride = 0 if tensorwise and not rowwise else 1
+    if stride == 1:
+        scale_a, scale_b = scale_a.reshape(-1).contiguous(), scale_b.reshape(-1).contiguous()
+    if bias is not None:
+        _cuda(bias, "bias")
+        if bias.dtype != torch.float32 or bias.numel() != N:
+            raise BsgemmError(BS_ERR_SHAPE, "bias must be float32 [N]")
+        bias = bias.reshape(-1).contiguous()
+    if A.stride(1) != 1 and M > 1:
+        raise BsgemmError(BS_ERR_LAYOUT, f"A must be row-major, got strides {A.stride()}")
+    if B.stride(0) != 1 and N > 1:
+        raise BsgemmError(BS_ERR_LAYOUT, f"B must be column-major, got strides {B.stride()}")
+    if out_dtype not in (torch.bfloat16, torch.float32):
+        raise BsgemmError(BS_ERR_DTYPE, f"out_dtype must be bfloat16 or float32, got {out_dtype}")
+    if out is None:
+        out = _empty_out((M,), N, out_dtype, A.device)
+    elif out.dtype != out_dtype or tuple(out.shape) != (M, N) or out.stride(1) != 1:
+        raise BsgemmError(BS_ERR_LAYOUT, "out must be a row-major [M, N] tensor of out_dtype")
+    with torch.cuda.device(A.device):
+        _check(lib().bs_gemm_fp8_rowwise(
+            _ptr(A), A.stride(0), _ptr(B), B.stride(1), _ptr(scale_a), stride, _ptr(scale_b), stride, _ptr(bias),
+            _ptr(out), out.stride(0), _OUT_CODE[out_dtype], M, N, K, _stream(A.device)))
+    return out
+
+
 def int_scaled_mm(A: torch.Tensor, B: torch.Tensor, s_a: torch.Tensor | None, s_b: torch.Tensor | None = None,
                   out_dtype: torch.dtype = torch.float32, out: torch.Tensor | None = None) -> torch.Tensor:
     """INT8 GEMM with fused (float(acc) * s_a[m]) * s_b[n].
@@ -252,7 +303,7 @@ def bmm_a8w8_blockscale(x: torch.Tensor, w: torch.Tensor, x_scale: torch.Tensor,
 # ---------------------------------------------------------------------------
 # host-side helpers
 # ---------------------------------------------------------------------------
-OP_FP8_BLOCKWISE, OP_INT_SCALED_MM, OP_BMM = 1, 2, 3
+OP_FP8_BLOCKWISE, OP_INT_SCALED_MM, OP_BMM, OP_FP8_ROWWISE = 1, 2, 3, 4
 
 
 def plan_for(op: int, M: int, G: int, N: int, K: int, num_sms: int = 148) -> dict:

@@ -140,7 +140,7 @@ Plan make_plan(int op, int64_t M, int64_t G, int64_t N, int64_t K, int sms) {
   }
   const int KB = static_cast<int>((K + 127) / 128);
   const int ov = g_path_override.load();
-  const bool skinny_ok = op != 2;
+  const bool skinny_ok = op == 1 || op == 3;  // block-scaled FP8 only
   const bool skinny = skinny_ok && (ov == 2 || (ov == 0 && M <= kSkinnyMaxM));
   if (skinny) {
     const int bmt = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128;
@@ -333,7 +333,7 @@ int32_t bs_set_path_override(int32_t path) { return g_path_override.exchange(pat
 bs_status bs_plan_for(int32_t op, int64_t M, int64_t G, int64_t N, int64_t K, int32_t num_sms, bs_plan* plan) {
   clear_msg();
   if (!plan) return fail(BS_ERR_NULL, "plan is NULL");
-  if (op < 1 || op > 3) return fail(BS_ERR_SHAPE, "op must be 1, 2 or 3");
+  if (op < 1 || op > 4) return fail(BS_ERR_SHAPE, "op must be 1, 2, 3 or 4");
   if (M < 0 || N < 0 || K < 0 || G < 0 || num_sms <= 0) return fail(BS_ERR_SHAPE, "negative size");
   *plan = make_plan(op, M, G, N, K, num_sms).pub;
   return BS_OK;
@@ -459,6 +459,72 @@ bs_status bmm_a8w8_blockscale(const void* x, int64_t x_sm, int64_t x_sg, const v
   return run_fp8(q, args, static_cast<cudaStream_t>(stream), dc);
 }
 
+bs_status bs_gemm_fp8_rowwise(const void* A, int64_t lda, const void* B, int64_t ldb, const float* scale_a,
+                              int64_t sa_stride, const float* scale_b, int64_t sb_stride, const float* bias, void* out,
+                              int64_t ldo, bs_out_dtype out_dtype, int64_t M, int64_t N, int64_t K, void* stream) {
+  clear_msg();
+  if (M < 0 || N < 0 || K < 0) return fail(BS_ERR_SHAPE, "negative size");
+  if (M > kMaxDim || N > kMaxDim || K > kMaxDim) return fail(BS_ERR_SHAPE, "size exceeds 2^31-1");
+  if (sa_stride != sb_stride || (sa_stride != 0 && sa_stride != 1))
+    return fail(BS_ERR_SHAPE,
+                "scales must be both tensorwise (strides 0: scalars) or both rowwise (strides 1: scale_a (M, 1), "
+                "scale_b (1, N)); got strides %lld and %lld",
+                (long long)sa_stride, (long long)sb_stride);
+  if (out_dtype != BS_OUT_BF16 && out_dtype != BS_OUT_F32)
+    return fail(BS_ERR_DTYPE, "bs_gemm_fp8_rowwise writes bf16 or f32 only");
+  if (M == 0 || N == 0) return BS_OK;
+  if (!out) return fail(BS_ERR_NULL, "out is NULL");
+  if (ldo < N) return fail(BS_ERR_LAYOUT, "ldo < N");
+  if (!aligned16(out) || (ldo * out_size(out_dtype)) % 16 != 0)
+    return fail(BS_ERR_ALIGNMENT, "out must be 16-byte aligned with a row stride that is a multiple of 16 bytes");
+  if (bias && !aligned4(bias)) return fail(BS_ERR_ALIGNMENT, "bias must be 4-byte aligned");
+  if (K > 0) {
+    if (!A || !B || !scale_a || !scale_b) return fail(BS_ERR_NULL, "A, B, scale_a and scale_b must be non-NULL");
+    if (lda < K || ldb < K) return fail(BS_ERR_LAYOUT, "lda/ldb must be >= K (A row-major, B column-major)");
+    if (!aligned16(A) || !aligned16(B) || lda % 16 != 0 || ldb % 16 != 0)
+      return fail(BS_ERR_ALIGNMENT, "A and B must be 16-byte aligned with lda, ldb multiples of 16");
+    if (!aligned4(scale_a) || !aligned4(scale_b)) return fail(BS_ERR_ALIGNMENT, "scales must be 4-byte aligned");
+  }
+  DeviceCtx* dc = nullptr;
+  bs_status st = device_ctx(&dc);
+  if (st != BS_OK) return st;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  const Plan pl = make_plan(4, M, 1, N, K, dc->sms);
+  if (pl.pub.kernel == 3)
+    return check_launch(launch_fill_zero(out, out_size(out_dtype), M, N, ldo, 1, 0, cs, bias), "bias-fill launch");
+
+  GemmArgs args;
+  std::memset(&args, 0, sizeof(args));
+  args.M = static_cast<int>(M);
+  args.N = static_cast<int>(N);
+  args.K = static_cast<int>(K);
+  args.G = 1;
+  args.KB = static_cast<int>((K + 127) / 128);
+  args.NB = static_cast<int>((N + 127) / 128);
+  args.s_row = scale_a;
+  args.s_col = scale_b;
+  args.s_row_stride = sa_stride;
+  args.s_col_stride = sb_stride;
+  args.bias = bias;
+  args.grid_m = pl.grid_m;
+  args.grid_n = pl.grid_n;
+  args.num_tiles = pl.num_tiles;
+  args.group_m = kGroupM;
+  args.splits = 1;
+  args.err = dc->err;
+  CUtensorMap ta, tb, td;
+  if ((st = encode_3d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, A, K, M, 1, lda, lda * M, 128, 128, "A"))) return st;
+  if ((st = encode_3d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, B, K, N, 1, ldb, ldb * N, 128, wide_b_box_rows(pl.cg),
+                      "B")))
+    return st;
+  const int es = out_size(out_dtype);
+  if ((st = encode_3d(&td, out_tmap_type(out_dtype), es, out, N, M, 1, ldo, ldo * M, static_cast<uint32_t>(64 / es),
+                      32, "out", CU_TENSOR_MAP_SWIZZLE_64B)))
+    return st;
+  return check_launch(launch_wide(Mode::kFp8Rowwise, out_kind(out_dtype), pl.cg, ta, tb, td, args, pl.pub.ctas, cs),
+                      "fp8 rowwise kernel launch");
+}
+
 bs_status int_scaled_mm(const int8_t* A, int64_t lda, const int8_t* B, int64_t ldb, const float* s_a,
                         const float* s_b, void* out, int64_t ldo, bs_out_dtype out_dtype, int64_t M, int64_t N,
                         int64_t K, void* stream) {
@@ -499,6 +565,8 @@ bs_status int_scaled_mm(const int8_t* A, int64_t lda, const int8_t* B, int64_t l
   args.NB = static_cast<int>((N + 127) / 128);
   args.s_row = s_a;
   args.s_col = s_b;
+  args.s_row_stride = 1;
+  args.s_col_stride = 1;
   args.grid_m = pl.grid_m;
   args.grid_n = pl.grid_n;
   args.num_tiles = pl.num_tiles;
@@ -521,12 +589,14 @@ bs_status int_scaled_mm(const int8_t* A, int64_t lda, const int8_t* B, int64_t l
 }  // extern "C"
 
 // ---------------------------------------------------------------------------
-// zero fill (K == 0)
+// zero (or bias) fill, K == 0
 // ---------------------------------------------------------------------------
 namespace bsg {
 
+// out[b][r][c] = bias[c] (bias may be null: zero).  es = 2 stores bf16, es = 4
+// stores fp32 (or a zero int32).
 __global__ void fill_zero_kernel(char* out, int es, long long rows, long long cols, long long ld, long long batches,
-                                 long long bstride) {
+                                 long long bstride, const float* bias) {
   const long long total = rows * cols * batches;
   for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
        i += static_cast<long long>(gridDim.x) * blockDim.x) {
@@ -534,19 +604,21 @@ __global__ void fill_zero_kernel(char* out, int es, long long rows, long long co
     const long long rc = i - b * rows * cols;
     const long long r = rc / cols, c = rc - r * cols;
     char* p = out + (b * bstride + r * ld + c) * es;
+    const float v = bias ? bias[c] : 0.f;
     if (es == 2)
-      *reinterpret_cast<uint16_t*>(p) = 0;
+      *reinterpret_cast<__nv_bfloat16*>(p) = __float2bfloat16_rn(v);
     else
-      *reinterpret_cast<uint32_t*>(p) = 0;
+      *reinterpret_cast<float*>(p) = v;
   }
 }
 
 cudaError_t launch_fill_zero(void* out, int elem_size, long long rows, long long cols, long long ld,
-                             long long batches, long long bstride, cudaStream_t stream) {
+                             long long batches, long long bstride, cudaStream_t stream, const float* bias) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  fill_zero_kernel<<<2 * sms, 256, 0, stream>>>(static_cast<char*>(out), elem_size, rows, cols, ld, batches, bstride);
+  fill_zero_kernel<<<2 * sms, 256, 0, stream>>>(static_cast<char*>(out), elem_size, rows, cols, ld, batches, bstride,
+                                                bias);
   return cudaGetLastError();
 }
 

@@ -26,9 +26,11 @@ cudaError_t launch_wide(Mode mode, OutKind out, int cta_group, const CUtensorMap
 cudaError_t launch_skinny(Mode mode, OutKind out, int bmt, const CUtensorMap& a, const CUtensorMap& b,
                           const GemmArgs& args, const SkinnyOut& o, int n_tiles, int m_tiles, cudaStream_t stream);
 
-// Zero-fill of `batches` matrices [rows, cols] (row stride ld, batch stride
-// bstride, elements of `elem_size` bytes).
+// Fill of `batches` matrices [rows, cols] (row stride ld, batch stride
+// bstride, elements of `elem_size` bytes) with zero, or with bias[col] (fp32
+// [cols]) when bias is given.
 cudaError_t launch_fill_zero(void* out, int elem_size, long long rows, long long cols, long long ld,
-                             long long batches, long long bstride, cudaStream_t stream);
+                             long long batches, long long bstride, cudaStream_t stream,
+                             const float* bias = nullptr);
 
 }  // namespace bsg

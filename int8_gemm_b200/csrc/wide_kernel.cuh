@@ -43,7 +43,10 @@
 
 namespace bsg {
 
-enum class Mode : int { kFp8F32Scale = 0, kFp8E8M0 = 1, kInt8 = 2 };
+// kFp8Rowwise: e4m3 with one scale per row of A and per column of B (or one
+// per operand), constant along K, so the accumulator stays in TMEM for all of
+// K as in the INT8 mode.
+enum class Mode : int { kFp8F32Scale = 0, kFp8E8M0 = 1, kInt8 = 2, kFp8Rowwise = 3 };
 
 struct GemmArgs {
   int M, N, K, G;
@@ -59,9 +62,13 @@ struct GemmArgs {
   // FP8, e8m0 scales: xs[(m * G + g) * KB + kb], ws[(g * NB + nb) * KB + kb]
   const uint8_t* xs;
   const uint8_t* ws;
-  // INT8 per-row / per-column scales, either may be null
+  // INT8 and FP8-rowwise per-row / per-column scales: element m of s_row is
+  // s_row[m * s_row_stride] (stride 0: one scale for all rows), likewise for
+  // s_col; INT8 allows either to be null.  bias: fp32 [N] or null (FP8 rowwise).
   const float* s_row;
   const float* s_col;
+  long long s_row_stride, s_col_stride;
+  const float* bias;
   uint32_t* err;
 };
 
@@ -193,6 +200,7 @@ __global__ void __launch_bounds__(384, 1)
   constexpr int CONSUMER_WARPS = 8;
   constexpr uint32_t TMEM_COLS = 2 * BN;
   constexpr bool IS_INT8 = MODE == Mode::kInt8;
+  constexpr bool FULL_K = IS_INT8 || MODE == Mode::kFp8Rowwise;  // accumulate over all of K in TMEM
   constexpr uint32_t IDESC = IS_INT8 ? idesc_s8_s32<BM * CG, BN>() : idesc_e4m3_f32<BM * CG, BN>();
   constexpr int CPC = 64 / sizeof(OutT);  // output columns per 64-byte staging row
   static_assert(CG == 1 || CG == 2, "CTA group is 1 or 2");
@@ -317,7 +325,7 @@ __global__ void __launch_bounds__(384, 1)
           for (int kb = 0; kb < p.KB; ++kb) {
             // FP8: every K block starts a fresh partial in the next buffer;
             // INT8: the tile's accumulator is claimed once, at its first K block
-            if (!IS_INT8 || kb == 0) {
+            if (!FULL_K || kb == 0) {
               if (!wait_bounded(&sm.acc_empty[buf], bphase ^ 1u, abort, p.err, kErrTimeout | kRoleMma | kWaitAccEmpty)) {
                 ok = false;
                 break;
@@ -333,7 +341,7 @@ __global__ void __launch_bounds__(384, 1)
             const uint64_t bd = sdesc_k_sw128(smem_u32(sm.b[stage]));
 #pragma unroll
             for (int k = 0; k < BK / 32; ++k) {
-              const uint32_t acc = IS_INT8 ? ((kb > 0 || k > 0) ? 1u : 0u) : (k > 0 ? 1u : 0u);
+              const uint32_t acc = FULL_K ? ((kb > 0 || k > 0) ? 1u : 0u) : (k > 0 ? 1u : 0u);
               if constexpr (CG == 2) {
                 if constexpr (IS_INT8) {
                   mma_i8_pair(d, ad + 2 * k, bd + 2 * k, IDESC, acc);
@@ -353,12 +361,12 @@ __global__ void __launch_bounds__(384, 1)
             // tile's last K block also commits the accumulator barrier.
             if constexpr (CG == 2) {
               mma_commit_pair_mc(&sm.empty[stage], 0x3);
-              if (IS_INT8 && kb == p.KB - 1) mma_commit_pair_mc(&sm.acc_full[buf], 0x3);
+              if (FULL_K && kb == p.KB - 1) mma_commit_pair_mc(&sm.acc_full[buf], 0x3);
             } else {
               mma_commit(&sm.empty[stage]);
-              if (IS_INT8 && kb == p.KB - 1) mma_commit(&sm.acc_full[buf]);
+              if (FULL_K && kb == p.KB - 1) mma_commit(&sm.acc_full[buf]);
             }
-            if (!IS_INT8 || kb == p.KB - 1) {
+            if (!FULL_K || kb == p.KB - 1) {
               buf ^= 1;
               if (buf == 0) bphase ^= 1u;
             }
@@ -379,7 +387,7 @@ __global__ void __launch_bounds__(384, 1)
         }
       }
       __syncwarp();
-    } else if (!IS_INT8) {
+    } else if (!FULL_K) {
       // ---------------------------------------------------------- scale producer (warps 2, 3)
       // Stages scale_a of this CTA's 128 rows and scale_b of the tile's two
       // 128-column blocks for each K block into a ring kScaleRing blocks deep.
@@ -444,7 +452,7 @@ __global__ void __launch_bounds__(384, 1)
       const int m = m0 + row;
       const int ncol0 = n0 + half * 128;
       bool ok = true;
-      if constexpr (!IS_INT8) {
+      if constexpr (!FULL_K) {
         // fp32 accumulators; the promotion uses the packed two-wide FMA, which
         // halves the consumers' instruction count (the tensor pipe's issue
         // rate suffers when the consumer warps sharing its SM sub-partition
@@ -515,7 +523,7 @@ __global__ void __launch_bounds__(384, 1)
           break;
         tc_fence_after();
         const bool has_row = p.s_row != nullptr, has_col = p.s_col != nullptr;
-        const float sr = (has_row && m < p.M) ? __ldg(p.s_row + m) : 1.f;
+        const float sr = (has_row && m < p.M) ? __ldg(p.s_row + m * p.s_row_stride) : 1.f;
         const uint32_t tb = tmem + t_lane + static_cast<uint32_t>(buf * BN + half * 128);
 #pragma unroll
         for (int ch = 0; ch < 128 / CPC; ++ch) {
@@ -532,6 +540,15 @@ __global__ void __launch_bounds__(384, 1)
           if constexpr (sizeof(OutT) == 4 && !std::is_same<OutT, float>::value) {
 #pragma unroll
             for (int j = 0; j < CPC; ++j) v[j] = __uint_as_float(r[j]);  // raw int32 accumulator
+          } else if constexpr (!IS_INT8) {
+            // FP8 rowwise / tensorwise: acc * (s_a * s_b) + bias[n]
+#pragma unroll
+            for (int j = 0; j < CPC; ++j) {
+              const int n = ncol0 + c0 + j;
+              const float sc = n < p.N ? __ldg(p.s_col + n * p.s_col_stride) : 0.f;
+              const float bn = (p.bias != nullptr && n < p.N) ? __ldg(p.bias + n) : 0.f;
+              v[j] = fmaf(__uint_as_float(r[j]), sr * sc, bn);
+            }
           } else {
 #pragma unroll
             for (int j = 0; j < CPC; ++j) {
@@ -539,7 +556,7 @@ __global__ void __launch_bounds__(384, 1)
               if (has_row) f = __fmul_rn(f, sr);
               if (has_col) {
                 const int n = ncol0 + c0 + j;
-                const float sc = n < p.N ? __ldg(p.s_col + n) : 0.f;
+                const float sc = n < p.N ? __ldg(p.s_col + n * p.s_col_stride) : 0.f;
                 f = __fmul_rn(f, sc);
               }
               v[j] = f;

@@ -180,6 +180,37 @@ def test_fp8_validation_codes():
     assert _fp8(M=0) == bs.BS_OK and _fp8(N=0) == bs.BS_OK  # empty problem: no-op, no device needed
 
 
+def _rw(**kw):
+    a = dict(A=P16, lda=256, B=P16, ldb=256, sa=P16, sas=1, sb=P16, sbs=1, bias=None, out=P16, ldo=256,
+             dt=bs.BS_OUT_BF16, M=64, N=256, K=200)
+    a.update(kw)
+    v = ctypes.c_void_p
+    return bs.lib().bs_gemm_fp8_rowwise(v(a["A"]), a["lda"], v(a["B"]), a["ldb"], v(a["sa"]), a["sas"], v(a["sb"]),
+                                        a["sbs"], v(a["bias"]), v(a["out"]), a["ldo"], a["dt"], a["M"], a["N"], a["K"],
+                                        None)
+
+
+def test_fp8_rowwise_validation_codes():
+    # the issue's rule: both scales tensorwise (scalars) or both rowwise ((M, 1) and (1, N))
+    assert _rw(sas=0, sbs=1) == bs.BS_ERR_SHAPE and _rw(sas=1, sbs=0) == bs.BS_ERR_SHAPE
+    assert _rw(sas=2, sbs=2) == bs.BS_ERR_SHAPE
+    assert _rw(M=-1) == bs.BS_ERR_SHAPE
+    assert _rw(dt=bs.BS_OUT_I32) == bs.BS_ERR_DTYPE
+    assert _rw(out=0) == bs.BS_ERR_NULL and _rw(sa=0) == bs.BS_ERR_NULL and _rw(sb=0) == bs.BS_ERR_NULL
+    assert _rw(lda=128) == bs.BS_ERR_LAYOUT and _rw(ldo=100) == bs.BS_ERR_LAYOUT
+    assert _rw(lda=264) == bs.BS_ERR_ALIGNMENT and _rw(bias=P16 + 2) == bs.BS_ERR_ALIGNMENT
+    assert _rw(M=0) == bs.BS_OK and _rw(N=0) == bs.BS_OK
+    # K need not be a multiple of 128 here (scales are constant along K): a well-formed call only fails on the device
+    assert _rw(K=200) == bs.BS_ERR_DEVICE and _rw(sas=0, sbs=0, K=48) == bs.BS_ERR_DEVICE
+
+
+def test_plan_fp8_rowwise_is_the_wide_kernel_for_every_m():
+    for M in (1, 16, 300, 16640):
+        p = bs.plan_for(bs.OP_FP8_ROWWISE, M, 1, 5120, 8192, 148)
+        assert p["kernel"] == 1 and p["tile_n"] == 256 and p["cluster"] == 2
+    assert bs.plan_for(bs.OP_FP8_ROWWISE, 16, 1, 512, 0, 148)["kernel"] == 3  # K = 0: bias (or zero) fill
+
+
 def test_int8_and_bmm_validation_codes():
     h, v = bs.lib(), ctypes.c_void_p
     call = lambda **k: h.int_scaled_mm(v(k.get("A", P16)), k.get("lda", 128), v(k.get("B", P16)), k.get("ldb", 128),

@@ -150,6 +150,57 @@ def test_fp8_transposed_scale_a_layout():
 
 
 # ---------------------------------------------------------------------------
+# FP8 with tensorwise / rowwise scales and bias
+# ---------------------------------------------------------------------------
+def rowwise_run(d, out_dtype=torch.bfloat16, bias=True, out=None):
+    b = d["bias"].to(DEV) if (bias and d["bias"] is not None) else None
+    return bs.bs_gemm_fp8_rowwise(d["A"].to(DEV), d["B_t"].to(DEV).t(), d["scale_a"].to(DEV), d["scale_b"].to(DEV), b,
+                                  out_dtype=out_dtype, out=out)
+
+
+def oracle_rowwise(d, bias=True, rows=None):
+    return oracle.fp8_rowwise(d["A"], d["B_t"], d["scale_a"], d["scale_b"], d["bias"] if bias else None, rows=rows)
+
+
+@pytest.mark.parametrize("M,N,K", [(256, 256, 512), (300, 520, 640), (1, 256, 128), (129, 384, 176), (640, 1280, 1024),
+                                   (5, 259, 48)])
+@pytest.mark.parametrize("tensorwise", [False, True])
+@pytest.mark.parametrize("kernel", [bs.PATH_AUTO, bs.PATH_WIDE_SINGLE])
+def test_fp8_rowwise_and_tensorwise(M, N, K, tensorwise, kernel, path):
+    path(kernel)
+    d = wl.fp8_rowwise_inputs(M, N, K, seed=140 + M + N + K, tensorwise=tensorwise)
+    for out_dtype in (torch.bfloat16, torch.float32):
+        for bias in (True, False):
+            y, S = oracle_rowwise(d, bias)
+            fp8_check(rowwise_run(d, out_dtype, bias), y, S, out_dtype,
+                      f"fp8 rowwise {M}x{N}x{K} tensorwise={tensorwise} bias={bias}")
+
+
+def test_fp8_rowwise_k0_writes_bias_and_is_deterministic():
+    bias = torch.randn(200, generator=torch.Generator().manual_seed(150)).to(DEV)
+    A = torch.zeros(64, 0, dtype=torch.uint8, device=DEV)
+    B = torch.zeros(200, 0, dtype=torch.uint8, device=DEV).t()
+    out = bs.bs_gemm_fp8_rowwise(A, B, torch.ones(64, 1, device=DEV), torch.ones(1, 200, device=DEV), bias,
+                                 out_dtype=torch.float32)
+    assert torch.equal(out, bias.expand(64, 200))
+    out = bs.bs_gemm_fp8_rowwise(A, B, torch.ones((), device=DEV), torch.ones((), device=DEV), None)
+    assert torch.all(out == 0)
+    d = wl.fp8_rowwise_inputs(300, 512, 1024, seed=151)
+    first = rowwise_run(d)
+    assert torch.equal(first, rowwise_run(d))
+
+
+@pytest.mark.slow
+def test_fp8_rowwise_16640x5120x8192_sampled_rows():
+    w = wl.WORKLOADS["fp8_rowwise_16640x5120x8192"]
+    d = wl.workload_inputs(w)
+    out = rowwise_run(d)
+    rows = rows_sample(w.M, extra=6)
+    y, S = oracle_rowwise(d, rows=rows)
+    fp8_check(out[torch.tensor(rows, device=DEV)], y, S, torch.bfloat16, "fp8 rowwise 16640x5120x8192")
+
+
+# ---------------------------------------------------------------------------
 # operation 2: INT8, bit-exact
 # ---------------------------------------------------------------------------
 def int8_run(d, out_dtype, s_b=True):

@@ -44,7 +44,7 @@ GROUP = 128  # quantisation group / block edge along K (and N for weights)
 @dataclass(frozen=True)
 class Workload:
     name: str
-    op: str  # "fp8_blockwise" | "int_scaled_mm" | "bmm_a8w8_blockscale"
+    op: str  # "fp8_blockwise" | "int_scaled_mm" | "bmm_a8w8_blockscale" | "fp8_rowwise"
     M: int
     N: int
     K: int
@@ -57,6 +57,8 @@ WORKLOADS = {
     "fp8_tiny_256x256x512": Workload("fp8_tiny_256x256x512", "fp8_blockwise", 256, 256, 512, seed=0),
     "int8_4096x4096x4096": Workload("int8_4096x4096x4096", "int_scaled_mm", 4096, 4096, 4096, seed=1),
     "fp8_16640x5120x8192": Workload("fp8_16640x5120x8192", "fp8_blockwise", 16640, 5120, 8192, seed=2),
+    # the rowwise-scaled form of the same shape (the mode the blockwise issue's error message names)
+    "fp8_rowwise_16640x5120x8192": Workload("fp8_rowwise_16640x5120x8192", "fp8_rowwise", 16640, 5120, 8192, seed=5),
 }
 BMM_M_SWEEP = (1, 16, 128, 1024, 16384)
 BMM_G = (8, 2)
@@ -147,6 +149,34 @@ def fp8_blockwise_inputs(M: int, N: int, K: int, seed: int):
     return {"A": A, "B_t": Bkn.t().contiguous(), "scale_a": sa, "scale_b": sb}
 
 
+def fp8_rowwise_inputs(M: int, N: int, K: int, seed: int, tensorwise: bool = False, bias: bool = True):
+    """Inputs of ``bs_gemm_fp8_rowwise``: the same N(0,1)-with-outliers data quantised with one scale per
+    row of A and per column of B (amax / 448), or one per operand when ``tensorwise``.
+
+    Returns CPU tensors: A uint8 [M, K], B_t uint8 [N, K], scale_a fp32 [M, 1] or [], scale_b fp32 [1, N] or [],
+    bias fp32 [N] (N(0,1)) or None."""
+    a = normal_with_outliers((M, K), seed + 10 * 1)
+    b = normal_with_outliers((N, K), seed + 10 * 2)
+
+    def quant(x, per_row):
+        amax = x.abs().amax(dim=1, keepdim=True) if per_row else x.abs().amax().reshape(1, 1)
+        scale = amax / E4M3_MAX
+        scale[amax == 0] = 1.0
+        return to_e4m3_bytes(x / scale), scale
+
+    A, sa = quant(a, not tensorwise)
+    B_t, sb = quant(b, not tensorwise)
+    if tensorwise:
+        sa, sb = sa.reshape(()), sb.reshape(())
+    else:
+        sb = sb.reshape(1, N)
+    out = {"A": A.contiguous(), "B_t": B_t.contiguous(), "scale_a": sa.contiguous(), "scale_b": sb.contiguous(),
+           "bias": None}
+    if bias:
+        out["bias"] = torch.randn(N, generator=_gen(seed + 10 * 7), dtype=torch.float32)
+    return out
+
+
 # ---------------------------------------------------------------------------
 # INT8 row/column scaled
 # ---------------------------------------------------------------------------
@@ -221,4 +251,6 @@ def workload_inputs(w: Workload, sweep: int = 0, batch_first: bool = False):
         return fp8_blockwise_inputs(w.M, w.N, w.K, base)
     if w.op == "int_scaled_mm":
         return int8_inputs(w.M, w.N, w.K, base)
+    if w.op == "fp8_rowwise":
+        return fp8_rowwise_inputs(w.M, w.N, w.K, base)
     return bmm_inputs(w.M, w.G, w.N, w.K, base, batch_first=batch_first)
