@@ -143,15 +143,24 @@ Plan make_plan(int op, int64_t M, int64_t G, int64_t N, int64_t K, int sms) {
   const bool skinny_ok = op == 1 || op == 3;  // block-scaled FP8 only
   const bool skinny = skinny_ok && (ov == 2 || (ov == 0 && M <= kSkinnyMaxM));
   if (skinny) {
-    const int bmt = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128;
+    const long long n_tiles = (N + 127) / 128;
+    const long long sm_count = sms > 0 ? sms : 148;
+    int bmt = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128;
+    // Each CTA issues its K blocks' MMAs as one serial chain, so for long K
+    // (32 or more blocks) two co-resident CTAs per SM -- possible only for
+    // activation tiles of at most 32 rows -- beat one wider tile per SM, as
+    // long as the grid of 32-row tiles is still resident in one wave.
+    if (bmt > 32 && KB >= 32 &&
+        ((M + 31) / 32) * n_tiles * G <= static_cast<long long>(skinny_ctas_per_sm(32)) * sm_count)
+      bmt = 32;
     x.bmt = bmt;
     x.m_tiles = static_cast<int>((M + bmt - 1) / bmt);
-    x.n_tiles = static_cast<int>((N + 127) / 128);
+    x.n_tiles = static_cast<int>(n_tiles);
     const long long units = static_cast<long long>(x.m_tiles) * x.n_tiles * G;
     // Split K over a cluster of S CTAs only as far as every CTA stays resident
     // at once (a second partial wave would double the time of an HBM-bound
     // stream), S a power of two <= 8 and <= the number of K blocks.
-    const long long slots = static_cast<long long>(skinny_ctas_per_sm(bmt)) * (sms > 0 ? sms : 148);
+    const long long slots = static_cast<long long>(skinny_ctas_per_sm(bmt)) * sm_count;
     // Clusters of 8 CTAs that each fill an SM do not all fit in the GPCs at
     // once, so those kernels split at most 4 ways.
     const int max_s = skinny_ctas_per_sm(bmt) > 1 ? 8 : 4;

@@ -9,8 +9,9 @@
 // second launch) -- the same fp32 partial-sum-then-cast structure as the
 // split-K decomposition decomposeK in pytorch/torch/_inductor/kernel/mm.py.
 //
-// Roles: warp 0 TMA producer, warp 1 MMA issuer and TMEM owner, warp 2 scale
-// producer, warp 3 idle, warps 4.. consumers.  Consumer warp w reads TMEM lanes
+// Roles: warp 0 TMA producer, warp 1 TMEM owner and MMA issuer of the even K
+// blocks, warp 3 MMA issuer of the odd K blocks, warp 2 scale producer,
+// warps 4.. consumers.  Consumer warp w reads TMEM lanes
 // 32*(w%4).. (32 weight rows) and, when there are eight consumer warps, one
 // half of the BMT accumulator columns.  The scale producer writes, per K block,
 // s[j] = scale_a[m0+j, kb] * scale_b[kb, nb] (one value per activation row,
@@ -58,7 +59,7 @@ struct SkinnySmem {
   uint64_t acc_empty[kSkinnyAccBufs];
   uint64_t sc_full[SSTAGES];
   uint64_t sc_empty[SSTAGES];
-  uint64_t drain;
+  uint64_t drain[2];  // one per MMA-issuing thread (abort path)
   uint32_t tmem_base;
   int abort;
 };
@@ -246,7 +247,8 @@ __global__ void __launch_bounds__(SkinnyCfg<BMT>::THREADS, SkinnyCfg<BMT>::CTAS_
       mbar_init(&sm.sc_full[s], 32);
       mbar_init(&sm.sc_empty[s], CW);
     }
-    mbar_init(&sm.drain, 1);
+    mbar_init(&sm.drain[0], 1);
+    mbar_init(&sm.drain[1], 1);
     sm.abort = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
@@ -311,12 +313,19 @@ __global__ void __launch_bounds__(SkinnyCfg<BMT>::THREADS, SkinnyCfg<BMT>::CTAS_
       }
     }
     __syncwarp();
-  } else if (warp == 1) {
+  } else if (warp == 1 || warp == 3) {
+    // Two MMA-issuing threads: warp 1 takes the even K blocks and warp 3 the
+    // odd ones.  Consecutive K blocks use different stages and accumulator
+    // buffers, so the two streams are independent; each thread's commits
+    // track its own MMAs.  (One thread issuing everything spends most of a
+    // K block's time in the issue of its four MMAs.)
     if (lane == 0) {
-      int stage = 0, buf = 0;
-      uint32_t phase = 0, bphase = 0;
+      const int issuer = warp == 3 ? 1 : 0;
       bool ok = true;
-      for (int i = 0; i < nkb; ++i) {
+      for (int i = issuer; i < nkb; i += 2) {
+        const int stage = i % STAGES, buf = i % NBUF;
+        const uint32_t phase = static_cast<uint32_t>(i / STAGES) & 1u;
+        const uint32_t bphase = static_cast<uint32_t>(i / NBUF) & 1u;
         if (!wait_bounded(&sm.acc_empty[buf], bphase ^ 1u, abort, p.err, kErrTimeout | kRoleMma | kWaitAccEmpty) ||
             !wait_bounded(&sm.full[stage], phase, abort, p.err, kErrTimeout | kRoleMma | kWaitStageFull)) {
           ok = false;
@@ -330,19 +339,11 @@ __global__ void __launch_bounds__(SkinnyCfg<BMT>::THREADS, SkinnyCfg<BMT>::CTAS_
         for (int k = 0; k < BK / 32; ++k) mma_f8f6f4(d, ad + 2 * k, bd + 2 * k, IDESC, k > 0 ? 1u : 0u);
         mma_commit(&sm.empty[stage]);
         mma_commit(&sm.acc_full[buf]);
-        if (++buf == NBUF) {
-          buf = 0;
-          bphase ^= 1u;
-        }
-        if (++stage == STAGES) {
-          stage = 0;
-          phase ^= 1u;
-        }
       }
-      if (!ok) {
-        mma_commit(&sm.drain);
+      if (!ok) {  // wait until this thread's MMAs have finished with TMEM and shared memory
+        mma_commit(&sm.drain[issuer]);
         volatile int never = 0;
-        wait_bounded(&sm.drain, 0, &never, nullptr, 0);
+        wait_bounded(&sm.drain[issuer], 0, &never, nullptr, 0);
       }
     }
     __syncwarp();

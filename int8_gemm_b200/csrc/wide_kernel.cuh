@@ -62,9 +62,11 @@ struct GemmArgs {
   // FP8, e8m0 scales: xs[(m * G + g) * KB + kb], ws[(g * NB + nb) * KB + kb]
   const uint8_t* xs;
   const uint8_t* ws;
-  // INT8 and FP8-rowwise per-row / per-column scales: element m of s_row is
-  // s_row[m * s_row_stride] (stride 0: one scale for all rows), likewise for
-  // s_col; INT8 allows either to be null.  bias: fp32 [N] or null (FP8 rowwise).
+  // INT8 and FP8-rowwise per-row / per-column scales.  INT8 reads s_row[m]
+  // and s_col[n] and allows either to be null.  FP8 rowwise reads s_row[m]
+  // when s_row_stride is 1 and s_row[0] when it is 0 (tensorwise), likewise
+  // for s_col; the strides are 0 or 1 and are applied as a select.  bias:
+  // fp32 [N] or null (FP8 rowwise).
   const float* s_row;
   const float* s_col;
   long long s_row_stride, s_col_stride;
@@ -523,7 +525,10 @@ __global__ void __launch_bounds__(384, 1)
           break;
         tc_fence_after();
         const bool has_row = p.s_row != nullptr, has_col = p.s_col != nullptr;
-        const float sr = (has_row && m < p.M) ? __ldg(p.s_row + m * p.s_row_stride) : 1.f;
+        const float sr = (has_row && m < p.M) ? __ldg(p.s_row + (IS_INT8 || p.s_row_stride != 0 ? m : 0)) : 1.f;
+        // FP8 rowwise: this thread's column scales start at s_col_n and advance by col_step
+        const int col_step = !IS_INT8 && p.s_col_stride != 0 ? 1 : 0;
+        const float* s_col_n = IS_INT8 ? nullptr : p.s_col + ncol0 * col_step;
         const uint32_t tb = tmem + t_lane + static_cast<uint32_t>(buf * BN + half * 128);
 #pragma unroll
         for (int ch = 0; ch < 128 / CPC; ++ch) {
@@ -545,7 +550,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
             for (int j = 0; j < CPC; ++j) {
               const int n = ncol0 + c0 + j;
-              const float sc = n < p.N ? __ldg(p.s_col + n * p.s_col_stride) : 0.f;
+              const float sc = n < p.N ? __ldg(s_col_n + (c0 + j) * col_step) : 0.f;
               const float bn = (p.bias != nullptr && n < p.N) ? __ldg(p.bias + n) : 0.f;
               v[j] = fmaf(__uint_as_float(r[j]), sr * sc, bn);
             }
@@ -556,7 +561,7 @@ __global__ void __launch_bounds__(384, 1)
               if (has_row) f = __fmul_rn(f, sr);
               if (has_col) {
                 const int n = ncol0 + c0 + j;
-                const float sc = n < p.N ? __ldg(p.s_col + n * p.s_col_stride) : 0.f;
+                const float sc = n < p.N ? __ldg(p.s_col + n) : 0.f;
                 f = __fmul_rn(f, sc);
               }
               v[j] = f;

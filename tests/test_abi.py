@@ -103,6 +103,19 @@ def test_plan_skinny_split_k(M):
     assert p["ctas"] == m_tiles * (7168 // 128) * p["splits"]
 
 
+def test_plan_skinny_long_k_prefers_two_ctas_per_sm():
+    # 32 or more K blocks: 32-row activation tiles (two CTAs per SM) when that grid is one wave
+    b = bs.plan_for(bs.OP_BMM, 128, 8, 1024, 4096, 148)
+    assert (b["tile_m"], b["splits"], b["ctas"]) == (32, 1, 4 * 8 * 8)
+    b = bs.plan_for(bs.OP_BMM, 128, 2, 1024, 4096, 148)
+    assert (b["tile_m"], b["splits"], b["ctas"]) == (32, 4, 4 * 8 * 2 * 4)
+    p = bs.plan_for(bs.OP_FP8_BLOCKWISE, 70, 1, 640, 4096, 148)
+    assert (p["tile_m"], p["splits"], p["cluster"]) == (32, 8, 8)
+    # 16 K blocks, or a grid of 32-row tiles beyond one wave: the widest tile that covers M
+    assert bs.plan_for(bs.OP_FP8_BLOCKWISE, 127, 1, 7168, 2048, 148)["tile_m"] == 128
+    assert bs.plan_for(bs.OP_BMM, 255, 8, 1024, 4096, 148)["tile_m"] == 128
+
+
 def test_plan_int8_and_edges():
     assert bs.plan_for(bs.OP_INT_SCALED_MM, 4096, 1, 4096, 4096, 148)["kernel"] == 1
     assert bs.plan_for(bs.OP_INT_SCALED_MM, 1, 1, 4096, 4096, 148)["kernel"] == 1  # no skinny INT8 kernel

@@ -79,6 +79,17 @@ def test_fp8_n_not_multiple_of_four(M, N, K, kernel, out_dtype, path):
     fp8_check(out, y, S, out_dtype, f"fp8 {M}x{N}x{K} kernel={kernel}")
 
 
+@pytest.mark.parametrize("M,N,K", [(70, 640, 4096), (128, 1032, 4096), (33, 256, 8192)])
+def test_fp8_skinny_long_k_32_row_tiles(M, N, K):
+    """Long K: the planner takes 32-row activation tiles (several per M, the
+    last one ragged) and splits K up to eight ways."""
+    d = wl.fp8_blockwise_inputs(M, N, K, seed=95 + M + N)
+    p = bs.plan_for(bs.OP_FP8_BLOCKWISE, M, 1, N, K, torch.cuda.get_device_properties(0).multi_processor_count)
+    assert p["kernel"] == 2 and p["tile_m"] == 32
+    y, S = oracle_fp8(d)
+    fp8_check(fp8_run(d), y, S, torch.bfloat16, f"fp8 {M}x{N}x{K} 32-row tiles split {p['splits']}")
+
+
 @pytest.mark.parametrize("M", wl.SKINNY_M_SWEEP)
 def test_fp8_skinny_sweep_n7168_k2048(M):
     w = wl.WORKLOADS[f"fp8_skinny_m{M}"]
