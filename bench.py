@@ -329,8 +329,9 @@ def main():
     ap.add_argument("--shape", default=None,
                     help="ad-hoc problem 'M,N,K' (or 'M,G,N,K' for --op bmm) instead of a named workload")
     ap.add_argument("--op", default="fp8", choices=["fp8", "int8", "bmm"], help="operation for --shape")
-    ap.add_argument("--path", default="auto", choices=["auto", "wide", "skinny", "wide1"],
-                    help="force a kernel family (wide = CTA-pair persistent, wide1 = single-CTA persistent)")
+    ap.add_argument("--path", default="auto", choices=["auto", "wide", "skinny", "wide1", "promote"],
+                    help="force a kernel family (wide = CTA-pair persistent, wide1 = single-CTA persistent, "
+                         "promote = CTA-pair persistent with e8m0 block scales promoted on the CUDA cores)")
     args = ap.parse_args()
 
     rank = int(os.environ.get("RANK", "0"))
@@ -378,7 +379,7 @@ def main():
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         return float(t.item())
 
-    bs.set_path_override({"auto": 0, "wide": 1, "skinny": 2, "wide1": 3}[args.path])
+    bs.set_path_override({"auto": 0, "wide": 1, "skinny": 2, "wide1": 3, "promote": 4}[args.path])
     copies = max(1, math.ceil(3 * L2_BYTES / byts)) if byts < 3 * L2_BYTES else 1
     d, sets = build_step(w, device, copies)
     op = {"fp8_blockwise": 1, "int_scaled_mm": 2, "bmm_a8w8_blockscale": 3, "fp8_rowwise": 4}[w.op]

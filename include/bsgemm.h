@@ -204,7 +204,10 @@ bs_status bs_plan_for(int32_t op, int64_t M, int64_t G, int64_t N, int64_t K, in
 /* Force the kernel family for subsequent calls in this process (testing):
  * 0 = automatic (default), 1 = persistent wide kernel on CTA pairs (256 x 256
  * tiles), 2 = skinny split-K kernel where the operation has one, 3 = persistent
- * wide kernel on single CTAs (128 x 256 tiles).  Returns the previous setting. */
+ * wide kernel on single CTAs (128 x 256 tiles), 4 = as 1, but
+ * bmm_a8w8_blockscale promotes every 128-deep block on the CUDA cores instead
+ * of letting the tensor core apply its e8m0 scales (block-scaled MMA).
+ * Returns the previous setting. */
 int32_t bs_set_path_override(int32_t path);
 
 /* The persistent tile order: fills out[3*t .. 3*t+2] = (batch, tile_row,

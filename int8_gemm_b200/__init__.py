@@ -26,7 +26,7 @@ BS_OK, BS_ERR_NULL, BS_ERR_SHAPE, BS_ERR_LAYOUT, BS_ERR_ALIGNMENT = 0, 1, 2, 3, 
 BS_ERR_DTYPE, BS_ERR_DEVICE, BS_ERR_CUDA, BS_ERR_TIMEOUT = 5, 6, 7, 8
 BS_OUT_BF16, BS_OUT_F32, BS_OUT_I32 = 0, 1, 2
 
-PATH_AUTO, PATH_WIDE, PATH_SKINNY, PATH_WIDE_SINGLE = 0, 1, 2, 3
+PATH_AUTO, PATH_WIDE, PATH_SKINNY, PATH_WIDE_SINGLE, PATH_WIDE_PROMOTE = 0, 1, 2, 3, 4
 
 _OUT_CODE = {torch.bfloat16: BS_OUT_BF16, torch.float32: BS_OUT_F32, torch.int32: BS_OUT_I32}
 

@@ -280,7 +280,10 @@ bs_status run_fp8(const Fp8Problem& q, GemmArgs args, cudaStream_t stream, Devic
     if ((st = encode_3d(&td, out_tmap_type(q.out_dtype), es, q.out, q.N, q.M, q.G, q.o_rs, o_bs,
                         static_cast<uint32_t>(64 / es), 32, "out", CU_TENSOR_MAP_SWIZZLE_64B)))
       return st;
-    return check_launch(launch_wide(q.mode, out_kind(q.out_dtype), pl.cg, ta, tb, td, args, pl.pub.ctas, stream),
+    // e8m0 block scales on CTA pairs: applied by the tensor core (block-scaled
+    // MMA) unless path 4 asks for the per-block promotion on the CUDA cores
+    const Mode mode = q.mode == Mode::kFp8E8M0 && pl.cg == 2 && g_path_override.load() != 4 ? Mode::kFp8Mx : q.mode;
+    return check_launch(launch_wide(mode, out_kind(q.out_dtype), pl.cg, ta, tb, td, args, pl.pub.ctas, stream),
                         "wide kernel launch");
   }
   args.splits = pl.pub.splits;

@@ -61,6 +61,12 @@ cudaError_t launch_cg(Mode mode, OutKind out, const CUtensorMap& a, const CUtens
       if (out == OutKind::kBF16) return launch_one<Mode::kFp8Rowwise, CG, __nv_bfloat16>(a, b, d, args, grid, stream);
       if (out == OutKind::kF32) return launch_one<Mode::kFp8Rowwise, CG, float>(a, b, d, args, grid, stream);
       break;
+    case Mode::kFp8Mx:
+      if constexpr (CG == 2) {
+        if (out == OutKind::kBF16) return launch_one<Mode::kFp8Mx, CG, __nv_bfloat16>(a, b, d, args, grid, stream);
+        if (out == OutKind::kF32) return launch_one<Mode::kFp8Mx, CG, float>(a, b, d, args, grid, stream);
+      }
+      break;
     case Mode::kInt8:
       if (out == OutKind::kBF16) return launch_one<Mode::kInt8, CG, __nv_bfloat16>(a, b, d, args, grid, stream);
       if (out == OutKind::kF32) return launch_one<Mode::kInt8, CG, float>(a, b, d, args, grid, stream);

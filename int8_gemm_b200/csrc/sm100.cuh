@@ -263,11 +263,32 @@ __device__ __forceinline__ uint64_t sdesc_k_sw128(uint32_t saddr) {
   return d;
 }
 
+// Shared-memory descriptor of a K-major operand without swizzle: core matrices
+// of 8 rows x 16 bytes stored contiguously, consecutive 8-row groups `sbo`
+// bytes apart (the source of tcgen05.cp for scale factors).
+__device__ __forceinline__ uint64_t sdesc_k_plain(uint32_t saddr, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);  // start address, bits 0-13
+  d |= static_cast<uint64_t>(1) << 16;                    // leading byte offset (one core matrix along K)
+  d |= static_cast<uint64_t>(sbo >> 4) << 32;             // stride byte offset
+  d |= static_cast<uint64_t>(1) << 46;                    // descriptor version
+  return d;                                               // layout type 0: no swizzle
+}
+
 // Instruction descriptors (dense, K-major A and B, no negation).
 // e4m3 x e4m3 -> f32
 template <int M, int N>
 __host__ __device__ constexpr uint32_t idesc_e4m3_f32() {
   return (1u << 4) | (0u << 7) | (0u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
+}
+// e4m3 x e4m3 -> f32 with block scaling (kind::mxf8f6f4): e8m0 scale factors,
+// one per 32 K elements of every A row and B column, read from TMEM at the
+// byte selected by the scale-factor ids (bits 29-30 for A, 4-5 for B; 0 here).
+// Bit 23 selects the e8m0 scale format.
+template <int M, int N>
+__host__ __device__ constexpr uint32_t idesc_mx_e4m3_f32() {
+  return (0u << 7) | (0u << 10) | (static_cast<uint32_t>(N >> 3) << 17) | (1u << 23) |
          (static_cast<uint32_t>(M >> 4) << 24);
 }
 // s8 x s8 -> s32
@@ -307,6 +328,24 @@ __device__ __forceinline__ void mma_f8f6f4_pair(uint32_t d_tmem, uint64_t adesc,
       "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
+}
+// Block-scaled MMA on a CTA pair: D (+)= (A * sfA) x (B * sfB), the scale
+// factors at TMEM addresses sfa (the pair's 256 rows, 128 per CTA) and sfb
+// (the N columns).
+__device__ __forceinline__ void mma_mxf8f6f4_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                                  uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%4], [%5], p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
+      : "memory");
+}
+// Copy 32 rows x 16 bytes of shared memory (descriptor `sdesc`) into four
+// TMEM columns at `taddr`, the same data in each of the four 32-lane groups;
+// on a CTA pair, each CTA's shared memory into its own TMEM.
+__device__ __forceinline__ void tmem_cp_32x128b_x4_pair(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 __device__ __forceinline__ void mma_i8_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                             uint32_t accumulate) {

@@ -7,7 +7,8 @@
 //   warp 1      MMA issuer: four tcgen05.mma (K = 32 bytes each) per K block
 //               into a TMEM accumulator; owns the TMEM allocation.
 //   warps 2, 3  FP8 modes: scale producer (stages the block scales of the
-//               next K blocks in a shared ring); idle for INT8.
+//               next K blocks in a shared ring; for kFp8Mx, the e8m0 scale
+//               factors the tensor core reads); idle for INT8 and rowwise.
 //   warps 4..11 consumers (warpgroups 1 and 2).  Warp w reads TMEM lanes
 //               32*(w%4).. and one half (128 columns) of the tile.
 // Launched with 384 threads x 168 registers; warpgroup 0 keeps 56 each and the
@@ -24,13 +25,21 @@
 //   work with torch.compile" (1x128 / 128x128 scale shapes); ROCm/aiter PR
 //   "Add opus fp8 mxscale BMM kernels for gfx950" (m-major batched layout,
 //   e8m0 scales [M, G, K/128] and [G, N/128, K/128]).
+// kFp8Mx (the batched operation on CTA pairs): the e8m0 scales are powers of
+// two, so the tensor core applies them itself -- per K block the MMA thread
+// copies the scale factors of the pair's 256 rows and 256 columns from
+// shared memory into TMEM (tcgen05.cp) and issues block-scaled MMAs that
+// accumulate over all of K.  The second half of TMEM holds the scale factors,
+// so one accumulator buffer remains and the epilogue does not overlap the
+// next tile.  The power-of-two scales make every product exact, so this sums
+// the same terms as the per-block promotion, in a different order.
 // INT8 mode: s8 x s8 -> s32 accumulates over all of K in TMEM (double-buffered
 // across tiles); the epilogue computes (float(acc) * s_a[m]) * s_b[n] with two
 // round-to-nearest fp32 multiplies.
 //   Sources: pytorch/ao PR "Remove int_scaled_mm's dependency on triton for
 //   cpu" (int_scaled_matmul_cpu); pytorch/ao issue "Unify scaled INT8 matmul"
 //   (cast acc_i32 to f32, then multiply by the fp32 scales).
-// Epilogue: registers -> 128B-swizzled shared staging (4 KB per consumer warp)
+// Epilogue: registers -> 64B-swizzled shared staging (2 KB per consumer warp)
 // -> TMA store, which clips rows >= M and columns >= N (the masked store of
 // mm_template in pytorch/torch/_inductor/kernel/mm.py).  Rows >= M of A are
 // zero-filled by the TMA loads, so ragged M needs no padding copies.
@@ -46,7 +55,11 @@ namespace bsg {
 // kFp8Rowwise: e4m3 with one scale per row of A and per column of B (or one
 // per operand), constant along K, so the accumulator stays in TMEM for all of
 // K as in the INT8 mode.
-enum class Mode : int { kFp8F32Scale = 0, kFp8E8M0 = 1, kInt8 = 2, kFp8Rowwise = 3 };
+// kFp8Mx: the batched operation's e8m0 (power-of-two) block scales applied by
+// the tensor core itself (tcgen05.mma kind::mxf8f6f4 with block scaling, one
+// scale per 32 K elements, each 128-deep block's scale repeated four times),
+// so the accumulator also stays in TMEM for all of K.  CTA pairs only.
+enum class Mode : int { kFp8F32Scale = 0, kFp8E8M0 = 1, kInt8 = 2, kFp8Rowwise = 3, kFp8Mx = 4 };
 
 struct GemmArgs {
   int M, N, K, G;
@@ -79,13 +92,22 @@ struct GemmArgs {
 // offsets in the peer.
 constexpr int kScaleRing = 16;  // K blocks of scales staged ahead of the consumers
 constexpr int kScaleBatch = 8;  // K blocks whose scale loads are in flight together
+constexpr int kSfRing = 5;      // kFp8Mx: K blocks of scale-factor chunks staged ahead of the MMA
+constexpr uint32_t kSfaCol = 256, kSfbCol = 260;  // kFp8Mx: TMEM columns of the scale factors
 
 template <int BNL, int STAGES>
 struct WideSmem {
   uint8_t a[STAGES][128 * 128];  // this CTA's 128 A rows of one K block
   uint8_t b[STAGES][BNL * 128];  // this CTA's BNL B rows (output columns) of one K block
   uint8_t stage_out[8][32 * 64];  // per consumer warp: 32 rows x 64 bytes, 64-byte swizzle
-  float sa[kScaleRing][128];     // scale_a of this CTA's rows, per K block
+  union {
+    float sa[kScaleRing][128];  // scale_a of this CTA's rows, per K block
+    // kFp8Mx, per K block: three 512-byte scale-factor chunks (this CTA's 128
+    // rows of A; B columns 0-127; B columns 128-255), each 32 lanes x 16 bytes
+    // as tcgen05.cp reads them: item i at byte 16*(i%32) + 4*(i/32), its
+    // byte repeated for the four 32-deep sub-blocks
+    alignas(16) uint8_t sf[kSfRing][3][512];
+  };
   float sb[kScaleRing][4];       // scale_b of the tile's two 128-column blocks, per K block
   uint64_t full[STAGES];
   uint64_t empty[STAGES];
@@ -202,8 +224,13 @@ __global__ void __launch_bounds__(384, 1)
   constexpr int CONSUMER_WARPS = 8;
   constexpr uint32_t TMEM_COLS = 2 * BN;
   constexpr bool IS_INT8 = MODE == Mode::kInt8;
-  constexpr bool FULL_K = IS_INT8 || MODE == Mode::kFp8Rowwise;  // accumulate over all of K in TMEM
-  constexpr uint32_t IDESC = IS_INT8 ? idesc_s8_s32<BM * CG, BN>() : idesc_e4m3_f32<BM * CG, BN>();
+  constexpr bool MX = MODE == Mode::kFp8Mx;  // block scales applied by the tensor core
+  constexpr bool FULL_K = IS_INT8 || MODE == Mode::kFp8Rowwise || MX;  // accumulate over all of K in TMEM
+  // accumulator buffers; kFp8Mx keeps the second half of TMEM for the scale factors
+  constexpr int NACC = MX ? 1 : 2;
+  constexpr uint32_t IDESC = IS_INT8 ? idesc_s8_s32<BM * CG, BN>()
+                                     : (MX ? idesc_mx_e4m3_f32<BM * CG, BN>() : idesc_e4m3_f32<BM * CG, BN>());
+  static_assert(!MX || CG == 2, "hardware block scaling is built for CTA pairs");
   constexpr int CPC = 64 / sizeof(OutT);  // output columns per 64-byte staging row
   static_assert(CG == 1 || CG == 2, "CTA group is 1 or 2");
   using Smem = WideSmem<BNL, STAGES>;
@@ -232,8 +259,11 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(&sm.acc_empty[b], CONSUMER_WARPS * CG);
     }
     for (int i = 0; i < kScaleRing; ++i) {
-      mbar_init(&sm.sc_full[i], 64);  // every thread of the two scale warps
-      mbar_init(&sm.sc_empty[i], CONSUMER_WARPS);
+      // FP8 block scales: every thread of the two scale warps fills, the
+      // consumer warps release.  kFp8Mx: one arrival per scale warp of both
+      // CTAs on the leader's barrier, released by the MMA's commit.
+      mbar_init(&sm.sc_full[i], MX ? 2 * CG : 64);
+      mbar_init(&sm.sc_empty[i], MX ? 1 : CONSUMER_WARPS);
     }
     mbar_init(&sm.drain, 1);
     sm.abort = 0;
@@ -322,6 +352,7 @@ __global__ void __launch_bounds__(384, 1)
       if (lane == 0 && leader) {
         int stage = 0, buf = 0;
         uint32_t phase = 0, bphase = 0;
+        uint32_t sfc = 0;  // kFp8Mx: K blocks whose scale factors were consumed (ring position)
         bool ok = true;
         for (int tile = unit; ok && tile < p.num_tiles; tile += units) {
           for (int kb = 0; kb < p.KB; ++kb) {
@@ -337,16 +368,34 @@ __global__ void __launch_bounds__(384, 1)
               ok = false;
               break;
             }
+            const int sslot = static_cast<int>(sfc % kSfRing);
+            if constexpr (MX) {  // both CTAs' scale-factor chunks of this K block are in shared memory
+              if (!wait_bounded<true>(&sm.sc_full[sslot], (sfc / kSfRing) & 1u, abort, p.err,
+                                      kErrTimeout | kRoleMma | kWaitScaleFull)) {
+                ok = false;
+                break;
+              }
+            }
             tc_fence_after();
             const uint32_t d = tmem + static_cast<uint32_t>(buf * BN);
             const uint64_t ad = sdesc_k_sw128(smem_u32(sm.a[stage]));
             const uint64_t bd = sdesc_k_sw128(smem_u32(sm.b[stage]));
+            if constexpr (MX) {
+              // scale factors to TMEM; issued by this thread, they are ordered
+              // after the previous K block's MMAs and before this block's
+              const uint32_t sf0 = smem_u32(sm.sf[sslot][0]);
+              tmem_cp_32x128b_x4_pair(tmem + kSfaCol, sdesc_k_plain(sf0, 128));
+              tmem_cp_32x128b_x4_pair(tmem + kSfbCol, sdesc_k_plain(sf0 + 512, 128));
+              tmem_cp_32x128b_x4_pair(tmem + kSfbCol + 4, sdesc_k_plain(sf0 + 1024, 128));
+            }
 #pragma unroll
             for (int k = 0; k < BK / 32; ++k) {
               const uint32_t acc = FULL_K ? ((kb > 0 || k > 0) ? 1u : 0u) : (k > 0 ? 1u : 0u);
               if constexpr (CG == 2) {
                 if constexpr (IS_INT8) {
                   mma_i8_pair(d, ad + 2 * k, bd + 2 * k, IDESC, acc);
+                } else if constexpr (MX) {
+                  mma_mxf8f6f4_pair(d, ad + 2 * k, bd + 2 * k, IDESC, tmem + kSfaCol, tmem + kSfbCol, acc);
                 } else {
                   mma_f8f6f4_pair(d, ad + 2 * k, bd + 2 * k, IDESC, acc);
                 }
@@ -363,14 +412,20 @@ __global__ void __launch_bounds__(384, 1)
             // tile's last K block also commits the accumulator barrier.
             if constexpr (CG == 2) {
               mma_commit_pair_mc(&sm.empty[stage], 0x3);
+              if constexpr (MX) {  // frees the scale-factor slot in both CTAs
+                mma_commit_pair_mc(&sm.sc_empty[sslot], 0x3);
+                ++sfc;
+              }
               if (FULL_K && kb == p.KB - 1) mma_commit_pair_mc(&sm.acc_full[buf], 0x3);
             } else {
               mma_commit(&sm.empty[stage]);
               if (FULL_K && kb == p.KB - 1) mma_commit(&sm.acc_full[buf]);
             }
             if (!FULL_K || kb == p.KB - 1) {
-              buf ^= 1;
-              if (buf == 0) bphase ^= 1u;
+              if (++buf == NACC) {
+                buf = 0;
+                bphase ^= 1u;
+              }
             }
             if (++stage == STAGES) {
               stage = 0;
@@ -389,6 +444,59 @@ __global__ void __launch_bounds__(384, 1)
         }
       }
       __syncwarp();
+    } else if constexpr (MX) {
+      // ---------------------------------------------------------- scale-factor producer (warps 2, 3)
+      // For each K block, this CTA's 128 row scales (x_scale) and the tile's
+      // two 128-column scales (w_scale) as e8m0 bytes in the chunk layout
+      // tcgen05.cp reads.  Both CTAs signal the leader's barrier; the MMA's
+      // commit frees the slot in both.  Rows and column blocks outside the
+      // problem get 2^0 (their operands are zero-filled).
+      const int t = threadIdx.x - 64;  // 0..63: rows t and t + 64
+      const uint32_t sc_full0 = CG == 2 ? mapa_shared(smem_u32(&sm.sc_full[0]), 0) : smem_u32(&sm.sc_full[0]);
+      uint32_t cnt = 0;  // K blocks staged so far (ring position)
+      bool ok = true;
+      for (int tile = unit; ok && tile < p.num_tiles; tile += units) {
+        const TileCoord tc = tile_coord(tile, p.grid_m, p.grid_n, p.group_m);
+        const int m0 = tc.pm * (BM * CG) + rank * BM, nb0 = tc.pn * 2;
+        const int ma = m0 + t, mc = m0 + t + 64;
+        for (int kb0 = 0; ok && kb0 < p.KB; kb0 += kScaleBatch) {
+          const int nb = p.KB - kb0 < kScaleBatch ? p.KB - kb0 : kScaleBatch;
+          uint32_t ea[kScaleBatch], ec[kScaleBatch], e0[kScaleBatch], e1[kScaleBatch];
+#pragma unroll
+          for (int i = 0; i < kScaleBatch; ++i) {
+            if (i < nb) {
+              const long long kb = kb0 + i;
+              ea[i] = ma < p.M ? __ldg(p.xs + (static_cast<long long>(ma) * p.G + tc.g) * p.KB + kb) : 127u;
+              ec[i] = mc < p.M ? __ldg(p.xs + (static_cast<long long>(mc) * p.G + tc.g) * p.KB + kb) : 127u;
+              e0[i] = nb0 < p.NB ? __ldg(p.ws + (static_cast<long long>(tc.g) * p.NB + nb0) * p.KB + kb) : 127u;
+              e1[i] = nb0 + 1 < p.NB ? __ldg(p.ws + (static_cast<long long>(tc.g) * p.NB + nb0 + 1) * p.KB + kb)
+                                     : 127u;
+            }
+          }
+#pragma unroll
+          for (int i = 0; i < kScaleBatch; ++i) {
+            if (i < nb) {
+              const uint32_t c = cnt + static_cast<uint32_t>(i);
+              const int slot = static_cast<int>(c % kSfRing);
+              if (!warp_wait(&sm.sc_empty[slot], ((c / kSfRing) & 1u) ^ 1u, abort, p.err,
+                             kErrTimeout | kRoleScale | kWaitScaleEmpty)) {
+                ok = false;
+                break;
+              }
+              uint32_t* sfa = reinterpret_cast<uint32_t*>(sm.sf[slot][0]);
+              uint32_t* sfb = reinterpret_cast<uint32_t*>(sm.sf[slot][1]);  // chunks 1 and 2: 256 words
+              sfa[4 * (t & 31) + (t >> 5)] = ea[i] * 0x01010101u;           // row t
+              sfa[4 * (t & 31) + (t >> 5) + 2] = ec[i] * 0x01010101u;       // row t + 64
+#pragma unroll
+              for (int q = 0; q < 4; ++q) sfb[t + 64 * q] = (q < 2 ? e0[i] : e1[i]) * 0x01010101u;
+              fence_proxy_async_smem();  // visible to tcgen05.cp
+              __syncwarp();
+              if (lane == 0) mbar_arrive_cluster(sc_full0 + static_cast<uint32_t>(slot * sizeof(uint64_t)));
+            }
+          }
+          cnt += static_cast<uint32_t>(nb);
+        }
+      }
     } else if (!FULL_K) {
       // ---------------------------------------------------------- scale producer (warps 2, 3)
       // Stages scale_a of this CTA's 128 rows and scale_b of the tile's two
@@ -545,6 +653,9 @@ __global__ void __launch_bounds__(384, 1)
           if constexpr (sizeof(OutT) == 4 && !std::is_same<OutT, float>::value) {
 #pragma unroll
             for (int j = 0; j < CPC; ++j) v[j] = __uint_as_float(r[j]);  // raw int32 accumulator
+          } else if constexpr (MX) {
+#pragma unroll
+            for (int j = 0; j < CPC; ++j) v[j] = __uint_as_float(r[j]);  // scales already applied
           } else if constexpr (!IS_INT8) {
             // FP8 rowwise / tensorwise: acc * (s_a * s_b) + bias[n]
 #pragma unroll
@@ -578,8 +689,10 @@ __global__ void __launch_bounds__(384, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(acc_empty0 + static_cast<uint32_t>(buf * sizeof(uint64_t)));
-        buf ^= 1;
-        if (buf == 0) bphase ^= 1u;
+        if (++buf == NACC) {
+          buf = 0;
+          bphase ^= 1u;
+        }
       }
     }
     if (lane == 0) bulk_wait_all();

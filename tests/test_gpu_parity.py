@@ -291,6 +291,19 @@ def test_bmm_n_not_multiple_of_four(M, G, N, path):
 def test_bmm_both_kernels_agree_with_oracle(path):
     d = wl.bmm_inputs(200, 3, 384, 512, seed=81)
     y, S = oracle.bmm_blockscale(d["x"], d["w"], d["x_scale"], d["w_scale"])
-    for k in (bs.PATH_WIDE, bs.PATH_WIDE_SINGLE, bs.PATH_SKINNY):
+    for k in (bs.PATH_WIDE, bs.PATH_WIDE_PROMOTE, bs.PATH_WIDE_SINGLE, bs.PATH_SKINNY):
         path(k)
         fp8_check(bmm_run(d), y, S, torch.bfloat16, f"bmm kernel={k}")
+
+
+@pytest.mark.parametrize("M,G,N,K", [(300, 2, 520, 640), (1024, 3, 264, 1280), (513, 1, 1024, 4096)])
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_bmm_block_scaled_mma_and_promotion(M, G, N, K, out_dtype, path):
+    """CTA pairs apply the e8m0 scales in the tensor core (block-scaled MMA);
+    path 4 promotes every 128-deep block on the CUDA cores instead.  Both meet
+    the bound, on ragged M, N and K tails and partial column blocks."""
+    d = wl.bmm_inputs(M, G, N, K, seed=86 + M + N + K)
+    y, S = oracle.bmm_blockscale(d["x"], d["w"], d["x_scale"], d["w_scale"])
+    for k in (bs.PATH_WIDE, bs.PATH_WIDE_PROMOTE):
+        path(k)
+        fp8_check(bmm_run(d, out_dtype), y, S, out_dtype, f"bmm {M}x{G}x{N}x{K} kernel={k}")
