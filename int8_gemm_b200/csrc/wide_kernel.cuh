@@ -29,10 +29,11 @@
 // two, so the tensor core applies them itself -- per K block the MMA thread
 // copies the scale factors of the pair's 256 rows and 256 columns from
 // shared memory into TMEM (tcgen05.cp) and issues block-scaled MMAs that
-// accumulate over all of K.  The second half of TMEM holds the scale factors,
-// so one accumulator buffer remains and the epilogue does not overlap the
-// next tile.  The power-of-two scales make every product exact, so this sums
-// the same terms as the per-block promotion, in a different order.
+// accumulate over all of K.  To leave room for the scale factors the two
+// accumulator buffers overlap in 32 columns: the epilogue reads those first
+// and releases them early, so it still overlaps the next tile's MMAs.  The
+// power-of-two scales make every product exact, so this sums the same terms
+// as the per-block promotion, in a different order.
 // INT8 mode: s8 x s8 -> s32 accumulates over all of K in TMEM (double-buffered
 // across tiles); the epilogue computes (float(acc) * s_a[m]) * s_b[n] with two
 // round-to-nearest fp32 multiplies.
@@ -92,8 +93,10 @@ struct GemmArgs {
 // offsets in the peer.
 constexpr int kScaleRing = 16;  // K blocks of scales staged ahead of the consumers
 constexpr int kScaleBatch = 8;  // K blocks whose scale loads are in flight together
-constexpr int kSfRing = 5;      // kFp8Mx: K blocks of scale-factor chunks staged ahead of the MMA
-constexpr uint32_t kSfaCol = 256, kSfbCol = 260;  // kFp8Mx: TMEM columns of the scale factors
+constexpr int kSfRing = 5;      // kFp8Mx: scale-factor slots (four K blocks each) staged ahead of the MMA
+// kFp8Mx TMEM columns: accumulator buffer 1 starts at kAcc1Col, so the two
+// 256-column buffers share 32 columns and the scale factors fit behind them.
+constexpr uint32_t kAcc1Col = 224, kSfaCol = 480, kSfbCol = 484;
 
 template <int BNL, int STAGES>
 struct WideSmem {
@@ -102,10 +105,11 @@ struct WideSmem {
   uint8_t stage_out[8][32 * 64];  // per consumer warp: 32 rows x 64 bytes, 64-byte swizzle
   union {
     float sa[kScaleRing][128];  // scale_a of this CTA's rows, per K block
-    // kFp8Mx, per K block: three 512-byte scale-factor chunks (this CTA's 128
-    // rows of A; B columns 0-127; B columns 128-255), each 32 lanes x 16 bytes
-    // as tcgen05.cp reads them: item i at byte 16*(i%32) + 4*(i/32), its
-    // byte repeated for the four 32-deep sub-blocks
+    // kFp8Mx, per four K blocks: three 512-byte scale-factor chunks (this
+    // CTA's 128 rows of A; B columns 0-127; B columns 128-255), each 32 lanes
+    // x 16 bytes as tcgen05.cp reads them: item i in the 32-bit word at byte
+    // 16*(i%32) + 4*(i/32), byte j of that word for the slot's K block j (the
+    // MMAs of K block kb select byte kb % 4 through the scale-factor ids)
     alignas(16) uint8_t sf[kSfRing][3][512];
   };
   float sb[kScaleRing][4];       // scale_b of the tile's two 128-column blocks, per K block
@@ -113,6 +117,7 @@ struct WideSmem {
   uint64_t empty[STAGES];
   uint64_t acc_full[2];   // INT8: tile accumulator complete (FP8 uses the stage barriers)
   uint64_t acc_empty[2];  // accumulator buffer released by every consumer warp (of both CTAs)
+  uint64_t ovl_empty[2];  // kFp8Mx: the buffer's 32 shared columns read by the warps holding them
   uint64_t sc_full[kScaleRing];
   uint64_t sc_empty[kScaleRing];
   uint64_t drain;
@@ -226,8 +231,9 @@ __global__ void __launch_bounds__(384, 1)
   constexpr bool IS_INT8 = MODE == Mode::kInt8;
   constexpr bool MX = MODE == Mode::kFp8Mx;  // block scales applied by the tensor core
   constexpr bool FULL_K = IS_INT8 || MODE == Mode::kFp8Rowwise || MX;  // accumulate over all of K in TMEM
-  // accumulator buffers; kFp8Mx keeps the second half of TMEM for the scale factors
-  constexpr int NACC = MX ? 1 : 2;
+  constexpr int NACC = 2;  // accumulator buffers
+  // first TMEM column of accumulator buffer b (kFp8Mx: the buffers overlap)
+  auto acc_col = [](int b) -> uint32_t { return MX ? (b ? kAcc1Col : 0u) : static_cast<uint32_t>(b * BN); };
   constexpr uint32_t IDESC = IS_INT8 ? idesc_s8_s32<BM * CG, BN>()
                                      : (MX ? idesc_mx_e4m3_f32<BM * CG, BN>() : idesc_e4m3_f32<BM * CG, BN>());
   static_assert(!MX || CG == 2, "hardware block scaling is built for CTA pairs");
@@ -257,6 +263,7 @@ __global__ void __launch_bounds__(384, 1)
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sm.acc_full[b], 1);
       mbar_init(&sm.acc_empty[b], CONSUMER_WARPS * CG);
+      mbar_init(&sm.ovl_empty[b], (CONSUMER_WARPS / 2) * CG);  // the half holding the shared columns
     }
     for (int i = 0; i < kScaleRing; ++i) {
       // FP8 block scales: every thread of the two scale warps fills, the
@@ -352,7 +359,7 @@ __global__ void __launch_bounds__(384, 1)
       if (lane == 0 && leader) {
         int stage = 0, buf = 0;
         uint32_t phase = 0, bphase = 0;
-        uint32_t sfc = 0;  // kFp8Mx: K blocks whose scale factors were consumed (ring position)
+        uint32_t sfc = 0;  // kFp8Mx: scale-factor slots consumed (ring position)
         bool ok = true;
         for (int tile = unit; ok && tile < p.num_tiles; tile += units) {
           for (int kb = 0; kb < p.KB; ++kb) {
@@ -363,30 +370,41 @@ __global__ void __launch_bounds__(384, 1)
                 ok = false;
                 break;
               }
+              // kFp8Mx: the previous tile, in the other buffer, has also read
+              // the columns the two buffers share
+              if (MX && !wait_bounded(&sm.ovl_empty[buf ^ 1], buf == 1 ? bphase : (bphase ^ 1u), abort, p.err,
+                                      kErrTimeout | kRoleMma | kWaitAccEmpty)) {
+                ok = false;
+                break;
+              }
             }
             if (!wait_bounded(&sm.full[stage], phase, abort, p.err, kErrTimeout | kRoleMma | kWaitStageFull)) {
               ok = false;
               break;
             }
             const int sslot = static_cast<int>(sfc % kSfRing);
-            if constexpr (MX) {  // both CTAs' scale-factor chunks of this K block are in shared memory
-              if (!wait_bounded<true>(&sm.sc_full[sslot], (sfc / kSfRing) & 1u, abort, p.err,
-                                      kErrTimeout | kRoleMma | kWaitScaleFull)) {
+            const uint32_t sf_id = static_cast<uint32_t>(kb & 3);  // kFp8Mx: this K block's byte in the slot
+            if constexpr (MX) {  // both CTAs' scale factors of K blocks kb..kb+3 are in shared memory
+              if (sf_id == 0 && !wait_bounded<true>(&sm.sc_full[sslot], (sfc / kSfRing) & 1u, abort, p.err,
+                                                    kErrTimeout | kRoleMma | kWaitScaleFull)) {
                 ok = false;
                 break;
               }
             }
             tc_fence_after();
-            const uint32_t d = tmem + static_cast<uint32_t>(buf * BN);
+            const uint32_t d = tmem + acc_col(buf);
             const uint64_t ad = sdesc_k_sw128(smem_u32(sm.a[stage]));
             const uint64_t bd = sdesc_k_sw128(smem_u32(sm.b[stage]));
             if constexpr (MX) {
-              // scale factors to TMEM; issued by this thread, they are ordered
-              // after the previous K block's MMAs and before this block's
-              const uint32_t sf0 = smem_u32(sm.sf[sslot][0]);
-              tmem_cp_32x128b_x4_pair(tmem + kSfaCol, sdesc_k_plain(sf0, 128));
-              tmem_cp_32x128b_x4_pair(tmem + kSfbCol, sdesc_k_plain(sf0 + 512, 128));
-              tmem_cp_32x128b_x4_pair(tmem + kSfbCol + 4, sdesc_k_plain(sf0 + 1024, 128));
+              if (sf_id == 0) {
+                // scale factors of four K blocks to TMEM; issued by this
+                // thread, the copies are ordered after the previous blocks'
+                // MMAs and before this block's
+                const uint32_t sf0 = smem_u32(sm.sf[sslot][0]);
+                tmem_cp_32x128b_x4_pair(tmem + kSfaCol, sdesc_k_plain(sf0, 128));
+                tmem_cp_32x128b_x4_pair(tmem + kSfbCol, sdesc_k_plain(sf0 + 512, 128));
+                tmem_cp_32x128b_x4_pair(tmem + kSfbCol + 4, sdesc_k_plain(sf0 + 1024, 128));
+              }
             }
 #pragma unroll
             for (int k = 0; k < BK / 32; ++k) {
@@ -395,7 +413,8 @@ __global__ void __launch_bounds__(384, 1)
                 if constexpr (IS_INT8) {
                   mma_i8_pair(d, ad + 2 * k, bd + 2 * k, IDESC, acc);
                 } else if constexpr (MX) {
-                  mma_mxf8f6f4_pair(d, ad + 2 * k, bd + 2 * k, IDESC, tmem + kSfaCol, tmem + kSfbCol, acc);
+                  mma_mxf8f6f4_pair(d, ad + 2 * k, bd + 2 * k, IDESC | (sf_id << 29) | (sf_id << 4),
+                                    tmem + kSfaCol, tmem + kSfbCol, acc);
                 } else {
                   mma_f8f6f4_pair(d, ad + 2 * k, bd + 2 * k, IDESC, acc);
                 }
@@ -412,9 +431,11 @@ __global__ void __launch_bounds__(384, 1)
             // tile's last K block also commits the accumulator barrier.
             if constexpr (CG == 2) {
               mma_commit_pair_mc(&sm.empty[stage], 0x3);
-              if constexpr (MX) {  // frees the scale-factor slot in both CTAs
-                mma_commit_pair_mc(&sm.sc_empty[sslot], 0x3);
-                ++sfc;
+              if constexpr (MX) {  // after the slot's last K block: free it in both CTAs
+                if (sf_id == 3 || kb == p.KB - 1) {
+                  mma_commit_pair_mc(&sm.sc_empty[sslot], 0x3);
+                  ++sfc;
+                }
               }
               if (FULL_K && kb == p.KB - 1) mma_commit_pair_mc(&sm.acc_full[buf], 0x3);
             } else {
@@ -446,55 +467,58 @@ __global__ void __launch_bounds__(384, 1)
       __syncwarp();
     } else if constexpr (MX) {
       // ---------------------------------------------------------- scale-factor producer (warps 2, 3)
-      // For each K block, this CTA's 128 row scales (x_scale) and the tile's
-      // two 128-column scales (w_scale) as e8m0 bytes in the chunk layout
-      // tcgen05.cp reads.  Both CTAs signal the leader's barrier; the MMA's
-      // commit frees the slot in both.  Rows and column blocks outside the
-      // problem get 2^0 (their operands are zero-filled).
+      // For every four K blocks of a tile, this CTA's 128 row scales
+      // (x_scale) and the tile's two 128-column scales (w_scale) as e8m0
+      // bytes in the chunk layout tcgen05.cp reads, byte j of each word for
+      // the slot's K block j.  Both CTAs signal the leader's barrier; the
+      // MMA's commit frees the slot in both.  Rows, column blocks and K blocks
+      // outside the problem get 2^0 (their operands are zero-filled or their
+      // byte is never selected).
       const int t = threadIdx.x - 64;  // 0..63: rows t and t + 64
       const uint32_t sc_full0 = CG == 2 ? mapa_shared(smem_u32(&sm.sc_full[0]), 0) : smem_u32(&sm.sc_full[0]);
-      uint32_t cnt = 0;  // K blocks staged so far (ring position)
+      uint32_t cnt = 0;  // slots staged so far (ring position)
       bool ok = true;
       for (int tile = unit; ok && tile < p.num_tiles; tile += units) {
         const TileCoord tc = tile_coord(tile, p.grid_m, p.grid_n, p.group_m);
         const int m0 = tc.pm * (BM * CG) + rank * BM, nb0 = tc.pn * 2;
         const int ma = m0 + t, mc = m0 + t + 64;
-        for (int kb0 = 0; ok && kb0 < p.KB; kb0 += kScaleBatch) {
-          const int nb = p.KB - kb0 < kScaleBatch ? p.KB - kb0 : kScaleBatch;
-          uint32_t ea[kScaleBatch], ec[kScaleBatch], e0[kScaleBatch], e1[kScaleBatch];
+        for (int kb0 = 0; ok && kb0 < p.KB; kb0 += 4) {
+          // the 16 loads of a slot are in flight together
+          uint32_t wa = 0, wc = 0, w0 = 0, w1 = 0;
 #pragma unroll
-          for (int i = 0; i < kScaleBatch; ++i) {
-            if (i < nb) {
-              const long long kb = kb0 + i;
-              ea[i] = ma < p.M ? __ldg(p.xs + (static_cast<long long>(ma) * p.G + tc.g) * p.KB + kb) : 127u;
-              ec[i] = mc < p.M ? __ldg(p.xs + (static_cast<long long>(mc) * p.G + tc.g) * p.KB + kb) : 127u;
-              e0[i] = nb0 < p.NB ? __ldg(p.ws + (static_cast<long long>(tc.g) * p.NB + nb0) * p.KB + kb) : 127u;
-              e1[i] = nb0 + 1 < p.NB ? __ldg(p.ws + (static_cast<long long>(tc.g) * p.NB + nb0 + 1) * p.KB + kb)
-                                     : 127u;
-            }
+          for (int j = 0; j < 4; ++j) {
+            const long long kb = kb0 + j;
+            const bool in_k = kb < p.KB;
+            const uint32_t a = in_k && ma < p.M ? __ldg(p.xs + (static_cast<long long>(ma) * p.G + tc.g) * p.KB + kb)
+                                                : 127u;
+            const uint32_t c = in_k && mc < p.M ? __ldg(p.xs + (static_cast<long long>(mc) * p.G + tc.g) * p.KB + kb)
+                                                : 127u;
+            const uint32_t b0 =
+                in_k && nb0 < p.NB ? __ldg(p.ws + (static_cast<long long>(tc.g) * p.NB + nb0) * p.KB + kb) : 127u;
+            const uint32_t b1 = in_k && nb0 + 1 < p.NB
+                                    ? __ldg(p.ws + (static_cast<long long>(tc.g) * p.NB + nb0 + 1) * p.KB + kb)
+                                    : 127u;
+            wa |= a << (8 * j);
+            wc |= c << (8 * j);
+            w0 |= b0 << (8 * j);
+            w1 |= b1 << (8 * j);
           }
-#pragma unroll
-          for (int i = 0; i < kScaleBatch; ++i) {
-            if (i < nb) {
-              const uint32_t c = cnt + static_cast<uint32_t>(i);
-              const int slot = static_cast<int>(c % kSfRing);
-              if (!warp_wait(&sm.sc_empty[slot], ((c / kSfRing) & 1u) ^ 1u, abort, p.err,
-                             kErrTimeout | kRoleScale | kWaitScaleEmpty)) {
-                ok = false;
-                break;
-              }
-              uint32_t* sfa = reinterpret_cast<uint32_t*>(sm.sf[slot][0]);
-              uint32_t* sfb = reinterpret_cast<uint32_t*>(sm.sf[slot][1]);  // chunks 1 and 2: 256 words
-              sfa[4 * (t & 31) + (t >> 5)] = ea[i] * 0x01010101u;           // row t
-              sfa[4 * (t & 31) + (t >> 5) + 2] = ec[i] * 0x01010101u;       // row t + 64
-#pragma unroll
-              for (int q = 0; q < 4; ++q) sfb[t + 64 * q] = (q < 2 ? e0[i] : e1[i]) * 0x01010101u;
-              fence_proxy_async_smem();  // visible to tcgen05.cp
-              __syncwarp();
-              if (lane == 0) mbar_arrive_cluster(sc_full0 + static_cast<uint32_t>(slot * sizeof(uint64_t)));
-            }
+          const int slot = static_cast<int>(cnt % kSfRing);
+          if (!warp_wait(&sm.sc_empty[slot], ((cnt / kSfRing) & 1u) ^ 1u, abort, p.err,
+                         kErrTimeout | kRoleScale | kWaitScaleEmpty)) {
+            ok = false;
+            break;
           }
-          cnt += static_cast<uint32_t>(nb);
+          uint32_t* sfa = reinterpret_cast<uint32_t*>(sm.sf[slot][0]);
+          uint32_t* sfb = reinterpret_cast<uint32_t*>(sm.sf[slot][1]);  // chunks 1 and 2: 256 words
+          sfa[4 * (t & 31) + (t >> 5)] = wa;      // row t
+          sfa[4 * (t & 31) + (t >> 5) + 2] = wc;  // row t + 64
+#pragma unroll
+          for (int q = 0; q < 4; ++q) sfb[t + 64 * q] = q < 2 ? w0 : w1;
+          fence_proxy_async_smem();  // visible to tcgen05.cp
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(sc_full0 + static_cast<uint32_t>(slot * sizeof(uint64_t)));
+          ++cnt;
         }
       }
     } else if (!FULL_K) {
@@ -553,6 +577,8 @@ __global__ void __launch_bounds__(384, 1)
     // release target of this warpgroup's accumulator half: the leader's barrier
     const uint32_t acc_empty0 =
         CG == 2 ? mapa_shared(smem_u32(&sm.acc_empty[0]), 0) : smem_u32(&sm.acc_empty[0]);
+    const uint32_t ovl_empty0 =
+        CG == 2 ? mapa_shared(smem_u32(&sm.ovl_empty[0]), 0) : smem_u32(&sm.ovl_empty[0]);
     int buf = 0, sslot = 0;
     uint32_t bphase = 0, ssph = 0;
     uint32_t kbc = 0;  // K blocks of this CTA's tiles seen so far (stage = kbc % STAGES)
@@ -637,17 +663,31 @@ __global__ void __launch_bounds__(384, 1)
         // FP8 rowwise: this thread's column scales start at s_col_n and advance by col_step
         const int col_step = !IS_INT8 && p.s_col_stride != 0 ? 1 : 0;
         const float* s_col_n = IS_INT8 ? nullptr : p.s_col + ncol0 * col_step;
-        const uint32_t tb = tmem + t_lane + static_cast<uint32_t>(buf * BN + half * 128);
+        const uint32_t tb = tmem + t_lane + acc_col(buf) + static_cast<uint32_t>(half * 128);
+        // kFp8Mx: the 32 columns this buffer shares with the other one are
+        // the last of half 1 (buffer 0) or the first of half 0 (buffer 1);
+        // the warps holding them read those chunks first and release them,
+        // so the next tile's MMAs can start while the rest drains
+        constexpr int NCH = 128 / CPC, OVC = 32 / CPC;
+        const bool ovl_here = MX && (buf == 0 ? half == 1 : half == 0);
+        const int rot = MX && buf == 0 && half == 1 ? NCH - OVC : 0;
 #pragma unroll
-        for (int ch = 0; ch < 128 / CPC; ++ch) {
+        for (int ch = 0; ch < NCH; ++ch) {
           if (lane == 0) bulk_wait_read_all();
           __syncwarp();
-          const int c0 = ch * CPC;
+          const int c0 = (MX ? (ch + rot) % NCH : ch) * CPC;
           uint32_t r[CPC];
           if constexpr (CPC == 32) {
             tmem_ld32(tb + c0, r);
           } else {
             tmem_ld16(tb + c0, r);
+          }
+          if constexpr (MX) {
+            if (ovl_here && ch == OVC - 1) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive_cluster(ovl_empty0 + static_cast<uint32_t>(buf * sizeof(uint64_t)));
+            }
           }
           float v[CPC];
           if constexpr (sizeof(OutT) == 4 && !std::is_same<OutT, float>::value) {
@@ -681,8 +721,8 @@ __global__ void __launch_bounds__(384, 1)
           stage_row64<OutT, CPC>(stg, lane, v);
           fence_proxy_async_smem();
           __syncwarp();
-          if (lane == 0 && m0 + lg * 32 < p.M && ncol0 + ch * CPC < p.N) {
-            tma_store_3d(&tmD, stg, ncol0 + ch * CPC, m0 + lg * 32, tc.g);
+          if (lane == 0 && m0 + lg * 32 < p.M && ncol0 + c0 < p.N) {
+            tma_store_3d(&tmD, stg, ncol0 + c0, m0 + lg * 32, tc.g);
             bulk_commit();
           }
         }
