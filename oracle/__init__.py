@@ -17,6 +17,11 @@ Parity status of each function (what pins it in ``tests/test_oracle_pins.py``):
   int_scaled_mm     -- bit-exact against torch._int_mm and torch fp32 ops on CPU
   bmm_blockscale    -- fp64 einsum of bf16-dequantised operands, per-g agreement
                        with fp8_blockwise, one-hot w_scale orientation
+  e4m3_encode       -- round trip of every finite code, midpoints (ties to the
+                       even code), saturation; torch's float8_e4m3fn cast
+  quantize_1x128    -- torch's float8_e4m3fn cast of x / scale (the library
+                       routine the recipe reduces to), amax -> +-448, zero
+                       groups, e8m0 exponent at and around 448 * 2^e, ragged K
 """
 from __future__ import annotations
 
@@ -62,7 +67,10 @@ def _load():
                                                i64, i64, i64, i64, p, i64, p, p]
             lib.orc_int_scaled_mm.argtypes = [p, i64, p, i64, p, p, i64, i64, i64, p, i64, p, p, p]
             lib.orc_fp8_rowwise.argtypes = [p, i64, p, i64, p, i64, p, i64, p, i64, i64, i64, p, i64, p, p]
-            for f in (lib.orc_fp8_blockwise, lib.orc_bmm_blockscale, lib.orc_int_scaled_mm, lib.orc_fp8_rowwise):
+            lib.orc_e4m3_encode.argtypes = [p, p, i64]
+            lib.orc_quantize_1x128.argtypes = [p, i64, i64, i64, ctypes.c_int, p, i64, p, p]
+            for f in (lib.orc_fp8_blockwise, lib.orc_bmm_blockscale, lib.orc_int_scaled_mm, lib.orc_fp8_rowwise,
+                      lib.orc_quantize_1x128):
                 f.restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -223,3 +231,31 @@ def fp8_rowwise(A, B_t, scale_a, scale_b, bias=None, rows=None):
     if rc != 0:
         raise ValueError(f"oracle fp8_rowwise failed with code {rc}")
     return y, S
+
+
+def e4m3_encode(v) -> np.ndarray:
+    """fp64 values -> e4m3 codes (uint8): round to nearest, ties to the even
+    code, |v| >= 448 saturates to +-448, NaN -> 0x7F."""
+    v = np.ascontiguousarray(_np(v), dtype=np.float64)
+    out = np.empty(v.shape, dtype=np.uint8)
+    _load().orc_e4m3_encode(_ptr(v), _ptr(out), v.size)
+    return out
+
+
+def quantize_1x128(x, fmt: int = 0):
+    """1x128 group quantisation of x [M, K] (fp32 or bf16, any row stride).
+
+    fmt 0: returns (codes uint8 [M, K], scale fp32 [M, ceil(K/128)]), scale = amax / 448;
+    fmt 1: returns (codes, e8m0 bytes uint8 [M, ceil(K/128)]).  See orc_quantize_1x128."""
+    xt = _np(x.float() if hasattr(x, "float") and not isinstance(x, np.ndarray) else x)
+    xt = np.ascontiguousarray(xt, dtype=np.float32)
+    assert xt.ndim == 2
+    M, K = xt.shape
+    KB = -(-K // 128)
+    q = np.empty((M, K), dtype=np.uint8)
+    sf = np.empty((M, KB), dtype=np.float32) if fmt == 0 else None
+    se = np.empty((M, KB), dtype=np.uint8) if fmt == 1 else None
+    rc = _load().orc_quantize_1x128(_ptr(xt), M, K, K, fmt, _ptr(q), K, _ptr(sf), _ptr(se))
+    if rc != 0:
+        raise ValueError(f"orc_quantize_1x128 failed ({rc})")
+    return q, (sf if fmt == 0 else se)

@@ -349,3 +349,93 @@ int orc_int_scaled_mm(const int8_t *A, int64_t lda, const int8_t *B, int64_t ldb
     }
     return overflow ? ORC_ERR_OVERFLOW : ORC_OK;
 }
+
+/*
+ * e4m3 encoding with round-to-nearest-even and saturation, straight from the
+ * decode table: the finite magnitudes are the table values of codes 0..126
+ * (ascending); v is mapped to the nearest one, a tie to the code with an even
+ * mantissa (last bit 0), anything beyond 448 to 448, NaN to 0x7F.  The sign
+ * is carried separately (so -0.0 and values rounding to zero keep the sign
+ * bit, as the format's own conversion does).
+ */
+uint8_t orc_e4m3_from_f64(double v)
+{
+    build_e4m3_table();
+    if (isnan(v)) return 0x7F;
+    const uint8_t sign = signbit(v) ? 0x80 : 0x00;
+    const double a = fabs(v);
+    if (a >= 448.0) return sign | 0x7E;                 /* saturation */
+    int lo = 0, hi = 126;                                /* table[lo] <= a < table[hi] */
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) / 2;
+        if (e4m3_value[mid] <= a) lo = mid; else hi = mid;
+    }
+    const double dlo = a - e4m3_value[lo], dhi = e4m3_value[hi] - a;
+    int code;
+    if (dlo < dhi) code = lo;
+    else if (dhi < dlo) code = hi;
+    else code = (lo & 1) ? hi : lo;                      /* tie: even mantissa */
+    return sign | (uint8_t)code;
+}
+
+void orc_e4m3_encode(const double *v, uint8_t *out, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = orc_e4m3_from_f64(v[i]);
+}
+
+/*
+ * 1x128 activation-group quantisation (the recipe the blockwise operation's
+ * inputs follow): for row m and group g (elements 128g .. min(128g+128, K)-1)
+ *   amax = max |x|
+ *   fmt 0: scale = fp32(amax / 448) (1 when amax == 0),
+ *          q = e4m3_rne(sat(fp32(x / scale)))
+ *   fmt 1: e = the smallest integer with amax <= 448 * 2^e, i.e.
+ *          ceil(log2(amax / 448)) (0 when amax == 0); byte = clamp(e + 127,
+ *          0, 254); q = e4m3_rne(sat(x * 2^-(byte - 127)))
+ * x is fp32 here (bf16 inputs widen exactly).  scale_f32 / scale_e8m0 are
+ * [M, ceil(K/128)] row-major; q is [M, K] with row stride ldq.
+ *   Sources: pytorch issue "torch._scaled_mm with blockwise scaling doesn't
+ *   work with torch.compile" (1x128 groups of A with an fp32 scale each,
+ *   scale_a [M, K/128]); ROCm/aiter PR "Add opus fp8 mxscale BMM kernels for
+ *   gfx950" (e8m0 power-of-two scales per 128-element group).  The amax / 448
+ *   scale and the saturating RNE cast are the plain reading of "scaled e4m3":
+ *   448 is the largest finite e4m3 magnitude.
+ */
+int orc_quantize_1x128(const float *x, int64_t M, int64_t K, int64_t ldx, int fmt,
+                       uint8_t *q, int64_t ldq, float *scale_f32, uint8_t *scale_e8m0)
+{
+    if (M < 0 || K < 0 || ldx < K || ldq < K || (fmt != 0 && fmt != 1)) return ORC_ERR_SHAPE;
+    const int64_t KB = (K + 127) / 128;
+#pragma omp parallel for schedule(dynamic, 16)
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t g = 0; g < KB; ++g) {
+            const int64_t k0 = 128 * g, k1 = k0 + 128 < K ? k0 + 128 : K;
+            float amax = 0.0f;
+            for (int64_t k = k0; k < k1; ++k) {
+                const float a = fabsf(x[m * ldx + k]);
+                if (a > amax) amax = a;
+            }
+            if (fmt == 0) {
+                const float s = amax == 0.0f ? 1.0f : amax / 448.0f;
+                scale_f32[m * KB + g] = s;
+                for (int64_t k = k0; k < k1; ++k) {
+                    const float v = x[m * ldx + k] / s;
+                    q[m * ldq + k] = orc_e4m3_from_f64((double)v);
+                }
+            } else {
+                int e = 0;
+                if (amax != 0.0f) {
+                    e = ilogb((double)amax) - 10;                /* 448 * 2^e < amax here */
+                    while (!((double)amax <= ldexp(448.0, e))) ++e;
+                }
+                int byte = e + 127;
+                if (byte < 0) byte = 0;
+                if (byte > 254) byte = 254;
+                scale_e8m0[m * KB + g] = (uint8_t)byte;
+                for (int64_t k = k0; k < k1; ++k)
+                    q[m * ldq + k] = orc_e4m3_from_f64(ldexp((double)x[m * ldx + k], -(byte - 127)));
+            }
+        }
+    }
+    return ORC_OK;
+}

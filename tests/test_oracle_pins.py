@@ -412,3 +412,122 @@ def test_oracle_rows_subset_matches_full():
     ys, Ss = oracle.fp8_blockwise(d["A"], d["B_t"], d["scale_a"], d["scale_b"], rows=[39, 0, 17])
     np.testing.assert_array_equal(ys, y[[39, 0, 17]])
     np.testing.assert_array_equal(Ss, S[[39, 0, 17]])
+
+
+# ---------------------------------------------------------------------------
+# e4m3 encoding and the 1x128 activation quantiser (fused-quantiser operation)
+# ---------------------------------------------------------------------------
+def _finite_magnitudes():
+    t = oracle.e4m3_table()
+    return t[:127]  # codes 0..126: 0, subnormals, normals up to 448, ascending
+
+
+def test_e4m3_encode_round_trips_every_finite_code():
+    t = oracle.e4m3_table()
+    codes = np.array([c for c in range(256) if not math.isnan(t[c])], dtype=np.uint8)
+    assert np.array_equal(oracle.e4m3_encode(t[codes]), codes)
+
+
+def test_e4m3_encode_midpoints_go_to_the_even_code_and_neighbours_to_the_nearest():
+    mags = _finite_magnitudes()
+    for c in range(126):
+        lo, hi = mags[c], mags[c + 1]
+        mid = (lo + hi) / 2  # exact in fp64
+        even = c if c % 2 == 0 else c + 1
+        assert oracle.e4m3_encode([mid])[0] == even, (c, mid)
+        assert oracle.e4m3_encode([-mid])[0] == 0x80 | even
+        assert oracle.e4m3_encode([np.nextafter(mid, 0)])[0] == c
+        assert oracle.e4m3_encode([np.nextafter(mid, 1e9)])[0] == c + 1
+
+
+def test_e4m3_encode_saturates_and_keeps_nan():
+    enc = oracle.e4m3_encode([448.0, 460.0, 464.0, 1e30, -1e30, -448.0, float("nan")])
+    assert list(enc) == [0x7E, 0x7E, 0x7E, 0x7E, 0xFE, 0xFE, 0x7F]
+
+
+def test_e4m3_encode_agrees_with_torch_cast_inside_the_range():
+    g = torch.Generator().manual_seed(7)
+    v = (torch.randn(200000, generator=g, dtype=torch.float64) * torch.pow(2.0, torch.randint(-12, 9, (200000,), generator=g)))
+    v = v.clamp(-448, 448)
+    ref = v.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(oracle.e4m3_encode(v.numpy()), ref)
+
+
+def _torch_quantize_f32(x):
+    """The recipe through torch's own cast: scale = amax / 448 (1 if 0), codes = cast(sat(x / scale))."""
+    M, K = x.shape
+    KB = -(-K // 128)
+    xp = torch.zeros(M, KB * 128)
+    xp[:, :K] = x
+    amax = xp.view(M, KB, 128).abs().amax(-1)
+    s = amax / 448.0
+    s[amax == 0] = 1.0
+    q = (xp / s.repeat_interleave(128, 1)).clamp(-448, 448).to(torch.float8_e4m3fn).view(torch.uint8)
+    return q[:, :K].numpy(), s.numpy()
+
+
+@pytest.mark.parametrize("M,K", [(3, 128), (5, 300), (2, 1000)])
+def test_quantize_fp32_scale_matches_torch_cast_of_x_over_scale(M, K):
+    x = wl.normal_with_outliers((M, K), 4321 + K)
+    q, s = oracle.quantize_1x128(x, 0)
+    rq, rs = _torch_quantize_f32(x)
+    assert s.dtype == np.float32 and s.shape == (M, -(-K // 128))
+    assert np.array_equal(s, rs) and np.array_equal(q, rq)
+
+
+def test_quantize_group_amax_maps_to_448_and_zero_groups_get_scale_one():
+    x = torch.zeros(2, 256)
+    x[0, :128] = torch.linspace(-3.0, 2.0, 128)
+    x[1, 128:] = torch.linspace(0.5, 7.0, 128)
+    q, s = oracle.quantize_1x128(x, 0)
+    assert q[0, 0] == 0xFE  # -3.0 is the group's amax, negative
+    assert q[1, 255] == 0x7E
+    assert s[0, 1] == 1.0 and s[1, 0] == 1.0 and np.all(q[0, 128:] == 0) and np.all(q[1, :128] == 0)
+    assert s[0, 0] == np.float32(3.0) / np.float32(448.0)
+    # a 1x128 group is one scale: rows and groups do not mix
+    q2, s2 = oracle.quantize_1x128(x[:, :128], 0)
+    assert np.array_equal(q2, q[:, :128]) and np.array_equal(s2[:, 0], s[:, 0])
+
+
+def test_quantize_e8m0_exponent_at_and_around_448_times_powers_of_two():
+    cases = []
+    for k in (-20, -3, 0, 1, 5, 40):
+        exact = 448.0 * 2.0 ** k
+        cases += [(exact, 127 + k),
+                  (float(np.nextafter(np.float32(exact), np.float32(1e38))), 128 + k),
+                  (float(np.float32(exact * 0.6)), 127 + k),
+                  (float(np.float32(exact * 0.5)), 126 + k)]
+    x = torch.zeros(len(cases), 128)
+    for i, (amax, _) in enumerate(cases):
+        x[i, 0] = amax
+        x[i, 1] = -amax / 3
+    q, e = oracle.quantize_1x128(x, 1)
+    assert [int(b) for b in e[:, 0]] == [b for _, b in cases]
+    for i, (amax, byte) in enumerate(cases):
+        assert q[i, 0] == oracle.e4m3_encode([amax * 2.0 ** -(byte - 127)])[0]
+    assert oracle.quantize_1x128(torch.zeros(1, 128), 1)[1][0, 0] == 127
+
+
+@pytest.mark.parametrize("M,K", [(4, 256), (3, 777)])
+def test_quantize_e8m0_matches_the_bmm_recipe_through_torch_cast(M, K):
+    x = wl.normal_with_outliers((M, K), 99 + K)
+    q, e = oracle.quantize_1x128(x, 1)
+    KB = -(-K // 128)
+    xp = torch.zeros(M, KB * 128)
+    xp[:, :K] = x
+    amax = xp.view(M, KB, 128).abs().amax(-1).double()
+    # ceil(log2(amax / 448)) in exact rational arithmetic
+    want = np.zeros((M, KB), dtype=np.int64)
+    for i in range(M):
+        for g in range(KB):
+            a = Fraction(float(amax[i, g]))
+            ee = 0
+            if a > 0:
+                ee = math.floor(math.log2(float(a / 448))) - 2
+                while a > 448 * Fraction(2) ** ee:
+                    ee += 1
+            want[i, g] = min(max(ee + 127, 0), 254)
+    assert np.array_equal(e.astype(np.int64), want)
+    sc = torch.pow(2.0, -(torch.tensor(want, dtype=torch.float64) - 127)).repeat_interleave(128, 1)
+    ref = (xp.double() * sc).clamp(-448, 448).to(torch.float8_e4m3fn).view(torch.uint8)[:, :K].numpy()
+    assert np.array_equal(q, ref)
