@@ -195,6 +195,50 @@ typedef struct {
   int32_t launches;/* kernel launches the call makes */
 } bs_plan;
 
+/*
+ * Fused quantiser -- 1x128 activation groups to e4m3 (the input side of
+ * operations 1 and 3).
+ *
+ * For every row m of x and every group g of 128 consecutive elements along K
+ * (the last group of a row holds K - 128*(ceil(K/128) - 1) elements):
+ *   amax = max |x[m, k]| over the group
+ *   BS_SCALE_F32:  scale[m, g] = amax / 448 (fp32 division; 1 when amax == 0)
+ *                  q[m, k]     = e4m3(x[m, k] / scale[m, g])   (fp32 division)
+ *   BS_SCALE_E8M0: scale[m, g] = clamp(ceil(log2(amax / 448)) + 127, 0, 254),
+ *                  the e8m0 byte of the smallest power of two 2^e with
+ *                  amax <= 448 * 2^e (127 when amax == 0)
+ *                  q[m, k]     = e4m3(x[m, k] * 2^-(scale[m, g] - 127))
+ * where e4m3() rounds to nearest, ties to even, saturates at +-448 and maps
+ * NaN to NaN (0x7F / 0xFF).  448 is the largest finite e4m3 magnitude, so the
+ * group's amax element becomes +-448.  The fp32 form gives exactly the A and
+ * scale_a [M, K/128] of bs_gemm_fp8_blockwise (pytorch issue
+ * "torch._scaled_mm with blockwise scaling doesn't work with torch.compile":
+ * 1x128 groups, one fp32 scale each); the e8m0 form gives the power-of-two
+ * group scales of bmm_a8w8_blockscale (ROCm/aiter PR "Add opus fp8 mxscale
+ * BMM kernels for gfx950").  Results are bit-exact (integer codes and exact
+ * scales); non-finite inputs other than NaN give unspecified codes.
+ *
+ *   x      bf16 or fp32 [M, K], row m at x + m*ldx (ldx >= K, in elements)
+ *   q      e4m3 codes [M, K], row m at q + m*ldq bytes (ldq >= K)
+ *   scale  [M, ceil(K/128)] fp32 or e8m0 bytes, row stride ld_scale elements
+ *   x must be aligned to its element size and fp32 scales to 4 bytes; any
+ *   row strides work (groups whose x row segment is 16-byte aligned and whose
+ *   q segment is 4-byte aligned use vector loads and stores).
+ *   M * ceil(K/512) must stay below 2^31.  M == 0 or K == 0 is a no-op.
+ */
+typedef enum {
+  BS_IN_BF16 = 0, /* bfloat16 */
+  BS_IN_F32 = 1   /* float32 */
+} bs_in_dtype;
+
+typedef enum {
+  BS_SCALE_F32 = 0, /* fp32 scale = amax / 448 */
+  BS_SCALE_E8M0 = 1 /* e8m0 byte: power-of-two scale 2^(byte - 127) */
+} bs_scale_fmt;
+
+bs_status bs_quantize_fp8_1x128(const void* x, bs_in_dtype x_dtype, int64_t M, int64_t K, int64_t ldx, void* q,
+                                int64_t ldq, void* scale, bs_scale_fmt scale_fmt, int64_t ld_scale, void* stream);
+
 /* Plan of operation `op` (1 = bs_gemm_fp8_blockwise, 2 = int_scaled_mm,
  * 3 = bmm_a8w8_blockscale, 4 = bs_gemm_fp8_rowwise; G = 1 for ops 1, 2 and 4)
  * on a GPU with `num_sms`

@@ -66,7 +66,9 @@ def lib() -> ctypes.CDLL:
                                               i64, i64, i64, p]
             h.bmm_a8w8_blockscale.argtypes = [p, i64, i64, p, i64, i64, p, p, p, i64, i64, ctypes.c_int,
                                               i64, i64, i64, i64, p]
-            for f in (h.bs_gemm_fp8_blockwise, h.int_scaled_mm, h.bmm_a8w8_blockscale, h.bs_gemm_fp8_rowwise):
+            h.bs_quantize_fp8_1x128.argtypes = [p, ctypes.c_int, i64, i64, i64, p, i64, p, ctypes.c_int, i64, p]
+            for f in (h.bs_gemm_fp8_blockwise, h.int_scaled_mm, h.bmm_a8w8_blockscale, h.bs_gemm_fp8_rowwise,
+                      h.bs_quantize_fp8_1x128):
                 f.restype = ctypes.c_int
             h.bs_status_string.argtypes = [ctypes.c_int]
             h.bs_status_string.restype = ctypes.c_char_p
@@ -304,6 +306,39 @@ def bmm_a8w8_blockscale(x: torch.Tensor, w: torch.Tensor, x_scale: torch.Tensor,
 # host-side helpers
 # ---------------------------------------------------------------------------
 OP_FP8_BLOCKWISE, OP_INT_SCALED_MM, OP_BMM, OP_FP8_ROWWISE = 1, 2, 3, 4
+
+
+def quantize_fp8_1x128(x: torch.Tensor, scale_format: str = "f32", q: torch.Tensor | None = None,
+                       scale: torch.Tensor | None = None):
+    """1x128 group quantisation of x [M, K] (bf16 or fp32, unit stride along K) to e4m3.
+
+    scale_format "f32": scale fp32 [M, ceil(K/128)] = amax / 448 (1 for an all-zero group);
+    scale_format "e8m0": scale uint8 [M, ceil(K/128)], the e8m0 byte of ceil(log2(amax / 448)).
+    Returns (q, scale) with q as uint8 e4m3 codes [M, K] (rows padded to 16 bytes in memory).
+    """
+    _cuda(x, "x")
+    if x.dim() != 2 or x.stride(1) != 1:
+        raise BsgemmError(BS_ERR_LAYOUT, "x must be [M, K] with unit stride along K")
+    if x.dtype == torch.bfloat16:
+        xd = 0
+    elif x.dtype == torch.float32:
+        xd = 1
+    else:
+        raise BsgemmError(BS_ERR_DTYPE, f"x must be bfloat16 or float32, got {x.dtype}")
+    if scale_format not in ("f32", "e8m0"):
+        raise BsgemmError(BS_ERR_DTYPE, f"unknown scale_format {scale_format!r}")
+    M, K = x.shape
+    KB = -(-K // 128)
+    if q is None:
+        q = _empty_out((M,), K, torch.uint8, x.device)
+    if scale is None:
+        scale = torch.empty((M, KB), dtype=torch.float32 if scale_format == "f32" else torch.uint8, device=x.device)
+    _cuda(q, "q"), _cuda(scale, "scale")
+    if q.shape != (M, K) or q.stride(1) != 1 or scale.shape != (M, KB) or scale.stride(1) != 1:
+        raise BsgemmError(BS_ERR_SHAPE, "q must be [M, K] and scale [M, ceil(K/128)], unit stride along the last dim")
+    _check(lib().bs_quantize_fp8_1x128(_ptr(x), xd, M, K, x.stride(0), _ptr(q), q.stride(0), _ptr(scale),
+                                       0 if scale_format == "f32" else 1, scale.stride(0), _stream(x.device)))
+    return q, scale
 
 
 def plan_for(op: int, M: int, G: int, N: int, K: int, num_sms: int = 148) -> dict:

@@ -9,6 +9,7 @@
 
 #include "bsgemm.h"
 #include "launch.h"
+#include "quantize.h"
 
 using namespace bsg;
 
@@ -535,6 +536,31 @@ bs_status bs_gemm_fp8_rowwise(const void* A, int64_t lda, const void* B, int64_t
     return st;
   return check_launch(launch_wide(Mode::kFp8Rowwise, out_kind(out_dtype), pl.cg, ta, tb, td, args, pl.pub.ctas, cs),
                       "fp8 rowwise kernel launch");
+}
+
+bs_status bs_quantize_fp8_1x128(const void* x, bs_in_dtype x_dtype, int64_t M, int64_t K, int64_t ldx, void* q,
+                                int64_t ldq, void* scale, bs_scale_fmt scale_fmt, int64_t ld_scale, void* stream) {
+  clear_msg();
+  if (M < 0 || K < 0) return fail(BS_ERR_SHAPE, "negative size");
+  if (M > kMaxDim || K > kMaxDim) return fail(BS_ERR_SHAPE, "size exceeds 2^31-1");
+  if (x_dtype != BS_IN_BF16 && x_dtype != BS_IN_F32) return fail(BS_ERR_DTYPE, "x must be bf16 or f32");
+  if (scale_fmt != BS_SCALE_F32 && scale_fmt != BS_SCALE_E8M0) return fail(BS_ERR_DTYPE, "unknown scale format");
+  if (M == 0 || K == 0) return BS_OK;
+  if (!x || !q || !scale) return fail(BS_ERR_NULL, "x, q and scale must be non-NULL");
+  const int64_t KB = (K + 127) / 128;
+  if (ldx < K || ldq < K || ld_scale < KB)
+    return fail(BS_ERR_LAYOUT, "ldx and ldq must be >= K and ld_scale >= ceil(K/128) = %lld", (long long)KB);
+  if (M * ((KB + 3) / 4) > kMaxDim) return fail(BS_ERR_SHAPE, "M * ceil(K/512) exceeds 2^31-1");
+  const uintptr_t es = x_dtype == BS_IN_BF16 ? 2 : 4;
+  if (reinterpret_cast<uintptr_t>(x) % es != 0) return fail(BS_ERR_ALIGNMENT, "x must be aligned to its element size");
+  if (scale_fmt == BS_SCALE_F32 && !aligned4(scale)) return fail(BS_ERR_ALIGNMENT, "fp32 scales must be 4-byte aligned");
+  DeviceCtx* dc = nullptr;
+  bs_status st = device_ctx(&dc);
+  if (st != BS_OK) return st;
+  return check_launch(launch_quantize_1x128(x, x_dtype == BS_IN_BF16, M, K, ldx, static_cast<uint8_t*>(q), ldq, scale,
+                                            scale_fmt == BS_SCALE_E8M0, ld_scale, dc->sms,
+                                            static_cast<cudaStream_t>(stream)),
+                      "quantise launch");
 }
 
 bs_status int_scaled_mm(const int8_t* A, int64_t lda, const int8_t* B, int64_t ldb, const float* s_a,

@@ -266,3 +266,26 @@ def test_default_output_rows_start_on_16_byte_boundaries(N, dtype):
     out3 = bs._empty_out((3, 4), N, dtype, "cpu")
     assert out3.shape == (3, 4, N)
     assert all((s * out3.element_size()) % 16 == 0 for s in out3.stride()[:2])
+
+
+def _qz(**kw):
+    a = dict(x=P16, dt=0, M=64, K=300, ldx=304, q=P16, ldq=304, s=P16, fmt=0, lds=3)
+    a.update(kw)
+    v = ctypes.c_void_p
+    return bs.lib().bs_quantize_fp8_1x128(v(a["x"]), a["dt"], a["M"], a["K"], a["ldx"], v(a["q"]), a["ldq"],
+                                          v(a["s"]), a["fmt"], a["lds"], None)
+
+
+def test_quantize_validation_codes():
+    assert _qz(M=-1) == bs.BS_ERR_SHAPE and _qz(K=-5) == bs.BS_ERR_SHAPE
+    assert _qz(M=1 << 31) == bs.BS_ERR_SHAPE
+    assert _qz(dt=2) == bs.BS_ERR_DTYPE and _qz(fmt=2) == bs.BS_ERR_DTYPE
+    assert _qz(x=0) == bs.BS_ERR_NULL and _qz(q=0) == bs.BS_ERR_NULL and _qz(s=0) == bs.BS_ERR_NULL
+    assert _qz(ldx=200) == bs.BS_ERR_LAYOUT and _qz(ldq=299) == bs.BS_ERR_LAYOUT
+    assert _qz(lds=2) == bs.BS_ERR_LAYOUT  # ceil(300 / 128) = 3 scales per row
+    assert _qz(x=P16 + 1) == bs.BS_ERR_ALIGNMENT and _qz(dt=1, x=P16 + 2) == bs.BS_ERR_ALIGNMENT
+    assert _qz(s=P16 + 2) == bs.BS_ERR_ALIGNMENT
+    assert _qz(M=0) == bs.BS_OK and _qz(K=0) == bs.BS_OK
+    if not HAS_GPU:  # well-formed calls reach the device check (never launched with fake pointers on a GPU)
+        for kw in ({}, {"x": P16 + 2}, {"q": P16 + 1}, {"ldx": 300}, {"ldq": 301}, {"fmt": 1, "s": P16 + 3}):
+            assert _qz(**kw) == bs.BS_ERR_DEVICE, kw

@@ -307,3 +307,68 @@ def test_bmm_block_scaled_mma_and_promotion(M, G, N, K, out_dtype, path):
     for k in (bs.PATH_WIDE, bs.PATH_WIDE_PROMOTE):
         path(k)
         fp8_check(bmm_run(d, out_dtype), y, S, out_dtype, f"bmm {M}x{G}x{N}x{K} kernel={k}")
+
+
+# ---------------------------------------------------------------------------
+# fused quantiser: 1x128 groups to e4m3 with fp32 or e8m0 scales (bit-exact)
+# ---------------------------------------------------------------------------
+def _quant_check(x_dev, fmt, rows=None, **kw):
+    q, s = bs.quantize_fp8_1x128(x_dev, "f32" if fmt == 0 else "e8m0", **kw)
+    if rows is not None:
+        r = torch.as_tensor(rows, device=x_dev.device)
+        x_dev, q, s = x_dev[r], q[r], s[r]
+    xr = x_dev.float().cpu()
+    rq, rs = oracle.quantize_1x128(xr, fmt)
+    gq, gs = q.cpu().numpy(), s.cpu().numpy()
+    bad = np.argwhere(gq != rq)
+    assert bad.size == 0, f"{len(bad)} codes differ, first at {bad[0]}: gpu {gq[tuple(bad[0])]:#x} oracle {rq[tuple(bad[0])]:#x}"
+    if fmt == 0:
+        assert np.array_equal(gs.view(np.uint32), rs.view(np.uint32)), "fp32 scales differ"
+    else:
+        assert np.array_equal(gs, rs), "e8m0 bytes differ"
+
+
+@pytest.mark.parametrize("M,K", [(1, 128), (7, 300), (64, 1000), (256, 4096), (33, 8200)])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("fmt", [0, 1])
+def test_quantize_1x128_bit_exact(M, K, dtype, fmt):
+    x = wl.normal_with_outliers((M, K), 7000 + M + K).to(dtype)
+    _quant_check(x.to(DEV), fmt)
+
+
+@pytest.mark.parametrize("fmt", [0, 1])
+def test_quantize_special_groups_and_strides(fmt):
+    x = torch.zeros(6, 520)
+    x[1] = wl.normal_with_outliers((1, 520), 7100)[0] * 1e-30     # tiny values
+    x[2, :128] = 448.0 * 2.0 ** 5                                   # amax exactly 448 * 2^5, constant group
+    x[2, 128:256] = torch.linspace(-1.0, 1.0, 128)                  # a tie-rich ramp
+    x[3] = -0.0
+    x[4] = wl.normal_with_outliers((1, 520), 7101)[0] * 1e20       # huge values
+    x[5, 7] = 1.0                                                   # one non-zero element per group
+    base = torch.zeros(6, 640)
+    base[:, :520] = x
+    xv = base.to(DEV)[:, :520]                                      # row stride 640 > K
+    q = torch.full((6, 544), 0x55, dtype=torch.uint8, device=DEV)[:, :520]
+    s = torch.zeros((6, 8), dtype=torch.float32 if fmt == 0 else torch.uint8, device=DEV)[:, :5]
+    _quant_check(xv, fmt, q=q, scale=s)
+    full = torch.as_strided(q, (6, 544), (544, 1))
+    assert torch.all(full[:, 520:] == 0x55), "wrote past K"
+
+
+def test_quantize_full_size_activations_sampled_rows():
+    M, K = 16640, 8192
+    x = wl.normal_with_outliers((M, K), 7200).to(torch.bfloat16).to(DEV)
+    rows = rows_sample(M, extra=4)
+    _quant_check(x, 0, rows=rows)
+
+
+def test_quantize_then_blockwise_gemm_matches_the_oracle():
+    M, N, K = 300, 384, 1024
+    x = wl.normal_with_outliers((M, K), 7300)
+    w = wl.normal_with_outliers((K, N), 7301)
+    Bq, sb = wl.quantize_blocks_128x128(w)
+    q, sa = bs.quantize_fp8_1x128(x.to(DEV), "f32")
+    out = bs.bs_gemm_fp8_blockwise(q, Bq.t().contiguous().to(DEV).t(), sa, sb.to(DEV))
+    rq, rsa = oracle.quantize_1x128(x, 0)
+    y, S = oracle.fp8_blockwise(rq, Bq.t().contiguous(), rsa, sb)
+    fp8_check(out, y, S, torch.bfloat16, "quantise + blockwise GEMM")
