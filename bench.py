@@ -62,14 +62,23 @@ def tensor_peak(peaks: dict, timed_s: float):
     return bf16 * FP8_PER_BF16, f"{peaks.get('source')}: bf16 {kind} x 2 (fp8:bf16 nominal ratio)"
 
 
-def source_digest() -> str:
-    """Hash of the CUDA sources: a stored ncu traffic figure is only valid for the kernel it was taken on."""
+# The device-code files of each kernel (its template, the PTX helpers it includes,
+# the translation unit that instantiates and launches it, and the compile-time
+# constants in launch.h).
+KERNEL_SOURCES = {
+    "wide": ["sm100.cuh", "tile_order.h", "wide_kernel.cuh", "kernels_wide.cu", "launch.h"],
+    "skinny": ["sm100.cuh", "tile_order.h", "wide_kernel.cuh", "skinny_kernel.cuh", "kernels_skinny.cu", "launch.h"],
+    "quantize": ["quantize.h", "kernels_quantize.cu"],
+}
+
+
+def source_digest(kernel: str = "wide") -> str:
+    """Hash of one kernel's CUDA sources: a stored ncu traffic figure is only valid for the kernel it was taken on."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "int8_gemm_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode() + b"\0" + f.read())
+    for name in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + b"\0" + f.read())
     return h.hexdigest()[:16]
 
 
@@ -81,7 +90,7 @@ def stored_traffic(workload: str):
     except (OSError, ValueError):
         return None
     e = t.get(workload)
-    if not e or e.get("source_digest") != source_digest():
+    if not e or e.get("kernel") not in KERNEL_SOURCES or e.get("source_digest") != source_digest(e["kernel"]):
         return None
     return e.get("dram_bytes_per_launch")
 
@@ -137,6 +146,10 @@ def describe(w):
         flops = 2.0 * w.M * w.N * w.K
         byts = w.M * w.K + w.N * w.K + 2 * w.M * w.N + 4 * (w.M + 2 * w.N)  # scales and bias
         dtype = "e4m3 (fp32 accumulate)"
+    elif w.op == "quantize_1x128":
+        flops = 0.0  # no tensor work: the metric is bytes moved
+        byts = 2 * w.M * w.K + w.M * w.K + 4 * w.M * (-(-w.K // 128))  # bf16 in, e4m3 codes + fp32 scales out
+        dtype = "bf16 -> e4m3 (fp32 group scales)"
     else:
         flops = 2.0 * w.M * w.G * w.N * w.K
         kb, nb = w.K // 128, -(-w.N // 128)
@@ -171,6 +184,11 @@ def build_step(w, device, copies):
             out = torch.empty(w.M, w.N, dtype=torch.bfloat16, device=device)
             sets.append(lambda A=A, B=B, sa=sa, sb=sb, bias=bias, out=out:
                         bs.bs_gemm_fp8_rowwise(A, B, sa, sb, bias, out=out))
+        elif w.op == "quantize_1x128":
+            x = d["x"].to(device)
+            q = torch.empty(w.M, w.K, dtype=torch.uint8, device=device)
+            sc = torch.empty(w.M, -(-w.K // 128), dtype=torch.float32, device=device)
+            sets.append(lambda x=x, q=q, sc=sc: bs.quantize_fp8_1x128(x, "f32", q=q, scale=sc))
         else:
             x, wt = d["x"].to(device), d["w"].to(device)
             xs, ws = d["x_scale"].to(device), d["w_scale"].to(device)
@@ -293,6 +311,8 @@ def oracle_rows_run(w, d, rows):
         oracle.int_scaled_mm(d["A"], d["B_t"], d["s_a"], d["s_b"], rows=rows)
     elif w.op == "fp8_rowwise":
         oracle.fp8_rowwise(d["A"], d["B_t"], d["scale_a"], d["scale_b"], d["bias"], rows=rows)
+    elif w.op == "quantize_1x128":
+        oracle.quantize_1x128(d["x"][rows], 0)
     else:
         oracle.bmm_blockscale(d["x"], d["w"], d["x_scale"], d["w_scale"], rows=rows)
 
@@ -301,7 +321,8 @@ def cpu_oracle_baseline(w, d, budget_s: float = 20.0):
     """Times the oracle on a bounded row sample sized to about `budget_s` seconds."""
     import oracle
     threads = oracle.num_threads()
-    flops_per_row = describe(w)[0] / w.M
+    quant = w.op == "quantize_1x128"
+    flops_per_row = describe(w)[1 if quant else 0] / w.M  # bytes per row for the quantiser
     n = max(1, min(w.M, threads))
     t0 = time.perf_counter()
     oracle_rows_run(w, d, list(range(n)))
@@ -310,7 +331,8 @@ def cpu_oracle_baseline(w, d, budget_s: float = 20.0):
     t0 = time.perf_counter()
     oracle_rows_run(w, d, list(range(rows)))
     dt = time.perf_counter() - t0
-    return {"value": flops_per_row * rows / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+    return {"value": flops_per_row * rows / dt / (1e9 if quant else 1e12), "unit": "GB/s" if quant else "TFLOP/s",
+            "cores": threads, "kind": "oracle",
             "sample": f"{rows} of {w.M} output rows of {w.name} (all columns), fp64 oracle, {dt:.1f} s"}
 
 
@@ -382,8 +404,12 @@ def main():
     bs.set_path_override({"auto": 0, "wide": 1, "skinny": 2, "wide1": 3, "promote": 4}[args.path])
     copies = max(1, math.ceil(3 * L2_BYTES / byts)) if byts < 3 * L2_BYTES else 1
     d, sets = build_step(w, device, copies)
-    op = {"fp8_blockwise": 1, "int_scaled_mm": 2, "bmm_a8w8_blockscale": 3, "fp8_rowwise": 4}[w.op]
-    plan = bs.plan_for(op, w.M, w.G, w.N, w.K, torch.cuda.get_device_properties(device).multi_processor_count)
+    quant = w.op == "quantize_1x128"
+    if quant:
+        plan = {"kernel": "quantize_1x128", "launches": 1}
+    else:
+        op = {"fp8_blockwise": 1, "int_scaled_mm": 2, "bmm_a8w8_blockscale": 3, "fp8_rowwise": 4}[w.op]
+        plan = bs.plan_for(op, w.M, w.G, w.N, w.K, torch.cuda.get_device_properties(device).multi_processor_count)
 
     for i in range(max(3, args.warmup)):
         sets[i % copies]()
@@ -423,12 +449,12 @@ def main():
     del graph
     err = bs.device_error()
     assert err == 0, f"device error word 0x{err:x}"
-    step_ms, value = aggregate(local_ms / K, flops, world, reduce_max)
-    value /= 1e12
+    step_ms, value = aggregate(local_ms / K, byts if quant else flops, world, reduce_max)
+    value /= 1e9 if quant else 1e12
 
     # end to end through the public API with pinned host buffers
     e2e = None
-    if args.e2e_steps > 0:
+    if args.e2e_steps > 0 and not quant:
         e2e_run, h2d, d2h = e2e_runner(w, d, device, stream)
         e2e_run(2)
         torch.cuda.synchronize()
@@ -454,9 +480,9 @@ def main():
     traffic = stored_traffic(w.name)
 
     result = {
-        "metric": METRIC if w.name == DEFAULT_WORKLOAD else f"{w.name} TFLOP/s",
+        "metric": METRIC if w.name == DEFAULT_WORKLOAD else f"{w.name} {'GB/s' if quant else 'TFLOP/s'}",
         "value": round(value, 2),
-        "unit": "TFLOP/s",
+        "unit": "GB/s" if quant else "TFLOP/s",
         "n_gpus": world,
         "steps": K,
         "warmup": args.warmup,
@@ -467,13 +493,14 @@ def main():
         "dtype": dtype,
         "data": "synthetic (seeded N(0,1) with 1% x20 outliers, quantised per the workload recipe)",
         "config": {"workload": w.name, "op": w.op, "M": w.M, "N": w.N, "K": w.K, "G": w.G,
-                   "out_dtype": "float32" if w.op == "int_scaled_mm" else "bfloat16",
+                   "out_dtype": "float32" if w.op == "int_scaled_mm" else ("e4m3" if quant else "bfloat16"),
                    "l2": (f"inputs larger than L2 ({byts / 1e6:.0f} MB per step)" if copies == 1 else
                           f"{copies} rotating input copies ({copies * byts / 1e6:.0f} MB) to defeat L2"),
                    "parallelism": f"replicas x{world}", "plan": plan},
         "roofline": {"bound": bound, "achieved": round(achieved, 2), "peak": round(peak, 1), "unit": unit,
                      "frac": round(achieved / peak, 4), "traffic": traffic,
-                     "kernel": "wide_gemm_kernel" if plan["kernel"] == 1 else "skinny_gemm_kernel",
+                     "kernel": "quantize_1x128_kernel" if quant else
+                               ("wide_gemm_kernel" if plan["kernel"] == 1 else "skinny_gemm_kernel"),
                      "peak_source": peak_source},
         "e2e": e2e,
         "gpu_launches": K * plan["launches"],
@@ -507,15 +534,17 @@ def run_reference(args, w, rank, world, flops):
     for _ in range(steps):
         oracle_rows_run(w, d, sample)
     dt = (time.perf_counter() - t0) / steps
-    value = flops / w.M * rows_per_step / dt / 1e12
+    quant = w.op == "quantize_1x128"
+    unit = "GB/s" if quant else "TFLOP/s"
+    value = (describe(w)[1] if quant else flops) / w.M * rows_per_step / dt / (1e9 if quant else 1e12)
     out = {
-        "impl": "reference", "metric": METRIC if w.name == DEFAULT_WORKLOAD else f"{w.name} TFLOP/s",
-        "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": steps, "warmup": args.warmup,
+        "impl": "reference", "metric": METRIC if w.name == DEFAULT_WORKLOAD else f"{w.name} {unit}",
+        "value": value, "unit": unit, "n_gpus": world, "steps": steps, "warmup": args.warmup,
         "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64 (oracle)", "data": "synthetic", "config": {"workload": w.name, "M": w.M, "N": w.N, "K": w.K},
-        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+        "cpu_baseline": {"value": value, "unit": unit, "cores": threads, "kind": "oracle",
                          "sample": f"{rows_per_step} of {w.M} output rows per step (all columns)"},
-        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(out), flush=True)
 

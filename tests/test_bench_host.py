@@ -35,16 +35,23 @@ def test_stored_traffic_requires_current_kernel_sources(tmp_path, monkeypatch):
     prof = tmp_path / "profiles"
     prof.mkdir()
     (prof / "traffic.json").write_text(json.dumps({
-        "w_ok": {"source_digest": bench.source_digest(), "dram_bytes_per_launch": 123},
-        "w_stale": {"source_digest": "0" * 16, "dram_bytes_per_launch": 456}}))
+        "w_ok": {"kernel": "wide", "source_digest": bench.source_digest("wide"), "dram_bytes_per_launch": 123},
+        "s_ok": {"kernel": "skinny", "source_digest": bench.source_digest("skinny"), "dram_bytes_per_launch": 7},
+        "w_stale": {"kernel": "wide", "source_digest": "0" * 16, "dram_bytes_per_launch": 456},
+        "w_nokernel": {"source_digest": bench.source_digest("wide"), "dram_bytes_per_launch": 9}}))
     csrc = tmp_path / "int8_gemm_b200" / "csrc"
     csrc.mkdir(parents=True)
     for name in os.listdir(os.path.join(ROOT, "int8_gemm_b200", "csrc")):
         (csrc / name).write_bytes(open(os.path.join(ROOT, "int8_gemm_b200", "csrc", name), "rb").read())
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
-    assert bench.stored_traffic("w_ok") == 123
-    assert bench.stored_traffic("w_stale") is None
+    assert bench.stored_traffic("w_ok") == 123 and bench.stored_traffic("s_ok") == 7
+    assert bench.stored_traffic("w_stale") is None and bench.stored_traffic("w_nokernel") is None
     assert bench.stored_traffic("absent") is None
+    # a change to the skinny kernel leaves the wide kernel's figure valid, and not the reverse
+    (csrc / "skinny_kernel.cuh").write_bytes(b"// changed\n" + (csrc / "skinny_kernel.cuh").read_bytes())
+    assert bench.stored_traffic("w_ok") == 123 and bench.stored_traffic("s_ok") is None
+    (csrc / "wide_kernel.cuh").write_bytes(b"// changed\n" + (csrc / "wide_kernel.cuh").read_bytes())
+    assert bench.stored_traffic("w_ok") is None
 
 
 def test_peaks_fall_back_when_file_missing(tmp_path):
