@@ -69,8 +69,9 @@ def _load():
             lib.orc_fp8_rowwise.argtypes = [p, i64, p, i64, p, i64, p, i64, p, i64, i64, i64, p, i64, p, p]
             lib.orc_e4m3_encode.argtypes = [p, p, i64]
             lib.orc_quantize_1x128.argtypes = [p, i64, i64, i64, ctypes.c_int, p, i64, p, p]
+            lib.orc_quantize_t.argtypes = [p, i64, i64, i64, ctypes.c_int, ctypes.c_int, p, i64, p, p]
             for f in (lib.orc_fp8_blockwise, lib.orc_bmm_blockscale, lib.orc_int_scaled_mm, lib.orc_fp8_rowwise,
-                      lib.orc_quantize_1x128):
+                      lib.orc_quantize_1x128, lib.orc_quantize_t):
                 f.restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -258,4 +259,25 @@ def quantize_1x128(x, fmt: int = 0):
     rc = _load().orc_quantize_1x128(_ptr(xt), M, K, K, fmt, _ptr(q), K, _ptr(sf), _ptr(se))
     if rc != 0:
         raise ValueError(f"orc_quantize_1x128 failed ({rc})")
+    return q, (sf if fmt == 0 else se)
+
+
+def quantize_t(x, group: int = 0, fmt: int = 0):
+    """Transposed-output quantisation of x [R, C] (fp32 or bf16) for the backward GEMMs.
+
+    Returns (codes uint8 [C, R], q_t[c, r] the code of x[r, c]; scales).  group 0 (128x1 groups along
+    the rows): scales [C, ceil(R/128)]; group 1 (128x128 blocks): scales [ceil(R/128), ceil(C/128)].
+    fmt 0: fp32 scales (amax / 448); fmt 1: e8m0 bytes.  See orc_quantize_t."""
+    xt = _np(x.float() if hasattr(x, "float") and not isinstance(x, np.ndarray) else x)
+    xt = np.ascontiguousarray(xt, dtype=np.float32)
+    assert xt.ndim == 2
+    R, C = xt.shape
+    RB, CB = -(-R // 128), -(-C // 128)
+    sshape = (C, RB) if group == 0 else (RB, CB)
+    q = np.empty((C, R), dtype=np.uint8)
+    sf = np.empty(sshape, dtype=np.float32) if fmt == 0 else None
+    se = np.empty(sshape, dtype=np.uint8) if fmt == 1 else None
+    rc = _load().orc_quantize_t(_ptr(xt), R, C, C, group, fmt, _ptr(q), R, _ptr(sf), _ptr(se))
+    if rc != 0:
+        raise ValueError(f"orc_quantize_t failed ({rc})")
     return q, (sf if fmt == 0 else se)

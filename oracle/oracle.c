@@ -383,6 +383,35 @@ void orc_e4m3_encode(const double *v, uint8_t *out, int64_t n)
     for (int64_t i = 0; i < n; ++i) out[i] = orc_e4m3_from_f64(v[i]);
 }
 
+/* fp32 group scale: amax / 448 in fp32, 1 for an all-zero group. */
+static float group_scale_f32(float amax)
+{
+    return amax == 0.0f ? 1.0f : amax / 448.0f;
+}
+
+/* e8m0 group scale byte: clamp(e + 127, 0, 254), e the smallest integer with
+ * amax <= 448 * 2^e (0 for an all-zero group). */
+static int group_scale_e8m0(float amax)
+{
+    int e = 0;
+    if (amax != 0.0f) {
+        e = ilogb((double)amax) - 10;                /* 448 * 2^e < amax here */
+        while (!((double)amax <= ldexp(448.0, e))) ++e;
+    }
+    int byte = e + 127;
+    if (byte < 0) byte = 0;
+    if (byte > 254) byte = 254;
+    return byte;
+}
+
+/* The e4m3 code of element v of a group with fp32 scale s (fmt 0) or e8m0
+ * byte b (fmt 1). */
+static uint8_t group_code(float v, int fmt, float s, int b)
+{
+    if (fmt == 0) return orc_e4m3_from_f64((double)(v / s));
+    return orc_e4m3_from_f64(ldexp((double)v, -(b - 127)));
+}
+
 /*
  * 1x128 activation-group quantisation (the recipe the blockwise operation's
  * inputs follow): for row m and group g (elements 128g .. min(128g+128, K)-1)
@@ -415,27 +444,60 @@ int orc_quantize_1x128(const float *x, int64_t M, int64_t K, int64_t ldx, int fm
                 const float a = fabsf(x[m * ldx + k]);
                 if (a > amax) amax = a;
             }
-            if (fmt == 0) {
-                const float s = amax == 0.0f ? 1.0f : amax / 448.0f;
-                scale_f32[m * KB + g] = s;
-                for (int64_t k = k0; k < k1; ++k) {
-                    const float v = x[m * ldx + k] / s;
-                    q[m * ldq + k] = orc_e4m3_from_f64((double)v);
-                }
-            } else {
-                int e = 0;
-                if (amax != 0.0f) {
-                    e = ilogb((double)amax) - 10;                /* 448 * 2^e < amax here */
-                    while (!((double)amax <= ldexp(448.0, e))) ++e;
-                }
-                int byte = e + 127;
-                if (byte < 0) byte = 0;
-                if (byte > 254) byte = 254;
-                scale_e8m0[m * KB + g] = (uint8_t)byte;
-                for (int64_t k = k0; k < k1; ++k)
-                    q[m * ldq + k] = orc_e4m3_from_f64(ldexp((double)x[m * ldx + k], -(byte - 127)));
-            }
+            const float s = group_scale_f32(amax);
+            const int b = group_scale_e8m0(amax);
+            if (fmt == 0) scale_f32[m * KB + g] = s;
+            else scale_e8m0[m * KB + g] = (uint8_t)b;
+            for (int64_t k = k0; k < k1; ++k) q[m * ldq + k] = group_code(x[m * ldx + k], fmt, s, b);
         }
+    }
+    return ORC_OK;
+}
+
+/*
+ * Quantisation for the backward pass of a blockwise fp8 linear layer: the
+ * codes are written transposed, so that the dimension the backward GEMMs
+ * contract over (the rows of x) becomes the contiguous one.  x is [R, C]
+ * (row stride ldx); q_t is [C, R] (row stride ldq), q_t[c][r] the code of
+ * x[r][c].  Groups, with the same scale and code rules as orc_quantize_1x128:
+ *   group 0 (128x1): rows 128rb .. min(128rb + 128, R) - 1 of one column c;
+ *                    scale[c * RB + rb]  ([C, RB], RB = ceil(R / 128)), i.e.
+ *                    the 1x128 groups of x transposed
+ *   group 1 (128x128): the block rows 128rb.., columns 128cb..;
+ *                    scale[rb * CB + cb]  ([RB, CB], CB = ceil(C / 128))
+ *   Sources: pytorch issue "torch._scaled_mm with blockwise scaling doesn't
+ *   work with torch.compile" (the forward and backward benchmark of the
+ *   blockwise fp8 linear layer; the 1x128 activation groups with scale_a
+ *   [M, K/128] and the 128x128 weight blocks with scale_b [K/128, N/128] are
+ *   the only two group shapes it fixes, so the backward operands take those
+ *   two shapes along their contraction dimension).
+ */
+int orc_quantize_t(const float *x, int64_t R, int64_t C, int64_t ldx, int group, int fmt,
+                   uint8_t *q_t, int64_t ldq, float *scale_f32, uint8_t *scale_e8m0)
+{
+    if (R < 0 || C < 0 || ldx < C || ldq < R || (fmt != 0 && fmt != 1) || (group != 0 && group != 1))
+        return ORC_ERR_SHAPE;
+    const int64_t RB = (R + 127) / 128, CB = (C + 127) / 128;
+    const int64_t CW = group == 0 ? 1 : 128;          /* columns per group */
+    const int64_t NG = group == 0 ? C : CB;            /* groups per row block */
+#pragma omp parallel for schedule(dynamic, 4)
+    for (int64_t gi = 0; gi < RB * NG; ++gi) {
+        const int64_t rb = gi / NG, g = gi % NG;
+        const int64_t r0 = 128 * rb, r1 = r0 + 128 < R ? r0 + 128 : R;
+        const int64_t c0 = g * CW, c1 = c0 + CW < C ? c0 + CW : C;
+        float amax = 0.0f;
+        for (int64_t r = r0; r < r1; ++r)
+            for (int64_t c = c0; c < c1; ++c) {
+                const float a = fabsf(x[r * ldx + c]);
+                if (a > amax) amax = a;
+            }
+        const float s = group_scale_f32(amax);
+        const int b = group_scale_e8m0(amax);
+        const int64_t si = group == 0 ? g * RB + rb : rb * CB + g;
+        if (fmt == 0) scale_f32[si] = s;
+        else scale_e8m0[si] = (uint8_t)b;
+        for (int64_t r = r0; r < r1; ++r)
+            for (int64_t c = c0; c < c1; ++c) q_t[c * ldq + r] = group_code(x[r * ldx + c], fmt, s, b);
     }
     return ORC_OK;
 }

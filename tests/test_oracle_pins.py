@@ -531,3 +531,71 @@ def test_quantize_e8m0_matches_the_bmm_recipe_through_torch_cast(M, K):
     sc = torch.pow(2.0, -(torch.tensor(want, dtype=torch.float64) - 127)).repeat_interleave(128, 1)
     ref = (xp.double() * sc).clamp(-448, 448).to(torch.float8_e4m3fn).view(torch.uint8)[:, :K].numpy()
     assert np.array_equal(q, ref)
+
+
+# ---------------------------------------------------------------------------
+# transposed-output quantiser for the backward GEMMs (128x1 and 128x128 groups)
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("R,C", [(128, 3), (300, 5), (1000, 2)])
+@pytest.mark.parametrize("fmt", [0, 1])
+def test_quantize_t_128x1_is_the_1x128_quantiser_of_the_transpose(R, C, fmt):
+    x = wl.normal_with_outliers((R, C), 77 + R + C)
+    q, s = oracle.quantize_t(x, 0, fmt)
+    rq, rs = oracle.quantize_1x128(x.t().contiguous(), fmt)
+    assert q.shape == (C, R) and s.shape == (C, -(-R // 128))
+    assert np.array_equal(q, rq) and np.array_equal(s, rs)
+
+
+def _torch_quantize_128x128_t(x):
+    """128x128 blocks through torch's own cast, codes transposed: scale = amax / 448 (1 if 0)."""
+    R, C = x.shape
+    RB, CB = -(-R // 128), -(-C // 128)
+    xp = torch.zeros(RB * 128, CB * 128)
+    xp[:R, :C] = x
+    amax = xp.view(RB, 128, CB, 128).abs().amax(dim=(1, 3))
+    s = amax / 448.0
+    s[amax == 0] = 1.0
+    full = s.repeat_interleave(128, 0).repeat_interleave(128, 1)
+    q = (xp / full).clamp(-448, 448).to(torch.float8_e4m3fn).view(torch.uint8)
+    return q[:R, :C].t().contiguous().numpy(), s.numpy()
+
+
+@pytest.mark.parametrize("R,C", [(128, 128), (300, 200), (256, 1000)])
+def test_quantize_t_128x128_matches_torch_cast_of_x_over_block_scale(R, C):
+    x = wl.normal_with_outliers((R, C), 55 + R + C)
+    q, s = oracle.quantize_t(x, 1, 0)
+    rq, rs = _torch_quantize_128x128_t(x)
+    assert s.dtype == np.float32 and s.shape == (-(-R // 128), -(-C // 128))
+    assert np.array_equal(s, rs) and np.array_equal(q, rq)
+
+
+def test_quantize_t_orientation_block_amax_and_isolation():
+    x = torch.zeros(256, 256)
+    x[3, 200] = -5.0  # block (0, 1): its amax, negative
+    x[130, 7] = 2.0   # block (1, 0)
+    x[131, 8] = 1.0
+    q, s = oracle.quantize_t(x, 1, 0)
+    assert q[200, 3] == 0xFE and q[7, 130] == 0x7E  # q_t[c, r] is the code of x[r, c]
+    assert q[8, 131] == oracle.e4m3_encode([1.0 / float(np.float32(2.0) / np.float32(448.0))])[0]
+    assert s[0, 0] == 1.0 and s[1, 1] == 1.0  # all-zero blocks
+    assert s[0, 1] == np.float32(5.0) / np.float32(448.0) and s[1, 0] == np.float32(2.0) / np.float32(448.0)
+    assert int(np.count_nonzero(q)) == 3
+    # 128x1: each column of a 128-row block is its own group
+    q1, s1 = oracle.quantize_t(x, 0, 0)
+    assert q1[7, 130] == 0x7E and q1[8, 131] == 0x7E and s1[8, 1] == np.float32(1.0) / np.float32(448.0)
+
+
+@pytest.mark.parametrize("fmt", [0, 1])
+def test_quantize_t_block_scale_is_the_largest_column_scale_of_the_block(fmt):
+    # amax / 448 and ceil(log2(amax / 448)) are monotone in amax: a block's
+    # scale is the largest 128x1 scale among its columns, and the column that
+    # holds the block amax gets identical codes either way
+    x = wl.normal_with_outliers((384, 256), 31 + fmt)
+    qb, sb = oracle.quantize_t(x, 1, fmt)
+    qc, sc = oracle.quantize_t(x, 0, fmt)
+    for rb in range(3):
+        for cb in range(2):
+            cols = sc[128 * cb:128 * cb + 128, rb]
+            assert sb[rb, cb] == cols.max()
+            c = 128 * cb + int(np.argmax(cols))
+            assert np.array_equal(qb[c, 128 * rb:128 * rb + 128], qc[c, 128 * rb:128 * rb + 128])
