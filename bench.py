@@ -68,7 +68,8 @@ def tensor_peak(peaks: dict, timed_s: float):
 KERNEL_SOURCES = {
     "wide": ["sm100.cuh", "tile_order.h", "wide_kernel.cuh", "kernels_wide.cu", "launch.h"],
     "skinny": ["sm100.cuh", "tile_order.h", "wide_kernel.cuh", "skinny_kernel.cuh", "kernels_skinny.cu", "launch.h"],
-    "quantize": ["quantize.h", "kernels_quantize.cu"],
+    "quantize": ["group_quant.cuh", "quantize.h", "kernels_quantize.cu"],
+    "quantize_t": ["group_quant.cuh", "quantize.h", "kernels_quantize_t.cu"],
 }
 
 
@@ -132,6 +133,9 @@ def parse_clock_csv(text: str):
 # ---------------------------------------------------------------------------
 # workloads
 # ---------------------------------------------------------------------------
+QUANT_OPS = ("quantize_1x128", "quantize_t")  # HBM-bound quantisers: GB/s, not TFLOP/s
+
+
 def describe(w):
     import workloads as wl
     if w.op == "fp8_blockwise":
@@ -144,18 +148,33 @@ def describe(w):
         dtype = "s8 (s32 accumulate)"
     elif w.op == "fp8_rowwise":
         flops = 2.0 * w.M * w.N * w.K
-        byts = w.M * w.K + w.N * w.K + 2 * w.M * w.N + 4 * (w.M + 2 * w.N)  # scales and bias
+        out_es = 1 if w.extra.get("out") == "e4m3" else 2
+        byts = w.M * w.K + w.N * w.K + out_es * w.M * w.N + 4 * (w.M + 2 * w.N)  # scales and bias
         dtype = "e4m3 (fp32 accumulate)"
     elif w.op == "quantize_1x128":
         flops = 0.0  # no tensor work: the metric is bytes moved
         byts = 2 * w.M * w.K + w.M * w.K + 4 * w.M * (-(-w.K // 128))  # bf16 in, e4m3 codes + fp32 scales out
         dtype = "bf16 -> e4m3 (fp32 group scales)"
+    elif w.op == "quantize_t":
+        flops = 0.0
+        rb, cb = -(-w.M // 128), -(-w.K // 128)
+        nscales = w.K * rb if w.extra["group"] == "128x1" else rb * cb
+        byts = 2 * w.M * w.K + w.M * w.K + 4 * nscales  # bf16 x [M, K] in, transposed codes + fp32 scales out
+        dtype = f"bf16 -> e4m3, transposed ({w.extra['group']} groups, fp32 scales)"
     else:
         flops = 2.0 * w.M * w.G * w.N * w.K
         kb, nb = w.K // 128, -(-w.N // 128)
         byts = w.M * w.G * w.K + w.G * w.N * w.K + 2 * w.M * w.G * w.N + w.M * w.G * kb + w.G * nb * kb
         dtype = "e4m3 (fp32 accumulate)"
     return flops, float(byts), dtype
+
+
+def rowwise_out(w, device):
+    """(output dtype, scale_result tensor or None) of an fp8_rowwise workload."""
+    import torch
+    if w.extra.get("out") == "e4m3":
+        return torch.float8_e4m3fn, torch.tensor([w.extra["scale_result"]], dtype=torch.float32, device=device)
+    return torch.bfloat16, None
 
 
 def build_step(w, device, copies):
@@ -181,14 +200,19 @@ def build_step(w, device, copies):
         elif w.op == "fp8_rowwise":
             A, B = d["A"].to(device), d["B_t"].to(device).t()
             sa, sb, bias = d["scale_a"].to(device), d["scale_b"].to(device), d["bias"].to(device)
-            out = torch.empty(w.M, w.N, dtype=torch.bfloat16, device=device)
-            sets.append(lambda A=A, B=B, sa=sa, sb=sb, bias=bias, out=out:
-                        bs.bs_gemm_fp8_rowwise(A, B, sa, sb, bias, out=out))
+            odt, sr = rowwise_out(w, device)
+            out = torch.empty(w.M, w.N, dtype=odt, device=device)
+            sets.append(lambda A=A, B=B, sa=sa, sb=sb, bias=bias, out=out, odt=odt, sr=sr:
+                        bs.bs_gemm_fp8_rowwise(A, B, sa, sb, bias, out_dtype=odt, out=out, scale_result=sr))
         elif w.op == "quantize_1x128":
             x = d["x"].to(device)
             q = torch.empty(w.M, w.K, dtype=torch.uint8, device=device)
             sc = torch.empty(w.M, -(-w.K // 128), dtype=torch.float32, device=device)
             sets.append(lambda x=x, q=q, sc=sc: bs.quantize_fp8_1x128(x, "f32", q=q, scale=sc))
+        elif w.op == "quantize_t":
+            x = d["x"].to(device)
+            q, sc = bs.quantize_fp8_t(x, w.extra["group"], "f32")  # allocates the outputs once
+            sets.append(lambda x=x, q=q, sc=sc: bs.quantize_fp8_t(x, w.extra["group"], "f32", q_t=q, scale=sc))
         else:
             x, wt = d["x"].to(device), d["w"].to(device)
             xs, ws = d["x_scale"].to(device), d["w_scale"].to(device)
@@ -207,7 +231,10 @@ def e2e_runner(w, d, device, stream):
     import int8_gemm_b200 as bs
 
     pin = {k: v.contiguous().pin_memory() for k, v in d.items() if v is not None}
-    if w.op in ("fp8_blockwise", "fp8_rowwise"):
+    s_res = None
+    if w.op == "fp8_rowwise":
+        out_shape, (out_dtype, s_res) = (w.M, w.N), rowwise_out(w, device)
+    elif w.op == "fp8_blockwise":
         out_shape, out_dtype = (w.M, w.N), torch.bfloat16
     elif w.op == "int_scaled_mm":
         out_shape, out_dtype = (w.M, w.N), torch.float32
@@ -228,7 +255,8 @@ def e2e_runner(w, d, device, stream):
         elif w.op == "int_scaled_mm":
             bs.int_scaled_mm(x["A"], x["B_t"].t(), x["s_a"], x["s_b"], out_dtype=torch.float32, out=out)
         elif w.op == "fp8_rowwise":
-            bs.bs_gemm_fp8_rowwise(x["A"], x["B_t"].t(), x["scale_a"], x["scale_b"], x.get("bias"), out=out)
+            bs.bs_gemm_fp8_rowwise(x["A"], x["B_t"].t(), x["scale_a"], x["scale_b"], x.get("bias"),
+                                   out_dtype=out_dtype, out=out, scale_result=s_res)
         else:
             bs.bmm_a8w8_blockscale(x["x"], x["w"], x["x_scale"], x["w_scale"], out=out)
 
@@ -310,9 +338,13 @@ def oracle_rows_run(w, d, rows):
     elif w.op == "int_scaled_mm":
         oracle.int_scaled_mm(d["A"], d["B_t"], d["s_a"], d["s_b"], rows=rows)
     elif w.op == "fp8_rowwise":
-        oracle.fp8_rowwise(d["A"], d["B_t"], d["scale_a"], d["scale_b"], d["bias"], rows=rows)
+        y, _ = oracle.fp8_rowwise(d["A"], d["B_t"], d["scale_a"], d["scale_b"], d["bias"], rows=rows)
+        if w.extra.get("out") == "e4m3":
+            oracle.e4m3_encode(w.extra["scale_result"] * y)
     elif w.op == "quantize_1x128":
         oracle.quantize_1x128(d["x"][rows], 0)
+    elif w.op == "quantize_t":
+        oracle.quantize_t(d["x"][rows], 0 if w.extra["group"] == "128x1" else 1, 0)
     else:
         oracle.bmm_blockscale(d["x"], d["w"], d["x_scale"], d["w_scale"], rows=rows)
 
@@ -321,7 +353,7 @@ def cpu_oracle_baseline(w, d, budget_s: float = 20.0):
     """Times the oracle on a bounded row sample sized to about `budget_s` seconds."""
     import oracle
     threads = oracle.num_threads()
-    quant = w.op == "quantize_1x128"
+    quant = w.op in QUANT_OPS
     flops_per_row = describe(w)[1 if quant else 0] / w.M  # bytes per row for the quantiser
     n = max(1, min(w.M, threads))
     t0 = time.perf_counter()
@@ -404,9 +436,9 @@ def main():
     bs.set_path_override({"auto": 0, "wide": 1, "skinny": 2, "wide1": 3, "promote": 4}[args.path])
     copies = max(1, math.ceil(3 * L2_BYTES / byts)) if byts < 3 * L2_BYTES else 1
     d, sets = build_step(w, device, copies)
-    quant = w.op == "quantize_1x128"
+    quant = w.op in QUANT_OPS
     if quant:
-        plan = {"kernel": "quantize_1x128", "launches": 1}
+        plan = {"kernel": w.op, "launches": 1}
     else:
         op = {"fp8_blockwise": 1, "int_scaled_mm": 2, "bmm_a8w8_blockscale": 3, "fp8_rowwise": 4}[w.op]
         plan = bs.plan_for(op, w.M, w.G, w.N, w.K, torch.cuda.get_device_properties(device).multi_processor_count)
@@ -493,13 +525,15 @@ def main():
         "dtype": dtype,
         "data": "synthetic (seeded N(0,1) with 1% x20 outliers, quantised per the workload recipe)",
         "config": {"workload": w.name, "op": w.op, "M": w.M, "N": w.N, "K": w.K, "G": w.G,
-                   "out_dtype": "float32" if w.op == "int_scaled_mm" else ("e4m3" if quant else "bfloat16"),
+                   "out_dtype": "float32" if w.op == "int_scaled_mm" else
+                   ("e4m3" if quant or w.extra.get("out") == "e4m3" else "bfloat16"),
+                   **({"scale_result": w.extra["scale_result"]} if "scale_result" in w.extra else {}),
                    "l2": (f"inputs larger than L2 ({byts / 1e6:.0f} MB per step)" if copies == 1 else
                           f"{copies} rotating input copies ({copies * byts / 1e6:.0f} MB) to defeat L2"),
                    "parallelism": f"replicas x{world}", "plan": plan},
         "roofline": {"bound": bound, "achieved": round(achieved, 2), "peak": round(peak, 1), "unit": unit,
                      "frac": round(achieved / peak, 4), "traffic": traffic,
-                     "kernel": "quantize_1x128_kernel" if quant else
+                     "kernel": f"{w.op}_kernel" if quant else
                                ("wide_gemm_kernel" if plan["kernel"] == 1 else "skinny_gemm_kernel"),
                      "peak_source": peak_source},
         "e2e": e2e,
@@ -534,7 +568,7 @@ def run_reference(args, w, rank, world, flops):
     for _ in range(steps):
         oracle_rows_run(w, d, sample)
     dt = (time.perf_counter() - t0) / steps
-    quant = w.op == "quantize_1x128"
+    quant = w.op in QUANT_OPS
     unit = "GB/s" if quant else "TFLOP/s"
     value = (describe(w)[1] if quant else flops) / w.M * rows_per_step / dt / (1e9 if quant else 1e12)
     out = {

@@ -52,7 +52,9 @@ typedef enum {
 typedef enum {
   BS_OUT_BF16 = 0, /* bfloat16, round-to-nearest-even from the fp32 result */
   BS_OUT_F32 = 1,  /* float32 */
-  BS_OUT_I32 = 2   /* raw int32 accumulator (int_scaled_mm only) */
+  BS_OUT_I32 = 2,  /* raw int32 accumulator (int_scaled_mm only) */
+  BS_OUT_E4M3 = 3  /* e4m3 bytes: round-to-nearest-even, saturated at +-448, of
+                      scale_result * result (bs_gemm_fp8_rowwise only) */
 } bs_out_dtype;
 
 /*
@@ -103,15 +105,24 @@ bs_status bs_gemm_fp8_blockwise(const void* A, int64_t lda, const void* B, int64
  *   scale_b  fp32; sb_stride = 0: one scale (tensorwise), 1: [N] (rowwise)
  *            (both strides equal: the two operands use the same mode)
  *   bias     fp32 [N] or NULL
- *   out      [M, N] row-major, row stride ldo (>= N), BS_OUT_BF16 or BS_OUT_F32
+ *   scale_result  fp32 scalar or NULL (1): with BS_OUT_E4M3 the result is
+ *            multiplied by it before the saturating e4m3 cast, the output
+ *            scale of an fp8 result (tuned_scaled_mm's scale_result, same
+ *            file); it must be NULL for the other output types
+ *   out      [M, N] row-major, row stride ldo (>= N), BS_OUT_BF16, BS_OUT_F32
+ *            or BS_OUT_E4M3
  *   K is free (lda and ldb multiples of 16); K == 0 writes bias (or zeros).
+ * The accumulator is fp32 in tensor memory over all of K; tuned_scaled_mm's
+ * use_fast_accum chooses between accumulating inside the MMA and adding each
+ * K tile's product in fp32, and on this hardware both are the fp32
+ * accumulation done here, so it is not a parameter.
  * Not a block-scaled operation: it has no counterpart in the block-scaled
  * statement of the problem above and follows the mm.py scaling modes.
  */
 bs_status bs_gemm_fp8_rowwise(const void* A, int64_t lda, const void* B, int64_t ldb,
                               const float* scale_a, int64_t sa_stride, const float* scale_b, int64_t sb_stride,
-                              const float* bias, void* out, int64_t ldo, bs_out_dtype out_dtype,
-                              int64_t M, int64_t N, int64_t K, void* stream);
+                              const float* bias, const float* scale_result, void* out, int64_t ldo,
+                              bs_out_dtype out_dtype, int64_t M, int64_t N, int64_t K, void* stream);
 
 /*
  * Operation 2 -- INT8 GEMM with a fused, fixed-order fp32 dequantisation.
@@ -238,6 +249,43 @@ typedef enum {
 
 bs_status bs_quantize_fp8_1x128(const void* x, bs_in_dtype x_dtype, int64_t M, int64_t K, int64_t ldx, void* q,
                                 int64_t ldq, void* scale, bs_scale_fmt scale_fmt, int64_t ld_scale, void* stream);
+
+/*
+ * Transposed-output quantiser -- the operands of the backward GEMMs of a
+ * blockwise fp8 linear layer y = x W^T (x [M, K] in 1x128 groups, W [N, K] in
+ * 128x128 blocks; the forward and backward benchmark of the pytorch issue
+ * "torch._scaled_mm with blockwise scaling doesn't work with torch.compile").
+ * The backward GEMMs contract over the rows of their inputs (the M tokens for
+ * the weight gradient dW = dy^T x, the N outputs for the input gradient
+ * dx = dy W), so the codes are written transposed, with groups along those
+ * rows:
+ *   q_t[c, r] = code of x[r, c],  q_t [C, R], row c at q_t + c*ldq (ldq >= R)
+ *   BS_GROUP_128x1:   one scale per column c and 128-row block rb (rows
+ *                     128rb .. min(128rb + 128, R) - 1), scale[c, rb] at
+ *                     scale + c*ld_scale + rb, [C, ceil(R/128)]: the 1x128
+ *                     groups of x^T, i.e. scale_a of bs_gemm_fp8_blockwise
+ *                     for A = q_t
+ *   BS_GROUP_128x128: one scale per 128 x 128 block, scale[rb, cb] at
+ *                     scale + rb*ld_scale + cb, [ceil(R/128), ceil(C/128)]:
+ *                     scale_b of bs_gemm_fp8_blockwise for B_t = q_t (B the
+ *                     column-major view of q_t)
+ * with the scale and code rules of bs_quantize_fp8_1x128 (amax over the group;
+ * fp32 amax / 448 or the e8m0 byte; saturating RNE e4m3 codes).  Bit-exact.
+ *   dW = dy^T x:  A = q_t(dy, 128x1), B_t = q_t(x, 128x128)
+ *   dx = dy W:    A = bs_quantize_fp8_1x128(dy), B_t = q_t(W, 128x128)
+ *   x      bf16 or fp32 [R, C], row r at x + r*ldx (ldx >= C, in elements),
+ *          aligned to its element size
+ *   fp32 scales must be 4-byte aligned.  R == 0 or C == 0 is a no-op.
+ *   16-byte loads and stores are used where x, ldx, q_t and ldq allow them.
+ */
+typedef enum {
+  BS_GROUP_128x1 = 0,  /* 128 rows of one column */
+  BS_GROUP_128x128 = 1 /* 128 x 128 blocks */
+} bs_group;
+
+bs_status bs_quantize_fp8_t(const void* x, bs_in_dtype x_dtype, int64_t R, int64_t C, int64_t ldx, void* q_t,
+                           int64_t ldq, void* scale, bs_scale_fmt scale_fmt, bs_group group, int64_t ld_scale,
+                           void* stream);
 
 /* Plan of operation `op` (1 = bs_gemm_fp8_blockwise, 2 = int_scaled_mm,
  * 3 = bmm_a8w8_blockscale, 4 = bs_gemm_fp8_rowwise; G = 1 for ops 1, 2 and 4)

@@ -24,11 +24,12 @@ LIB_PATH = os.path.join(_HERE, "libbsgemm.so")
 
 BS_OK, BS_ERR_NULL, BS_ERR_SHAPE, BS_ERR_LAYOUT, BS_ERR_ALIGNMENT = 0, 1, 2, 3, 4
 BS_ERR_DTYPE, BS_ERR_DEVICE, BS_ERR_CUDA, BS_ERR_TIMEOUT = 5, 6, 7, 8
-BS_OUT_BF16, BS_OUT_F32, BS_OUT_I32 = 0, 1, 2
+BS_OUT_BF16, BS_OUT_F32, BS_OUT_I32, BS_OUT_E4M3 = 0, 1, 2, 3
 
 PATH_AUTO, PATH_WIDE, PATH_SKINNY, PATH_WIDE_SINGLE, PATH_WIDE_PROMOTE = 0, 1, 2, 3, 4
 
-_OUT_CODE = {torch.bfloat16: BS_OUT_BF16, torch.float32: BS_OUT_F32, torch.int32: BS_OUT_I32}
+_OUT_CODE = {torch.bfloat16: BS_OUT_BF16, torch.float32: BS_OUT_F32, torch.int32: BS_OUT_I32,
+             torch.float8_e4m3fn: BS_OUT_E4M3}
 
 
 class BsgemmError(RuntimeError):
@@ -62,13 +63,15 @@ def lib() -> ctypes.CDLL:
             h.bs_gemm_fp8_blockwise.argtypes = [p, i64, p, i64, p, i64, i64, p, i64, i64, p, i64, ctypes.c_int,
                                                 i64, i64, i64, p]
             h.int_scaled_mm.argtypes = [p, i64, p, i64, p, p, p, i64, ctypes.c_int, i64, i64, i64, p]
-            h.bs_gemm_fp8_rowwise.argtypes = [p, i64, p, i64, p, i64, p, i64, p, p, i64, ctypes.c_int,
+            h.bs_gemm_fp8_rowwise.argtypes = [p, i64, p, i64, p, i64, p, i64, p, p, p, i64, ctypes.c_int,
                                               i64, i64, i64, p]
             h.bmm_a8w8_blockscale.argtypes = [p, i64, i64, p, i64, i64, p, p, p, i64, i64, ctypes.c_int,
                                               i64, i64, i64, i64, p]
             h.bs_quantize_fp8_1x128.argtypes = [p, ctypes.c_int, i64, i64, i64, p, i64, p, ctypes.c_int, i64, p]
+            h.bs_quantize_fp8_t.argtypes = [p, ctypes.c_int, i64, i64, i64, p, i64, p, ctypes.c_int, ctypes.c_int,
+                                            i64, p]
             for f in (h.bs_gemm_fp8_blockwise, h.int_scaled_mm, h.bmm_a8w8_blockscale, h.bs_gemm_fp8_rowwise,
-                      h.bs_quantize_fp8_1x128):
+                      h.bs_quantize_fp8_1x128, h.bs_quantize_fp8_t):
                 f.restype = ctypes.c_int
             h.bs_status_string.argtypes = [ctypes.c_int]
             h.bs_status_string.restype = ctypes.c_char_p
@@ -169,14 +172,21 @@ def bs_gemm_fp8_blockwise(A: torch.Tensor, B: torch.Tensor, scale_a: torch.Tenso
 
 def bs_gemm_fp8_rowwise(A: torch.Tensor, B: torch.Tensor, scale_a: torch.Tensor, scale_b: torch.Tensor,
                         bias: torch.Tensor | None = None, out_dtype: torch.dtype = torch.bfloat16,
-                        out: torch.Tensor | None = None) -> torch.Tensor:
+                        out: torch.Tensor | None = None, scale_result: torch.Tensor | None = None,
+                        use_fast_accum: bool = False) -> torch.Tensor:
     """FP8 GEMM with tensorwise or rowwise scales: out = (A @ B) * (scale_a * scale_b) + bias.
 
     A       e4m3 [M, K] row-major;  B e4m3 [K, N] column-major (``B_t.t()`` for B_t [N, K])
     scale_a fp32 scalar (tensorwise) or [M] / [M, 1] (rowwise)
     scale_b fp32 scalar (tensorwise) or [N] / [1, N] (rowwise), the same kind as scale_a
     bias    fp32 [N] or None
+    out_dtype bfloat16, float32 or float8_e4m3fn (saturating round-to-nearest-even cast)
+    scale_result fp32 scalar or None: an e4m3 result is scale_result * (the above) before
+            its cast (the output scale of _scaled_mm); only with out_dtype float8_e4m3fn
+    use_fast_accum accepted for _scaled_mm's signature; the tensor cores accumulate in fp32
+            over all of K either way, so it changes nothing
     """
+    del use_fast_accum
     for t, n in ((A, "A"), (B, "B"), (scale_a, "scale_a"), (scale_b, "scale_b")):
         _cuda(t, n)
     _bytes8(A, "A"), _bytes8(B, "B")
@@ -199,12 +209,17 @@ def bs_gemm_fp8_rowwise(A: torch.Tensor, B: torch.Tensor, scale_a: torch.Tensor,
         if bias.dtype != torch.float32 or bias.numel() != N:
             raise BsgemmError(BS_ERR_SHAPE, "bias must be float32 [N]")
         bias = bias.reshape(-1).contiguous()
+    if scale_result is not None:
+        _cuda(scale_result, "scale_result")
+        if scale_result.dtype != torch.float32 or scale_result.numel() != 1:
+            raise BsgemmError(BS_ERR_SHAPE, "scale_result must be a float32 scalar")
+        scale_result = scale_result.reshape(-1).contiguous()
     if A.stride(1) != 1 and M > 1:
         raise BsgemmError(BS_ERR_LAYOUT, f"A must be row-major, got strides {A.stride()}")
     if B.stride(0) != 1 and N > 1:
         raise BsgemmError(BS_ERR_LAYOUT, f"B must be column-major, got strides {B.stride()}")
-    if out_dtype not in (torch.bfloat16, torch.float32):
-        raise BsgemmError(BS_ERR_DTYPE, f"out_dtype must be bfloat16 or float32, got {out_dtype}")
+    if out_dtype not in (torch.bfloat16, torch.float32, torch.float8_e4m3fn):
+        raise BsgemmError(BS_ERR_DTYPE, f"out_dtype must be bfloat16, float32 or float8_e4m3fn, got {out_dtype}")
     if out is None:
         out = _empty_out((M,), N, out_dtype, A.device)
     elif out.dtype != out_dtype or tuple(out.shape) != (M, N) or out.stride(1) != 1:
@@ -212,7 +227,7 @@ def bs_gemm_fp8_rowwise(A: torch.Tensor, B: torch.Tensor, scale_a: torch.Tensor,
     with torch.cuda.device(A.device):
         _check(lib().bs_gemm_fp8_rowwise(
             _ptr(A), A.stride(0), _ptr(B), B.stride(1), _ptr(scale_a), stride, _ptr(scale_b), stride, _ptr(bias),
-            _ptr(out), out.stride(0), _OUT_CODE[out_dtype], M, N, K, _stream(A.device)))
+            _ptr(scale_result), _ptr(out), out.stride(0), _OUT_CODE[out_dtype], M, N, K, _stream(A.device)))
     return out
 
 
@@ -334,11 +349,55 @@ def quantize_fp8_1x128(x: torch.Tensor, scale_format: str = "f32", q: torch.Tens
     if scale is None:
         scale = torch.empty((M, KB), dtype=torch.float32 if scale_format == "f32" else torch.uint8, device=x.device)
     _cuda(q, "q"), _cuda(scale, "scale")
+    _check_quant_out(q, scale, scale_format)
     if q.shape != (M, K) or q.stride(1) != 1 or scale.shape != (M, KB) or scale.stride(1) != 1:
         raise BsgemmError(BS_ERR_SHAPE, "q must be [M, K] and scale [M, ceil(K/128)], unit stride along the last dim")
     _check(lib().bs_quantize_fp8_1x128(_ptr(x), xd, M, K, x.stride(0), _ptr(q), q.stride(0), _ptr(scale),
                                        0 if scale_format == "f32" else 1, scale.stride(0), _stream(x.device)))
     return q, scale
+
+
+def _check_quant_out(q: torch.Tensor, scale: torch.Tensor, scale_format: str):
+    if q.dtype not in (torch.uint8, torch.float8_e4m3fn):
+        raise BsgemmError(BS_ERR_DTYPE, f"q must hold e4m3 bytes (uint8 or float8_e4m3fn), got {q.dtype}")
+    want = torch.float32 if scale_format == "f32" else torch.uint8
+    if scale.dtype != want:
+        raise BsgemmError(BS_ERR_DTYPE, f"scale_format {scale_format!r} writes {want} scales, got {scale.dtype}")
+
+
+def quantize_fp8_t(x: torch.Tensor, group: str = "128x1", scale_format: str = "f32", q_t: torch.Tensor | None = None,
+                   scale: torch.Tensor | None = None):
+    """Transposed-output e4m3 quantisation of x [R, C] (bf16 or fp32, unit stride along C) for the
+    backward GEMMs: q_t [C, R] (uint8 codes, rows padded to 16 bytes in memory), q_t[c, r] the code of x[r, c].
+
+    group "128x1": one scale per column and 128-row block, scale [C, ceil(R/128)] (scale_a of A = q_t);
+    group "128x128": one scale per 128 x 128 block, scale [ceil(R/128), ceil(C/128)] (scale_b of B_t = q_t).
+    scale_format "f32" (amax / 448) or "e8m0" (uint8 bytes).  Returns (q_t, scale).
+    """
+    _cuda(x, "x")
+    if x.dim() != 2 or x.stride(1) != 1:
+        raise BsgemmError(BS_ERR_LAYOUT, "x must be [R, C] with unit stride along C")
+    if x.dtype not in (torch.bfloat16, torch.float32):
+        raise BsgemmError(BS_ERR_DTYPE, f"x must be bfloat16 or float32, got {x.dtype}")
+    if scale_format not in ("f32", "e8m0"):
+        raise BsgemmError(BS_ERR_DTYPE, f"unknown scale_format {scale_format!r}")
+    if group not in ("128x1", "128x128"):
+        raise BsgemmError(BS_ERR_SHAPE, f"unknown group {group!r}")
+    R, C = x.shape
+    RB, CB = -(-R // 128), -(-C // 128)
+    sshape = (C, RB) if group == "128x1" else (RB, CB)
+    if q_t is None:
+        q_t = _empty_out((C,), R, torch.uint8, x.device)
+    if scale is None:
+        scale = torch.empty(sshape, dtype=torch.float32 if scale_format == "f32" else torch.uint8, device=x.device)
+    _cuda(q_t, "q_t"), _cuda(scale, "scale")
+    _check_quant_out(q_t, scale, scale_format)
+    if q_t.shape != (C, R) or q_t.stride(1) != 1 or scale.shape != sshape or scale.stride(1) != 1:
+        raise BsgemmError(BS_ERR_SHAPE, f"q_t must be [C, R] and scale {list(sshape)}, unit stride along the last dim")
+    _check(lib().bs_quantize_fp8_t(_ptr(x), 0 if x.dtype == torch.bfloat16 else 1, R, C, x.stride(0), _ptr(q_t),
+                                   q_t.stride(0), _ptr(scale), 0 if scale_format == "f32" else 1,
+                                   0 if group == "128x1" else 1, scale.stride(0), _stream(x.device)))
+    return q_t, scale
 
 
 def plan_for(op: int, M: int, G: int, N: int, K: int, num_sms: int = 148) -> dict:

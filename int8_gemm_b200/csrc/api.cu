@@ -7,6 +7,8 @@
 #include <cstring>
 #include <mutex>
 
+#include <cuda_fp8.h>
+
 #include "bsgemm.h"
 #include "launch.h"
 #include "quantize.h"
@@ -219,14 +221,16 @@ uint32_t wide_b_box_rows(int cg) { return static_cast<uint32_t>(kWideBN / cg); }
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
-int out_size(bs_out_dtype t) { return t == BS_OUT_BF16 ? 2 : 4; }
+int out_size(bs_out_dtype t) { return t == BS_OUT_E4M3 ? 1 : (t == BS_OUT_BF16 ? 2 : 4); }
 
 CUtensorMapDataType out_tmap_type(bs_out_dtype t) {
+  if (t == BS_OUT_E4M3) return CU_TENSOR_MAP_DATA_TYPE_UINT8;
   return t == BS_OUT_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                           : (t == BS_OUT_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_INT32);
 }
 
 OutKind out_kind(bs_out_dtype t) {
+  if (t == BS_OUT_E4M3) return OutKind::kE4M3;
   return t == BS_OUT_BF16 ? OutKind::kBF16 : (t == BS_OUT_F32 ? OutKind::kF32 : OutKind::kI32);
 }
 
@@ -473,8 +477,9 @@ bs_status bmm_a8w8_blockscale(const void* x, int64_t x_sm, int64_t x_sg, const v
 }
 
 bs_status bs_gemm_fp8_rowwise(const void* A, int64_t lda, const void* B, int64_t ldb, const float* scale_a,
-                              int64_t sa_stride, const float* scale_b, int64_t sb_stride, const float* bias, void* out,
-                              int64_t ldo, bs_out_dtype out_dtype, int64_t M, int64_t N, int64_t K, void* stream) {
+                              int64_t sa_stride, const float* scale_b, int64_t sb_stride, const float* bias,
+                              const float* scale_result, void* out, int64_t ldo, bs_out_dtype out_dtype, int64_t M,
+                              int64_t N, int64_t K, void* stream) {
   clear_msg();
   if (M < 0 || N < 0 || K < 0) return fail(BS_ERR_SHAPE, "negative size");
   if (M > kMaxDim || N > kMaxDim || K > kMaxDim) return fail(BS_ERR_SHAPE, "size exceeds 2^31-1");
@@ -483,14 +488,17 @@ bs_status bs_gemm_fp8_rowwise(const void* A, int64_t lda, const void* B, int64_t
                 "scales must be both tensorwise (strides 0: scalars) or both rowwise (strides 1: scale_a (M, 1), "
                 "scale_b (1, N)); got strides %lld and %lld",
                 (long long)sa_stride, (long long)sb_stride);
-  if (out_dtype != BS_OUT_BF16 && out_dtype != BS_OUT_F32)
-    return fail(BS_ERR_DTYPE, "bs_gemm_fp8_rowwise writes bf16 or f32 only");
+  if (out_dtype != BS_OUT_BF16 && out_dtype != BS_OUT_F32 && out_dtype != BS_OUT_E4M3)
+    return fail(BS_ERR_DTYPE, "bs_gemm_fp8_rowwise writes bf16, f32 or e4m3 only");
+  if (scale_result && out_dtype != BS_OUT_E4M3)
+    return fail(BS_ERR_DTYPE, "scale_result applies to an e4m3 output only");
   if (M == 0 || N == 0) return BS_OK;
   if (!out) return fail(BS_ERR_NULL, "out is NULL");
   if (ldo < N) return fail(BS_ERR_LAYOUT, "ldo < N");
   if (!aligned16(out) || (ldo * out_size(out_dtype)) % 16 != 0)
     return fail(BS_ERR_ALIGNMENT, "out must be 16-byte aligned with a row stride that is a multiple of 16 bytes");
   if (bias && !aligned4(bias)) return fail(BS_ERR_ALIGNMENT, "bias must be 4-byte aligned");
+  if (scale_result && !aligned4(scale_result)) return fail(BS_ERR_ALIGNMENT, "scale_result must be 4-byte aligned");
   if (K > 0) {
     if (!A || !B || !scale_a || !scale_b) return fail(BS_ERR_NULL, "A, B, scale_a and scale_b must be non-NULL");
     if (lda < K || ldb < K) return fail(BS_ERR_LAYOUT, "lda/ldb must be >= K (A row-major, B column-major)");
@@ -504,7 +512,8 @@ bs_status bs_gemm_fp8_rowwise(const void* A, int64_t lda, const void* B, int64_t
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   const Plan pl = make_plan(4, M, 1, N, K, dc->sms);
   if (pl.pub.kernel == 3)
-    return check_launch(launch_fill_zero(out, out_size(out_dtype), M, N, ldo, 1, 0, cs, bias), "bias-fill launch");
+    return check_launch(launch_fill_zero(out, out_size(out_dtype), M, N, ldo, 1, 0, cs, bias, scale_result),
+                        "bias-fill launch");
 
   GemmArgs args;
   std::memset(&args, 0, sizeof(args));
@@ -519,6 +528,7 @@ bs_status bs_gemm_fp8_rowwise(const void* A, int64_t lda, const void* B, int64_t
   args.s_row_stride = sa_stride;
   args.s_col_stride = sb_stride;
   args.bias = bias;
+  args.s_result = scale_result;
   args.grid_m = pl.grid_m;
   args.grid_n = pl.grid_n;
   args.num_tiles = pl.num_tiles;
@@ -561,6 +571,34 @@ bs_status bs_quantize_fp8_1x128(const void* x, bs_in_dtype x_dtype, int64_t M, i
                                             scale_fmt == BS_SCALE_E8M0, ld_scale, dc->sms,
                                             static_cast<cudaStream_t>(stream)),
                       "quantise launch");
+}
+
+bs_status bs_quantize_fp8_t(const void* x, bs_in_dtype x_dtype, int64_t R, int64_t C, int64_t ldx, void* q_t,
+                           int64_t ldq, void* scale, bs_scale_fmt scale_fmt, bs_group group, int64_t ld_scale,
+                           void* stream) {
+  clear_msg();
+  if (R < 0 || C < 0) return fail(BS_ERR_SHAPE, "negative size");
+  if (R > kMaxDim || C > kMaxDim) return fail(BS_ERR_SHAPE, "size exceeds 2^31-1");
+  if (x_dtype != BS_IN_BF16 && x_dtype != BS_IN_F32) return fail(BS_ERR_DTYPE, "x must be bf16 or f32");
+  if (scale_fmt != BS_SCALE_F32 && scale_fmt != BS_SCALE_E8M0) return fail(BS_ERR_DTYPE, "unknown scale format");
+  if (group != BS_GROUP_128x1 && group != BS_GROUP_128x128) return fail(BS_ERR_SHAPE, "unknown group shape");
+  if (R == 0 || C == 0) return BS_OK;
+  if (!x || !q_t || !scale) return fail(BS_ERR_NULL, "x, q_t and scale must be non-NULL");
+  const int64_t RB = (R + 127) / 128, CB = (C + 127) / 128;
+  const int64_t min_lds = group == BS_GROUP_128x1 ? RB : CB;
+  if (ldx < C || ldq < R || ld_scale < min_lds)
+    return fail(BS_ERR_LAYOUT, "ldx must be >= C, ldq >= R and ld_scale >= %lld", (long long)min_lds);
+  if (RB * CB > kMaxDim) return fail(BS_ERR_SHAPE, "more than 2^31-1 tiles of 128 x 128");
+  const uintptr_t es = x_dtype == BS_IN_BF16 ? 2 : 4;
+  if (reinterpret_cast<uintptr_t>(x) % es != 0) return fail(BS_ERR_ALIGNMENT, "x must be aligned to its element size");
+  if (scale_fmt == BS_SCALE_F32 && !aligned4(scale)) return fail(BS_ERR_ALIGNMENT, "fp32 scales must be 4-byte aligned");
+  DeviceCtx* dc = nullptr;
+  bs_status st = device_ctx(&dc);
+  if (st != BS_OK) return st;
+  return check_launch(launch_quantize_t(x, x_dtype == BS_IN_BF16, R, C, ldx, static_cast<uint8_t*>(q_t), ldq, scale,
+                                        scale_fmt == BS_SCALE_E8M0, group == BS_GROUP_128x128, ld_scale, dc->sms,
+                                        static_cast<cudaStream_t>(stream)),
+                      "transposed quantise launch");
 }
 
 bs_status int_scaled_mm(const int8_t* A, int64_t lda, const int8_t* B, int64_t ldb, const float* s_a,
@@ -632,9 +670,11 @@ bs_status int_scaled_mm(const int8_t* A, int64_t lda, const int8_t* B, int64_t l
 namespace bsg {
 
 // out[b][r][c] = bias[c] (bias may be null: zero).  es = 2 stores bf16, es = 4
-// stores fp32 (or a zero int32).
+// stores fp32 (or a zero int32), es = 1 stores the saturating e4m3 code of
+// s_result[0] * bias[c] (s_result null: 1).
 __global__ void fill_zero_kernel(char* out, int es, long long rows, long long cols, long long ld, long long batches,
-                                 long long bstride, const float* bias) {
+                                 long long bstride, const float* bias, const float* s_result) {
+  const float sr = s_result ? *s_result : 1.f;
   const long long total = rows * cols * batches;
   for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
        i += static_cast<long long>(gridDim.x) * blockDim.x) {
@@ -643,7 +683,9 @@ __global__ void fill_zero_kernel(char* out, int es, long long rows, long long co
     const long long r = rc / cols, c = rc - r * cols;
     char* p = out + (b * bstride + r * ld + c) * es;
     const float v = bias ? bias[c] : 0.f;
-    if (es == 2)
+    if (es == 1)
+      *reinterpret_cast<__nv_fp8_storage_t*>(p) = __nv_cvt_float_to_fp8(v * sr, __NV_SATFINITE, __NV_E4M3);
+    else if (es == 2)
       *reinterpret_cast<__nv_bfloat16*>(p) = __float2bfloat16_rn(v);
     else
       *reinterpret_cast<float*>(p) = v;
@@ -651,12 +693,13 @@ __global__ void fill_zero_kernel(char* out, int es, long long rows, long long co
 }
 
 cudaError_t launch_fill_zero(void* out, int elem_size, long long rows, long long cols, long long ld,
-                             long long batches, long long bstride, cudaStream_t stream, const float* bias) {
+                             long long batches, long long bstride, cudaStream_t stream, const float* bias,
+                             const float* s_result) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   fill_zero_kernel<<<2 * sms, 256, 0, stream>>>(static_cast<char*>(out), elem_size, rows, cols, ld, batches, bstride,
-                                                bias);
+                                                bias, s_result);
   return cudaGetLastError();
 }
 

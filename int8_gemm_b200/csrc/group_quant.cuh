@@ -1,0 +1,48 @@
+// Group-scale and e4m3 code arithmetic shared by the quantiser kernels.
+//
+// For a group with largest magnitude amax:
+//   fp32 scale:  s = amax / 448 (1 when amax == 0), code = e4m3(x / s)
+//   e8m0 scale:  byte = clamp(ceil(log2(amax / 448)) + 127, 0, 254) (127 when
+//                amax == 0), code = e4m3(x * 2^-(byte - 127))
+// with e4m3() rounding to nearest even and saturating at +-448, the largest
+// finite e4m3 magnitude (pytorch issue "torch._scaled_mm with blockwise
+// scaling doesn't work with torch.compile": one fp32 scale per group; ROCm/
+// aiter PR "Add opus fp8 mxscale BMM kernels for gfx950": power-of-two scales).
+#pragma once
+
+#include <cuda_fp8.h>
+#include <stdint.h>
+
+namespace bsg {
+
+// Two saturating round-to-nearest-even e4m3 codes (first value in the low byte).
+__device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
+  return static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3));
+}
+
+__device__ __forceinline__ float group_scale_f32(float amax) { return amax == 0.f ? 1.f : __fdiv_rn(amax, 448.f); }
+
+// fp32(v / s) without an fp32 division per element: v times the fp64
+// reciprocal of s (rinv = __drcp_rn(s)), rounded to fp32.  The fp64 product is
+// within 2^-52 (relative) of v / s, while a quotient of two 24-bit-significand
+// numbers is never an fp32 rounding midpoint and, when it is not exactly
+// representable, lies at least 2^-49 (relative) away from every midpoint, so
+// both round to the same fp32 value.  Quotients in the fp32 subnormal range
+// map to e4m3 zero either way.
+__device__ __forceinline__ float over_scale(float v, double rinv) {
+  return __double2float_rn(__dmul_rn(static_cast<double>(v), rinv));
+}
+
+// The e8m0 byte: ceil(log2(amax / 448)) from amax = f * 2^ex, f in [0.5, 1):
+// with 448 = 0.875 * 2^9 it is ex - 9, plus one when f > 0.875.
+__device__ __forceinline__ int group_e8m0(float amax) {
+  int e = 0;
+  if (amax != 0.f) {
+    int ex;
+    const float f = frexpf(amax, &ex);
+    e = ex - 9 + (f > 0.875f ? 1 : 0);
+  }
+  return e + 127 < 0 ? 0 : (e + 127 > 254 ? 254 : e + 127);
+}
+
+}  // namespace bsg

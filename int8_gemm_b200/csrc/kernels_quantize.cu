@@ -21,8 +21,8 @@
 // warp takes chunks of eight groups (two passes) and keeps all their loads in
 // flight before it reduces any of them.
 #include <cuda_bf16.h>
-#include <cuda_fp8.h>
 
+#include "group_quant.cuh"
 #include "quantize.h"
 
 namespace bsg {
@@ -74,11 +74,6 @@ __device__ __forceinline__ void load16(const InT* row, long long k, long long K,
   }
 }
 
-// Two saturating round-to-nearest-even e4m3 codes (first value in the low byte).
-__device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
-  return static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3));
-}
-
 template <typename InT, int FMT>
 __global__ void __launch_bounds__(kQuantThreads)
     quantize_1x128_kernel(const InT* __restrict__ x, int M, long long K, long long ldx, uint8_t* __restrict__ q,
@@ -116,28 +111,13 @@ __global__ void __launch_bounds__(kQuantThreads)
         amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
       float y[16];
       if constexpr (FMT == 0) {
-        const float s = amax == 0.f ? 1.f : __fdiv_rn(amax, 448.f);
-        // fp32(x / s) without an fp32 division per element: x times the fp64
-        // reciprocal of s, rounded to fp32.  The fp64 product is within 2^-52
-        // (relative) of x / s, while a quotient of two 24-bit-significand
-        // numbers is never an fp32 rounding midpoint and, when it is not
-        // exactly representable, lies at least 2^-49 (relative) away from
-        // every midpoint, so both round to the same fp32 value.  Quotients in
-        // the fp32 subnormal range map to e4m3 zero either way.
+        const float s = group_scale_f32(amax);
         const double rinv = __drcp_rn(static_cast<double>(s));
 #pragma unroll
-        for (int i = 0; i < 16; ++i) y[i] = __double2float_rn(__dmul_rn(static_cast<double>(v[ps][i]), rinv));
+        for (int i = 0; i < 16; ++i) y[i] = over_scale(v[ps][i], rinv);
         if (j == 0 && g < KB) static_cast<float*>(scale)[static_cast<long long>(m) * lds + g] = s;
       } else {
-        // ceil(log2(amax / 448)) from amax = f * 2^ex, f in [0.5, 1): with
-        // 448 = 0.875 * 2^9 it is ex - 9, plus one when f > 0.875
-        int e = 0;
-        if (amax != 0.f) {
-          int ex;
-          const float f = frexpf(amax, &ex);
-          e = ex - 9 + (f > 0.875f ? 1 : 0);
-        }
-        const int byte = e + 127 < 0 ? 0 : (e + 127 > 254 ? 254 : e + 127);
+        const int byte = group_e8m0(amax);
         const float mul = ldexpf(1.f, 127 - byte);  // exact power of two
 #pragma unroll
         for (int i = 0; i < 16; ++i) y[i] = v[ps][i] * mul;

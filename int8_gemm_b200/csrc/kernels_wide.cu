@@ -60,6 +60,7 @@ cudaError_t launch_cg(Mode mode, OutKind out, const CUtensorMap& a, const CUtens
     case Mode::kFp8Rowwise:
       if (out == OutKind::kBF16) return launch_one<Mode::kFp8Rowwise, CG, __nv_bfloat16>(a, b, d, args, grid, stream);
       if (out == OutKind::kF32) return launch_one<Mode::kFp8Rowwise, CG, float>(a, b, d, args, grid, stream);
+      if (out == OutKind::kE4M3) return launch_one<Mode::kFp8Rowwise, CG, uint8_t>(a, b, d, args, grid, stream);
       break;
     case Mode::kFp8Mx:
       if constexpr (CG == 2) {

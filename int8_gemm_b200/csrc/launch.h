@@ -10,7 +10,7 @@
 
 namespace bsg {
 
-enum class OutKind : int { kBF16 = 0, kF32 = 1, kI32 = 2 };
+enum class OutKind : int { kBF16 = 0, kF32 = 1, kI32 = 2, kE4M3 = 3 };
 
 constexpr int kWideBN = 256;
 constexpr int kWideStages = 4;      // single-CTA tiles: 48 KB per stage
@@ -27,10 +27,11 @@ cudaError_t launch_skinny(Mode mode, OutKind out, int bmt, const CUtensorMap& a,
                           const GemmArgs& args, const SkinnyOut& o, int n_tiles, int m_tiles, cudaStream_t stream);
 
 // Fill of `batches` matrices [rows, cols] (row stride ld, batch stride
-// bstride, elements of `elem_size` bytes) with zero, or with bias[col] (fp32
-// [cols]) when bias is given.
+// bstride, elements of `elem_size` bytes: bf16, fp32, or 1 = e4m3) with zero,
+// or with bias[col] (fp32 [cols]) when bias is given; e4m3 elements take the
+// saturating e4m3 of s_result[0] * value (s_result NULL: 1).
 cudaError_t launch_fill_zero(void* out, int elem_size, long long rows, long long cols, long long ld,
                              long long batches, long long bstride, cudaStream_t stream,
-                             const float* bias = nullptr);
+                             const float* bias = nullptr, const float* s_result = nullptr);
 
 }  // namespace bsg

@@ -1,5 +1,5 @@
-// Internal interface of the 1x128 group quantiser (kernels_quantize.cu) for the
-// C-ABI layer.  Not part of the public header.
+// Internal interface of the quantiser kernels (kernels_quantize.cu,
+// kernels_quantize_t.cu) for the C-ABI layer.  Not part of the public header.
 #pragma once
 
 #include <cuda_runtime.h>
@@ -13,5 +13,14 @@ namespace bsg {
 cudaError_t launch_quantize_1x128(const void* x, bool x_bf16, long long M, long long K, long long ldx, uint8_t* q,
                                   long long ldq, void* scale, bool e8m0, long long lds, int sms,
                                   cudaStream_t stream);
+
+// Transposed-output quantisation of x [R, C] (bf16 or fp32, row stride ldx
+// elements) to e4m3 codes q_t [C, R] (row stride ldq bytes), q_t[c][r] the
+// code of x[r][c].  block128 = false: 128x1 groups (rows 128rb.. of one
+// column), scale [C, ceil(R/128)]; true: 128x128 blocks, scale
+// [ceil(R/128), ceil(C/128)]; scale row stride lds, fp32 or e8m0 bytes.
+cudaError_t launch_quantize_t(const void* x, bool x_bf16, long long R, long long C, long long ldx, uint8_t* q_t,
+                              long long ldq, void* scale, bool e8m0, bool block128, long long lds, int sms,
+                              cudaStream_t stream);
 
 }  // namespace bsg

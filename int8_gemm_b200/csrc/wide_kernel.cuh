@@ -46,6 +46,8 @@
 // zero-filled by the TMA loads, so ragged M needs no padding copies.
 #pragma once
 
+#include <cuda_fp8.h>
+
 #include <type_traits>
 
 #include "sm100.cuh"
@@ -80,11 +82,13 @@ struct GemmArgs {
   // and s_col[n] and allows either to be null.  FP8 rowwise reads s_row[m]
   // when s_row_stride is 1 and s_row[0] when it is 0 (tensorwise), likewise
   // for s_col; the strides are 0 or 1 and are applied as a select.  bias:
-  // fp32 [N] or null (FP8 rowwise).
+  // fp32 [N] or null (FP8 rowwise).  s_result: fp32 scalar or null, the
+  // factor an e4m3 output of FP8 rowwise takes before its cast.
   const float* s_row;
   const float* s_col;
   long long s_row_stride, s_col_stride;
   const float* bias;
+  const float* s_result;
   uint32_t* err;
 };
 
@@ -165,7 +169,8 @@ __device__ __forceinline__ float block_scale(const GemmArgs& p, int g, int m, in
 // Write one 64-byte staging row (this lane's output row; CPC = 64 / sizeof(OutT)
 // values) with the 64-byte swizzle of the output tensor map: 16-byte unit u of
 // row r lives at unit u ^ ((r >> 1) & 3), which also keeps the 8 rows a
-// quarter-warp writes at once on distinct banks.
+// quarter-warp writes at once on distinct banks.  One-byte outputs are e4m3
+// codes, rounded to nearest even and saturated at +-448.
 template <typename OutT, int CPC>
 __device__ __forceinline__ void stage_row64(uint8_t* stg, int lane, const float (&v)[CPC]) {
   uint8_t* row = stg + lane * 64;
@@ -173,7 +178,14 @@ __device__ __forceinline__ void stage_row64(uint8_t* stg, int lane, const float 
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
     uint4 w;
-    if constexpr (sizeof(OutT) == 2) {
+    if constexpr (sizeof(OutT) == 1) {
+      uint32_t c[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        c[i] = __nv_cvt_float2_to_fp8x2(make_float2(v[q * 16 + 2 * i], v[q * 16 + 2 * i + 1]), __NV_SATFINITE,
+                                        __NV_E4M3);
+      w = make_uint4(c[0] | (c[1] << 16), c[2] | (c[3] << 16), c[4] | (c[5] << 16), c[6] | (c[7] << 16));
+    } else if constexpr (sizeof(OutT) == 2) {
       __nv_bfloat162 h0 = __floats2bfloat162_rn(v[q * 8 + 0], v[q * 8 + 1]);
       __nv_bfloat162 h1 = __floats2bfloat162_rn(v[q * 8 + 2], v[q * 8 + 3]);
       __nv_bfloat162 h2 = __floats2bfloat162_rn(v[q * 8 + 4], v[q * 8 + 5]);
@@ -663,6 +675,7 @@ __global__ void __launch_bounds__(384, 1)
         // FP8 rowwise: this thread's column scales start at s_col_n and advance by col_step
         const int col_step = !IS_INT8 && p.s_col_stride != 0 ? 1 : 0;
         const float* s_col_n = IS_INT8 ? nullptr : p.s_col + ncol0 * col_step;
+        const float s_res = sizeof(OutT) == 1 && p.s_result != nullptr ? __ldg(p.s_result) : 1.f;
         const uint32_t tb = tmem + t_lane + acc_col(buf) + static_cast<uint32_t>(half * 128);
         // kFp8Mx: the 32 columns this buffer shares with the other one are
         // the last of half 1 (buffer 0) or the first of half 0 (buffer 1);
@@ -677,7 +690,9 @@ __global__ void __launch_bounds__(384, 1)
           __syncwarp();
           const int c0 = (MX ? (ch + rot) % NCH : ch) * CPC;
           uint32_t r[CPC];
-          if constexpr (CPC == 32) {
+          if constexpr (CPC == 64) {
+            tmem_ld64(tb + c0, r);
+          } else if constexpr (CPC == 32) {
             tmem_ld32(tb + c0, r);
           } else {
             tmem_ld16(tb + c0, r);
@@ -704,6 +719,10 @@ __global__ void __launch_bounds__(384, 1)
               const float sc = n < p.N ? __ldg(s_col_n + (c0 + j) * col_step) : 0.f;
               const float bn = (p.bias != nullptr && n < p.N) ? __ldg(p.bias + n) : 0.f;
               v[j] = fmaf(__uint_as_float(r[j]), sr * sc, bn);
+            }
+            if constexpr (sizeof(OutT) == 1) {
+#pragma unroll
+              for (int j = 0; j < CPC; ++j) v[j] *= s_res;  // output scale of the e4m3 result
             }
           } else {
 #pragma unroll

@@ -12,6 +12,11 @@ of magnitude below 1e-3 * S; the ulp term covers the final rounding.
 
 INT8 (operation 2): bit-exact for the int32 accumulator, the fp32
 (float(acc) * s_a) * s_b and its bf16 rounding.
+
+e4m3 outputs (scale_result of the rowwise operation): the kernel rounds an
+fp32 value z within |s_r| * (1e-3 * S + ulp_f32(y)) + ulp_f32(s_r * y) of
+s_r * y, and e4m3 rounding is monotone, so its code must lie between the codes
+of the two ends of that interval.
 """
 from __future__ import annotations
 
@@ -72,3 +77,22 @@ def rows_sample(M: int, tile: int = 128, extra: int = 8, seed: int = 0):
 
 def oracle_fp8(d, rows=None):
     return oracle.fp8_blockwise(d["A"], d["B_t"], d["scale_a"], d["scale_b"], rows=rows)
+
+
+def e4m3_check(gpu: torch.Tensor, y: np.ndarray, S: np.ndarray, s_r: float, label: str = ""):
+    """Asserts an e4m3 output against the oracle value y before the output scale s_r;
+    returns the fraction of codes equal to the oracle's own rounding of s_r * y."""
+    codes = gpu.detach().cpu().view(torch.uint8).numpy()
+    assert codes.shape == y.shape, (codes.shape, y.shape)
+    table = oracle.e4m3_table()
+    g = table[codes]
+    assert not np.any(np.isnan(g)), f"{label}: NaN codes in a saturating output"
+    z = s_r * y
+    d = abs(s_r) * (1e-3 * S + ulp_at(y, torch.float32)) + ulp_at(z, torch.float32)
+    lo, hi = table[oracle.e4m3_encode(z - d)], table[oracle.e4m3_encode(z + d)]
+    bad = (g < lo) | (g > hi)
+    if np.any(bad):
+        idx = np.unravel_index(int(np.argmax(bad)), bad.shape)
+        raise AssertionError(f"{label}: {int(bad.sum())} of {bad.size} codes outside the rounding window; first at "
+                             f"{idx}: gpu={g[idx]!r} oracle s_r*y={z[idx]!r} window=[{lo[idx]!r}, {hi[idx]!r}]")
+    return float(np.mean(codes == oracle.e4m3_encode(z)))

@@ -194,13 +194,13 @@ def test_fp8_validation_codes():
 
 
 def _rw(**kw):
-    a = dict(A=P16, lda=256, B=P16, ldb=256, sa=P16, sas=1, sb=P16, sbs=1, bias=None, out=P16, ldo=256,
+    a = dict(A=P16, lda=256, B=P16, ldb=256, sa=P16, sas=1, sb=P16, sbs=1, bias=None, sres=None, out=P16, ldo=256,
              dt=bs.BS_OUT_BF16, M=64, N=256, K=200)
     a.update(kw)
     v = ctypes.c_void_p
     return bs.lib().bs_gemm_fp8_rowwise(v(a["A"]), a["lda"], v(a["B"]), a["ldb"], v(a["sa"]), a["sas"], v(a["sb"]),
-                                        a["sbs"], v(a["bias"]), v(a["out"]), a["ldo"], a["dt"], a["M"], a["N"], a["K"],
-                                        None)
+                                        a["sbs"], v(a["bias"]), v(a["sres"]), v(a["out"]), a["ldo"], a["dt"], a["M"],
+                                        a["N"], a["K"], None)
 
 
 def test_fp8_rowwise_validation_codes():
@@ -213,8 +213,16 @@ def test_fp8_rowwise_validation_codes():
     assert _rw(lda=128) == bs.BS_ERR_LAYOUT and _rw(ldo=100) == bs.BS_ERR_LAYOUT
     assert _rw(lda=264) == bs.BS_ERR_ALIGNMENT and _rw(bias=P16 + 2) == bs.BS_ERR_ALIGNMENT
     assert _rw(M=0) == bs.BS_OK and _rw(N=0) == bs.BS_OK
-    # K need not be a multiple of 128 here (scales are constant along K): a well-formed call only fails on the device
-    assert _rw(K=200) == bs.BS_ERR_DEVICE and _rw(sas=0, sbs=0, K=48) == bs.BS_ERR_DEVICE
+    # e4m3 output: an optional output scale, rows of N bytes on 16-byte boundaries
+    e8 = bs.BS_OUT_E4M3
+    assert _rw(sres=P16) == bs.BS_ERR_DTYPE and _rw(dt=bs.BS_OUT_F32, sres=P16) == bs.BS_ERR_DTYPE
+    assert _rw(dt=e8, sres=P16 + 2) == bs.BS_ERR_ALIGNMENT
+    assert _rw(dt=e8, N=200, ldo=200) == bs.BS_ERR_ALIGNMENT and _rw(dt=e8, ldo=100) == bs.BS_ERR_LAYOUT
+    assert _rw(dt=e8, sres=P16, N=0) == bs.BS_OK
+    if not HAS_GPU:  # well-formed calls reach the device check (never launched with fake pointers on a GPU)
+        # K need not be a multiple of 128 here (scales are constant along K)
+        assert _rw(K=200) == bs.BS_ERR_DEVICE and _rw(sas=0, sbs=0, K=48) == bs.BS_ERR_DEVICE
+        assert _rw(dt=e8, sres=P16, N=200, ldo=208) == bs.BS_ERR_DEVICE and _rw(dt=e8, K=0) == bs.BS_ERR_DEVICE
 
 
 def test_plan_fp8_rowwise_is_the_wide_kernel_for_every_m():
@@ -289,3 +297,28 @@ def test_quantize_validation_codes():
     if not HAS_GPU:  # well-formed calls reach the device check (never launched with fake pointers on a GPU)
         for kw in ({}, {"x": P16 + 2}, {"q": P16 + 1}, {"ldx": 300}, {"ldq": 301}, {"fmt": 1, "s": P16 + 3}):
             assert _qz(**kw) == bs.BS_ERR_DEVICE, kw
+
+
+def _qt(**kw):
+    a = dict(x=P16, dt=0, R=300, C=200, ldx=208, q=P16, ldq=304, s=P16, fmt=0, grp=0, lds=3)
+    a.update(kw)
+    v = ctypes.c_void_p
+    return bs.lib().bs_quantize_fp8_t(v(a["x"]), a["dt"], a["R"], a["C"], a["ldx"], v(a["q"]), a["ldq"], v(a["s"]),
+                                      a["fmt"], a["grp"], a["lds"], None)
+
+
+def test_quantize_t_validation_codes():
+    assert _qt(R=-1) == bs.BS_ERR_SHAPE and _qt(C=-5) == bs.BS_ERR_SHAPE and _qt(R=1 << 31) == bs.BS_ERR_SHAPE
+    assert _qt(grp=2) == bs.BS_ERR_SHAPE
+    assert _qt(R=1 << 30, C=1 << 30, ldx=1 << 30, ldq=1 << 30, lds=1 << 23) == bs.BS_ERR_SHAPE  # 2^46 tiles
+    assert _qt(dt=2) == bs.BS_ERR_DTYPE and _qt(fmt=2) == bs.BS_ERR_DTYPE
+    assert _qt(x=0) == bs.BS_ERR_NULL and _qt(q=0) == bs.BS_ERR_NULL and _qt(s=0) == bs.BS_ERR_NULL
+    assert _qt(ldx=199) == bs.BS_ERR_LAYOUT and _qt(ldq=299) == bs.BS_ERR_LAYOUT
+    assert _qt(lds=2) == bs.BS_ERR_LAYOUT               # 128x1: ceil(300 / 128) = 3 scales per column
+    assert _qt(grp=1, lds=1) == bs.BS_ERR_LAYOUT        # 128x128: ceil(200 / 128) = 2 scales per block row
+    assert _qt(x=P16 + 1) == bs.BS_ERR_ALIGNMENT and _qt(dt=1, x=P16 + 2) == bs.BS_ERR_ALIGNMENT
+    assert _qt(s=P16 + 2) == bs.BS_ERR_ALIGNMENT
+    assert _qt(R=0) == bs.BS_OK and _qt(C=0) == bs.BS_OK
+    if not HAS_GPU:  # well-formed calls reach the device check (never launched with fake pointers on a GPU)
+        for kw in ({}, {"grp": 1, "lds": 2}, {"x": P16 + 2}, {"q": P16 + 1}, {"ldx": 201}, {"fmt": 1, "s": P16 + 3}):
+            assert _qt(**kw) == bs.BS_ERR_DEVICE, kw

@@ -15,7 +15,7 @@ import torch
 import int8_gemm_b200 as bs
 import oracle
 import workloads as wl
-from parity import bf16_bits, f32_bits, fp8_check, oracle_fp8, rows_sample, to_f64
+from parity import bf16_bits, e4m3_check, f32_bits, fp8_check, oracle_fp8, rows_sample, to_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -163,10 +163,11 @@ def test_fp8_transposed_scale_a_layout():
 # ---------------------------------------------------------------------------
 # FP8 with tensorwise / rowwise scales and bias
 # ---------------------------------------------------------------------------
-def rowwise_run(d, out_dtype=torch.bfloat16, bias=True, out=None):
+def rowwise_run(d, out_dtype=torch.bfloat16, bias=True, out=None, scale_result=None):
     b = d["bias"].to(DEV) if (bias and d["bias"] is not None) else None
+    sr = None if scale_result is None else torch.tensor(scale_result, dtype=torch.float32, device=DEV)
     return bs.bs_gemm_fp8_rowwise(d["A"].to(DEV), d["B_t"].to(DEV).t(), d["scale_a"].to(DEV), d["scale_b"].to(DEV), b,
-                                  out_dtype=out_dtype, out=out)
+                                  out_dtype=out_dtype, out=out, scale_result=sr)
 
 
 def oracle_rowwise(d, bias=True, rows=None):
@@ -185,6 +186,48 @@ def test_fp8_rowwise_and_tensorwise(M, N, K, tensorwise, kernel, path):
             y, S = oracle_rowwise(d, bias)
             fp8_check(rowwise_run(d, out_dtype, bias), y, S, out_dtype,
                       f"fp8 rowwise {M}x{N}x{K} tensorwise={tensorwise} bias={bias}")
+
+
+@pytest.mark.parametrize("M,N,K", [(256, 256, 512), (300, 520, 640), (1, 256, 128), (129, 384, 176), (5, 259, 48)])
+@pytest.mark.parametrize("tensorwise", [False, True])
+@pytest.mark.parametrize("kernel", [bs.PATH_AUTO, bs.PATH_WIDE_SINGLE])
+def test_fp8_rowwise_e4m3_output_with_scale_result(M, N, K, tensorwise, kernel, path):
+    path(kernel)
+    d = wl.fp8_rowwise_inputs(M, N, K, seed=160 + M + N + K, tensorwise=tensorwise)
+    for bias in (True, False):
+        y, S = oracle_rowwise(d, bias)
+        top = float(np.abs(y).max())
+        # no output scale; one that maps the largest |y| to 300 (no saturation);
+        # one that maps it to 3000, so the largest outputs saturate at +-448
+        for s_r in (None, np.float32(300.0 / top), np.float32(3000.0 / top)):
+            out = rowwise_run(d, torch.float8_e4m3fn, bias, scale_result=None if s_r is None else float(s_r))
+            assert out.dtype == torch.float8_e4m3fn and tuple(out.shape) == (M, N)
+            same = e4m3_check(out, y, S, 1.0 if s_r is None else float(s_r),
+                              f"fp8 rowwise e4m3 {M}x{N}x{K} tensorwise={tensorwise} bias={bias} s_r={s_r}")
+            assert same > 0.97, f"only {same:.3f} of codes equal the oracle's rounding"
+        sat = rowwise_run(d, torch.float8_e4m3fn, bias, scale_result=float(np.float32(3000.0 / top)))
+        assert float(sat.float().abs().max()) == 448.0
+
+
+def test_fp8_rowwise_e4m3_output_k0_and_use_fast_accum():
+    bias = torch.randn(208, generator=torch.Generator().manual_seed(161)).to(DEV) * 100
+    A = torch.zeros(16, 0, dtype=torch.uint8, device=DEV)
+    B = torch.zeros(208, 0, dtype=torch.uint8, device=DEV).t()
+    sr = torch.tensor([2.0], device=DEV)  # a power of two: the fp32 product is exact
+    out = bs.bs_gemm_fp8_rowwise(A, B, torch.ones(16, 1, device=DEV), torch.ones(1, 208, device=DEV), bias,
+                                 out_dtype=torch.float8_e4m3fn, scale_result=sr)
+    want = oracle.e4m3_encode(2.0 * bias.cpu().double().numpy())  # |2 bias| reaches past 448: saturation too
+    assert np.array_equal(out.cpu().view(torch.uint8).numpy(), np.broadcast_to(want, (16, 208)))
+    # use_fast_accum selects nothing on this hardware: the results are identical
+    d = wl.fp8_rowwise_inputs(300, 512, 1024, seed=162)
+    for dt in (torch.bfloat16, torch.float8_e4m3fn):
+        a = bs.bs_gemm_fp8_rowwise(d["A"].to(DEV), d["B_t"].to(DEV).t(), d["scale_a"].to(DEV), d["scale_b"].to(DEV),
+                                   d["bias"].to(DEV), out_dtype=dt, use_fast_accum=True)
+        b = rowwise_run(d, dt)
+        assert torch.equal(a.view(torch.uint8) if dt != torch.bfloat16 else a,
+                           b.view(torch.uint8) if dt != torch.bfloat16 else b)
+    with pytest.raises(bs.BsgemmError):  # an output scale is only defined for an e4m3 result
+        rowwise_run(d, torch.bfloat16, scale_result=2.0)
 
 
 def test_fp8_rowwise_k0_writes_bias_and_is_deterministic():
@@ -209,6 +252,9 @@ def test_fp8_rowwise_16640x5120x8192_sampled_rows():
     rows = rows_sample(w.M, extra=6)
     y, S = oracle_rowwise(d, rows=rows)
     fp8_check(out[torch.tensor(rows, device=DEV)], y, S, torch.bfloat16, "fp8 rowwise 16640x5120x8192")
+    s_r = float(np.float32(400.0 / float(np.abs(y).max())))
+    out8 = rowwise_run(d, torch.float8_e4m3fn, scale_result=s_r)
+    e4m3_check(out8[torch.tensor(rows, device=DEV)], y, S, s_r, "fp8 rowwise e4m3 16640x5120x8192")
 
 
 # ---------------------------------------------------------------------------
@@ -372,3 +418,80 @@ def test_quantize_then_blockwise_gemm_matches_the_oracle():
     rq, rsa = oracle.quantize_1x128(x, 0)
     y, S = oracle.fp8_blockwise(rq, Bq.t().contiguous(), rsa, sb)
     fp8_check(out, y, S, torch.bfloat16, "quantise + blockwise GEMM")
+
+
+# ---------------------------------------------------------------------------
+# transposed-output quantiser (128x1 and 128x128 groups) and the backward GEMMs
+# ---------------------------------------------------------------------------
+def _quant_t_check(x_dev, group, fmt, **kw):
+    qt, s = bs.quantize_fp8_t(x_dev, group, "f32" if fmt == 0 else "e8m0", **kw)
+    rq, rs = oracle.quantize_t(x_dev.float().cpu(), 0 if group == "128x1" else 1, fmt)
+    gq, gs = qt.cpu().numpy(), s.cpu().numpy()
+    assert gq.shape == rq.shape and gs.shape == rs.shape
+    bad = np.argwhere(gq != rq)
+    assert bad.size == 0, f"{len(bad)} codes differ, first at {bad[0]}: gpu {gq[tuple(bad[0])]:#x} oracle {rq[tuple(bad[0])]:#x}"
+    if fmt == 0:
+        assert np.array_equal(gs.view(np.uint32), rs.view(np.uint32)), "fp32 scales differ"
+    else:
+        assert np.array_equal(gs, rs), "e8m0 bytes differ"
+    return qt, s
+
+
+@pytest.mark.parametrize("R,C", [(1, 1), (128, 128), (300, 5), (5, 300), (130, 260), (1000, 384), (4096, 640)])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("group", ["128x1", "128x128"])
+@pytest.mark.parametrize("fmt", [0, 1])
+def test_quantize_t_bit_exact(R, C, dtype, group, fmt):
+    x = wl.normal_with_outliers((R, C), 7400 + R + C).to(dtype)
+    _quant_t_check(x.to(DEV), group, fmt)
+
+
+@pytest.mark.parametrize("group", ["128x1", "128x128"])
+@pytest.mark.parametrize("fmt", [0, 1])
+def test_quantize_t_special_blocks_strides_and_canaries(group, fmt):
+    R, C = 260, 136
+    x = wl.normal_with_outliers((R, C), 7500)
+    x[:128, :128] = 0.0                                  # an all-zero block / columns
+    x[128:256, 0] = 448.0 * 2.0 ** 5                     # amax exactly 448 * 2^5
+    x[128:256, 1] = torch.linspace(-1.0, 1.0, 128)      # a tie-rich ramp
+    x[256:, 5] = 1e-30                                   # tiny values
+    x[3, 130] = 3e20                                     # one huge value
+    base = torch.zeros(R, 141)                           # row stride 141: no 16-byte loads
+    base[:, :C] = x
+    xv = base.to(DEV)[:, :C]
+    q = torch.full((C, 288), 0x55, dtype=torch.uint8, device=DEV)[:, :R]  # rows of 288 bytes, R = 260 used
+    sshape = (C, 3) if group == "128x1" else (3, 2)
+    s = torch.zeros((sshape[0], sshape[1] + 3), dtype=torch.float32 if fmt == 0 else torch.uint8,
+                    device=DEV)[:, :sshape[1]]
+    _quant_t_check(xv, group, fmt, q_t=q, scale=s)
+    full = torch.as_strided(q, (C, 288), (288, 1))
+    assert torch.all(full[:, R:] == 0x55), "wrote past R"
+
+
+def test_quantize_t_full_size_output_gradient():
+    dy = wl.normal_with_outliers((16640, 5120), 7600).to(torch.bfloat16).to(DEV)
+    _quant_t_check(dy, "128x1", 0)
+
+
+def test_backward_gemms_through_the_transposed_quantiser():
+    M, N, K = 384, 256, 640  # tokens, output features, input features of y = x W^T
+    x = wl.normal_with_outliers((M, K), 7700)
+    dy = wl.normal_with_outliers((M, N), 7701)
+    W = wl.normal_with_outliers((N, K), 7702)
+    # weight gradient dW [N, K] = dy^T x: contraction over the M tokens
+    a, sa = bs.quantize_fp8_t(dy.to(DEV), "128x1")
+    b, sb = bs.quantize_fp8_t(x.to(DEV), "128x128")
+    dW = bs.bs_gemm_fp8_blockwise(a, b.t(), sa, sb)
+    ra, rsa = oracle.quantize_t(dy, 0, 0)
+    rb, rsb = oracle.quantize_t(x, 1, 0)
+    assert np.array_equal(a.cpu().numpy(), ra) and np.array_equal(b.cpu().numpy(), rb)
+    y, S = oracle.fp8_blockwise(ra, rb, rsa, rsb)
+    fp8_check(dW, y, S, torch.bfloat16, "weight gradient")
+    # input gradient dx [M, K] = dy W: contraction over the N outputs
+    a2, sa2 = bs.quantize_fp8_1x128(dy.to(DEV), "f32")
+    b2, sb2 = bs.quantize_fp8_t(W.to(DEV), "128x128")
+    dx = bs.bs_gemm_fp8_blockwise(a2, b2.t(), sa2, sb2)
+    ra2, rsa2 = oracle.quantize_1x128(dy, 0)
+    rb2, rsb2 = oracle.quantize_t(W, 1, 0)
+    y2, S2 = oracle.fp8_blockwise(ra2, rb2, rsa2, rsb2)
+    fp8_check(dx, y2, S2, torch.bfloat16, "input gradient")

@@ -599,3 +599,23 @@ def test_quantize_t_block_scale_is_the_largest_column_scale_of_the_block(fmt):
             assert sb[rb, cb] == cols.max()
             c = 128 * cb + int(np.argmax(cols))
             assert np.array_equal(qb[c, 128 * rb:128 * rb + 128], qc[c, 128 * rb:128 * rb + 128])
+
+
+def test_backward_gemms_of_the_quantised_operands_approximate_the_exact_gradients():
+    # dW = dy^T x and dx = dy W through the transposed quantiser: e4m3 keeps 3
+    # mantissa bits, so the result is the exact gradient within a few percent
+    # (a transposed or misgrouped operand gives an unrelated matrix)
+    M, N, K = 256, 128, 384
+    x = wl.normal_with_outliers((M, K), 901)
+    dy = wl.normal_with_outliers((M, N), 902)
+    W = wl.normal_with_outliers((N, K), 903)
+    xd, dyd, Wd = x.double().numpy(), dy.double().numpy(), W.double().numpy()
+    a, sa = oracle.quantize_t(dy, 0, 0)
+    b, sb = oracle.quantize_t(x, 1, 0)
+    dW, _ = oracle.fp8_blockwise(a, b, sa, sb)
+    a2, sa2 = oracle.quantize_1x128(dy, 0)
+    b2, sb2 = oracle.quantize_t(W, 1, 0)
+    dx, _ = oracle.fp8_blockwise(a2, b2, sa2, sb2)
+    for got, want in ((dW, dyd.T @ xd), (dx, dyd @ Wd)):
+        assert got.shape == want.shape
+        assert np.linalg.norm(got - want) / np.linalg.norm(want) < 0.06

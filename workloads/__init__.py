@@ -44,7 +44,7 @@ GROUP = 128  # quantisation group / block edge along K (and N for weights)
 @dataclass(frozen=True)
 class Workload:
     name: str
-    op: str  # "fp8_blockwise" | "int_scaled_mm" | "bmm_a8w8_blockscale" | "fp8_rowwise" | "quantize_1x128"
+    op: str  # "fp8_blockwise" | "int_scaled_mm" | "bmm_a8w8_blockscale" | "fp8_rowwise" | "quantize_1x128" | "quantize_t"
     M: int
     N: int
     K: int
@@ -59,8 +59,17 @@ WORKLOADS = {
     "fp8_16640x5120x8192": Workload("fp8_16640x5120x8192", "fp8_blockwise", 16640, 5120, 8192, seed=2),
     # the rowwise-scaled form of the same shape (the mode the blockwise issue's error message names)
     "fp8_rowwise_16640x5120x8192": Workload("fp8_rowwise_16640x5120x8192", "fp8_rowwise", 16640, 5120, 8192, seed=5),
+    # the same, with an e4m3 result: output scale 448 / 4096 (a result amax of 4096, just above this data's)
+    "fp8_rowwise_e4m3out_16640x5120x8192": Workload("fp8_rowwise_e4m3out_16640x5120x8192", "fp8_rowwise", 16640, 5120,
+                                                    8192, seed=5, extra={"out": "e4m3", "scale_result": 0.109375}),
     # the activations of the 16640x5120x8192 shape, bf16, quantised to e4m3 per 1x128 group (fp32 scales)
     "quant_1x128_16640x8192_bf16": Workload("quant_1x128_16640x8192_bf16", "quantize_1x128", 16640, 0, 8192, seed=6),
+    # the backward operands of the same layer, quantised transposed: the output gradient dy [16640, 5120] in
+    # 128x1 groups (A of the weight gradient) and the activations x [16640, 8192] in 128x128 blocks (its B)
+    "quant_t_128x1_16640x5120_bf16": Workload("quant_t_128x1_16640x5120_bf16", "quantize_t", 16640, 0, 5120, seed=7,
+                                              extra={"group": "128x1"}),
+    "quant_t_128x128_16640x8192_bf16": Workload("quant_t_128x128_16640x8192_bf16", "quantize_t", 16640, 0, 8192,
+                                                seed=8, extra={"group": "128x128"}),
 }
 BMM_M_SWEEP = (1, 16, 128, 1024, 16384)
 BMM_G = (8, 2)
@@ -255,6 +264,6 @@ def workload_inputs(w: Workload, sweep: int = 0, batch_first: bool = False):
         return int8_inputs(w.M, w.N, w.K, base)
     if w.op == "fp8_rowwise":
         return fp8_rowwise_inputs(w.M, w.N, w.K, base)
-    if w.op == "quantize_1x128":
+    if w.op in ("quantize_1x128", "quantize_t"):
         return {"x": normal_with_outliers((w.M, w.K), base + 10 * 7).to(torch.bfloat16)}
     return bmm_inputs(w.M, w.G, w.N, w.K, base, batch_first=batch_first)
