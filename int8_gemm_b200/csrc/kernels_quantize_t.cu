@@ -15,12 +15,14 @@
 // GEMM), and 128x128 blocks give its scale_b.
 //
 // One CTA quantises a 128 x 128 tile at a time (persistent over tiles).  The
-// tile is read row by row with 16-byte loads into shared memory as fp32;
-// thread t then owns column t % 128, rows 64 (t / 128) .. + 63, reading them
-// down the column (a warp reads 32 consecutive floats of one row per step, no
-// bank conflicts).  The column halves' amaxes meet in shared memory (128x1),
-// or the whole tile's in a block reduction (128x128).  Each thread writes its
-// 64 codes, contiguous in q_t, as four 16-byte stores.
+// tile is read row by row with 16-byte loads and kept in shared memory in the
+// input type; thread t then owns column t % 128, rows 64 (t / 128) .. + 63,
+// reading them down the column (a warp reads 32 consecutive elements of one
+// row per step, no bank conflicts) once for the amax and once to quantise, so
+// few registers are live and several CTAs share an SM: while one quantises,
+// the others' loads are in flight.  The column halves' amaxes meet in shared
+// memory (128x1), or the whole tile's in a block reduction (128x128).  Each
+// thread writes its 64 codes, contiguous in q_t, as four 16-byte stores.
 #include <cuda_bf16.h>
 
 #include <cstring>
@@ -34,12 +36,20 @@ namespace {
 
 constexpr int kTile = 128;
 constexpr int kThreads = 256;
+// CTAs per SM the register budget is sized for: four bf16 tiles (32 KB each),
+// three fp32 tiles (64 KB each, which also hold twice the loads in flight)
+template <typename InT>
+constexpr int kMinBlocks = sizeof(InT) == 2 ? 4 : 3;
 
+template <typename InT>
 struct TileSmem {
-  float v[kTile][kTile];  // the tile as fp32, [row][column]
-  float part[2][kTile];   // per-column amax of the two row halves
+  InT v[kTile][kTile];   // the tile, [row][column]
+  float part[2][kTile];  // per-column amax of the two row halves
   float wmax[kThreads / 32];
 };
+
+__device__ __forceinline__ float to_f32(float v) { return v; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
 
 // Tile rows are read as 16-byte vectors: 8 bf16 or 4 fp32 elements.
 template <typename InT>
@@ -49,34 +59,16 @@ struct Vec {
   static constexpr int kPerThread = kTile * kPerRow / kThreads;
 };
 
-template <typename InT>
-__device__ __forceinline__ void unpack(const uint4& u, float* out) {
-  if constexpr (sizeof(InT) == 4) {
-    out[0] = __uint_as_float(u.x);
-    out[1] = __uint_as_float(u.y);
-    out[2] = __uint_as_float(u.z);
-    out[3] = __uint_as_float(u.w);
-  } else {
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const __nv_bfloat162 h = *reinterpret_cast<const __nv_bfloat162*>(&w[j]);
-      out[2 * j] = __low2float(h);
-      out[2 * j + 1] = __high2float(h);
-    }
-  }
-}
-
 // GROUP 0: 128x1 groups; GROUP 1: 128x128 blocks.  FMT 0: fp32 scales; 1: e8m0.
 // vec_x: x and its row stride allow 16-byte loads; vec_q: q_t and its row
 // stride allow 16-byte stores.
 template <typename InT, int FMT, int GROUP>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, kMinBlocks<InT>)
     quantize_t_kernel(const InT* __restrict__ x, long long R, long long C, long long ldx, uint8_t* __restrict__ q,
                       long long ldq, void* __restrict__ scale, long long lds, long long ctiles, long long ntiles,
                       bool vec_x, bool vec_q) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
-  TileSmem& sm = *reinterpret_cast<TileSmem*>(smem_raw);
+  TileSmem<InT>& sm = *reinterpret_cast<TileSmem<InT>*>(smem_raw);
   using V = Vec<InT>;
   const int t = threadIdx.x;
   const int col = t % kTile;   // this thread's column in the compute phase
@@ -104,22 +96,14 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll
     for (int k = 0; k < V::kPerThread; ++k) {
       const int i = k * kThreads + t;
-      float f[V::kElems];
-      unpack<InT>(raw[k], f);
-      float* dst = &sm.v[i / V::kPerRow][(i % V::kPerRow) * V::kElems];
-#pragma unroll
-      for (int j = 0; j < V::kElems; j += 4)
-        *reinterpret_cast<float4*>(dst + j) = make_float4(f[j], f[j + 1], f[j + 2], f[j + 3]);
+      *reinterpret_cast<uint4*>(&sm.v[i / V::kPerRow][(i % V::kPerRow) * V::kElems]) = raw[k];
     }
     __syncthreads();
-    // this thread's 64 values, down its column
-    float v[64];
+    // the amax of this thread's 64 values, down its column
+    const InT* colp = &sm.v[64 * half][col];
     float amax = 0.f;
-#pragma unroll
-    for (int i = 0; i < 64; ++i) {
-      v[i] = sm.v[64 * half + i][col];
-      amax = fmaxf(amax, fabsf(v[i]));
-    }
+#pragma unroll 16
+    for (int i = 0; i < 64; ++i) amax = fmaxf(amax, fabsf(to_f32(colp[i * kTile])));
     if constexpr (GROUP == 0) {
       sm.part[half][col] = amax;
       __syncthreads();
@@ -159,7 +143,10 @@ __global__ void __launch_bounds__(kThreads)
     for (int k = 0; k < 4; ++k) {
       float y[16];
 #pragma unroll
-      for (int j = 0; j < 16; ++j) y[j] = FMT == 0 ? over_scale(v[16 * k + j], rinv) : v[16 * k + j] * mul;
+      for (int j = 0; j < 16; ++j) {
+        const float e = to_f32(colp[(16 * k + j) * kTile]);
+        y[j] = FMT == 0 ? over_scale(e, rinv) : e * mul;
+      }
       uint4 codes;
       codes.x = e4m3x2(y[0], y[1]) | (e4m3x2(y[2], y[3]) << 16);
       codes.y = e4m3x2(y[4], y[5]) | (e4m3x2(y[6], y[7]) << 16);
@@ -183,7 +170,7 @@ cudaError_t launch_t(const void* x, long long R, long long C, long long ldx, uin
                      long long lds, int sms, cudaStream_t stream) {
   const long long ctiles = (C + kTile - 1) / kTile;
   const long long ntiles = ((R + kTile - 1) / kTile) * ctiles;
-  const size_t smem = sizeof(TileSmem);
+  const size_t smem = sizeof(TileSmem<InT>);
   cudaError_t e = cudaFuncSetAttribute(quantize_t_kernel<InT, FMT, GROUP>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
