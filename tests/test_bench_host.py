@@ -109,3 +109,44 @@ def test_reference_arm_prints_contract_line():
     assert line["impl"] == "reference" and line["value"] > 0 and line["unit"] == "TFLOP/s"
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
+
+
+def test_algorithmic_work_of_every_workload():
+    # the roofline's algorithmic FLOPs and bytes: operands read once, results written once
+    import workloads as wl
+    for name, w in wl.WORKLOADS.items():
+        flops, byts, _ = bench.describe(w)
+        kb, nb = -(-w.K // 128), -(-w.N // 128)
+        if w.op == "fp8_blockwise":
+            want_f = 2 * w.M * w.N * w.K
+            want_b = w.M * w.K + w.N * w.K + 2 * w.M * w.N + 4 * w.M * kb + 4 * kb * nb
+        elif w.op == "int_scaled_mm":
+            want_f = 2 * w.M * w.N * w.K
+            want_b = w.M * w.K + w.N * w.K + 4 * w.M * w.N + 4 * (w.M + w.N)
+        elif w.op == "fp8_rowwise":
+            out_es = 1 if w.extra.get("out") == "e4m3" else 2
+            want_f = 2 * w.M * w.N * w.K
+            want_b = w.M * w.K + w.N * w.K + out_es * w.M * w.N + 4 * w.M + 8 * w.N
+        elif w.op == "quantize_1x128":
+            want_f, want_b = 0, 3 * w.M * w.K + 4 * w.M * kb
+        elif w.op == "quantize_t":
+            rb = -(-w.M // 128)
+            scales = w.K * rb if w.extra["group"] == "128x1" else rb * kb
+            want_f, want_b = 0, 3 * w.M * w.K + 4 * scales
+        else:
+            want_f = 2 * w.M * w.G * w.N * w.K
+            want_b = w.M * w.G * w.K + w.G * w.N * w.K + 2 * w.M * w.G * w.N + w.M * w.G * kb + w.G * nb * kb
+        assert (flops, byts) == (want_f, want_b), name
+    # the e4m3 result halves the output bytes of the same GEMM
+    bf = bench.describe(wl.WORKLOADS["fp8_rowwise_16640x5120x8192"])[1]
+    e4 = bench.describe(wl.WORKLOADS["fp8_rowwise_e4m3out_16640x5120x8192"])[1]
+    assert bf - e4 == 16640 * 5120
+
+
+def test_reference_arm_of_a_quantiser_workload():
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload",
+                        "quant_t_128x1_16640x5120_bf16", "--steps", "2", "--warmup", "1"],
+                       capture_output=True, text=True, timeout=300, cwd=ROOT)
+    assert r.returncode == 0, r.stderr
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["value"] > 0 and line["unit"] == "GB/s"
