@@ -330,7 +330,7 @@ const char* bs_status_string(bs_status s) {
 
 const char* bs_last_error_message(void) { return g_msg; }
 
-int32_t bs_version(void) { return 100; }
+int32_t bs_version(void) { return 200; }  // 0.2.0: rowwise e4m3 output (scale_result), transposed quantiser
 
 bs_status bs_check_blockwise_scale_shapes(int64_t M, int64_t N, int64_t K, int64_t sa_rows, int64_t sa_cols,
                                           int64_t sb_rows, int64_t sb_cols) {
