@@ -4,14 +4,15 @@
  *
  * C ABI.  Every pointer argument is a DEVICE pointer unless stated otherwise,
  * owned by the caller; the library keeps no reference after the call returns
- * and allocates no device memory.  All GEMM calls are asynchronous on the
- * given stream (a cudaStream_t passed as void*; NULL = legacy default stream).
+ * and allocates no device memory.  Every call that launches work (the GEMMs
+ * and the quantisers) is asynchronous on the given stream (a cudaStream_t
+ * passed as void*; NULL = legacy default stream).
  * Argument checks run synchronously on the host before anything is launched;
  * a call that returns an error status has launched nothing.  There is no CPU
  * fallback: on a device other than compute capability 10.0 the calls return
  * BS_ERR_DEVICE.
  *
- * Conventions shared by the three operations
+ * Conventions shared by the GEMM operations
  *   - Sizes are in elements, strides ("ld", "s_*") in elements of the tensor
  *     they describe.
  *   - FP8 operands are OCP e4m3 ("float8_e4m3fn") bytes; INT8 operands are
