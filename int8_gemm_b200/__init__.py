@@ -10,6 +10,11 @@ calls raise.
     bs_gemm_fp8_blockwise(A, B, scale_a, scale_b, out_dtype=torch.bfloat16)
     int_scaled_mm(A, B, s_a, s_b=None, out_dtype=torch.float32)
     bmm_a8w8_blockscale(x, w, x_scale, w_scale, out_dtype=torch.bfloat16)
+    bs_gemm_fp8_rowwise(A, B, scale_a, scale_b, bias=None, out_dtype=torch.bfloat16, scale_result=None)
+    bs_quantize_fp8_1x128(x, scale_format="f32")            -> (q, scale)
+    bs_quantize_fp8_t(x, group="128x1", scale_format="f32")  -> (q_t, scale)
+
+The quantisers are also available as ``quantize_fp8_1x128`` and ``quantize_fp8_t``.
 """
 from __future__ import annotations
 
@@ -323,8 +328,8 @@ def bmm_a8w8_blockscale(x: torch.Tensor, w: torch.Tensor, x_scale: torch.Tensor,
 OP_FP8_BLOCKWISE, OP_INT_SCALED_MM, OP_BMM, OP_FP8_ROWWISE = 1, 2, 3, 4
 
 
-def quantize_fp8_1x128(x: torch.Tensor, scale_format: str = "f32", q: torch.Tensor | None = None,
-                       scale: torch.Tensor | None = None):
+def bs_quantize_fp8_1x128(x: torch.Tensor, scale_format: str = "f32", q: torch.Tensor | None = None,
+                          scale: torch.Tensor | None = None):
     """1x128 group quantisation of x [M, K] (bf16 or fp32, unit stride along K) to e4m3.
 
     scale_format "f32": scale fp32 [M, ceil(K/128)] = amax / 448 (1 for an all-zero group);
@@ -365,8 +370,8 @@ def _check_quant_out(q: torch.Tensor, scale: torch.Tensor, scale_format: str):
         raise BsgemmError(BS_ERR_DTYPE, f"scale_format {scale_format!r} writes {want} scales, got {scale.dtype}")
 
 
-def quantize_fp8_t(x: torch.Tensor, group: str = "128x1", scale_format: str = "f32", q_t: torch.Tensor | None = None,
-                   scale: torch.Tensor | None = None):
+def bs_quantize_fp8_t(x: torch.Tensor, group: str = "128x1", scale_format: str = "f32",
+                      q_t: torch.Tensor | None = None, scale: torch.Tensor | None = None):
     """Transposed-output e4m3 quantisation of x [R, C] (bf16 or fp32, unit stride along C) for the
     backward GEMMs: q_t [C, R] (uint8 codes, rows padded to 16 bytes in memory), q_t[c, r] the code of x[r, c].
 
@@ -398,6 +403,10 @@ def quantize_fp8_t(x: torch.Tensor, group: str = "128x1", scale_format: str = "f
                                    q_t.stride(0), _ptr(scale), 0 if scale_format == "f32" else 1,
                                    0 if group == "128x1" else 1, scale.stride(0), _stream(x.device)))
     return q_t, scale
+
+
+quantize_fp8_1x128 = bs_quantize_fp8_1x128
+quantize_fp8_t = bs_quantize_fp8_t
 
 
 def plan_for(op: int, M: int, G: int, N: int, K: int, num_sms: int = 148) -> dict:
