@@ -349,23 +349,33 @@ def oracle_rows_run(w, d, rows):
         oracle.bmm_blockscale(d["x"], d["w"], d["x_scale"], d["w_scale"], rows=rows)
 
 
+def sample_unit(w, threads: int) -> int:
+    """Rows of the smallest oracle sample: one per host thread, and for the transposed quantiser whole
+    128-row groups, so the sample quantises complete groups."""
+    n = max(1, min(w.M, threads))
+    if w.op == "quantize_t":
+        n = min(w.M, -(-n // 128) * 128)
+    return n
+
+
 def cpu_oracle_baseline(w, d, budget_s: float = 20.0):
     """Times the oracle on a bounded row sample sized to about `budget_s` seconds."""
     import oracle
     threads = oracle.num_threads()
     quant = w.op in QUANT_OPS
     flops_per_row = describe(w)[1 if quant else 0] / w.M  # bytes per row for the quantiser
-    n = max(1, min(w.M, threads))
+    n = sample_unit(w, threads)
     t0 = time.perf_counter()
     oracle_rows_run(w, d, list(range(n)))
     dt = time.perf_counter() - t0
-    rows = max(n, min(w.M, int(n * budget_s / max(dt, 1e-3) / threads) * threads))
+    rows = max(n, min(w.M, int(n * budget_s / max(dt, 1e-3) / n) * n))
     t0 = time.perf_counter()
     oracle_rows_run(w, d, list(range(rows)))
     dt = time.perf_counter() - t0
     return {"value": flops_per_row * rows / dt / (1e9 if quant else 1e12), "unit": "GB/s" if quant else "TFLOP/s",
             "cores": threads, "kind": "oracle",
-            "sample": f"{rows} of {w.M} output rows of {w.name} (all columns), fp64 oracle, {dt:.1f} s"}
+            "sample": f"{rows} of {w.M} {'input' if quant else 'output'} rows of {w.name} (all columns), "
+                      f"fp64 oracle, {dt:.1f} s"}
 
 
 # ---------------------------------------------------------------------------
@@ -559,7 +569,7 @@ def run_reference(args, w, rank, world, flops):
     import workloads as wl
     d = wl.workload_inputs(w)
     threads = oracle.num_threads()
-    rows_per_step = max(1, min(w.M, threads))
+    rows_per_step = sample_unit(w, threads)
     sample = list(range(rows_per_step))
     for _ in range(max(1, args.warmup if args.warmup < 3 else 3)):
         oracle_rows_run(w, d, sample)
@@ -577,7 +587,7 @@ def run_reference(args, w, rank, world, flops):
         "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64 (oracle)", "data": "synthetic", "config": {"workload": w.name, "M": w.M, "N": w.N, "K": w.K},
         "cpu_baseline": {"value": value, "unit": unit, "cores": threads, "kind": "oracle",
-                         "sample": f"{rows_per_step} of {w.M} output rows per step (all columns)"},
+                         "sample": f"{rows_per_step} of {w.M} {'input rows' if quant else 'output rows'} per step (all columns)"},
         "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(out), flush=True)
