@@ -587,7 +587,8 @@ def run_reference(args, w, rank, world, flops):
         "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64 (oracle)", "data": "synthetic", "config": {"workload": w.name, "M": w.M, "N": w.N, "K": w.K},
         "cpu_baseline": {"value": value, "unit": unit, "cores": threads, "kind": "oracle",
-                         "sample": f"{rows_per_step} of {w.M} {'input rows' if quant else 'output rows'} per step (all columns)"},
+                         "sample": f"{rows_per_step} of {w.M} {'input' if quant else 'output'} rows per step "
+                                   "(all columns)"},
         "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(out), flush=True)

@@ -96,3 +96,15 @@ def e4m3_check(gpu: torch.Tensor, y: np.ndarray, S: np.ndarray, s_r: float, labe
         raise AssertionError(f"{label}: {int(bad.sum())} of {bad.size} codes outside the rounding window; first at "
                              f"{idx}: gpu={g[idx]!r} oracle s_r*y={z[idx]!r} window=[{lo[idx]!r}, {hi[idx]!r}]")
     return float(np.mean(codes == oracle.e4m3_encode(z)))
+
+
+def assert_quantised(gq: np.ndarray, gs: np.ndarray, rq: np.ndarray, rs: np.ndarray, fmt: int):
+    """Quantiser parity: codes and scales bit-exact (fmt 0: fp32 scales by bit pattern; 1: e8m0 bytes)."""
+    assert gq.shape == rq.shape and gs.shape == rs.shape, (gq.shape, rq.shape, gs.shape, rs.shape)
+    bad = np.argwhere(gq != rq)
+    assert bad.size == 0, (f"{len(bad)} codes differ, first at {bad[0]}: "
+                           f"gpu {gq[tuple(bad[0])]:#x} oracle {rq[tuple(bad[0])]:#x}")
+    if fmt == 0:
+        assert np.array_equal(gs.view(np.uint32), rs.view(np.uint32)), "fp32 scales differ"
+    else:
+        assert np.array_equal(gs, rs), "e8m0 bytes differ"

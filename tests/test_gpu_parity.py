@@ -15,7 +15,8 @@ import torch
 import int8_gemm_b200 as bs
 import oracle
 import workloads as wl
-from parity import bf16_bits, e4m3_check, f32_bits, fp8_check, oracle_fp8, rows_sample, to_f64
+from parity import (assert_quantised, bf16_bits, e4m3_check, f32_bits, fp8_check, oracle_fp8, rows_sample,
+                    to_f64)
 
 pytestmark = pytest.mark.gpu
 
@@ -365,13 +366,7 @@ def _quant_check(x_dev, fmt, rows=None, **kw):
         x_dev, q, s = x_dev[r], q[r], s[r]
     xr = x_dev.float().cpu()
     rq, rs = oracle.quantize_1x128(xr, fmt)
-    gq, gs = q.cpu().numpy(), s.cpu().numpy()
-    bad = np.argwhere(gq != rq)
-    assert bad.size == 0, f"{len(bad)} codes differ, first at {bad[0]}: gpu {gq[tuple(bad[0])]:#x} oracle {rq[tuple(bad[0])]:#x}"
-    if fmt == 0:
-        assert np.array_equal(gs.view(np.uint32), rs.view(np.uint32)), "fp32 scales differ"
-    else:
-        assert np.array_equal(gs, rs), "e8m0 bytes differ"
+    assert_quantised(q.cpu().numpy(), s.cpu().numpy(), rq, rs, fmt)
 
 
 @pytest.mark.parametrize("M,K", [(1, 128), (7, 300), (64, 1000), (256, 4096), (33, 8200)])
@@ -426,14 +421,7 @@ def test_quantize_then_blockwise_gemm_matches_the_oracle():
 def _quant_t_check(x_dev, group, fmt, **kw):
     qt, s = bs.quantize_fp8_t(x_dev, group, "f32" if fmt == 0 else "e8m0", **kw)
     rq, rs = oracle.quantize_t(x_dev.float().cpu(), 0 if group == "128x1" else 1, fmt)
-    gq, gs = qt.cpu().numpy(), s.cpu().numpy()
-    assert gq.shape == rq.shape and gs.shape == rs.shape
-    bad = np.argwhere(gq != rq)
-    assert bad.size == 0, f"{len(bad)} codes differ, first at {bad[0]}: gpu {gq[tuple(bad[0])]:#x} oracle {rq[tuple(bad[0])]:#x}"
-    if fmt == 0:
-        assert np.array_equal(gs.view(np.uint32), rs.view(np.uint32)), "fp32 scales differ"
-    else:
-        assert np.array_equal(gs, rs), "e8m0 bytes differ"
+    assert_quantised(qt.cpu().numpy(), s.cpu().numpy(), rq, rs, fmt)
     return qt, s
 
 

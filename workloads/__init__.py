@@ -44,7 +44,8 @@ GROUP = 128  # quantisation group / block edge along K (and N for weights)
 @dataclass(frozen=True)
 class Workload:
     name: str
-    op: str  # "fp8_blockwise" | "int_scaled_mm" | "bmm_a8w8_blockscale" | "fp8_rowwise" | "quantize_1x128" | "quantize_t"
+    # "fp8_blockwise" | "int_scaled_mm" | "bmm_a8w8_blockscale" | "fp8_rowwise" | "quantize_1x128" | "quantize_t"
+    op: str
     M: int
     N: int
     K: int
