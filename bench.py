@@ -66,7 +66,7 @@ def tensor_peak(peaks: dict, timed_s: float):
 # the translation unit that instantiates and launches it, and the compile-time
 # constants in launch.h).
 KERNEL_SOURCES = {
-    "wide": ["sm100.cuh", "tile_order.h", "wide_kernel.cuh", "kernels_wide.cu", "launch.h"],
+    "wide": ["sm100.cuh", "tile_order.h", "wide_kernel.cuh", "skinny_kernel.cuh", "kernels_wide.cu", "launch.h"],
     "skinny": ["sm100.cuh", "tile_order.h", "wide_kernel.cuh", "skinny_kernel.cuh", "kernels_skinny.cu", "launch.h"],
     "quantize": ["group_quant.cuh", "quantize.h", "kernels_quantize.cu"],
     "quantize_t": ["group_quant.cuh", "quantize.h", "kernels_quantize_t.cu"],

@@ -47,8 +47,11 @@ def test_stored_traffic_requires_current_kernel_sources(tmp_path, monkeypatch):
     assert bench.stored_traffic("w_ok") == 123 and bench.stored_traffic("s_ok") == 7
     assert bench.stored_traffic("w_stale") is None and bench.stored_traffic("w_nokernel") is None
     assert bench.stored_traffic("absent") is None
-    # a change to the skinny kernel leaves the wide kernel's figure valid, and not the reverse
-    (csrc / "skinny_kernel.cuh").write_bytes(b"// changed\n" + (csrc / "skinny_kernel.cuh").read_bytes())
+    # a change to a quantiser leaves both GEMM figures valid; a change to the
+    # skinny kernel's own unit leaves the wide kernel's figure valid, not the reverse
+    (csrc / "kernels_quantize.cu").write_bytes(b"// changed\n" + (csrc / "kernels_quantize.cu").read_bytes())
+    assert bench.stored_traffic("w_ok") == 123 and bench.stored_traffic("s_ok") == 7
+    (csrc / "kernels_skinny.cu").write_bytes(b"// changed\n" + (csrc / "kernels_skinny.cu").read_bytes())
     assert bench.stored_traffic("w_ok") == 123 and bench.stored_traffic("s_ok") is None
     (csrc / "wide_kernel.cuh").write_bytes(b"// changed\n" + (csrc / "wide_kernel.cuh").read_bytes())
     assert bench.stored_traffic("w_ok") is None
@@ -150,3 +153,24 @@ def test_reference_arm_of_a_quantiser_workload():
     assert r.returncode == 0, r.stderr
     line = json.loads(r.stdout.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["value"] > 0 and line["unit"] == "GB/s"
+
+
+def test_kernel_source_lists_cover_every_local_include():
+    # a stored ncu traffic figure is tied to a digest of its kernel's sources:
+    # every header a kernel's translation unit includes must be part of it
+    import re
+    csrc = os.path.join(ROOT, "int8_gemm_b200", "csrc")
+
+    def local_includes(name, seen):
+        if name in seen:
+            return seen
+        seen.add(name)
+        for inc in re.findall(r'^#include "([^"]+)"', open(os.path.join(csrc, name)).read(), flags=re.M):
+            if os.path.exists(os.path.join(csrc, inc)):
+                local_includes(inc, seen)
+        return seen
+
+    for kernel, files in bench.KERNEL_SOURCES.items():
+        units = [f for f in files if f.endswith(".cu")]
+        assert len(units) == 1, kernel
+        assert local_includes(units[0], set()) <= set(files), kernel
