@@ -214,7 +214,8 @@ typedef struct {
  * For every row m of x and every group g of 128 consecutive elements along K
  * (the last group of a row holds K - 128*(ceil(K/128) - 1) elements):
  *   amax = max |x[m, k]| over the group
- *   BS_SCALE_F32:  scale[m, g] = amax / 448 (fp32 division; 1 when amax == 0)
+ *   BS_SCALE_F32:  scale[m, g] = amax / 448 (fp32 division; 1 when that is 0:
+ *                  amax == 0, or amax < 448 * 2^-150 and the quotient underflows)
  *                  q[m, k]     = e4m3(x[m, k] / scale[m, g])   (fp32 division)
  *   BS_SCALE_E8M0: scale[m, g] = clamp(ceil(log2(amax / 448)) + 127, 0, 254),
  *                  the e8m0 byte of the smallest power of two 2^e with

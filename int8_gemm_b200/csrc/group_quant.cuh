@@ -1,7 +1,7 @@
 // Group-scale and e4m3 code arithmetic shared by the quantiser kernels.
 //
 // For a group with largest magnitude amax:
-//   fp32 scale:  s = amax / 448 (1 when amax == 0), code = e4m3(x / s)
+//   fp32 scale:  s = amax / 448 (1 when that quotient is 0), code = e4m3(x / s)
 //   e8m0 scale:  byte = clamp(ceil(log2(amax / 448)) + 127, 0, 254) (127 when
 //                amax == 0), code = e4m3(x * 2^-(byte - 127))
 // with e4m3() rounding to nearest even and saturating at +-448, the largest
@@ -20,7 +20,12 @@ __device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
   return static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3));
 }
 
-__device__ __forceinline__ float group_scale_f32(float amax) { return amax == 0.f ? 1.f : __fdiv_rn(amax, 448.f); }
+// amax / 448, or 1 where that fp32 quotient is zero: an all-zero group, or a
+// group whose amax is below 448 * 2^-150 so that the quotient underflows.
+__device__ __forceinline__ float group_scale_f32(float amax) {
+  const float s = __fdiv_rn(amax, 448.f);
+  return s == 0.f ? 1.f : s;
+}
 
 // fp32(v / s) without an fp32 division per element: v times the fp64
 // reciprocal of s (rinv = __drcp_rn(s)), rounded to fp32.  The fp64 product is

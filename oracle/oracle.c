@@ -383,10 +383,14 @@ void orc_e4m3_encode(const double *v, uint8_t *out, int64_t n)
     for (int64_t i = 0; i < n; ++i) out[i] = orc_e4m3_from_f64(v[i]);
 }
 
-/* fp32 group scale: amax / 448 in fp32, 1 for an all-zero group. */
+/* fp32 group scale: amax / 448 in fp32, and 1 where that quotient is zero:
+ * an all-zero group, or one whose largest magnitude is below 448 * 2^-150, so
+ * that the fp32 quotient underflows (a zero scale would leave the codes
+ * undefined).  Both cases keep the all-zero group's convention. */
 static float group_scale_f32(float amax)
 {
-    return amax == 0.0f ? 1.0f : amax / 448.0f;
+    const float s = amax / 448.0f;
+    return s == 0.0f ? 1.0f : s;
 }
 
 /* e8m0 group scale byte: clamp(e + 127, 0, 254), e the smallest integer with
@@ -416,7 +420,7 @@ static uint8_t group_code(float v, int fmt, float s, int b)
  * 1x128 activation-group quantisation (the recipe the blockwise operation's
  * inputs follow): for row m and group g (elements 128g .. min(128g+128, K)-1)
  *   amax = max |x|
- *   fmt 0: scale = fp32(amax / 448) (1 when amax == 0),
+ *   fmt 0: scale = fp32(amax / 448) (1 when that is zero),
  *          q = e4m3_rne(sat(fp32(x / scale)))
  *   fmt 1: e = the smallest integer with amax <= 448 * 2^e, i.e.
  *          ceil(log2(amax / 448)) (0 when amax == 0); byte = clamp(e + 127,

@@ -461,7 +461,7 @@ def _torch_quantize_f32(x):
     xp[:, :K] = x
     amax = xp.view(M, KB, 128).abs().amax(-1)
     s = amax / 448.0
-    s[amax == 0] = 1.0
+    s[s == 0] = 1.0
     q = (xp / s.repeat_interleave(128, 1)).clamp(-448, 448).to(torch.float8_e4m3fn).view(torch.uint8)
     return q[:, :K].numpy(), s.numpy()
 
@@ -487,6 +487,29 @@ def test_quantize_group_amax_maps_to_448_and_zero_groups_get_scale_one():
     # a 1x128 group is one scale: rows and groups do not mix
     q2, s2 = oracle.quantize_1x128(x[:, :128], 0)
     assert np.array_equal(q2, q[:, :128]) and np.array_equal(s2[:, 0], s[:, 0])
+
+
+def test_quantize_scale_that_underflows_takes_the_zero_group_scale():
+    """amax / 448 is computed in fp32: below 448 * 2^-150 it rounds to zero, and
+    such a group takes scale 1 like an all-zero group (its codes are e4m3(x),
+    zero here) instead of dividing by zero.  Just above, the scale is the
+    smallest fp32 subnormal and the amax element still maps to x / 2^-149."""
+    x = torch.zeros(3, 128)
+    x[0, :5] = torch.tensor([2.0 ** -142, -2.0 ** -143, 2.0 ** -149, 0.0, -2.0 ** -142])  # quotient 2^-150.8 -> 0
+    x[1, 0] = 2.0 ** -141                      # quotient 0.57 * 2^-149 -> the smallest subnormal
+    x[1, 1] = -2.0 ** -145
+    q, s = oracle.quantize_1x128(x, 0)
+    table = oracle.e4m3_table()
+    assert np.float32(np.float32(2.0 ** -142) / np.float32(448.0)) == 0.0  # the underflow itself
+    assert s[0, 0] == 1.0 and np.all(table[q[0]] == 0.0)  # +-0 codes
+    assert q[0, 1] == 0x80 and q[0, 0] == 0x00              # the signs survive
+    assert s[1, 0] == np.float32(2.0 ** -149)
+    assert table[q[1, 0]] == 256.0 and table[q[1, 1]] == -16.0
+    assert s[2, 0] == 1.0 and np.all(q[2] == 0)  # all-zero group
+    assert not np.any(np.isin(q, [0x7F, 0xFF]))
+    # the transposed quantiser follows the same rule (128 x 1 groups of x^T)
+    qt, st = oracle.quantize_t(x.t().contiguous(), 0, 0)
+    assert np.array_equal(qt, q) and np.array_equal(st, s)
 
 
 def test_quantize_e8m0_exponent_at_and_around_448_times_powers_of_two():
@@ -554,7 +577,7 @@ def _torch_quantize_128x128_t(x):
     xp[:R, :C] = x
     amax = xp.view(RB, 128, CB, 128).abs().amax(dim=(1, 3))
     s = amax / 448.0
-    s[amax == 0] = 1.0
+    s[s == 0] = 1.0
     full = s.repeat_interleave(128, 0).repeat_interleave(128, 1)
     q = (xp / full).clamp(-448, 448).to(torch.float8_e4m3fn).view(torch.uint8)
     return q[:R, :C].t().contiguous().numpy(), s.numpy()

@@ -126,7 +126,7 @@ def quantize_groups_1x128(x: torch.Tensor):
     xp[:, :K] = x
     amax = xp.view(R, KB, GROUP).abs().amax(dim=-1)
     scale = amax / E4M3_MAX
-    scale[amax == 0] = 1.0
+    scale[scale == 0] = 1.0  # all-zero groups (and quotients that underflow)
     q = to_e4m3_bytes(xp / scale.repeat_interleave(GROUP, dim=1))
     return q[:, :K].contiguous(), scale.contiguous()
 
@@ -139,7 +139,7 @@ def quantize_blocks_128x128(w_kn: torch.Tensor):
     wp[:K, :N] = w_kn
     amax = wp.view(KB, GROUP, NB, GROUP).abs().amax(dim=(1, 3))
     scale = amax / E4M3_MAX
-    scale[amax == 0] = 1.0
+    scale[scale == 0] = 1.0  # all-zero groups (and quotients that underflow)
     full = scale.repeat_interleave(GROUP, dim=0).repeat_interleave(GROUP, dim=1)
     q = to_e4m3_bytes(wp / full)
     return q[:K, :N].contiguous(), scale.contiguous()
@@ -173,7 +173,7 @@ def fp8_rowwise_inputs(M: int, N: int, K: int, seed: int, tensorwise: bool = Fal
     def quant(x, per_row):
         amax = x.abs().amax(dim=1, keepdim=True) if per_row else x.abs().amax().reshape(1, 1)
         scale = amax / E4M3_MAX
-        scale[amax == 0] = 1.0
+        scale[scale == 0] = 1.0  # all-zero groups (and quotients that underflow)
         return to_e4m3_bytes(x / scale), scale
 
     A, sa = quant(a, not tensorwise)
