@@ -35,6 +35,9 @@ DEFAULT_WORKLOAD = "fp8_16640x5120x8192"
 L2_BYTES = 126 * 1024 * 1024
 FP8_PER_BF16 = 2.0  # nominal dense fp8 : bf16 tensor throughput on B200 (4.5 : 2.25 PFLOP/s)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+# B200 datasheet figures (dense): FP8 and INT8 tensor 4.5 PFLOP/s (POPS), HBM3e 8 TB/s
+DENSE_TENSOR_TFLOPS = 4500.0
+DATASHEET_HBM_GBS = 8000.0
 
 
 # ---------------------------------------------------------------------------
@@ -167,6 +170,24 @@ def describe(w):
         byts = w.M * w.G * w.K + w.G * w.N * w.K + 2 * w.M * w.G * w.N + w.M * w.G * kb + w.G * nb * kb
         dtype = "e4m3 (fp32 accumulate)"
     return flops, float(byts), dtype
+
+
+def copies_for(byts: float) -> int:
+    """Independent input sets rotated per step so that consecutive steps never find their inputs in L2."""
+    return max(1, math.ceil(3 * L2_BYTES / byts)) if byts < 3 * L2_BYTES else 1
+
+
+def workload_config(w, world: int, byts: float) -> dict:
+    """The `config` object of the JSON line; both arms print the same one for the same workload."""
+    quant = w.op in QUANT_OPS
+    copies = copies_for(byts)
+    return {"workload": w.name, "op": w.op, "M": w.M, "N": w.N, "K": w.K, "G": w.G,
+            "out_dtype": "float32" if w.op == "int_scaled_mm" else
+            ("e4m3" if quant or w.extra.get("out") == "e4m3" else "bfloat16"),
+            **({"scale_result": w.extra["scale_result"]} if "scale_result" in w.extra else {}),
+            "l2": (f"inputs larger than L2 ({byts / 1e6:.0f} MB per step)" if copies == 1 else
+                   f"{copies} rotating input copies ({copies * byts / 1e6:.0f} MB) to defeat L2"),
+            "parallelism": f"replicas x{world}"}
 
 
 def rowwise_out(w, device):
@@ -444,7 +465,7 @@ def main():
         return float(t.item())
 
     bs.set_path_override({"auto": 0, "wide": 1, "skinny": 2, "wide1": 3, "promote": 4}[args.path])
-    copies = max(1, math.ceil(3 * L2_BYTES / byts)) if byts < 3 * L2_BYTES else 1
+    copies = copies_for(byts)
     d, sets = build_step(w, device, copies)
     quant = w.op in QUANT_OPS
     if quant:
@@ -514,10 +535,12 @@ def main():
     if w.op in ("fp8_blockwise", "bmm_a8w8_blockscale", "fp8_rowwise") and flops / byts > 690 or w.op == "int_scaled_mm":
         bound, unit = "tensor", "TFLOP/s"
         peak, peak_source = tensor_peak(peaks, step_ms * K / 1e3)
+        dense_peak = DENSE_TENSOR_TFLOPS
         achieved = flops / (per_launch_ms / 1e3) / 1e12
     else:
         bound, unit = "hbm", "GB/s"
         peak, peak_source = peaks["hbm_gbs"], f"{peaks.get('source')}: HBM copy"
+        dense_peak = DATASHEET_HBM_GBS
         achieved = byts / (per_launch_ms / 1e3) / 1e9
     traffic = stored_traffic(w.name)
 
@@ -534,18 +557,16 @@ def main():
         "vs_baseline": None,
         "dtype": dtype,
         "data": "synthetic (seeded N(0,1) with 1% x20 outliers, quantised per the workload recipe)",
-        "config": {"workload": w.name, "op": w.op, "M": w.M, "N": w.N, "K": w.K, "G": w.G,
-                   "out_dtype": "float32" if w.op == "int_scaled_mm" else
-                   ("e4m3" if quant or w.extra.get("out") == "e4m3" else "bfloat16"),
-                   **({"scale_result": w.extra["scale_result"]} if "scale_result" in w.extra else {}),
-                   "l2": (f"inputs larger than L2 ({byts / 1e6:.0f} MB per step)" if copies == 1 else
-                          f"{copies} rotating input copies ({copies * byts / 1e6:.0f} MB) to defeat L2"),
-                   "parallelism": f"replicas x{world}", "plan": plan},
+        "config": workload_config(w, world, byts),
+        "plan": plan,
         "roofline": {"bound": bound, "achieved": round(achieved, 2), "peak": round(peak, 1), "unit": unit,
-                     "frac": round(achieved / peak, 4), "traffic": traffic,
+                     "frac": round(achieved / peak, 4), "frac_basis": "of " + peak_source,
+                     "traffic": traffic,
                      "kernel": f"{w.op}_kernel" if quant else
                                ("wide_gemm_kernel" if plan["kernel"] == 1 else "skinny_gemm_kernel"),
-                     "peak_source": peak_source},
+                     "peak_source": peak_source,
+                     "dense_peak": dense_peak,
+                     "frac_dense_peak": round(achieved / dense_peak, 4)},
         "e2e": e2e,
         "gpu_launches": K * plan["launches"],
         "timing": f"{replays} replays of a CUDA graph holding {graph_steps} launches; CUDA events on the replay stream",
@@ -585,7 +606,7 @@ def run_reference(args, w, rank, world, flops):
         "impl": "reference", "metric": METRIC if w.name == DEFAULT_WORKLOAD else f"{w.name} {unit}",
         "value": value, "unit": unit, "n_gpus": world, "steps": steps, "warmup": args.warmup,
         "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "f64 (oracle)", "data": "synthetic", "config": {"workload": w.name, "M": w.M, "N": w.N, "K": w.K},
+        "dtype": "f64 (oracle)", "data": "synthetic", "config": workload_config(w, world, describe(w)[1]),
         "cpu_baseline": {"value": value, "unit": unit, "cores": threads, "kind": "oracle",
                          "sample": f"{rows_per_step} of {w.M} {'input' if quant else 'output'} rows per step "
                                    "(all columns)"},

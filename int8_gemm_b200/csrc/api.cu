@@ -59,10 +59,12 @@ EncodeTiledFn encode_fn() {
 // ---------------------------------------------------------------------------
 // per-device facts
 // ---------------------------------------------------------------------------
+// `ready` is published with release order after the other fields are written,
+// and read with acquire order, so a thread that sees it set also sees them.
 struct DeviceCtx {
   int sms = 0;
   uint32_t* err = nullptr;
-  bool ready = false;
+  std::atomic<bool> ready{false};
   bs_status status = BS_OK;
 };
 
@@ -76,9 +78,9 @@ bs_status device_ctx(DeviceCtx** out) {
   if (e != cudaSuccess) return fail(BS_ERR_DEVICE, "no CUDA device: %s", cudaGetErrorString(e));
   if (dev < 0 || dev >= kMaxDevices) return fail(BS_ERR_DEVICE, "device index %d out of range", dev);
   DeviceCtx& d = g_dev[dev];
-  if (!d.ready) {
+  if (!d.ready.load(std::memory_order_acquire)) {
     std::lock_guard<std::mutex> lk(g_dev_mu);
-    if (!d.ready) {
+    if (!d.ready.load(std::memory_order_relaxed)) {
       int major = 0, minor = 0, sms = 0;
       cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
       cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
@@ -96,7 +98,7 @@ bs_status device_ctx(DeviceCtx** out) {
           d.status = BS_OK;
         }
       }
-      d.ready = true;
+      d.ready.store(true, std::memory_order_release);
     }
   }
   if (d.status == BS_ERR_DEVICE) return fail(BS_ERR_DEVICE, "device %d is not an sm_100 GPU", dev);

@@ -112,6 +112,11 @@ def test_reference_arm_prints_contract_line():
     assert line["impl"] == "reference" and line["value"] > 0 and line["unit"] == "TFLOP/s"
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
+    # the same `config` object the GPU arm prints for this workload (one process, world size 1)
+    import workloads as wl
+    w = wl.WORKLOADS["fp8_tiny_256x256x512"]
+    assert line["config"] == bench.workload_config(w, 1, bench.describe(w)[1])
+    assert set(line["config"]) >= {"workload", "op", "M", "N", "K", "G", "out_dtype", "l2", "parallelism"}
 
 
 def test_algorithmic_work_of_every_workload():
