@@ -73,6 +73,7 @@ KERNEL_SOURCES = {
     "skinny": ["sm100.cuh", "tile_order.h", "wide_kernel.cuh", "skinny_kernel.cuh", "kernels_skinny.cu", "launch.h"],
     "quantize": ["group_quant.cuh", "quantize.h", "kernels_quantize.cu"],
     "quantize_t": ["group_quant.cuh", "quantize.h", "kernels_quantize_t.cu"],
+    "quantize_blocks": ["group_quant.cuh", "quantize.h", "kernels_quantize_blocks.cu"],
 }
 
 
@@ -136,7 +137,7 @@ def parse_clock_csv(text: str):
 # ---------------------------------------------------------------------------
 # workloads
 # ---------------------------------------------------------------------------
-QUANT_OPS = ("quantize_1x128", "quantize_t")  # HBM-bound quantisers: GB/s, not TFLOP/s
+QUANT_OPS = ("quantize_1x128", "quantize_t", "quantize_128x128")  # HBM-bound quantisers: GB/s, not TFLOP/s
 
 
 def describe(w):
@@ -164,6 +165,10 @@ def describe(w):
         nscales = w.K * rb if w.extra["group"] == "128x1" else rb * cb
         byts = 2 * w.M * w.K + w.M * w.K + 4 * nscales  # bf16 x [M, K] in, transposed codes + fp32 scales out
         dtype = f"bf16 -> e4m3, transposed ({w.extra['group']} groups, fp32 scales)"
+    elif w.op == "quantize_128x128":
+        flops = 0.0
+        byts = 2 * w.M * w.K + w.M * w.K + 4 * (-(-w.M // 128)) * (-(-w.K // 128))  # bf16 in, codes + block scales
+        dtype = "bf16 -> e4m3 (128x128 blocks, fp32 scales)"
     else:
         flops = 2.0 * w.M * w.G * w.N * w.K
         kb, nb = w.K // 128, -(-w.N // 128)
@@ -234,6 +239,10 @@ def build_step(w, device, copies):
             x = d["x"].to(device)
             q, sc = bs.quantize_fp8_t(x, w.extra["group"], "f32")  # allocates the outputs once
             sets.append(lambda x=x, q=q, sc=sc: bs.quantize_fp8_t(x, w.extra["group"], "f32", q_t=q, scale=sc))
+        elif w.op == "quantize_128x128":
+            x = d["x"].to(device)
+            q, sc = bs.bs_quantize_fp8_128x128(x, "f32")  # allocates the outputs once
+            sets.append(lambda x=x, q=q, sc=sc: bs.bs_quantize_fp8_128x128(x, "f32", q=q, scale=sc))
         else:
             x, wt = d["x"].to(device), d["w"].to(device)
             xs, ws = d["x_scale"].to(device), d["w_scale"].to(device)
@@ -366,6 +375,8 @@ def oracle_rows_run(w, d, rows):
         oracle.quantize_1x128(d["x"][rows], 0)
     elif w.op == "quantize_t":
         oracle.quantize_t(d["x"][rows], 0 if w.extra["group"] == "128x1" else 1, 0)
+    elif w.op == "quantize_128x128":
+        oracle.quantize_128x128(d["x"][rows], 0)
     else:
         oracle.bmm_blockscale(d["x"], d["w"], d["x_scale"], d["w_scale"], rows=rows)
 
@@ -374,7 +385,7 @@ def sample_unit(w, threads: int) -> int:
     """Rows of the smallest oracle sample: one per host thread, and for the transposed quantiser whole
     128-row groups, so the sample quantises complete groups."""
     n = max(1, min(w.M, threads))
-    if w.op == "quantize_t":
+    if w.op in ("quantize_t", "quantize_128x128"):
         n = min(w.M, -(-n // 128) * 128)
     return n
 
@@ -411,12 +422,18 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-baseline-s", type=float, default=20.0,
+                    help="seconds of host-core work the cpu_baseline row sample is sized to")
     ap.add_argument("--shape", default=None,
                     help="ad-hoc problem 'M,N,K' (or 'M,G,N,K' for --op bmm) instead of a named workload")
     ap.add_argument("--op", default="fp8", choices=["fp8", "int8", "bmm"], help="operation for --shape")
     ap.add_argument("--path", default="auto", choices=["auto", "wide", "skinny", "wide1", "promote"],
                     help="force a kernel family (wide = CTA-pair persistent, wide1 = single-CTA persistent, "
                          "promote = CTA-pair persistent with e8m0 block scales promoted on the CUDA cores)")
+    ap.add_argument("--splits", type=int, default=0, choices=[0, 1, 2, 4, 8],
+                    help="force the skinny kernel's split-K factor (0 = the planner's choice)")
+    ap.add_argument("--stream-k", default="on", choices=["on", "off"],
+                    help="off: compute every tile of the wide kernel whole (no split of the last wave)")
     args = ap.parse_args()
 
     rank = int(os.environ.get("RANK", "0"))
@@ -465,6 +482,8 @@ def main():
         return float(t.item())
 
     bs.set_path_override({"auto": 0, "wide": 1, "skinny": 2, "wide1": 3, "promote": 4}[args.path])
+    bs.set_stream_k(args.stream_k == "on")
+    bs.set_split_override(args.splits)
     copies = copies_for(byts)
     d, sets = build_step(w, device, copies)
     quant = w.op in QUANT_OPS
@@ -575,7 +594,7 @@ def main():
     if clocks:
         result["clocks"] = clocks
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        result["cpu_baseline"] = cpu_oracle_baseline(w, d)
+        result["cpu_baseline"] = cpu_oracle_baseline(w, d, args.cpu_baseline_s)
     if world > 1:
         dist.destroy_process_group()
     if rank == 0:

@@ -47,7 +47,8 @@ typedef enum {
   BS_ERR_DTYPE = 5,     /* output dtype not supported by this operation */
   BS_ERR_DEVICE = 6,    /* current device is not an sm_100 (B200-class) GPU */
   BS_ERR_CUDA = 7,      /* a CUDA runtime call failed (launch, encode, ...) */
-  BS_ERR_TIMEOUT = 8    /* a kernel gave up on a bounded wait (bs_get_device_error) */
+  BS_ERR_TIMEOUT = 8,   /* a kernel gave up on a bounded wait (bs_get_device_error) */
+  BS_ERR_WORKSPACE = 9  /* workspace smaller than bs_workspace_size() */
 } bs_status;
 
 typedef enum {
@@ -78,6 +79,12 @@ typedef enum {
  *            scale_b[kb*sb_sk + nb*sb_sn]
  *   out      [M, N] row-major, row stride ldo (>= N), BS_OUT_BF16 or BS_OUT_F32
  *   K must be a multiple of 128 (one scale per 128-deep group).
+ * Zero and subnormal scales are accepted.  Each block's scale product
+ * scale_a * scale_b is formed in fp32: below 2^-140 in magnitude, where fp32
+ * subnormals keep fewer than ten significant bits, that block contributes with
+ * an absolute error of up to 2^-150 times its sum of |A*B|.  bf16 outputs are
+ * coarser than that error; fp32 outputs whose blocks all have products of zero
+ * or at least 2^-140 meet the relative bound of the other inputs.
  */
 bs_status bs_gemm_fp8_blockwise(const void* A, int64_t lda, const void* B, int64_t ldb,
                                 const float* scale_a, int64_t sa_sm, int64_t sa_sk,
@@ -168,6 +175,9 @@ bs_status int_scaled_mm(const int8_t* A, int64_t lda, const int8_t* B, int64_t l
  *   w_scale  e8m0 bytes [G, ceil(N/128), K/128], contiguous
  *   out      element (m, g, n) at out[m*o_sm + g*o_sg + n]; BS_OUT_BF16 or BS_OUT_F32
  *   K must be a multiple of 128.  Scale byte 255 encodes NaN and is not checked.
+ * Every byte 0..254 is decoded exactly (byte 0 is 2^-127, an fp32 subnormal),
+ * whether the tensor core applies the scales (CTA pairs) or the CUDA cores
+ * promote each block; block products that underflow fp32 contribute zero.
  */
 bs_status bmm_a8w8_blockscale(const void* x, int64_t x_sm, int64_t x_sg,
                               const void* w, int64_t w_sg, int64_t w_sn,
@@ -205,6 +215,8 @@ typedef struct {
   int32_t ctas;    /* CTAs launched */
   int32_t cluster; /* CTAs per thread-block cluster (2 for the CTA-pair wide kernel) */
   int32_t launches;/* kernel launches the call makes */
+  int32_t sk_tiles;/* wide kernel: tiles whose K blocks are split over several CTA pairs (or CTAs)
+                      to balance the last wave (stream-K); 0 = every tile is computed whole */
 } bs_plan;
 
 /*
@@ -289,6 +301,33 @@ bs_status bs_quantize_fp8_t(const void* x, bs_in_dtype x_dtype, int64_t R, int64
                            int64_t ldq, void* scale, bs_scale_fmt scale_fmt, bs_group group, int64_t ld_scale,
                            void* stream);
 
+/*
+ * Weight quantiser -- 128x128 blocks to e4m3 in the input's own orientation
+ * (the weight operand of the forward GEMM).
+ *
+ * For every block of rows 128rb .. min(128rb + 128, R) - 1 and columns
+ * 128cb .. min(128cb + 128, C) - 1 of x, one scale from the block's amax and
+ * one code per element, with the scale and code rules of
+ * bs_quantize_fp8_1x128:
+ *   q[r, c] = code of x[r, c],  q [R, C], row r at q + r*ldq bytes (ldq >= C)
+ *   scale of block (rb, cb) at scale[rb*s_rb + cb*s_cb] (element strides)
+ * A weight W [N, K] (y = x W^T) becomes the B_t [N, K] codes that
+ * bs_gemm_fp8_blockwise reads as its column-major B, and with
+ * (s_rb, s_cb) = (1, ceil(N/128)) the scales land as its
+ * scale_b [K/128, N/128] -- no transpose copy of either.  Source: pytorch
+ * issue "torch._scaled_mm with blockwise scaling doesn't work with
+ * torch.compile" (128x128 weight blocks, one fp32 scale each: scale_b
+ * (64, 40) for K = 8192, N = 5120).  Bit-exact (integer codes, exact scales).
+ *   x      bf16 or fp32 [R, C], row r at x + r*ldx (ldx >= C, in elements),
+ *          aligned to its element size
+ *   s_rb, s_cb >= 0, and non-zero along a dimension that has several blocks.
+ *   fp32 scales must be 4-byte aligned.  R == 0 or C == 0 is a no-op.
+ *   16-byte loads are used where x and ldx allow them.
+ */
+bs_status bs_quantize_fp8_128x128(const void* x, bs_in_dtype x_dtype, int64_t R, int64_t C, int64_t ldx, void* q,
+                                  int64_t ldq, void* scale, bs_scale_fmt scale_fmt, int64_t s_rb, int64_t s_cb,
+                                  void* stream);
+
 /* Plan of operation `op` (1 = bs_gemm_fp8_blockwise, 2 = int_scaled_mm,
  * 3 = bmm_a8w8_blockscale, 4 = bs_gemm_fp8_rowwise; G = 1 for ops 1, 2 and 4)
  * on a GPU with `num_sms`
@@ -303,6 +342,47 @@ bs_status bs_plan_for(int32_t op, int64_t M, int64_t G, int64_t N, int64_t K, in
  * of letting the tensor core apply its e8m0 scales (block-scaled MMA).
  * Returns the previous setting. */
 int32_t bs_set_path_override(int32_t path);
+
+/* Force the skinny kernel's split-K factor (1, 2, 4 or 8 CTAs per cluster, at
+ * most the number of K blocks) for subsequent calls in this process (testing
+ * and tuning); 0 restores the planner's choice.  Returns the previous setting. */
+int32_t bs_set_split_override(int32_t splits);
+
+/*
+ * Stream-K workspace.  When a problem's tiles would leave the last round of
+ * the persistent wide kernel's CTA pairs (or CTAs) badly filled, the K blocks
+ * of the remaining tiles are spread evenly over all of them and the pieces of
+ * a split tile meet in this workspace: fp32 (int32 for int_scaled_mm) partial
+ * sums, added in a fixed order by the CTA that holds the tile's first K block,
+ * so results are deterministic.  Without a registered workspace (or with
+ * bs_set_stream_k(0)) every tile is computed whole.
+ *
+ * bs_workspace_size(num_sms): bytes needed on a GPU with num_sms SMs
+ *   (num_sms * 131,104 rounded up; about 19.4 MB on a 148-SM B200).  Pure host logic.
+ * bs_set_workspace(ptr, bytes): registers a caller-owned device buffer for the
+ *   current device (NULL unregisters).  `ptr` must be 256-byte aligned and
+ *   zero-filled before its first use; every call that completes leaves its
+ *   flag words zero again.  The library keeps the pointer until it is replaced
+ *   or unregistered and never frees it.  Calls that may split K share this
+ *   buffer, so they must not run concurrently on different streams of the
+ *   device (as with a library handle's workspace).  Returns BS_ERR_WORKSPACE
+ *   if `bytes` < bs_workspace_size(device SMs), BS_ERR_ALIGNMENT if misaligned.
+ * bs_set_stream_k(enable): 0 disables the split process-wide (for testing);
+ *   returns the previous setting.
+ */
+size_t bs_workspace_size(int32_t num_sms);
+bs_status bs_set_workspace(void* workspace, size_t bytes);
+int32_t bs_set_stream_k(int32_t enable);
+
+/* The work items of one unit (CTA pair or CTA) `unit` of `units` in the
+ * persistent wide kernel, in processing order: tiles [0, dp_tiles) whole
+ * (tile t by unit t % units), then that unit's share of the sk_iters =
+ * (num_tiles - dp_tiles) * kb split K blocks.  Writes (tile, first K block,
+ * end K block) triples to out[3*i ..] for the first `capacity` items and
+ * returns the number of items, or -1 for inconsistent arguments.  Pure host
+ * logic (the host copy of the kernels' decomposition). */
+int32_t bs_work_items(int32_t num_tiles, int32_t dp_tiles, int64_t sk_iters, int32_t kb, int32_t units, int32_t unit,
+                      int32_t* out, int32_t capacity);
 
 /* The persistent tile order: fills out[3*t .. 3*t+2] = (batch, tile_row,
  * tile_col) of linear tile t for t < count (host copy of the mapping the

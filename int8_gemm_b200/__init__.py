@@ -13,8 +13,9 @@ calls raise.
     bs_gemm_fp8_rowwise(A, B, scale_a, scale_b, bias=None, out_dtype=torch.bfloat16, scale_result=None)
     bs_quantize_fp8_1x128(x, scale_format="f32")            -> (q, scale)
     bs_quantize_fp8_t(x, group="128x1", scale_format="f32")  -> (q_t, scale)
+    bs_quantize_fp8_128x128(w, scale_format="f32")           -> (q, scale_b)
 
-The quantisers are also available as ``quantize_fp8_1x128`` and ``quantize_fp8_t``.
+The quantisers are also available as ``quantize_fp8_1x128``, ``quantize_fp8_t`` and ``quantize_fp8_128x128``.
 """
 from __future__ import annotations
 
@@ -28,7 +29,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libbsgemm.so")
 
 BS_OK, BS_ERR_NULL, BS_ERR_SHAPE, BS_ERR_LAYOUT, BS_ERR_ALIGNMENT = 0, 1, 2, 3, 4
-BS_ERR_DTYPE, BS_ERR_DEVICE, BS_ERR_CUDA, BS_ERR_TIMEOUT = 5, 6, 7, 8
+BS_ERR_DTYPE, BS_ERR_DEVICE, BS_ERR_CUDA, BS_ERR_TIMEOUT, BS_ERR_WORKSPACE = 5, 6, 7, 8, 9
 BS_OUT_BF16, BS_OUT_F32, BS_OUT_I32, BS_OUT_E4M3 = 0, 1, 2, 3
 
 PATH_AUTO, PATH_WIDE, PATH_SKINNY, PATH_WIDE_SINGLE, PATH_WIDE_PROMOTE = 0, 1, 2, 3, 4
@@ -46,7 +47,7 @@ class BsgemmError(RuntimeError):
 class Plan(ctypes.Structure):
     _fields_ = [("kernel", ctypes.c_int32), ("tile_m", ctypes.c_int32), ("tile_n", ctypes.c_int32),
                 ("splits", ctypes.c_int32), ("ctas", ctypes.c_int32), ("cluster", ctypes.c_int32),
-                ("launches", ctypes.c_int32)]
+                ("launches", ctypes.c_int32), ("sk_tiles", ctypes.c_int32)]
 
     def as_dict(self):
         return {f: getattr(self, f) for f, _ in self._fields_}
@@ -75,8 +76,10 @@ def lib() -> ctypes.CDLL:
             h.bs_quantize_fp8_1x128.argtypes = [p, ctypes.c_int, i64, i64, i64, p, i64, p, ctypes.c_int, i64, p]
             h.bs_quantize_fp8_t.argtypes = [p, ctypes.c_int, i64, i64, i64, p, i64, p, ctypes.c_int, ctypes.c_int,
                                             i64, p]
+            h.bs_quantize_fp8_128x128.argtypes = [p, ctypes.c_int, i64, i64, i64, p, i64, p, ctypes.c_int, i64, i64,
+                                                  p]
             for f in (h.bs_gemm_fp8_blockwise, h.int_scaled_mm, h.bmm_a8w8_blockscale, h.bs_gemm_fp8_rowwise,
-                      h.bs_quantize_fp8_1x128, h.bs_quantize_fp8_t):
+                      h.bs_quantize_fp8_1x128, h.bs_quantize_fp8_t, h.bs_quantize_fp8_128x128):
                 f.restype = ctypes.c_int
             h.bs_status_string.argtypes = [ctypes.c_int]
             h.bs_status_string.restype = ctypes.c_char_p
@@ -93,6 +96,16 @@ def lib() -> ctypes.CDLL:
             h.bs_get_device_error.argtypes = [p, u32p]
             h.bs_get_device_error.restype = ctypes.c_int
             h.bs_version.restype = i32
+            h.bs_workspace_size.argtypes = [i32]
+            h.bs_workspace_size.restype = ctypes.c_size_t
+            h.bs_set_workspace.argtypes = [p, ctypes.c_size_t]
+            h.bs_set_workspace.restype = ctypes.c_int
+            h.bs_set_split_override.argtypes = [i32]
+            h.bs_set_split_override.restype = i32
+            h.bs_set_stream_k.argtypes = [i32]
+            h.bs_set_stream_k.restype = i32
+            h.bs_work_items.argtypes = [i32, i32, i64, i32, i32, i32, ctypes.POINTER(ctypes.c_int32), i32]
+            h.bs_work_items.restype = i32
             _handle = h
     return _handle
 
@@ -107,6 +120,29 @@ def _check(status: int):
 
 def status_string(status: int) -> str:
     return lib().bs_status_string(status).decode()
+
+
+_workspaces = {}  # device index -> the zero-filled stream-K workspace registered with the library
+
+
+def _ensure_workspace(device) -> None:
+    """Registers a stream-K workspace for `device` on its first GEMM call (bs_set_workspace): allocated
+    from torch's caching allocator, zero-filled, and waited for once so that calls on any stream see it
+    zeroed.  Inside a CUDA-graph capture nothing is registered (the calls run whole tiles) until a later
+    call outside a capture."""
+    idx = torch.device(device).index
+    idx = torch.cuda.current_device() if idx is None else idx
+    if idx in _workspaces:
+        return
+    with torch.cuda.device(idx):
+        if torch.cuda.is_current_stream_capturing():
+            return
+        n = lib().bs_workspace_size(torch.cuda.get_device_properties(idx).multi_processor_count)
+        ws = torch.zeros(n + 256, dtype=torch.uint8, device=f"cuda:{idx}")
+        torch.cuda.current_stream().synchronize()
+        off = (-ws.data_ptr()) % 256
+        _check(lib().bs_set_workspace(ctypes.c_void_p(ws.data_ptr() + off), n))
+    _workspaces[idx] = ws
 
 
 def _stream(device) -> ctypes.c_void_p:
@@ -167,6 +203,7 @@ def bs_gemm_fp8_blockwise(A: torch.Tensor, B: torch.Tensor, scale_a: torch.Tenso
         out = _empty_out((M,), N, out_dtype, A.device)
     elif out.dtype != out_dtype or tuple(out.shape) != (M, N) or out.stride(1) != 1:
         raise BsgemmError(BS_ERR_LAYOUT, "out must be a row-major [M, N] tensor of out_dtype")
+    _ensure_workspace(A.device)
     with torch.cuda.device(A.device):
         _check(lib().bs_gemm_fp8_blockwise(
             _ptr(A), A.stride(0), _ptr(B), B.stride(1), _ptr(scale_a), scale_a.stride(0), scale_a.stride(1),
@@ -229,6 +266,7 @@ def bs_gemm_fp8_rowwise(A: torch.Tensor, B: torch.Tensor, scale_a: torch.Tensor,
         out = _empty_out((M,), N, out_dtype, A.device)
     elif out.dtype != out_dtype or tuple(out.shape) != (M, N) or out.stride(1) != 1:
         raise BsgemmError(BS_ERR_LAYOUT, "out must be a row-major [M, N] tensor of out_dtype")
+    _ensure_workspace(A.device)
     with torch.cuda.device(A.device):
         _check(lib().bs_gemm_fp8_rowwise(
             _ptr(A), A.stride(0), _ptr(B), B.stride(1), _ptr(scale_a), stride, _ptr(scale_b), stride, _ptr(bias),
@@ -271,6 +309,7 @@ def int_scaled_mm(A: torch.Tensor, B: torch.Tensor, s_a: torch.Tensor | None, s_
         out = _empty_out((M,), N, out_dtype, A.device)
     elif out.dtype != out_dtype or tuple(out.shape) != (M, N) or out.stride(1) != 1:
         raise BsgemmError(BS_ERR_LAYOUT, "out must be a row-major [M, N] tensor of out_dtype")
+    _ensure_workspace(A.device)
     with torch.cuda.device(A.device):
         _check(lib().int_scaled_mm(_ptr(A), A.stride(0), _ptr(B), B.stride(1), _ptr(sa), _ptr(sb), _ptr(out),
                                    out.stride(0), _OUT_CODE[out_dtype], M, N, K, _stream(A.device)))
@@ -315,6 +354,7 @@ def bmm_a8w8_blockscale(x: torch.Tensor, w: torch.Tensor, x_scale: torch.Tensor,
         out = _empty_out((M, G), N, out_dtype, x.device)
     elif out.dtype != out_dtype or tuple(out.shape) != (M, G, N) or out.stride(2) != 1:
         raise BsgemmError(BS_ERR_LAYOUT, "out must be [M, G, N] of out_dtype with unit stride along N")
+    _ensure_workspace(x.device)
     with torch.cuda.device(x.device):
         _check(lib().bmm_a8w8_blockscale(
             _ptr(x), x.stride(0), x.stride(1), _ptr(w), w.stride(0), w.stride(1), _ptr(xs), _ptr(ws), _ptr(out),
@@ -405,14 +445,73 @@ def bs_quantize_fp8_t(x: torch.Tensor, group: str = "128x1", scale_format: str =
     return q_t, scale
 
 
+def bs_quantize_fp8_128x128(x: torch.Tensor, scale_format: str = "f32", q: torch.Tensor | None = None,
+                            scale: torch.Tensor | None = None):
+    """128x128 block quantisation of a weight x = W [R, C] (bf16 or fp32, unit stride along C) to e4m3 codes in
+    its own orientation: q [R, C] (uint8, rows padded to 16 bytes in memory), q[r, c] the code of x[r, c].
+
+    The scales come back as [ceil(C/128), ceil(R/128)]: for W [N, K] that is the scale_b [K/128, N/128] of
+    bs_gemm_fp8_blockwise with B = q.t() (no transpose copy).  A ``scale`` passed in may have any strides;
+    element (cb, rb) is the scale of the block of rows 128rb.. and columns 128cb..
+    scale_format "f32" (amax / 448) or "e8m0" (uint8 bytes).  Returns (q, scale).
+    """
+    _cuda(x, "x")
+    if x.dim() != 2 or x.stride(1) != 1:
+        raise BsgemmError(BS_ERR_LAYOUT, "x must be [R, C] with unit stride along C")
+    if x.dtype not in (torch.bfloat16, torch.float32):
+        raise BsgemmError(BS_ERR_DTYPE, f"x must be bfloat16 or float32, got {x.dtype}")
+    if scale_format not in ("f32", "e8m0"):
+        raise BsgemmError(BS_ERR_DTYPE, f"unknown scale_format {scale_format!r}")
+    R, C = x.shape
+    RB, CB = -(-R // 128), -(-C // 128)
+    if q is None:
+        q = _empty_out((R,), C, torch.uint8, x.device)
+    if scale is None:
+        scale = torch.empty((CB, RB), dtype=torch.float32 if scale_format == "f32" else torch.uint8, device=x.device)
+    _cuda(q, "q"), _cuda(scale, "scale")
+    _check_quant_out(q, scale, scale_format)
+    if q.shape != (R, C) or q.stride(1) != 1 or scale.shape != (CB, RB):
+        raise BsgemmError(BS_ERR_SHAPE, f"q must be [R, C] with unit stride along C and scale [{CB}, {RB}]")
+    with torch.cuda.device(x.device):
+        _check(lib().bs_quantize_fp8_128x128(_ptr(x), 0 if x.dtype == torch.bfloat16 else 1, R, C, x.stride(0),
+                                             _ptr(q), q.stride(0), _ptr(scale), 0 if scale_format == "f32" else 1,
+                                             scale.stride(1), scale.stride(0), _stream(x.device)))
+    return q, scale
+
+
 quantize_fp8_1x128 = bs_quantize_fp8_1x128
 quantize_fp8_t = bs_quantize_fp8_t
+quantize_fp8_128x128 = bs_quantize_fp8_128x128
 
 
 def plan_for(op: int, M: int, G: int, N: int, K: int, num_sms: int = 148) -> dict:
     p = Plan()
     _check(lib().bs_plan_for(op, M, G, N, K, num_sms, ctypes.byref(p)))
     return p.as_dict()
+
+
+def set_split_override(splits: int) -> int:
+    """Forces the skinny kernel's split-K factor (1, 2, 4, 8; 0 = automatic); returns the previous value."""
+    return lib().bs_set_split_override(splits)
+
+
+def set_stream_k(enable: bool) -> bool:
+    """Enables or disables the stream-K split of the wide kernel's last wave; returns the previous setting."""
+    return bool(lib().bs_set_stream_k(1 if enable else 0))
+
+
+def workspace_size(num_sms: int) -> int:
+    return int(lib().bs_workspace_size(num_sms))
+
+
+def work_items(num_tiles: int, dp_tiles: int, sk_iters: int, kb: int, units: int, unit: int):
+    """Host copy of the wide kernel's work decomposition: the (tile, kb0, kb1) items of one unit, in order."""
+    n = lib().bs_work_items(num_tiles, dp_tiles, sk_iters, kb, units, unit, None, 0)
+    if n < 0:
+        raise BsgemmError(BS_ERR_SHAPE, "inconsistent work split")
+    buf = (ctypes.c_int32 * (3 * max(n, 1)))()
+    lib().bs_work_items(num_tiles, dp_tiles, sk_iters, kb, units, unit, buf, n)
+    return [tuple(buf[3 * i:3 * i + 3]) for i in range(n)]
 
 
 def set_path_override(path: int) -> int:

@@ -66,6 +66,9 @@ struct DeviceCtx {
   uint32_t* err = nullptr;
   std::atomic<bool> ready{false};
   bs_status status = BS_OK;
+  // stream-K workspace registered with bs_set_workspace (caller-owned)
+  std::atomic<void*> ws{nullptr};
+  std::atomic<size_t> ws_bytes{0};
 };
 
 constexpr int kMaxDevices = 64;
@@ -111,6 +114,17 @@ bs_status device_ctx(DeviceCtx** out) {
 // planning (pure host logic)
 // ---------------------------------------------------------------------------
 std::atomic<int32_t> g_path_override{0};
+std::atomic<int32_t> g_stream_k{1};
+std::atomic<int32_t> g_split_override{0};  // skinny kernel: forced split factor (0 = planner's choice)
+
+// Bytes of the stream-K workspace for a GPU with `sms` SMs: one partial-sum
+// slot per CTA (the 128 x 256 fp32 accumulator, 128 KB) and one flag word per
+// slot and consumer warp, the flags after the slots.
+size_t workspace_slots_bytes(int sms) { return static_cast<size_t>(sms) * kWsSlotWords * sizeof(uint32_t); }
+size_t workspace_bytes_for(int sms) {
+  const size_t flags = static_cast<size_t>(sms) * kWsFlagsPerSlot * sizeof(uint32_t);
+  return workspace_slots_bytes(sms) + ((flags + 255) / 256) * 256;
+}
 
 constexpr int kSkinnyMaxM = 256;
 
@@ -129,9 +143,35 @@ struct Plan {
   int bmt = 0;
   int m_tiles = 0, n_tiles = 0;
   int grid_m = 0, grid_n = 0, num_tiles = 0;
+  int dp_tiles = 0;        // wide kernel: tiles computed whole
+  long long sk_iters = 0;  // K blocks of the remaining tiles, split evenly over the units
 };
 
-Plan make_plan(int op, int64_t M, int64_t G, int64_t N, int64_t K, int sms) {
+// Stream-K split of the wide kernel's persistent loop (tile_order.h): when
+// the tiles leave the last round of units badly filled, that round's K
+// blocks (and, if that leaves fewer than kSkMinPerUnit per unit, one more
+// round's) are spread evenly over every unit.  Each unit then hands over at
+// most one partial sum and finishes at most one split tile.
+constexpr double kSkMinFill = 0.9;  // below this fraction of busy unit-rounds, split
+constexpr int kSkMinPerUnit = 4;    // K blocks per unit, at least
+void plan_stream_k(Plan& x, long long tiles, long long units, int KB) {
+  x.dp_tiles = static_cast<int>(tiles);
+  x.sk_iters = 0;
+  if (units <= 1 || KB < 2) return;
+  const long long full = tiles / units, rem = tiles % units;
+  if (rem == 0) return;
+  const double fill = static_cast<double>(tiles) / static_cast<double>((full + 1) * units);
+  if (fill >= kSkMinFill) return;
+  long long dp = full * units;
+  if ((tiles - dp) * KB < kSkMinPerUnit * units && full >= 1) dp -= units;
+  const long long iters = (tiles - dp) * KB;
+  if (iters < kSkMinPerUnit * units) return;
+  x.dp_tiles = static_cast<int>(dp);
+  x.sk_iters = iters;
+  x.pub.sk_tiles = static_cast<int32_t>(tiles - dp);
+}
+
+Plan make_plan(int op, int64_t M, int64_t G, int64_t N, int64_t K, int sms, bool stream_k_ok) {
   Plan x;
   std::memset(&x.pub, 0, sizeof(x.pub));
   if (M == 0 || N == 0 || G == 0) return x;  // kernel 0: nothing to do
@@ -171,6 +211,8 @@ Plan make_plan(int op, int64_t M, int64_t G, int64_t N, int64_t K, int sms) {
     const int max_s = skinny_ctas_per_sm(bmt) > 1 ? 8 : 4;
     int S = 1;
     while (S < max_s && 2 * S <= KB && units * 2 * S <= slots) S *= 2;
+    const int forced = g_split_override.load();
+    if (forced == 1 || forced == 2 || forced == 4 || forced == 8) S = forced <= KB ? forced : S;
     x.pub.kernel = 2;
     x.pub.tile_m = bmt;
     x.pub.tile_n = 128;
@@ -186,15 +228,35 @@ Plan make_plan(int op, int64_t M, int64_t G, int64_t N, int64_t K, int sms) {
     const long long tiles = static_cast<long long>(x.grid_m) * x.grid_n * G;
     const long long units = (sms > 0 ? sms : 148) / x.cg;  // persistent CTAs (or CTA pairs)
     x.num_tiles = static_cast<int>(tiles);
+    x.dp_tiles = x.num_tiles;
+    if (stream_k_ok && g_stream_k.load() != 0) plan_stream_k(x, tiles, units, KB);
     x.pub.kernel = 1;
     x.pub.tile_m = tile_m;
     x.pub.tile_n = kWideBN;
     x.pub.splits = 1;
     x.pub.cluster = x.cg;
-    x.pub.ctas = static_cast<int32_t>(x.cg * (tiles < units ? tiles : units));
+    // a split plan keeps every unit busy; otherwise no more units than tiles
+    x.pub.ctas = static_cast<int32_t>(x.cg * (x.sk_iters > 0 || tiles > units ? units : tiles));
     x.pub.launches = 1;
   }
   return x;
+}
+
+// A registered workspace large enough for this device's stream-K slots.
+bool workspace_ok(const DeviceCtx* dc) {
+  return dc->ws.load() != nullptr && dc->ws_bytes.load() >= workspace_bytes_for(dc->sms);
+}
+
+// The persistent loop's split (whole tiles, stream-K blocks) and, for a split
+// plan, the workspace slots and flags of this device.
+void set_work_split(GemmArgs& a, const Plan& pl, const DeviceCtx* dc) {
+  a.dp_tiles = pl.dp_tiles;
+  a.sk_iters = pl.sk_iters;
+  if (pl.sk_iters > 0) {
+    uint8_t* base = static_cast<uint8_t*>(dc->ws.load());
+    a.sk_ws = reinterpret_cast<uint32_t*>(base);
+    a.sk_flags = reinterpret_cast<uint32_t*>(base + workspace_slots_bytes(dc->sms));
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -261,7 +323,7 @@ struct Fp8Problem {
 };
 
 bs_status run_fp8(const Fp8Problem& q, GemmArgs args, cudaStream_t stream, DeviceCtx* dc) {
-  const Plan pl = make_plan(q.mode == Mode::kFp8E8M0 ? 3 : 1, q.M, q.G, q.N, q.K, dc->sms);
+  const Plan pl = make_plan(q.mode == Mode::kFp8E8M0 ? 3 : 1, q.M, q.G, q.N, q.K, dc->sms, workspace_ok(dc));
   if (pl.pub.kernel == 0) return BS_OK;
   if (pl.pub.kernel == 3)
     return check_launch(launch_fill_zero(q.out, out_size(q.out_dtype), q.M, q.N, q.o_rs, q.G, q.o_bs, stream),
@@ -278,6 +340,7 @@ bs_status run_fp8(const Fp8Problem& q, GemmArgs args, cudaStream_t stream, Devic
     args.num_tiles = pl.num_tiles;
     args.group_m = kGroupM;
     args.splits = 1;
+    set_work_split(args, pl, dc);
     if ((st = encode_3d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, q.a, q.K, q.M, q.G, q.a_rs, a_bs, 128, 128, "A")))
       return st;
     if ((st = encode_3d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, q.b, q.K, q.N, q.G, q.b_rs, b_bs, 128,
@@ -326,6 +389,7 @@ const char* bs_status_string(bs_status s) {
     case BS_ERR_DEVICE: return "BS_ERR_DEVICE";
     case BS_ERR_CUDA: return "BS_ERR_CUDA";
     case BS_ERR_TIMEOUT: return "BS_ERR_TIMEOUT";
+    case BS_ERR_WORKSPACE: return "BS_ERR_WORKSPACE";
   }
   return "BS_ERR_UNKNOWN";
 }
@@ -349,12 +413,58 @@ bs_status bs_check_blockwise_scale_shapes(int64_t M, int64_t N, int64_t K, int64
 
 int32_t bs_set_path_override(int32_t path) { return g_path_override.exchange(path); }
 
+int32_t bs_set_stream_k(int32_t enable) { return g_stream_k.exchange(enable != 0 ? 1 : 0); }
+
+int32_t bs_set_split_override(int32_t splits) { return g_split_override.exchange(splits); }
+
+size_t bs_workspace_size(int32_t num_sms) { return num_sms > 0 ? workspace_bytes_for(num_sms) : 0; }
+
+bs_status bs_set_workspace(void* workspace, size_t bytes) {
+  clear_msg();
+  DeviceCtx* dc = nullptr;
+  bs_status st = device_ctx(&dc);
+  if (st != BS_OK) return st;
+  if (workspace == nullptr) {
+    dc->ws.store(nullptr);
+    dc->ws_bytes.store(0);
+    return BS_OK;
+  }
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(BS_ERR_ALIGNMENT, "the workspace must be 256-byte aligned");
+  const size_t need = workspace_bytes_for(dc->sms);
+  if (bytes < need)
+    return fail(BS_ERR_WORKSPACE, "workspace of %zu bytes; this device needs %zu (bs_workspace_size)", bytes, need);
+  dc->ws_bytes.store(0);
+  dc->ws.store(workspace);
+  dc->ws_bytes.store(bytes);
+  return BS_OK;
+}
+
+int32_t bs_work_items(int32_t num_tiles, int32_t dp_tiles, int64_t sk_iters, int32_t kb, int32_t units, int32_t unit,
+                      int32_t* out, int32_t capacity) {
+  if (num_tiles < 0 || dp_tiles < 0 || dp_tiles > num_tiles || sk_iters < 0 || kb <= 0 || units <= 0 || unit < 0 ||
+      unit >= units || (sk_iters > 0 && sk_iters != static_cast<int64_t>(num_tiles - dp_tiles) * kb))
+    return -1;
+  WorkIter it(unit, units, sk_iters);
+  WorkItem w;
+  int32_t n = 0;
+  while (it.next(w, units, dp_tiles, kb)) {
+    if (out && n < capacity) {
+      out[3 * n + 0] = w.tile;
+      out[3 * n + 1] = w.kb0;
+      out[3 * n + 2] = w.kb1;
+    }
+    ++n;
+  }
+  return n;
+}
+
 bs_status bs_plan_for(int32_t op, int64_t M, int64_t G, int64_t N, int64_t K, int32_t num_sms, bs_plan* plan) {
   clear_msg();
   if (!plan) return fail(BS_ERR_NULL, "plan is NULL");
   if (op < 1 || op > 4) return fail(BS_ERR_SHAPE, "op must be 1, 2, 3 or 4");
   if (M < 0 || N < 0 || K < 0 || G < 0 || num_sms <= 0) return fail(BS_ERR_SHAPE, "negative size");
-  *plan = make_plan(op, M, G, N, K, num_sms).pub;
+  *plan = make_plan(op, M, G, N, K, num_sms, true).pub;
   return BS_OK;
 }
 
@@ -512,7 +622,7 @@ bs_status bs_gemm_fp8_rowwise(const void* A, int64_t lda, const void* B, int64_t
   bs_status st = device_ctx(&dc);
   if (st != BS_OK) return st;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  const Plan pl = make_plan(4, M, 1, N, K, dc->sms);
+  const Plan pl = make_plan(4, M, 1, N, K, dc->sms, workspace_ok(dc));
   if (pl.pub.kernel == 3)
     return check_launch(launch_fill_zero(out, out_size(out_dtype), M, N, ldo, 1, 0, cs, bias, scale_result),
                         "bias-fill launch");
@@ -537,6 +647,7 @@ bs_status bs_gemm_fp8_rowwise(const void* A, int64_t lda, const void* B, int64_t
   args.group_m = kGroupM;
   args.splits = 1;
   args.err = dc->err;
+  set_work_split(args, pl, dc);
   CUtensorMap ta, tb, td;
   if ((st = encode_3d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, A, K, M, 1, lda, lda * M, 128, 128, "A"))) return st;
   if ((st = encode_3d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, B, K, N, 1, ldb, ldb * N, 128, wide_b_box_rows(pl.cg),
@@ -603,6 +714,33 @@ bs_status bs_quantize_fp8_t(const void* x, bs_in_dtype x_dtype, int64_t R, int64
                       "transposed quantise launch");
 }
 
+bs_status bs_quantize_fp8_128x128(const void* x, bs_in_dtype x_dtype, int64_t R, int64_t C, int64_t ldx, void* q,
+                                  int64_t ldq, void* scale, bs_scale_fmt scale_fmt, int64_t s_rb, int64_t s_cb,
+                                  void* stream) {
+  clear_msg();
+  if (R < 0 || C < 0) return fail(BS_ERR_SHAPE, "negative size");
+  if (R > kMaxDim || C > kMaxDim) return fail(BS_ERR_SHAPE, "size exceeds 2^31-1");
+  if (x_dtype != BS_IN_BF16 && x_dtype != BS_IN_F32) return fail(BS_ERR_DTYPE, "x must be bf16 or f32");
+  if (scale_fmt != BS_SCALE_F32 && scale_fmt != BS_SCALE_E8M0) return fail(BS_ERR_DTYPE, "unknown scale format");
+  if (R == 0 || C == 0) return BS_OK;
+  if (!x || !q || !scale) return fail(BS_ERR_NULL, "x, q and scale must be non-NULL");
+  const int64_t RB = (R + 127) / 128, CB = (C + 127) / 128;
+  if (ldx < C || ldq < C) return fail(BS_ERR_LAYOUT, "ldx and ldq must be >= C");
+  if (s_rb < 0 || s_cb < 0 || (RB > 1 && s_rb == 0) || (CB > 1 && s_cb == 0))
+    return fail(BS_ERR_LAYOUT, "scale strides must be non-negative and non-zero along a dimension with several blocks");
+  if (RB * CB > kMaxDim) return fail(BS_ERR_SHAPE, "more than 2^31-1 blocks of 128 x 128");
+  const uintptr_t es = x_dtype == BS_IN_BF16 ? 2 : 4;
+  if (reinterpret_cast<uintptr_t>(x) % es != 0) return fail(BS_ERR_ALIGNMENT, "x must be aligned to its element size");
+  if (scale_fmt == BS_SCALE_F32 && !aligned4(scale)) return fail(BS_ERR_ALIGNMENT, "fp32 scales must be 4-byte aligned");
+  DeviceCtx* dc = nullptr;
+  bs_status st = device_ctx(&dc);
+  if (st != BS_OK) return st;
+  return check_launch(launch_quantize_blocks(x, x_dtype == BS_IN_BF16, R, C, ldx, static_cast<uint8_t*>(q), ldq, scale,
+                                             scale_fmt == BS_SCALE_E8M0, s_rb, s_cb, dc->sms,
+                                             static_cast<cudaStream_t>(stream)),
+                      "block quantise launch");
+}
+
 bs_status int_scaled_mm(const int8_t* A, int64_t lda, const int8_t* B, int64_t ldb, const float* s_a,
                         const float* s_b, void* out, int64_t ldo, bs_out_dtype out_dtype, int64_t M, int64_t N,
                         int64_t K, void* stream) {
@@ -629,7 +767,7 @@ bs_status int_scaled_mm(const int8_t* A, int64_t lda, const int8_t* B, int64_t l
   bs_status st = device_ctx(&dc);
   if (st != BS_OK) return st;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  const Plan pl = make_plan(2, M, 1, N, K, dc->sms);
+  const Plan pl = make_plan(2, M, 1, N, K, dc->sms, workspace_ok(dc));
   if (pl.pub.kernel == 3)
     return check_launch(launch_fill_zero(out, out_size(out_dtype), M, N, ldo, 1, 0, cs), "zero-fill launch");
 
@@ -651,6 +789,7 @@ bs_status int_scaled_mm(const int8_t* A, int64_t lda, const int8_t* B, int64_t l
   args.group_m = kGroupM;
   args.splits = 1;
   args.err = dc->err;
+  set_work_split(args, pl, dc);
   CUtensorMap ta, tb, td;
   if ((st = encode_3d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, A, K, M, 1, lda, lda * M, 128, 128, "A"))) return st;
   if ((st = encode_3d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, B, K, N, 1, ldb, ldb * N, 128, wide_b_box_rows(pl.cg),

@@ -10,11 +10,11 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 
-template <Mode MODE, int CG, typename OutT>
-cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& d, const GemmArgs& args,
-                       int grid, cudaStream_t stream) {
+template <Mode MODE, int CG, typename OutT, bool SPLIT>
+cudaError_t launch_split(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& d, const GemmArgs& args,
+                         int grid, cudaStream_t stream) {
   constexpr int STAGES = CG == 2 ? kWideStagesPair : kWideStages;
-  auto kernel = wide_gemm_kernel<MODE, CG, STAGES, OutT>;
+  auto kernel = wide_gemm_kernel<MODE, CG, STAGES, OutT, SPLIT>;
   constexpr size_t smem = sizeof(WideSmem<kWideBN / CG, STAGES>) + 1024;
   static std::atomic<uint64_t> configured{0};  // one bit per device
   int dev = 0;
@@ -43,6 +43,14 @@ cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b, const CUtenso
   cfg.attrs = attr;
   cfg.numAttrs = CG == 2 ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, kernel, a, b, d, args);
+}
+
+// The stream-K instantiation only for plans that split the last round.
+template <Mode MODE, int CG, typename OutT>
+cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& d, const GemmArgs& args,
+                       int grid, cudaStream_t stream) {
+  return args.sk_iters > 0 ? launch_split<MODE, CG, OutT, true>(a, b, d, args, grid, stream)
+                           : launch_split<MODE, CG, OutT, false>(a, b, d, args, grid, stream);
 }
 
 template <int CG>

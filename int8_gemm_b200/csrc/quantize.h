@@ -1,5 +1,6 @@
 // Internal interface of the quantiser kernels (kernels_quantize.cu,
-// kernels_quantize_t.cu) for the C-ABI layer.  Not part of the public header.
+// kernels_quantize_t.cu, kernels_quantize_blocks.cu) for the C-ABI layer.
+// Not part of the public header.
 #pragma once
 
 #include <cuda_runtime.h>
@@ -22,5 +23,13 @@ cudaError_t launch_quantize_1x128(const void* x, bool x_bf16, long long M, long 
 cudaError_t launch_quantize_t(const void* x, bool x_bf16, long long R, long long C, long long ldx, uint8_t* q_t,
                               long long ldq, void* scale, bool e8m0, bool block128, long long lds, int sms,
                               cudaStream_t stream);
+
+// 128x128 block quantisation of x [R, C] (bf16 or fp32, row stride ldx
+// elements) in its own orientation: codes q [R, C] (row stride ldq bytes),
+// q[r][c] the code of x[r][c], one scale per block (rb, cb) at
+// scale[rb * s_rb + cb * s_cb] (element strides), fp32 or e8m0 bytes.
+cudaError_t launch_quantize_blocks(const void* x, bool x_bf16, long long R, long long C, long long ldx, uint8_t* q,
+                                   long long ldq, void* scale, bool e8m0, long long s_rb, long long s_cb, int sms,
+                                   cudaStream_t stream);
 
 }  // namespace bsg

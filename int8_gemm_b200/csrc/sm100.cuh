@@ -32,6 +32,7 @@ enum : uint32_t {
   kWaitDrain = 5,
   kWaitScaleFull = 6,
   kWaitScaleEmpty = 7,
+  kWaitPartial = 8,  // a stream-K partial sum from another unit
 };
 constexpr uint64_t kTimeoutNs = 2000000000ull;  // 2 s per wait
 
@@ -60,6 +61,19 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 // after the wait.
 __device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void grid_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// One lane of the (converged) warp, the same one every time: the lowest
+// active lane.  Used so a whole warp runs an issue loop -- its waits, fences
+// and descriptor arithmetic stay warp-uniform -- while one thread issues.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\t"
+      "elect.sync _|P, 0xffffffff;\n\t"
+      "selp.b32 %0, 1, 0, P;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
 
 // Bytes of dynamic shared memory this launch provides.
 __device__ __forceinline__ uint32_t dynamic_smem_bytes() {
@@ -153,6 +167,37 @@ __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, vol
   const uint32_t a = smem_u32(bar);
   if (CLUSTER ? mbar_try_wait_cluster(a, parity) : mbar_try_wait(a, parity)) return true;
   return wait_slow<CLUSTER>(a, parity, abort, err, code);
+}
+
+// Flag words in global memory for hand-overs between CTAs: a release store
+// after the data it publishes, an acquire load before the data it guards.
+__device__ __forceinline__ void st_release_gpu(uint32_t* p, uint32_t v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Waits until *flag is non-zero, another role raised `abort`, or kTimeoutNs
+// elapsed (then records `code` and raises `abort`).
+__device__ __forceinline__ bool wait_flag_bounded(const uint32_t* flag, volatile int* abort, uint32_t* err,
+                                                  uint32_t code) {
+  if (ld_acquire_gpu(flag) != 0u) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t i = 0;; ++i) {
+    __nanosleep(64);
+    if (ld_acquire_gpu(flag) != 0u) return true;
+    if ((i & 15u) == 15u) {
+      if (*abort) return false;
+      if (globaltimer_ns() - t0 > kTimeoutNs) {
+        record_error(err, code);
+        *abort = 1;
+        return false;
+      }
+    }
+  }
 }
 
 // Bounded pause (used only on the abort path to let copies that the CTA

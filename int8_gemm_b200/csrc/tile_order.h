@@ -38,4 +38,63 @@ BSG_HD TileCoord tile_coord(int t, int grid_m, int grid_n, int group_m) {
   return c;
 }
 
+// Stream-K split of the persistent loop (balances the last, partial wave of
+// tiles over every unit -- a CTA pair or a single CTA).  Tiles
+// [0, dp_tiles) are processed whole, unit u taking tiles u, u + units, ...
+// (data-parallel rounds).  The K blocks of the remaining tiles form one
+// sequence of sk_iters = (num_tiles - dp_tiles) * KB blocks, tile by tile,
+// cut into `units` contiguous ranges: unit u takes indices
+// [u * sk_iters / units, (u + 1) * sk_iters / units).  A tile whose K blocks
+// fall into several ranges is finished by the unit holding its first block
+// (the "head", which reaches it last: it is at the end of that unit's range);
+// the others hand over their fp32 (int32) partial sums.
+struct WorkItem {
+  int tile;
+  int kb0, kb1;  // K blocks [kb0, kb1) of the tile
+};
+
+BSG_HD long long sk_range_begin(long long sk_iters, int unit, int units) {
+  return sk_iters * unit / units;
+}
+
+// The unit whose range holds stream-K block index i (the largest u with
+// sk_range_begin(u) <= i).
+BSG_HD int sk_unit_of(long long i, long long sk_iters, int units) {
+  return static_cast<int>(((i + 1) * units - 1) / sk_iters);
+}
+
+// Only the position is state; the split's constants come with each call, so
+// a kernel keeps three values live across its loops.
+struct WorkIter {
+  int next_dp;
+  long long sk, sk_end;
+
+  BSG_HD WorkIter(int unit, int units, long long sk_iters)
+      : next_dp(unit),
+        sk(sk_iters > 0 ? sk_range_begin(sk_iters, unit, units) : 0),
+        sk_end(sk_iters > 0 ? sk_range_begin(sk_iters, unit + 1, units) : 0) {}
+
+  // The next work item of this unit, in processing order; false when done.
+  BSG_HD bool next(WorkItem& w, int units, int dp_tiles, int KB) {
+    if (next_dp < dp_tiles) {
+      w.tile = next_dp;
+      w.kb0 = 0;
+      w.kb1 = KB;
+      next_dp += units;
+      return true;
+    }
+    if (sk < sk_end) {
+      const long long rel = sk / KB;
+      const long long tile_end = (rel + 1) * KB;
+      const long long stop = sk_end < tile_end ? sk_end : tile_end;
+      w.tile = dp_tiles + static_cast<int>(rel);
+      w.kb0 = static_cast<int>(sk - rel * KB);
+      w.kb1 = w.kb0 + static_cast<int>(stop - sk);
+      sk = stop;
+      return true;
+    }
+    return false;
+  }
+};
+
 }  // namespace bsg

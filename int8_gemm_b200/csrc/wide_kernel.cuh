@@ -90,7 +90,22 @@ struct GemmArgs {
   const float* bias;
   const float* s_result;
   uint32_t* err;
+  // Stream-K split of the wide kernel (tile_order.h): tiles [0, dp_tiles)
+  // whole, the sk_iters K blocks of the others cut evenly over the units
+  // (sk_iters == 0: no split).  sk_ws: one partial-sum slot per unit and
+  // CTA (kWsSlotWords words); sk_flags: one word per slot and consumer warp,
+  // zero between launches.
+  int dp_tiles;
+  long long sk_iters;
+  uint32_t* sk_ws;
+  uint32_t* sk_flags;
 };
+
+// A stream-K partial-sum slot: the 128 x 256 accumulator of one CTA, laid out
+// per consumer warp as [column / 4][lane][column % 4] (16-byte pieces, so a
+// warp's stores and loads of four columns cover 512 contiguous bytes).
+constexpr int kWsSlotWords = 8 * 128 * 32;
+constexpr int kWsFlagsPerSlot = 8;
 
 // Shared-memory layout of one CTA.  In the pair (cta_group::2) variant both
 // CTAs use the same layout: the leader's MMA descriptors address the same
@@ -127,6 +142,7 @@ struct WideSmem {
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
+  long long sk_pos[8];  // consumer warps: position in the stream-K range (kept out of registers)
 };
 
 // Row and column-block factors of the block scale (0 outside the problem; the
@@ -230,7 +246,10 @@ static_assert(128 * kWideProducerRegs + 256 * kWideConsumerRegs <= 384 * 168, "r
 // and more stages fit.  Both CTAs' TMA loads signal the leader's full barrier;
 // the leader's commits arrive on both CTAs' barriers; the peer's consumers
 // release the leader's accumulator barrier remotely.
-template <Mode MODE, int CG, int STAGES, typename OutT>
+// SPLIT: the plan splits the last round of tiles (stream-K, tile_order.h); a
+// separate instantiation, so the consumers of plans without a split keep
+// their registers for the promotion loop.
+template <Mode MODE, int CG, int STAGES, typename OutT, bool SPLIT>
 __global__ void __launch_bounds__(384, 1)
     wide_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmD, const GemmArgs p) {
@@ -319,11 +338,13 @@ __global__ void __launch_bounds__(384, 1)
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true;
-        for (int tile = unit; ok && tile < p.num_tiles; tile += units) {
-          const TileCoord tc = tile_coord(tile, p.grid_m, p.grid_n, p.group_m);
+        WorkIter it(unit, units, p.sk_iters);
+        WorkItem w;
+        while (ok && it.next(w, units, p.dp_tiles, p.KB)) {
+          const TileCoord tc = tile_coord(w.tile, p.grid_m, p.grid_n, p.group_m);
           const int m0 = tc.pm * (BM * CG) + rank * BM;
           const int nb0 = tc.pn * BN + rank * BNL;  // this CTA's B rows (tile columns)
-          for (int kb = 0; kb < p.KB; ++kb) {
+          for (int kb = w.kb0; kb < w.kb1; ++kb) {
             if (!wait_bounded(&sm.empty[stage], phase ^ 1u, abort, p.err,
                               kErrTimeout | kRoleProducer | kWaitStageEmpty)) {
               ok = false;
@@ -373,11 +394,14 @@ __global__ void __launch_bounds__(384, 1)
         uint32_t phase = 0, bphase = 0;
         uint32_t sfc = 0;  // kFp8Mx: scale-factor slots consumed (ring position)
         bool ok = true;
-        for (int tile = unit; ok && tile < p.num_tiles; tile += units) {
-          for (int kb = 0; kb < p.KB; ++kb) {
+        WorkIter it(unit, units, p.sk_iters);
+        WorkItem w;
+        while (ok && it.next(w, units, p.dp_tiles, p.KB)) {
+          for (int kb = w.kb0; kb < w.kb1; ++kb) {
+            const bool first = kb == w.kb0, last = kb == w.kb1 - 1;
             // FP8: every K block starts a fresh partial in the next buffer;
-            // INT8: the tile's accumulator is claimed once, at its first K block
-            if (!FULL_K || kb == 0) {
+            // INT8: the work item's accumulator is claimed once, at its first K block
+            if (!FULL_K || first) {
               if (!wait_bounded(&sm.acc_empty[buf], bphase ^ 1u, abort, p.err, kErrTimeout | kRoleMma | kWaitAccEmpty)) {
                 ok = false;
                 break;
@@ -395,7 +419,8 @@ __global__ void __launch_bounds__(384, 1)
               break;
             }
             const int sslot = static_cast<int>(sfc % kSfRing);
-            const uint32_t sf_id = static_cast<uint32_t>(kb & 3);  // kFp8Mx: this K block's byte in the slot
+            // kFp8Mx: this K block's byte in its slot (slots start at the item's first K block)
+            const uint32_t sf_id = static_cast<uint32_t>((kb - w.kb0) & 3);
             if constexpr (MX) {  // both CTAs' scale factors of K blocks kb..kb+3 are in shared memory
               if (sf_id == 0 && !wait_bounded<true>(&sm.sc_full[sslot], (sfc / kSfRing) & 1u, abort, p.err,
                                                     kErrTimeout | kRoleMma | kWaitScaleFull)) {
@@ -420,7 +445,7 @@ __global__ void __launch_bounds__(384, 1)
             }
 #pragma unroll
             for (int k = 0; k < BK / 32; ++k) {
-              const uint32_t acc = FULL_K ? ((kb > 0 || k > 0) ? 1u : 0u) : (k > 0 ? 1u : 0u);
+              const uint32_t acc = FULL_K ? ((!first || k > 0) ? 1u : 0u) : (k > 0 ? 1u : 0u);
               if constexpr (CG == 2) {
                 if constexpr (IS_INT8) {
                   mma_i8_pair(d, ad + 2 * k, bd + 2 * k, IDESC, acc);
@@ -444,17 +469,17 @@ __global__ void __launch_bounds__(384, 1)
             if constexpr (CG == 2) {
               mma_commit_pair_mc(&sm.empty[stage], 0x3);
               if constexpr (MX) {  // after the slot's last K block: free it in both CTAs
-                if (sf_id == 3 || kb == p.KB - 1) {
+                if (sf_id == 3 || last) {
                   mma_commit_pair_mc(&sm.sc_empty[sslot], 0x3);
                   ++sfc;
                 }
               }
-              if (FULL_K && kb == p.KB - 1) mma_commit_pair_mc(&sm.acc_full[buf], 0x3);
+              if (FULL_K && last) mma_commit_pair_mc(&sm.acc_full[buf], 0x3);
             } else {
               mma_commit(&sm.empty[stage]);
-              if (FULL_K && kb == p.KB - 1) mma_commit(&sm.acc_full[buf]);
+              if (FULL_K && last) mma_commit(&sm.acc_full[buf]);
             }
-            if (!FULL_K || kb == p.KB - 1) {
+            if (!FULL_K || last) {
               if (++buf == NACC) {
                 buf = 0;
                 bphase ^= 1u;
@@ -490,17 +515,19 @@ __global__ void __launch_bounds__(384, 1)
       const uint32_t sc_full0 = CG == 2 ? mapa_shared(smem_u32(&sm.sc_full[0]), 0) : smem_u32(&sm.sc_full[0]);
       uint32_t cnt = 0;  // slots staged so far (ring position)
       bool ok = true;
-      for (int tile = unit; ok && tile < p.num_tiles; tile += units) {
-        const TileCoord tc = tile_coord(tile, p.grid_m, p.grid_n, p.group_m);
+      WorkIter it(unit, units, p.sk_iters);
+      WorkItem w;
+      while (ok && it.next(w, units, p.dp_tiles, p.KB)) {
+        const TileCoord tc = tile_coord(w.tile, p.grid_m, p.grid_n, p.group_m);
         const int m0 = tc.pm * (BM * CG) + rank * BM, nb0 = tc.pn * 2;
         const int ma = m0 + t, mc = m0 + t + 64;
-        for (int kb0 = 0; ok && kb0 < p.KB; kb0 += 4) {
+        for (int kb0 = w.kb0; ok && kb0 < w.kb1; kb0 += 4) {
           // the 16 loads of a slot are in flight together
           uint32_t wa = 0, wc = 0, w0 = 0, w1 = 0;
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             const long long kb = kb0 + j;
-            const bool in_k = kb < p.KB;
+            const bool in_k = kb < w.kb1;
             const uint32_t a = in_k && ma < p.M ? __ldg(p.xs + (static_cast<long long>(ma) * p.G + tc.g) * p.KB + kb)
                                                 : 127u;
             const uint32_t c = in_k && mc < p.M ? __ldg(p.xs + (static_cast<long long>(mc) * p.G + tc.g) * p.KB + kb)
@@ -542,11 +569,13 @@ __global__ void __launch_bounds__(384, 1)
       const int t = threadIdx.x - 64;  // 0..63
       uint32_t cnt = 0;                // K blocks staged so far (ring position)
       bool ok = true;
-      for (int tile = unit; ok && tile < p.num_tiles; tile += units) {
-        const TileCoord tc = tile_coord(tile, p.grid_m, p.grid_n, p.group_m);
+      WorkIter it(unit, units, p.sk_iters);
+      WorkItem w;
+      while (ok && it.next(w, units, p.dp_tiles, p.KB)) {
+        const TileCoord tc = tile_coord(w.tile, p.grid_m, p.grid_n, p.group_m);
         const int m0 = tc.pm * (BM * CG) + rank * BM, n0 = tc.pn * BN;
-        for (int kb0 = 0; ok && kb0 < p.KB; kb0 += kScaleBatch) {
-          const int nb = p.KB - kb0 < kScaleBatch ? p.KB - kb0 : kScaleBatch;
+        for (int kb0 = w.kb0; ok && kb0 < w.kb1; kb0 += kScaleBatch) {
+          const int nb = w.kb1 - kb0 < kScaleBatch ? w.kb1 - kb0 : kScaleBatch;
           float va[kScaleBatch], vc[kScaleBatch], vb[kScaleBatch];
 #pragma unroll
           for (int i = 0; i < kScaleBatch; ++i) {
@@ -593,12 +622,29 @@ __global__ void __launch_bounds__(384, 1)
         CG == 2 ? mapa_shared(smem_u32(&sm.ovl_empty[0]), 0) : smem_u32(&sm.ovl_empty[0]);
     int buf = 0, sslot = 0;
     uint32_t bphase = 0, ssph = 0;
-    uint32_t kbc = 0;  // K blocks of this CTA's tiles seen so far (stage = kbc % STAGES)
-    for (int tile = unit; tile < p.num_tiles; tile += units) {
-      const TileCoord tc = tile_coord(tile, p.grid_m, p.grid_n, p.group_m);
-      const int m0 = tc.pm * (BM * CG) + rank * BM, n0 = tc.pn * BN;
-      const int m = m0 + row;
-      const int ncol0 = n0 + half * 128;
+    uint32_t kbc = 0;  // K blocks of this CTA's work items seen so far (stage = kbc % STAGES)
+    // stream-K hand-over: this warp's part of unit u's partial-sum slot (a
+    // [column / 4][lane] array of 16-byte pieces) and its flag word
+    auto slot_piece = [&](int u) -> uint4* {
+      return reinterpret_cast<uint4*>(p.sk_ws) + (static_cast<long long>(u * CG + rank) * 8 + cw) * (128 * 32 / 4);
+    };
+    auto slot_flag = [&](int u) -> uint32_t* {
+      return p.sk_flags + static_cast<long long>(u * CG + rank) * kWsFlagsPerSlot + cw;
+    };
+    auto has_range = [&](int u) {
+      return sk_range_begin(p.sk_iters, u, units) != sk_range_begin(p.sk_iters, u + 1, units);
+    };
+    // The item's stream-K role: a whole tile; a later part of a split tile (a
+    // giver: its partial goes to this unit's slot); or the head of a split
+    // tile, which adds the partials of units c_lo..c_hi, in that order, to its
+    // own and stores the result.  (Worked out after the promotion loop, so
+    // none of it is live across that loop.)
+    auto givers_of = [&](const WorkItem& wi, int& lo, int& hi) {
+      lo = unit + 1;
+      hi = sk_unit_of(static_cast<long long>(wi.tile - p.dp_tiles) * p.KB + p.KB - 1, p.sk_iters, units);
+    };
+    // one work item; false when a wait gave up (the CTA is winding down)
+    auto process = [&](const WorkItem& w) -> bool {
       bool ok = true;
       if constexpr (!FULL_K) {
         // fp32 accumulators; the promotion uses the packed two-wide FMA, which
@@ -608,7 +654,7 @@ __global__ void __launch_bounds__(384, 1)
         float acc[128];
 #pragma unroll
         for (int j = 0; j < 128; ++j) acc[j] = 0.f;
-        for (int kb = 0; kb < p.KB; ++kb) {
+        for (int kb = w.kb0; kb < w.kb1; ++kb) {
           if (!warp_wait(&sm.sc_full[sslot], ssph, abort, p.err, kErrTimeout | kRoleConsumer | kWaitScaleFull)) {
             ok = false;
             break;
@@ -650,7 +696,51 @@ __global__ void __launch_bounds__(384, 1)
           buf ^= 1;
           if (buf == 0) bphase ^= 1u;
         }
-        if (!ok) break;
+        if (!ok) return false;
+        const bool whole = w.kb0 == 0 && w.kb1 == p.KB;
+        if (w.kb0 > 0) {  // giver
+          uint4* dst = slot_piece(unit);
+#pragma unroll
+          for (int q = 0; q < 32; ++q)
+            dst[q * 32 + lane] = make_uint4(__float_as_uint(acc[4 * q]), __float_as_uint(acc[4 * q + 1]),
+                                            __float_as_uint(acc[4 * q + 2]), __float_as_uint(acc[4 * q + 3]));
+          __threadfence();
+          __syncwarp();
+          if (lane == 0) st_release_gpu(slot_flag(unit), 1u);
+          return true;
+        }
+        int c_lo = 0, c_hi = -1;
+        if (!whole) givers_of(w, c_lo, c_hi);
+        for (int u = c_lo; u <= c_hi; ++u) {
+          if (!has_range(u)) continue;
+          if (!wait_flag_bounded(slot_flag(u), abort, p.err, kErrTimeout | kRoleConsumer | kWaitPartial)) {
+            ok = false;
+            break;
+          }
+          const uint4* src = slot_piece(u);
+          // four 16-byte pieces in flight at a time: the 128 accumulators
+          // leave no registers for more
+#pragma unroll
+          for (int q0 = 0; q0 < 32; q0 += 4) {
+            uint4 v[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) v[q] = __ldcg(src + (q0 + q) * 32 + lane);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              acc[4 * (q0 + q)] += __uint_as_float(v[q].x);
+              acc[4 * (q0 + q) + 1] += __uint_as_float(v[q].y);
+              acc[4 * (q0 + q) + 2] += __uint_as_float(v[q].z);
+              acc[4 * (q0 + q) + 3] += __uint_as_float(v[q].w);
+            }
+            asm volatile("" ::: "memory");  // keep the next group's loads after these adds
+          }
+          __syncwarp();
+          if (lane == 0) *slot_flag(u) = 0u;  // zero again for the next launch
+        }
+        if (!ok) return false;
+        const TileCoord tc = tile_coord(w.tile, p.grid_m, p.grid_n, p.group_m);
+        const int m0 = tc.pm * (BM * CG) + rank * BM;
+        const int ncol0 = tc.pn * BN + half * 128;
 #pragma unroll
         for (int ch = 0; ch < 128 / CPC; ++ch) {
           if (lane == 0) bulk_wait_read_all();
@@ -667,9 +757,26 @@ __global__ void __launch_bounds__(384, 1)
           }
         }
       } else {
+        const TileCoord tc = tile_coord(w.tile, p.grid_m, p.grid_n, p.group_m);
+        const int m0 = tc.pm * (BM * CG) + rank * BM;
+        const int m = m0 + row;
+        const int ncol0 = tc.pn * BN + half * 128;
+        const bool whole = w.kb0 == 0 && w.kb1 == p.KB;
+        const bool giver = w.kb0 > 0;
+        int c_lo = 0, c_hi = -1;
+        if (!whole && !giver) givers_of(w, c_lo, c_hi);
         if (!warp_wait(&sm.acc_full[buf], bphase, abort, p.err, kErrTimeout | kRoleConsumer | kWaitAccFull))
-          break;
+          return false;
         tc_fence_after();
+        // the head waits for every giver's partial before it reads any
+        for (int u = c_lo; u <= c_hi; ++u) {
+          if (has_range(u) &&
+              !wait_flag_bounded(slot_flag(u), abort, p.err, kErrTimeout | kRoleConsumer | kWaitPartial)) {
+            ok = false;
+            break;
+          }
+        }
+        if (!ok) return false;
         const bool has_row = p.s_row != nullptr, has_col = p.s_col != nullptr;
         const float sr = (has_row && m < p.M) ? __ldg(p.s_row + (IS_INT8 || p.s_row_stride != 0 ? m : 0)) : 1.f;
         // FP8 rowwise: this thread's column scales start at s_col_n and advance by col_step
@@ -686,8 +793,10 @@ __global__ void __launch_bounds__(384, 1)
         const int rot = MX && buf == 0 && half == 1 ? NCH - OVC : 0;
 #pragma unroll
         for (int ch = 0; ch < NCH; ++ch) {
-          if (lane == 0) bulk_wait_read_all();
-          __syncwarp();
+          if (!giver) {
+            if (lane == 0) bulk_wait_read_all();
+            __syncwarp();
+          }
           const int c0 = (MX ? (ch + rot) % NCH : ch) * CPC;
           uint32_t r[CPC];
           if constexpr (CPC == 64) {
@@ -702,6 +811,29 @@ __global__ void __launch_bounds__(384, 1)
               tc_fence_before();
               __syncwarp();
               if (lane == 0) mbar_arrive_cluster(ovl_empty0 + static_cast<uint32_t>(buf * sizeof(uint64_t)));
+            }
+          }
+          if (giver) {  // the raw accumulator (fp32, or int32 for INT8) to this unit's slot
+            uint4* dst = slot_piece(unit) + (c0 / 4) * 32 + lane;
+#pragma unroll
+            for (int q = 0; q < CPC / 4; ++q) dst[q * 32] = make_uint4(r[4 * q], r[4 * q + 1], r[4 * q + 2], r[4 * q + 3]);
+            continue;
+          }
+          for (int u = c_lo; u <= c_hi; ++u) {  // the head adds the givers' partials in unit order
+            if (!has_range(u)) continue;
+            const uint4* src = slot_piece(u) + (c0 / 4) * 32 + lane;
+#pragma unroll
+            for (int q = 0; q < CPC / 4; ++q) {
+              const uint4 g = __ldcg(src + q * 32);
+              const uint32_t gv[4] = {g.x, g.y, g.z, g.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                if constexpr (IS_INT8) {
+                  r[4 * q + e] += gv[e];  // exact int32 sum (two's complement)
+                } else {
+                  r[4 * q + e] = __float_as_uint(__uint_as_float(r[4 * q + e]) + __uint_as_float(gv[e]));
+                }
+              }
             }
           }
           float v[CPC];
@@ -745,6 +877,15 @@ __global__ void __launch_bounds__(384, 1)
             bulk_commit();
           }
         }
+        if (giver) {
+          __threadfence();
+          __syncwarp();
+          if (lane == 0) st_release_gpu(slot_flag(unit), 1u);
+        } else if (!whole) {
+          __syncwarp();
+          if (lane == 0)
+            for (int u = c_lo; u <= c_hi; ++u) *slot_flag(u) = 0u;  // zero again for the next launch
+        }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(acc_empty0 + static_cast<uint32_t>(buf * sizeof(uint64_t)));
@@ -752,6 +893,27 @@ __global__ void __launch_bounds__(384, 1)
           buf = 0;
           bphase ^= 1u;
         }
+      }
+          return true;
+    };
+    // whole tiles (the data-parallel rounds), then this unit's stream-K range
+    bool live = true;
+    for (int tile = unit; live && tile < p.dp_tiles; tile += units) live = process(WorkItem{tile, 0, p.KB});
+    if (SPLIT && live && p.sk_iters > 0) {
+      // the range's position lives in shared memory, so no iterator state is
+      // held in registers across an item's promotion loop
+      if (lane == 0) sm.sk_pos[cw] = sk_range_begin(p.sk_iters, unit, units);
+      __syncwarp();
+      while (live) {
+        WorkIter it(unit, units, p.sk_iters);
+        it.next_dp = p.dp_tiles;  // the whole tiles are done
+        it.sk = sm.sk_pos[cw];
+        WorkItem w;
+        if (!it.next(w, units, p.dp_tiles, p.KB)) break;
+        __syncwarp();
+        if (lane == 0) sm.sk_pos[cw] = it.sk;
+        __syncwarp();
+        live = process(w);
       }
     }
     if (lane == 0) bulk_wait_all();

@@ -21,7 +21,17 @@ Parity status of each function (what pins it in ``tests/test_oracle_pins.py``):
                        even code), saturation; torch's float8_e4m3fn cast
   quantize_1x128    -- torch's float8_e4m3fn cast of x / scale (the library
                        routine the recipe reduces to), amax -> +-448, zero
-                       groups, e8m0 exponent at and around 448 * 2^e, ragged K
+                       groups, e8m0 exponent at and around 448 * 2^e, ragged K,
+                       scales that underflow take the zero group's scale
+  quantize_t        -- 128x1 groups = the 1x128 quantiser of the transpose;
+                       torch's cast of x over its 128x128 block scale; one-hot
+                       orientation and block isolation; a block's scale is its
+                       largest column scale; the backward GEMMs of the
+                       quantised operands approximate the exact gradients
+  quantize_128x128  -- torch's cast of x over its block scale; the transposed
+                       quantiser's 128x128 codes, transposed back; one-hot block
+                       isolation and orientation; the forward GEMM of the
+                       quantised weight approximates the exact product
 """
 from __future__ import annotations
 
@@ -70,8 +80,9 @@ def _load():
             lib.orc_e4m3_encode.argtypes = [p, p, i64]
             lib.orc_quantize_1x128.argtypes = [p, i64, i64, i64, ctypes.c_int, p, i64, p, p]
             lib.orc_quantize_t.argtypes = [p, i64, i64, i64, ctypes.c_int, ctypes.c_int, p, i64, p, p]
+            lib.orc_quantize_128x128.argtypes = [p, i64, i64, i64, ctypes.c_int, p, i64, p, p]
             for f in (lib.orc_fp8_blockwise, lib.orc_bmm_blockscale, lib.orc_int_scaled_mm, lib.orc_fp8_rowwise,
-                      lib.orc_quantize_1x128, lib.orc_quantize_t):
+                      lib.orc_quantize_1x128, lib.orc_quantize_t, lib.orc_quantize_128x128):
                 f.restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -280,4 +291,25 @@ def quantize_t(x, group: int = 0, fmt: int = 0):
     rc = _load().orc_quantize_t(_ptr(xt), R, C, C, group, fmt, _ptr(q), R, _ptr(sf), _ptr(se))
     if rc != 0:
         raise ValueError(f"orc_quantize_t failed ({rc})")
+    return q, (sf if fmt == 0 else se)
+
+
+def quantize_128x128(x, fmt: int = 0):
+    """128x128 block quantisation of x [R, C] (fp32 or bf16) keeping its orientation (a weight W [N, K]
+    becomes the B_t codes of the forward GEMM).
+
+    Returns (codes uint8 [R, C], q[r, c] the code of x[r, c]; scales [ceil(R/128), ceil(C/128)], fp32 for
+    fmt 0 or e8m0 bytes for fmt 1).  The transpose of the scales is scale_b [K/128, N/128] for x = W [N, K].
+    See orc_quantize_128x128."""
+    xt = _np(x.float() if hasattr(x, "float") and not isinstance(x, np.ndarray) else x)
+    xt = np.ascontiguousarray(xt, dtype=np.float32)
+    assert xt.ndim == 2
+    R, C = xt.shape
+    RB, CB = -(-R // 128), -(-C // 128)
+    q = np.empty((R, C), dtype=np.uint8)
+    sf = np.empty((RB, CB), dtype=np.float32) if fmt == 0 else None
+    se = np.empty((RB, CB), dtype=np.uint8) if fmt == 1 else None
+    rc = _load().orc_quantize_128x128(_ptr(xt), R, C, C, fmt, _ptr(q), C, _ptr(sf), _ptr(se))
+    if rc != 0:
+        raise ValueError(f"orc_quantize_128x128 failed ({rc})")
     return q, (sf if fmt == 0 else se)

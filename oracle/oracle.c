@@ -505,3 +505,42 @@ int orc_quantize_t(const float *x, int64_t R, int64_t C, int64_t ldx, int group,
     }
     return ORC_OK;
 }
+
+/*
+ * 128x128 block quantisation in the input's own orientation, for the forward
+ * GEMM's weight operand: a weight W [N, K] (x [R, C], row stride ldx) becomes
+ * codes q [R, C] (row stride ldq), q[r][c] the code of x[r][c], with one scale
+ * per block of rows 128rb .. min(128rb + 128, R) - 1 and columns
+ * 128cb .. min(128cb + 128, C) - 1, scale[rb * CB + cb] ([RB, CB]), and the
+ * scale and code rules of orc_quantize_1x128.  For x = W [N, K] the codes are
+ * the B_t [N, K] of the blockwise GEMM and the transposed scale matrix is its
+ * scale_b [K/128, N/128].
+ *   Source: pytorch issue "torch._scaled_mm with blockwise scaling doesn't
+ *   work with torch.compile" (128x128 weight blocks with one fp32 scale each,
+ *   scale_b (64, 40) for K = 8192, N = 5120).
+ */
+int orc_quantize_128x128(const float *x, int64_t R, int64_t C, int64_t ldx, int fmt,
+                         uint8_t *q, int64_t ldq, float *scale_f32, uint8_t *scale_e8m0)
+{
+    if (R < 0 || C < 0 || ldx < C || ldq < C || (fmt != 0 && fmt != 1)) return ORC_ERR_SHAPE;
+    const int64_t RB = (R + 127) / 128, CB = (C + 127) / 128;
+#pragma omp parallel for schedule(dynamic, 4)
+    for (int64_t bi = 0; bi < RB * CB; ++bi) {
+        const int64_t rb = bi / CB, cb = bi % CB;
+        const int64_t r0 = 128 * rb, r1 = r0 + 128 < R ? r0 + 128 : R;
+        const int64_t c0 = 128 * cb, c1 = c0 + 128 < C ? c0 + 128 : C;
+        float amax = 0.0f;
+        for (int64_t r = r0; r < r1; ++r)
+            for (int64_t c = c0; c < c1; ++c) {
+                const float a = fabsf(x[r * ldx + c]);
+                if (a > amax) amax = a;
+            }
+        const float s = group_scale_f32(amax);
+        const int b = group_scale_e8m0(amax);
+        if (fmt == 0) scale_f32[rb * CB + cb] = s;
+        else scale_e8m0[rb * CB + cb] = (uint8_t)b;
+        for (int64_t r = r0; r < r1; ++r)
+            for (int64_t c = c0; c < c1; ++c) q[r * ldq + c] = group_code(x[r * ldx + c], fmt, s, b);
+    }
+    return ORC_OK;
+}

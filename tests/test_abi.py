@@ -41,9 +41,9 @@ def declared_functions():
 def test_header_declares_the_entry_points():
     f = declared_functions()
     for name in ("bs_gemm_fp8_blockwise", "int_scaled_mm", "bmm_a8w8_blockscale", "bs_gemm_fp8_rowwise",
-                 "bs_quantize_fp8_1x128", "bs_quantize_fp8_t"):
+                 "bs_quantize_fp8_1x128", "bs_quantize_fp8_t", "bs_quantize_fp8_128x128"):
         assert name in f
-    assert len(f) >= 13
+    assert len(f) >= 14
 
 
 def test_library_exports_every_declared_symbol():
@@ -81,16 +81,26 @@ def test_blockwise_scale_shape_rule_from_the_issue():
 # ---------------------------------------------------------------------------
 def test_plan_large_fp8_is_persistent_wide_on_cta_pairs():
     p = bs.plan_for(bs.OP_FP8_BLOCKWISE, 16640, 1, 5120, 8192, 148)
-    assert p == {"kernel": 1, "tile_m": 256, "tile_n": 256, "splits": 1, "ctas": 148, "cluster": 2, "launches": 1}
+    assert p == {"kernel": 1, "tile_m": 256, "tile_n": 256, "splits": 1, "ctas": 148, "cluster": 2, "launches": 1,
+                 "sk_tiles": 0}
     prev = bs.set_path_override(bs.PATH_WIDE_SINGLE)
     try:
         p = bs.plan_for(bs.OP_FP8_BLOCKWISE, 16640, 1, 5120, 8192, 148)
-        assert p == {"kernel": 1, "tile_m": 128, "tile_n": 256, "splits": 1, "ctas": 148, "cluster": 1, "launches": 1}
+        assert p == {"kernel": 1, "tile_m": 128, "tile_n": 256, "splits": 1, "ctas": 148, "cluster": 1, "launches": 1,
+                     "sk_tiles": 0}
     finally:
         bs.set_path_override(prev)
-    # fewer tiles than CTA pairs: one pair per tile
+    # fewer tiles than CTA pairs and too few K blocks to spread: one pair per tile
     p = bs.plan_for(bs.OP_FP8_BLOCKWISE, 300, 1, 512, 1024, 148)
-    assert p["ctas"] == 2 * 2 * 2 and p["cluster"] == 2
+    assert p["ctas"] == 2 * 2 * 2 and p["cluster"] == 2 and p["sk_tiles"] == 0
+    # a badly filled last round with enough K blocks: split over every pair
+    p = bs.plan_for(bs.OP_FP8_BLOCKWISE, 1000, 1, 7168, 2048, 148)
+    assert p["ctas"] == 148 and p["sk_tiles"] == 112 - 74
+    prev = bs.set_stream_k(False)
+    try:
+        assert bs.plan_for(bs.OP_FP8_BLOCKWISE, 1000, 1, 7168, 2048, 148)["sk_tiles"] == 0
+    finally:
+        bs.set_stream_k(prev)
 
 
 @pytest.mark.parametrize("M", [1, 8, 16, 17, 32, 127, 128, 129, 255, 256])
@@ -323,3 +333,79 @@ def test_quantize_t_validation_codes():
     if not HAS_GPU:  # well-formed calls reach the device check (never launched with fake pointers on a GPU)
         for kw in ({}, {"grp": 1, "lds": 2}, {"x": P16 + 2}, {"q": P16 + 1}, {"ldx": 201}, {"fmt": 1, "s": P16 + 3}):
             assert _qt(**kw) == bs.BS_ERR_DEVICE, kw
+
+
+def _qb(**kw):
+    a = dict(x=P16, dt=0, R=300, C=200, ldx=208, q=P16, ldq=208, s=P16, fmt=0, srb=1, scb=3)
+    a.update(kw)
+    v = ctypes.c_void_p
+    return bs.lib().bs_quantize_fp8_128x128(v(a["x"]), a["dt"], a["R"], a["C"], a["ldx"], v(a["q"]), a["ldq"],
+                                            v(a["s"]), a["fmt"], a["srb"], a["scb"], None)
+
+
+def test_quantize_128x128_validation_codes():
+    assert _qb(R=-1) == bs.BS_ERR_SHAPE and _qb(C=-5) == bs.BS_ERR_SHAPE and _qb(R=1 << 31) == bs.BS_ERR_SHAPE
+    assert _qb(R=1 << 30, C=1 << 30, ldx=1 << 30, ldq=1 << 30) == bs.BS_ERR_SHAPE  # 2^46 blocks
+    assert _qb(dt=2) == bs.BS_ERR_DTYPE and _qb(fmt=2) == bs.BS_ERR_DTYPE
+    assert _qb(x=0) == bs.BS_ERR_NULL and _qb(q=0) == bs.BS_ERR_NULL and _qb(s=0) == bs.BS_ERR_NULL
+    assert _qb(ldx=199) == bs.BS_ERR_LAYOUT and _qb(ldq=199) == bs.BS_ERR_LAYOUT
+    assert _qb(srb=-1) == bs.BS_ERR_LAYOUT and _qb(scb=0) == bs.BS_ERR_LAYOUT  # 2 column blocks need a stride
+    assert _qb(srb=0) == bs.BS_ERR_LAYOUT                                        # 3 row blocks too
+    assert _qb(x=P16 + 1) == bs.BS_ERR_ALIGNMENT and _qb(dt=1, x=P16 + 2) == bs.BS_ERR_ALIGNMENT
+    assert _qb(s=P16 + 2) == bs.BS_ERR_ALIGNMENT
+    assert _qb(R=0) == bs.BS_OK and _qb(C=0) == bs.BS_OK
+    if not HAS_GPU:  # well-formed calls reach the device check (never launched with fake pointers on a GPU)
+        for kw in ({}, {"R": 100, "srb": 0}, {"C": 100, "scb": 0}, {"x": P16 + 2}, {"q": P16 + 1}, {"ldx": 201},
+                   {"fmt": 1, "s": P16 + 3}):
+            assert _qb(**kw) == bs.BS_ERR_DEVICE, kw
+
+
+@pytest.mark.parametrize("M,N,K,G,op", [(4096, 4096, 4096, 1, 2), (1000, 7168, 2048, 1, 1), (1024, 1024, 4096, 2, 3),
+                                        (1024, 1024, 4096, 8, 3), (300, 1024, 2048, 1, 1), (1024, 1024, 4096, 1, 2),
+                                        (16640, 5120, 8192, 1, 1)])
+@pytest.mark.parametrize("sms", [148, 132])
+def test_stream_k_split_covers_every_k_block_once(M, N, K, G, op, sms):
+    """The host copy of the wide kernel's decomposition: every (tile, K block) is computed by exactly one
+    unit; each split tile has one head (the unit holding its first block, where that block is the last
+    item of the unit); the other pieces are the first split item of their units, so each unit hands over
+    at most one partial and finishes at most one split tile."""
+    p = bs.plan_for(op, M, G, N, K, sms)
+    assert p["kernel"] == 1
+    units = p["ctas"] // p["cluster"]
+    tiles = -(-M // 256) * -(-N // 256) * G
+    KB = -(-K // 128)
+    sk_tiles = p["sk_tiles"]
+    dp = tiles - sk_tiles
+    cover = {}
+    heads, givers = {}, {}
+    for u in range(units):
+        items = bs.work_items(tiles, dp, sk_tiles * KB, KB, units, u)
+        split = [it for it in items if it[0] >= dp]
+        for n_it, (t, k0, k1) in enumerate(items):
+            assert 0 <= k0 < k1 <= KB and 0 <= t < tiles
+            for kb in range(k0, k1):
+                assert (t, kb) not in cover
+                cover[(t, kb)] = u
+            if (k0, k1) != (0, KB):
+                assert t >= dp
+                if k0 == 0:
+                    heads.setdefault(t, []).append(u)
+                    assert (t, k0, k1) == split[-1], "a head is the last item of its unit"
+                else:
+                    givers.setdefault(t, []).append(u)
+                    assert (t, k0, k1) == split[0], "a hand-over is the first split item of its unit"
+        assert sum(1 for it in split if it[1] > 0) <= 1
+    assert len(cover) == tiles * KB
+    for t in givers:
+        assert len(heads[t]) == 1 and all(g > heads[t][0] for g in givers[t])
+    if sk_tiles:
+        assert set(heads) == set(givers) and len(heads) > 0
+        assert p["ctas"] == p["cluster"] * (sms // p["cluster"])
+
+
+def test_workspace_size_and_registration_checks():
+    assert bs.workspace_size(148) >= 148 * 128 * 1024 and bs.workspace_size(0) == 0
+    assert bs.workspace_size(148) % 256 == 0
+    if not HAS_GPU:  # registration needs a device
+        assert bs.lib().bs_set_workspace(ctypes.c_void_p(P16), 1 << 30) == bs.BS_ERR_DEVICE
+    assert bs.status_string(bs.BS_ERR_WORKSPACE) == "BS_ERR_WORKSPACE"

@@ -141,6 +141,8 @@ def test_algorithmic_work_of_every_workload():
             rb = -(-w.M // 128)
             scales = w.K * rb if w.extra["group"] == "128x1" else rb * kb
             want_f, want_b = 0, 3 * w.M * w.K + 4 * scales
+        elif w.op == "quantize_128x128":
+            want_f, want_b = 0, 3 * w.M * w.K + 4 * (-(-w.M // 128)) * kb
         else:
             want_f = 2 * w.M * w.G * w.N * w.K
             want_b = w.M * w.G * w.K + w.G * w.N * w.K + 2 * w.M * w.G * w.N + w.M * w.G * kb + w.G * nb * kb

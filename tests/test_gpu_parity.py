@@ -379,20 +379,23 @@ def test_quantize_1x128_bit_exact(M, K, dtype, fmt):
 
 @pytest.mark.parametrize("fmt", [0, 1])
 def test_quantize_special_groups_and_strides(fmt):
-    x = torch.zeros(6, 520)
+    x = torch.zeros(7, 520)
     x[1] = wl.normal_with_outliers((1, 520), 7100)[0] * 1e-30     # tiny values
+    x[6] = wl.normal_with_outliers((1, 520), 7102)[0] * 1e-44     # amax / 448 underflows fp32: scale 1
     x[2, :128] = 448.0 * 2.0 ** 5                                   # amax exactly 448 * 2^5, constant group
     x[2, 128:256] = torch.linspace(-1.0, 1.0, 128)                  # a tie-rich ramp
     x[3] = -0.0
     x[4] = wl.normal_with_outliers((1, 520), 7101)[0] * 1e20       # huge values
     x[5, 7] = 1.0                                                   # one non-zero element per group
-    base = torch.zeros(6, 640)
+    base = torch.zeros(7, 640)
     base[:, :520] = x
     xv = base.to(DEV)[:, :520]                                      # row stride 640 > K
-    q = torch.full((6, 544), 0x55, dtype=torch.uint8, device=DEV)[:, :520]
-    s = torch.zeros((6, 8), dtype=torch.float32 if fmt == 0 else torch.uint8, device=DEV)[:, :5]
+    q = torch.full((7, 544), 0x55, dtype=torch.uint8, device=DEV)[:, :520]
+    s = torch.zeros((7, 8), dtype=torch.float32 if fmt == 0 else torch.uint8, device=DEV)[:, :5]
     _quant_check(xv, fmt, q=q, scale=s)
-    full = torch.as_strided(q, (6, 544), (544, 1))
+    if fmt == 0:
+        assert torch.all(s[6] == 1.0)
+    full = torch.as_strided(q, (7, 544), (544, 1))
     assert torch.all(full[:, 520:] == 0x55), "wrote past K"
 
 
@@ -444,6 +447,7 @@ def test_quantize_t_special_blocks_strides_and_canaries(group, fmt):
     x[128:256, 1] = torch.linspace(-1.0, 1.0, 128)      # a tie-rich ramp
     x[256:, 5] = 1e-30                                   # tiny values
     x[3, 130] = 3e20                                     # one huge value
+    x[:128, 133] = 3e-44 * torch.linspace(-1.0, 1.0, 128)  # a 128x1 group whose amax / 448 underflows
     base = torch.zeros(R, 141)                           # row stride 141: no 16-byte loads
     base[:, :C] = x
     xv = base.to(DEV)[:, :C]
@@ -483,3 +487,276 @@ def test_backward_gemms_through_the_transposed_quantiser():
     rb2, rsb2 = oracle.quantize_t(W, 1, 0)
     y2, S2 = oracle.fp8_blockwise(ra2, rb2, rsa2, rsb2)
     fp8_check(dx, y2, S2, torch.bfloat16, "input gradient")
+
+
+# ---------------------------------------------------------------------------
+# forward-orientation 128x128 weight quantiser (B_t [N, K] and scale_b) -- bit-exact
+# ---------------------------------------------------------------------------
+def _quant_b_check(x_dev, fmt, **kw):
+    q, s = bs.bs_quantize_fp8_128x128(x_dev, "f32" if fmt == 0 else "e8m0", **kw)
+    rq, rs = oracle.quantize_128x128(x_dev.float().cpu(), fmt)
+    assert_quantised(q.cpu().numpy(), s.t().cpu().numpy(), rq, rs, fmt)
+    return q, s
+
+
+@pytest.mark.parametrize("R,C", [(1, 1), (128, 128), (300, 5), (5, 300), (130, 260), (1000, 384), (384, 4104)])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("fmt", [0, 1])
+def test_quantize_128x128_bit_exact(R, C, dtype, fmt):
+    x = wl.normal_with_outliers((R, C), 9400 + R + C).to(dtype)
+    _quant_b_check(x.to(DEV), fmt)
+
+
+@pytest.mark.parametrize("fmt", [0, 1])
+def test_quantize_128x128_special_blocks_strides_and_canaries(fmt):
+    R, C = 260, 300
+    x = wl.normal_with_outliers((R, C), 9500)
+    x[:128, :128] = 0.0                                   # an all-zero block
+    x[:128, 128:256] = 3e-44 * torch.linspace(-1.0, 1.0, 128)[None, :]  # amax / 448 underflows: scale 1
+    x[128:256, :128] = torch.linspace(-1.0, 1.0, 128)[:, None] * 448.0 * 2.0 ** 5  # amax exactly 448 * 2^5
+    x[256:, 7] = 1e-30                                    # tiny values
+    x[200, 290] = 3e20                                    # one huge value
+    base = torch.zeros(R, 303)                            # row stride 303: no 16-byte loads
+    base[:, :C] = x
+    xv = base.to(DEV)[:, :C]
+    q = torch.full((R, 320), 0x55, dtype=torch.uint8, device=DEV)[:, :C]
+    sfull = torch.full((3, 5), 9, dtype=torch.float32 if fmt == 0 else torch.uint8, device=DEV)
+    s = sfull[:, :3]                                     # [CB, RB] with a padded row stride
+    _quant_b_check(xv, fmt, q=q, scale=s)
+    assert torch.all(torch.as_strided(q, (R, 320), (320, 1))[:, C:] == 0x55), "wrote past C"
+    assert torch.all(sfull[:, 3:] == 9), "wrote past the scale rows"
+    if fmt == 0:
+        assert float(s[1, 0]) == 1.0 and float(s[0, 0]) == 1.0
+
+
+def test_quantize_128x128_full_size_weight():
+    W = wl.normal_with_outliers((5120, 8192), 9600).to(torch.bfloat16).to(DEV)
+    _quant_b_check(W, 0)
+
+
+def test_forward_gemm_through_the_weight_quantiser():
+    """y = x W^T with x in 1x128 groups and W in 128x128 blocks, both quantised on the GPU and fed to the
+    blockwise GEMM without a copy (B = q.t(), scale_b as returned)."""
+    M, N, K = 300, 384, 1024
+    x = wl.normal_with_outliers((M, K), 9700)
+    W = wl.normal_with_outliers((N, K), 9701)
+    a, sa = bs.quantize_fp8_1x128(x.to(DEV), "f32")
+    b, sb = bs.bs_quantize_fp8_128x128(W.to(DEV), "f32")
+    y_gpu = bs.bs_gemm_fp8_blockwise(a, b.t(), sa, sb)
+    ra, rsa = oracle.quantize_1x128(x, 0)
+    rb, rsb = oracle.quantize_128x128(W, 0)
+    assert np.array_equal(b.cpu().numpy(), rb) and np.array_equal(sb.cpu().numpy(), rsb.T)
+    y, S = oracle.fp8_blockwise(ra, rb, rsa, rsb.T)
+    fp8_check(y_gpu, y, S, torch.bfloat16, "forward GEMM of the quantised weight")
+
+
+# ---------------------------------------------------------------------------
+# stream-K: the last, badly filled round of tiles split over every CTA pair
+# ---------------------------------------------------------------------------
+def _sk_tiles(op, M, G, N, K):
+    return bs.plan_for(op, M, G, N, K, torch.cuda.get_device_properties(0).multi_processor_count)["sk_tiles"]
+
+
+@pytest.fixture
+def no_stream_k():
+    def off():
+        bs.set_stream_k(False)
+    yield off
+    bs.set_stream_k(True)
+
+
+@pytest.mark.parametrize("M,N,K", [(1024, 1024, 4096), (1000, 1800, 2080), (300, 1040, 8192)])
+@pytest.mark.parametrize("kernel", [bs.PATH_WIDE, bs.PATH_WIDE_SINGLE])
+def test_int8_stream_k_bit_exact(M, N, K, kernel, path):
+    path(kernel)
+    assert _sk_tiles(bs.OP_INT_SCALED_MM, M, 1, N, K) > 0
+    _int8_assert(wl.int8_inputs(M, N, K, seed=950 + M), rows=None)
+
+
+@pytest.mark.parametrize("M,N,K", [(1024, 1024, 4096), (700, 1800, 2048), (300, 1040, 8192)])
+@pytest.mark.parametrize("kernel", [bs.PATH_WIDE, bs.PATH_WIDE_SINGLE])
+def test_fp8_stream_k_matches_the_oracle_and_is_deterministic(M, N, K, kernel, path, no_stream_k):
+    path(kernel)
+    assert _sk_tiles(bs.OP_FP8_BLOCKWISE, M, 1, N, K) > 0
+    d = wl.fp8_blockwise_inputs(M, N, K, seed=960 + M)
+    y, S = oracle_fp8(d)
+    for out_dtype in (torch.bfloat16, torch.float32):
+        first = fp8_run(d, out_dtype)
+        fp8_check(first, y, S, out_dtype, f"fp8 stream-K {M}x{N}x{K} kernel={kernel}")
+        assert torch.equal(first, fp8_run(d, out_dtype)), "split tiles are summed in a fixed order"
+    no_stream_k()
+    fp8_check(fp8_run(d, torch.float32), y, S, torch.float32, "fp8 without the split")
+
+
+@pytest.mark.parametrize("M,N,K", [(1024, 1024, 4096), (300, 1040, 8192)])
+def test_fp8_rowwise_stream_k(M, N, K):
+    assert _sk_tiles(bs.OP_FP8_ROWWISE, M, 1, N, K) > 0
+    d = wl.fp8_rowwise_inputs(M, N, K, seed=970 + M)
+    for out_dtype in (torch.bfloat16, torch.float32):
+        y, S = oracle_rowwise(d, True)
+        fp8_check(rowwise_run(d, out_dtype, True), y, S, out_dtype, f"fp8 rowwise stream-K {M}x{N}x{K}")
+    y, S = oracle_rowwise(d, True)
+    s_r = float(np.float32(300.0 / float(np.abs(y).max())))
+    e4m3_check(rowwise_run(d, torch.float8_e4m3fn, True, scale_result=s_r), y, S, s_r, "rowwise e4m3 stream-K")
+
+
+@pytest.mark.parametrize("M,G,N,K", [(1024, 2, 1024, 4096), (300, 3, 520, 4096)])
+@pytest.mark.parametrize("kernel", [bs.PATH_WIDE, bs.PATH_WIDE_PROMOTE])
+def test_bmm_stream_k(M, G, N, K, kernel, path):
+    path(kernel)
+    assert _sk_tiles(bs.OP_BMM, M, G, N, K) > 0
+    d = wl.bmm_inputs(M, G, N, K, seed=980 + M + G)
+    y, S = oracle.bmm_blockscale(d["x"], d["w"], d["x_scale"], d["w_scale"])
+    out = bmm_run(d, torch.float32)
+    fp8_check(out, y, S, torch.float32, f"bmm stream-K {M}x{G}x{N}x{K} kernel={kernel}")
+    assert torch.equal(out, bmm_run(d, torch.float32))
+
+
+def test_int8_stream_k_equals_the_unsplit_plan(no_stream_k):
+    d = wl.int8_inputs(4096, 4096, 4096, seed=990)
+    assert _sk_tiles(bs.OP_INT_SCALED_MM, 4096, 1, 4096, 4096) > 0
+    a = int8_run(d, torch.int32)
+    no_stream_k()
+    assert torch.equal(a, int8_run(d, torch.int32))
+
+
+# ---------------------------------------------------------------------------
+# edges of the input domain: extreme e8m0 bytes, the int32 limit, zero and
+# subnormal fp32 block scales
+# ---------------------------------------------------------------------------
+# e8m0 bytes planted per batch g (the w bytes are shared by every row, so each
+# batch holds one regime of w; the x bytes vary per row and K block):
+#   g=0: w in {0,1,2} (2^-127 .. 2^-125, byte 0 an fp32 subnormal); rows of
+#        the first half take x in {252,253,254}, so every block scale is
+#        2^-2 .. 2^2; the second half x in {126,127,128}: tiny results
+#        (2^-129 .. 2^-125 times the partials)
+#   g=1: w in {252,253,254}; x in {0,1,2} (first half) or {30,31,32}
+#   g=2: w in {126,127,128}; x drawn from {0,1,2,126,127,128,200,210,220}
+#        per block, so huge and tiny blocks meet in one sum
+#   g=3: w and x in {0,1,2}: every product underflows fp32 (2^-254 .. 2^-250)
+#   g=4: w in {107,108,109}, x in {0,1,2}: block scales 2^-147 .. 2^-143,
+#        results in the fp32 subnormal range
+E8M0_EDGE_W = ((0, 1, 2), (252, 253, 254), (126, 127, 128), (0, 1, 2), (107, 108, 109))
+E8M0_EDGE_X = (((252, 253, 254), (126, 127, 128)), ((0, 1, 2), (30, 31, 32)),
+               ((0, 1, 2, 126, 127, 128, 200, 210, 220),) * 2, ((0, 1, 2),) * 2, ((0, 1, 2),) * 2)
+
+
+def _bmm_edge_inputs(M, N, K, seed):
+    G = len(E8M0_EDGE_W)
+    d = wl.bmm_inputs(M, G, N, K, seed=seed)
+    gen = torch.Generator().manual_seed(seed)
+    xs, ws = d["x_scale"].clone(), d["w_scale"].clone()
+    for g in range(G):
+        wc = torch.tensor(E8M0_EDGE_W[g], dtype=torch.uint8)
+        ws[g] = wc[torch.randint(0, len(wc), tuple(ws[g].shape), generator=gen)]
+        for half, rows in enumerate((slice(0, M // 2), slice(M // 2, M))):
+            xc = torch.tensor(E8M0_EDGE_X[g][half], dtype=torch.uint8)
+            sub = xs[rows, g]
+            xs[rows, g] = xc[torch.randint(0, len(xc), tuple(sub.shape), generator=gen)]
+    d["x_scale"], d["w_scale"] = xs, ws
+    return d
+
+
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("kernel", [bs.PATH_WIDE, bs.PATH_WIDE_PROMOTE, bs.PATH_WIDE_SINGLE, bs.PATH_SKINNY])
+def test_bmm_extreme_e8m0_bytes(kernel, out_dtype, path):
+    """Scale bytes 0, 1, 2 and 252, 253, 254 (2^-127 .. 2^127) on every BMM path:
+    the tensor core's block-scaled MMA decodes the byte itself, the promotion
+    paths decode it in software; both must meet the bound, and products that
+    underflow fp32 must give zero, not NaN."""
+    M, N, K = 256, 384, 1024
+    d = _bmm_edge_inputs(M, N, K, seed=901)
+    y, S = oracle.bmm_blockscale(d["x"], d["w"], d["x_scale"], d["w_scale"])
+    assert np.all(np.isfinite(y)) and float(np.abs(y).max()) < 2.0 ** 120  # finite in fp32 by construction
+    path(kernel)
+    fp8_check(bmm_run(d, out_dtype), y, S, out_dtype, f"bmm extreme e8m0 kernel={kernel}")
+
+
+def test_int8_at_the_int32_limit():
+    """K = 131071 (the largest the header allows, lda = 131072) with -128 / 127
+    patterns: the accumulator reaches 16384 * 131071 = 2^31 - 16383 and
+    -16256 * 131071; int32, fp32 and bf16 outputs bit-exact on both wide
+    kernel variants."""
+    M, N, K = 128, 128, 131071
+    gen = torch.Generator().manual_seed(905)
+    vals = torch.tensor([-128, 127, -127, 0, 1, -1], dtype=torch.int8)
+    A = torch.zeros(M, K + 1, dtype=torch.int8)
+    Bt = torch.zeros(N, K + 1, dtype=torch.int8)
+    A[:, :K] = vals[torch.randint(0, len(vals), (M, K), generator=gen)]
+    Bt[:, :K] = vals[torch.randint(0, len(vals), (N, K), generator=gen)]
+    A[0, :K], A[1, :K], A[2, :K] = -128, 127, -128
+    Bt[0, :K], Bt[1, :K] = -128, 127
+    A[2, 1:K:2] = 127           # alternating row
+    Bt[2, :K] = -128
+    Bt[3, :K] = A[3, :K]         # a column equal to a random row: a large positive sum
+    d = {"A": A[:, :K], "B_t": Bt[:, :K], "s_a": wl.log_uniform(M, 1e-3, 1e-1, 906),
+         "s_b": wl.log_uniform(N, 1e-3, 1e-1, 907)}
+    acc, _, _ = oracle.int_scaled_mm(d["A"], d["B_t"], None, None)
+    assert acc[0, 0] == 16384 * K and acc[0, 1] == -16256 * K and acc[1, 0] == -16256 * K
+    for kernel in (bs.PATH_WIDE, bs.PATH_WIDE_SINGLE):
+        bs.set_path_override(kernel)
+        try:
+            Ad = A.to(DEV)[:, :K]
+            Bd = Bt.to(DEV)[:, :K].t()
+            assert Ad.stride(0) == K + 1
+            for out_dtype in (torch.int32, torch.float32, torch.bfloat16):
+                got = bs.int_scaled_mm(Ad, Bd, d["s_a"].to(DEV), d["s_b"].to(DEV), out_dtype=out_dtype)
+                acc_r, y_r, bf_r = oracle.int_scaled_mm(d["A"], d["B_t"], d["s_a"], d["s_b"])
+                if out_dtype == torch.int32:
+                    np.testing.assert_array_equal(got.cpu().numpy(), acc_r)
+                elif out_dtype == torch.float32:
+                    np.testing.assert_array_equal(f32_bits(got), y_r.view(np.uint32))
+                else:
+                    np.testing.assert_array_equal(bf16_bits(got), bf_r)
+        finally:
+            bs.set_path_override(bs.PATH_AUTO)
+
+
+def _blockwise_zero_and_subnormal_scales(M, N, K, seed):
+    """Block scales with zeros and fp32 subnormals planted:
+      scale_a row 3 all zero, row 4 zero at kb=2, rows 5..8 subnormal
+      (2^-149, 1e-40, 2^-130, 3e-39) in every block, row 9 subnormal in the
+      even blocks only; scale_b block (1, 0) zero, (2, 2) subnormal (1e-39);
+      column block 1 of scale_b scaled by 2^24 so the subnormal scale_a
+      entries meet a partner that lifts their product into the normal range."""
+    d = wl.fp8_blockwise_inputs(M, N, K, seed=seed)
+    sa, sb = d["scale_a"].clone(), d["scale_b"].clone()
+    sa[3] = 0.0
+    sa[4, 2] = 0.0
+    for r, v in zip(range(5, 9), (2.0 ** -149, 1e-40, 2.0 ** -130, 3e-39)):
+        sa[r] = v
+    sa[9, 0::2] = 1e-40
+    sb[1, 0] = 0.0
+    sb[2, 2] = 1e-39
+    sb[:, 1] *= 2.0 ** 24
+    d["scale_a"], d["scale_b"] = sa, sb
+    return d
+
+
+@pytest.mark.parametrize("kernel", [bs.PATH_WIDE, bs.PATH_WIDE_SINGLE, bs.PATH_SKINNY])
+def test_fp8_zero_and_subnormal_block_scales(kernel, path):
+    """Zero and subnormal fp32 entries in scale_a and scale_b.  bf16 outputs
+    meet the bound everywhere (its ulp floor covers the tiny results).  The
+    kernels form each block-scale product scale_a * scale_b in fp32, where a
+    subnormal product carries an absolute error of up to 2^-150; that is
+    within 1e-3 of the product when it is at least 2^-140.  fp32 outputs are
+    checked wherever every block's product is zero or at least 2^-140 (the
+    domain the header states for fp32 outputs)."""
+    M, N, K = 256, 384, 1024
+    d = _blockwise_zero_and_subnormal_scales(M, N, K, seed=910)
+    y, S = oracle_fp8(d)
+    assert np.all(y[3] == 0.0)
+    path(kernel)
+    fp8_check(fp8_run(d, torch.bfloat16), y, S, torch.bfloat16, f"zero/subnormal scales bf16 kernel={kernel}")
+    g = fp8_run(d, torch.float32)
+    sa = d["scale_a"].double().numpy()
+    sb = d["scale_b"].double().numpy()
+    prod = np.abs(sa[:, :, None] * sb[None, :, :])                 # [M, KB, NB], exact in fp64
+    ok_blk = (prod == 0.0) | (prod >= 2.0 ** -140)
+    ok = np.repeat(ok_blk.all(axis=1), 128, axis=1)[:, :N]         # [M, N]: every block of (m, n) is safe
+    assert ok[:10].sum() > 0 and (~ok).sum() > 0
+    gf = to_f64(g)
+    assert np.all(np.isfinite(gf))
+    rows, cols = np.nonzero(ok)
+    sub = torch.tensor(gf[rows, cols])
+    fp8_check(sub, y[rows, cols], S[rows, cols], torch.float32, f"zero/subnormal scales f32 kernel={kernel}")

@@ -642,3 +642,63 @@ def test_backward_gemms_of_the_quantised_operands_approximate_the_exact_gradient
     for got, want in ((dW, dyd.T @ xd), (dx, dyd @ Wd)):
         assert got.shape == want.shape
         assert np.linalg.norm(got - want) / np.linalg.norm(want) < 0.06
+
+
+# ---------------------------------------------------------------------------
+# forward-orientation 128x128 quantiser (the weight operand B_t [N, K])
+# ---------------------------------------------------------------------------
+def _torch_quantize_blocks(x):
+    """torch's own cast of x over its 128x128 block's scale (amax / 448, 1 if that is 0)."""
+    R, C = x.shape
+    RB, CB = -(-R // 128), -(-C // 128)
+    xp = torch.zeros(RB * 128, CB * 128)
+    xp[:R, :C] = x
+    amax = xp.view(RB, 128, CB, 128).abs().amax(dim=(1, 3))
+    s = amax / 448.0
+    s[s == 0] = 1.0
+    full = s.repeat_interleave(128, 0).repeat_interleave(128, 1)
+    q = (xp / full).clamp(-448, 448).to(torch.float8_e4m3fn).view(torch.uint8)
+    return q[:R, :C].numpy(), s.numpy()
+
+
+@pytest.mark.parametrize("R,C", [(128, 128), (300, 260), (5, 700), (1000, 1), (256, 384)])
+def test_quantize_128x128_matches_torch_cast_of_x_over_block_scale(R, C):
+    x = wl.normal_with_outliers((R, C), 9100 + R + C)
+    q, s = oracle.quantize_128x128(x, 0)
+    rq, rs = _torch_quantize_blocks(x)
+    assert q.shape == (R, C) and s.shape == (-(-R // 128), -(-C // 128))
+    assert np.array_equal(s, rs) and np.array_equal(q, rq)
+
+
+@pytest.mark.parametrize("fmt", [0, 1])
+def test_quantize_128x128_is_the_transposed_quantiser_transposed_back(fmt):
+    x = wl.normal_with_outliers((300, 520), 9200 + fmt)
+    q, s = oracle.quantize_128x128(x, fmt)
+    qt, st = oracle.quantize_t(x, 1, fmt)  # codes [C, R], block scales [RB, CB]
+    assert np.array_equal(q, qt.T) and np.array_equal(s, st)
+
+
+def test_quantize_128x128_orientation_and_block_isolation():
+    x = torch.zeros(256, 384)
+    x[5, 200] = 7.0     # block (0, 1): rows 0..127, columns 128..255
+    x[130, 3] = -2.0    # block (1, 0)
+    q, s = oracle.quantize_128x128(x, 0)
+    assert s[0, 1] == np.float32(7.0) / np.float32(448.0) and s[1, 0] == np.float32(2.0) / np.float32(448.0)
+    assert s[0, 0] == 1.0 and s[1, 1] == 1.0 and s[0, 2] == 1.0 and s[1, 2] == 1.0
+    assert q[5, 200] == 0x7E and q[130, 3] == 0xFE      # +-448
+    assert int(np.count_nonzero(q)) == 2
+    # e8m0: the byte of the block holding 7.0 is ceil(log2(7 / 448)) + 127 = -6 + 127
+    _, b = oracle.quantize_128x128(x, 1)
+    assert b[0, 1] == 121 and b[0, 0] == 127
+
+
+def test_quantize_128x128_weight_in_the_forward_gemm_approximates_the_exact_product():
+    M, N, K = 200, 384, 640
+    x = wl.normal_with_outliers((M, K), 9300)
+    W = wl.normal_with_outliers((N, K), 9301)
+    a, sa = oracle.quantize_1x128(x, 0)
+    b, sbT = oracle.quantize_128x128(W, 0)  # B_t [N, K], scales [N/128, K/128]
+    y, _ = oracle.fp8_blockwise(a, b, sa, sbT.T)
+    exact = x.double().numpy() @ W.double().numpy().T
+    rel = np.linalg.norm(y - exact) / np.linalg.norm(exact)
+    assert rel < 0.06, rel

@@ -45,6 +45,7 @@ GROUP = 128  # quantisation group / block edge along K (and N for weights)
 class Workload:
     name: str
     # "fp8_blockwise" | "int_scaled_mm" | "bmm_a8w8_blockscale" | "fp8_rowwise" | "quantize_1x128" | "quantize_t"
+    # | "quantize_128x128"
     op: str
     M: int
     N: int
@@ -71,6 +72,9 @@ WORKLOADS = {
                                               extra={"group": "128x1"}),
     "quant_t_128x128_16640x8192_bf16": Workload("quant_t_128x128_16640x8192_bf16", "quantize_t", 16640, 0, 8192,
                                                 seed=8, extra={"group": "128x128"}),
+    # the weight W [5120, 8192] of the same layer, bf16, quantised to the forward GEMM's B_t in 128x128 blocks
+    "quant_128x128_5120x8192_bf16": Workload("quant_128x128_5120x8192_bf16", "quantize_128x128", 5120, 0, 8192,
+                                             seed=9),
 }
 BMM_M_SWEEP = (1, 16, 128, 1024, 16384)
 BMM_G = (8, 2)
@@ -265,6 +269,6 @@ def workload_inputs(w: Workload, sweep: int = 0, batch_first: bool = False):
         return int8_inputs(w.M, w.N, w.K, base)
     if w.op == "fp8_rowwise":
         return fp8_rowwise_inputs(w.M, w.N, w.K, base)
-    if w.op in ("quantize_1x128", "quantize_t"):
+    if w.op in ("quantize_1x128", "quantize_t", "quantize_128x128"):
         return {"x": normal_with_outliers((w.M, w.K), base + 10 * 7).to(torch.bfloat16)}
     return bmm_inputs(w.M, w.G, w.N, w.K, base, batch_first=batch_first)
