@@ -71,6 +71,7 @@ def tensor_peak(peaks: dict, timed_s: float):
 KERNEL_SOURCES = {
     "wide": ["sm100.cuh", "tile_order.h", "wide_kernel.cuh", "skinny_kernel.cuh", "kernels_wide.cu", "launch.h"],
     "skinny": ["sm100.cuh", "tile_order.h", "wide_kernel.cuh", "skinny_kernel.cuh", "kernels_skinny.cu", "launch.h"],
+    "gemv": ["sm100.cuh", "tile_order.h", "wide_kernel.cuh", "skinny_kernel.cuh", "kernels_gemv.cu", "launch.h"],
     "quantize": ["group_quant.cuh", "quantize.h", "kernels_quantize.cu"],
     "quantize_t": ["group_quant.cuh", "quantize.h", "kernels_quantize_t.cu"],
     "quantize_blocks": ["group_quant.cuh", "quantize.h", "kernels_quantize_blocks.cu"],
@@ -427,12 +428,12 @@ def main():
     ap.add_argument("--shape", default=None,
                     help="ad-hoc problem 'M,N,K' (or 'M,G,N,K' for --op bmm) instead of a named workload")
     ap.add_argument("--op", default="fp8", choices=["fp8", "int8", "bmm"], help="operation for --shape")
-    ap.add_argument("--path", default="auto", choices=["auto", "wide", "skinny", "wide1", "promote"],
+    ap.add_argument("--path", default="auto", choices=["auto", "wide", "skinny", "wide1", "promote", "gemv"],
                     help="force a kernel family (wide = CTA-pair persistent, wide1 = single-CTA persistent, "
                          "promote = CTA-pair persistent with e8m0 block scales promoted on the CUDA cores)")
     ap.add_argument("--splits", type=int, default=0, choices=[0, 1, 2, 4, 8],
                     help="force the skinny kernel's split-K factor (0 = the planner's choice)")
-    ap.add_argument("--stream-k", default="on", choices=["on", "off"],
+    ap.add_argument("--stream-k", default="off", choices=["on", "off"],
                     help="off: compute every tile of the wide kernel whole (no split of the last wave)")
     args = ap.parse_args()
 
@@ -481,7 +482,7 @@ def main():
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         return float(t.item())
 
-    bs.set_path_override({"auto": 0, "wide": 1, "skinny": 2, "wide1": 3, "promote": 4}[args.path])
+    bs.set_path_override({"auto": 0, "wide": 1, "skinny": 2, "wide1": 3, "promote": 4, "gemv": 5}[args.path])
     bs.set_stream_k(args.stream_k == "on")
     bs.set_split_override(args.splits)
     copies = copies_for(byts)
@@ -582,7 +583,7 @@ def main():
                      "frac": round(achieved / peak, 4), "frac_basis": "of " + peak_source,
                      "traffic": traffic,
                      "kernel": f"{w.op}_kernel" if quant else
-                               ("wide_gemm_kernel" if plan["kernel"] == 1 else "skinny_gemm_kernel"),
+                               {1: "wide_gemm_kernel", 2: "skinny_gemm_kernel", 4: "gemv_kernel"}[plan["kernel"]],
                      "peak_source": peak_source,
                      "dense_peak": dense_peak,
                      "frac_dense_peak": round(achieved / dense_peak, 4)},

@@ -208,7 +208,8 @@ bs_status bs_check_blockwise_scale_shapes(int64_t M, int64_t N, int64_t K,
 
 /* Which kernel a call would launch, for tests and benchmarks. */
 typedef struct {
-  int32_t kernel;  /* 0: none (empty problem), 1: persistent wide, 2: skinny split-K, 3: zero fill */
+  int32_t kernel;  /* 0: none (empty problem), 1: persistent wide, 2: skinny split-K, 3: zero fill,
+                      4: small-M weight stream (warp-level MMA, M <= 8) */
   int32_t tile_m;  /* rows of A (M direction) per tile */
   int32_t tile_n;  /* columns of B (N direction) per tile */
   int32_t splits;  /* K splits reduced through cluster shared memory (1 = none) */
@@ -339,7 +340,8 @@ bs_status bs_plan_for(int32_t op, int64_t M, int64_t G, int64_t N, int64_t K, in
  * tiles), 2 = skinny split-K kernel where the operation has one, 3 = persistent
  * wide kernel on single CTAs (128 x 256 tiles), 4 = as 1, but
  * bmm_a8w8_blockscale promotes every 128-deep block on the CUDA cores instead
- * of letting the tensor core apply its e8m0 scales (block-scaled MMA).
+ * of letting the tensor core apply its e8m0 scales (block-scaled MMA), 5 = the
+ * small-M weight-stream kernel (operations 1 and 3 with M <= 8).
  * Returns the previous setting. */
 int32_t bs_set_path_override(int32_t path);
 
@@ -354,8 +356,11 @@ int32_t bs_set_split_override(int32_t splits);
  * of the remaining tiles are spread evenly over all of them and the pieces of
  * a split tile meet in this workspace: fp32 (int32 for int_scaled_mm) partial
  * sums, added in a fixed order by the CTA that holds the tile's first K block,
- * so results are deterministic.  Without a registered workspace (or with
- * bs_set_stream_k(0)) every tile is computed whole.
+ * so results are deterministic.  The split is off by default (on the B200
+ * shapes measured, INT8 4096^3, FP8 1000 x 7168 x 2048 and BMMs of 1024-row
+ * batches, it was 14-35% slower than computing every tile whole: a split
+ * tile's hand-over costs more than the idle part of the last round); it runs
+ * only after bs_set_stream_k(1) and with a registered workspace.
  *
  * bs_workspace_size(num_sms): bytes needed on a GPU with num_sms SMs
  *   (num_sms * 131,104 rounded up; about 19.4 MB on a 148-SM B200).  Pure host logic.
@@ -367,8 +372,8 @@ int32_t bs_set_split_override(int32_t splits);
  *   buffer, so they must not run concurrently on different streams of the
  *   device (as with a library handle's workspace).  Returns BS_ERR_WORKSPACE
  *   if `bytes` < bs_workspace_size(device SMs), BS_ERR_ALIGNMENT if misaligned.
- * bs_set_stream_k(enable): 0 disables the split process-wide (for testing);
- *   returns the previous setting.
+ * bs_set_stream_k(enable): 1 enables the split process-wide, 0 (the
+ *   default) disables it; returns the previous setting.
  */
 size_t bs_workspace_size(int32_t num_sms);
 bs_status bs_set_workspace(void* workspace, size_t bytes);

@@ -32,7 +32,7 @@ BS_OK, BS_ERR_NULL, BS_ERR_SHAPE, BS_ERR_LAYOUT, BS_ERR_ALIGNMENT = 0, 1, 2, 3, 
 BS_ERR_DTYPE, BS_ERR_DEVICE, BS_ERR_CUDA, BS_ERR_TIMEOUT, BS_ERR_WORKSPACE = 5, 6, 7, 8, 9
 BS_OUT_BF16, BS_OUT_F32, BS_OUT_I32, BS_OUT_E4M3 = 0, 1, 2, 3
 
-PATH_AUTO, PATH_WIDE, PATH_SKINNY, PATH_WIDE_SINGLE, PATH_WIDE_PROMOTE = 0, 1, 2, 3, 4
+PATH_AUTO, PATH_WIDE, PATH_SKINNY, PATH_WIDE_SINGLE, PATH_WIDE_PROMOTE, PATH_GEMV = 0, 1, 2, 3, 4, 5
 
 _OUT_CODE = {torch.bfloat16: BS_OUT_BF16, torch.float32: BS_OUT_F32, torch.int32: BS_OUT_I32,
              torch.float8_e4m3fn: BS_OUT_E4M3}
@@ -123,6 +123,7 @@ def status_string(status: int) -> str:
 
 
 _workspaces = {}  # device index -> the zero-filled stream-K workspace registered with the library
+_stream_k_on = False  # mirrors bs_set_stream_k: a workspace is registered only while the split is enabled
 
 
 def _ensure_workspace(device) -> None:
@@ -132,7 +133,7 @@ def _ensure_workspace(device) -> None:
     call outside a capture."""
     idx = torch.device(device).index
     idx = torch.cuda.current_device() if idx is None else idx
-    if idx in _workspaces:
+    if not _stream_k_on or idx in _workspaces:
         return
     with torch.cuda.device(idx):
         if torch.cuda.is_current_stream_capturing():
@@ -496,8 +497,13 @@ def set_split_override(splits: int) -> int:
 
 
 def set_stream_k(enable: bool) -> bool:
-    """Enables or disables the stream-K split of the wide kernel's last wave; returns the previous setting."""
-    return bool(lib().bs_set_stream_k(1 if enable else 0))
+    """Enables or disables the stream-K split of the wide kernel's last wave (off by default: it measured
+    slower than whole tiles on every shape tried); returns the previous setting.  While enabled, the
+    first GEMM call on a device registers a workspace for it."""
+    global _stream_k_on
+    prev = bool(lib().bs_set_stream_k(1 if enable else 0))
+    _stream_k_on = bool(enable)
+    return prev
 
 
 def workspace_size(num_sms: int) -> int:

@@ -114,7 +114,7 @@ bs_status device_ctx(DeviceCtx** out) {
 // planning (pure host logic)
 // ---------------------------------------------------------------------------
 std::atomic<int32_t> g_path_override{0};
-std::atomic<int32_t> g_stream_k{1};
+std::atomic<int32_t> g_stream_k{0};  // stream-K split: off unless enabled
 std::atomic<int32_t> g_split_override{0};  // skinny kernel: forced split factor (0 = planner's choice)
 
 // Bytes of the stream-K workspace for a GPU with `sms` SMs: one partial-sum
@@ -186,6 +186,17 @@ Plan make_plan(int op, int64_t M, int64_t G, int64_t N, int64_t K, int sms, bool
   const int KB = static_cast<int>((K + 127) / 128);
   const int ov = g_path_override.load();
   const bool skinny_ok = op == 1 || op == 3;  // block-scaled FP8 only
+  // M <= kGemvMaxM: the warp-MMA weight stream (kernels_gemv.cu)
+  if (skinny_ok && M <= kGemvMaxM && (ov == 5 || ov == 0)) {
+    x.pub.kernel = 4;
+    x.pub.tile_m = 8;
+    x.pub.tile_n = 16;
+    x.pub.splits = 1;
+    x.pub.cluster = 1;
+    x.pub.ctas = static_cast<int32_t>(((N + 15) / 16) * G);
+    x.pub.launches = 1;
+    return x;
+  }
   const bool skinny = skinny_ok && (ov == 2 || (ov == 0 && M <= kSkinnyMaxM));
   if (skinny) {
     const long long n_tiles = (N + 127) / 128;
@@ -211,6 +222,11 @@ Plan make_plan(int op, int64_t M, int64_t G, int64_t N, int64_t K, int sms, bool
     const int max_s = skinny_ctas_per_sm(bmt) > 1 ? 8 : 4;
     int S = 1;
     while (S < max_s && 2 * S <= KB && units * 2 * S <= slots) S *= 2;
+    // With 32-row or wider activation tiles, a CTA holding fewer than 8 K
+    // blocks spends more on its fixed costs than the extra CTAs gain, while
+    // the halved grid still has half as many CTAs as SMs (measured: M=32,
+    // N=7168, K=2048 takes 6.7 us split 2 ways against 7.2 us 4 ways).
+    while (bmt >= 32 && S > 1 && KB / S < 8 && units * (S / 2) >= sm_count / 2) S /= 2;
     const int forced = g_split_override.load();
     if (forced == 1 || forced == 2 || forced == 4 || forced == 8) S = forced <= KB ? forced : S;
     x.pub.kernel = 2;
@@ -328,6 +344,21 @@ bs_status run_fp8(const Fp8Problem& q, GemmArgs args, cudaStream_t stream, Devic
   if (pl.pub.kernel == 3)
     return check_launch(launch_fill_zero(q.out, out_size(q.out_dtype), q.M, q.N, q.o_rs, q.G, q.o_bs, stream),
                         "zero-fill launch");
+  if (pl.pub.kernel == 4) {
+    args.err = dc->err;
+    GemvProblem gq;
+    gq.a = q.a;
+    gq.a_sm = q.a_rs;
+    gq.a_sg = q.G > 1 ? q.a_bs : 0;
+    gq.b = q.b;
+    gq.b_sn = q.b_rs;
+    gq.b_sg = q.G > 1 ? q.b_bs : 0;
+    gq.out = q.out;
+    gq.o_sm = q.o_rs;
+    gq.o_sg = q.G > 1 ? q.o_bs : 0;
+    gq.sms = dc->sms;
+    return check_launch(launch_gemv(q.mode, out_kind(q.out_dtype), gq, args, stream), "small-M kernel launch");
+  }
   args.err = dc->err;
   CUtensorMap ta, tb, td;
   const uint64_t a_bs = q.G > 1 ? static_cast<uint64_t>(q.a_bs) : static_cast<uint64_t>(q.a_rs) * q.M;

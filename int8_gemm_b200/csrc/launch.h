@@ -26,6 +26,23 @@ cudaError_t launch_wide(Mode mode, OutKind out, int cta_group, const CUtensorMap
 cudaError_t launch_skinny(Mode mode, OutKind out, int bmt, const CUtensorMap& a, const CUtensorMap& b,
                           const GemmArgs& args, const SkinnyOut& o, int n_tiles, int m_tiles, cudaStream_t stream);
 
+// Small-M kernel (kernels_gemv.cu): M <= kGemvMaxM activation rows, FP8
+// modes kFp8F32Scale and kFp8E8M0.  Activation (m, g, k) at
+// a[m * a_sm + g * a_sg + k], weight (g, n, k) at b[g * b_sg + n * b_sn + k],
+// output (m, g, n) at out[m * o_sm + g * o_sg + n] (byte strides for a and b,
+// element strides for out).  Grid: ceil(N / 16) x G CTAs of 8 warps.
+constexpr int kGemvMaxM = 8;
+struct GemvProblem {
+  const void* a;
+  long long a_sm, a_sg;
+  const void* b;
+  long long b_sn, b_sg;
+  void* out;
+  long long o_sm, o_sg;
+  int sms;  // SMs of the device (grid size choice)
+};
+cudaError_t launch_gemv(Mode mode, OutKind out, const GemvProblem& q, const GemmArgs& args, cudaStream_t stream);
+
 // Fill of `batches` matrices [rows, cols] (row stride ld, batch stride
 // bstride, elements of `elem_size` bytes: bf16, fp32, or 1 = e4m3) with zero,
 // or with bias[col] (fp32 [cols]) when bias is given; e4m3 elements take the

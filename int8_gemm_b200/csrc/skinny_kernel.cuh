@@ -319,15 +319,17 @@ __global__ void __launch_bounds__(SkinnyCfg<BMT>::THREADS, SkinnyCfg<BMT>::CTAS_
     // buffers, so the two streams are independent; each thread's commits
     // track its own MMAs.  (One thread issuing everything spends most of a
     // K block's time in the issue of its four MMAs.)
-    if (lane == 0) {
+    // Each issuing warp runs its loop as a whole (warp-uniform waits and
+    // descriptor arithmetic); one elected lane issues the MMAs and commits.
+    {
       const int issuer = warp == 3 ? 1 : 0;
       bool ok = true;
       for (int i = issuer; i < nkb; i += 2) {
         const int stage = i % STAGES, buf = i % NBUF;
         const uint32_t phase = static_cast<uint32_t>(i / STAGES) & 1u;
         const uint32_t bphase = static_cast<uint32_t>(i / NBUF) & 1u;
-        if (!wait_bounded(&sm.acc_empty[buf], bphase ^ 1u, abort, p.err, kErrTimeout | kRoleMma | kWaitAccEmpty) ||
-            !wait_bounded(&sm.full[stage], phase, abort, p.err, kErrTimeout | kRoleMma | kWaitStageFull)) {
+        if (!warp_wait(&sm.acc_empty[buf], bphase ^ 1u, abort, p.err, kErrTimeout | kRoleMma | kWaitAccEmpty) ||
+            !warp_wait(&sm.full[stage], phase, abort, p.err, kErrTimeout | kRoleMma | kWaitStageFull)) {
           ok = false;
           break;
         }
@@ -335,13 +337,17 @@ __global__ void __launch_bounds__(SkinnyCfg<BMT>::THREADS, SkinnyCfg<BMT>::CTAS_
         const uint32_t d = tmem + static_cast<uint32_t>(buf) * ACC_COLS;
         const uint64_t ad = sdesc_k_sw128(smem_u32(sm.b[stage]));
         const uint64_t bd = sdesc_k_sw128(smem_u32(sm.a[stage]));
+        if (elect_one()) {
 #pragma unroll
-        for (int k = 0; k < BK / 32; ++k) mma_f8f6f4(d, ad + 2 * k, bd + 2 * k, IDESC, k > 0 ? 1u : 0u);
-        mma_commit(&sm.empty[stage]);
-        mma_commit(&sm.acc_full[buf]);
+          for (int k = 0; k < BK / 32; ++k) mma_f8f6f4(d, ad + 2 * k, bd + 2 * k, IDESC, k > 0 ? 1u : 0u);
+          mma_commit(&sm.empty[stage]);
+          mma_commit(&sm.acc_full[buf]);
+        }
+        __syncwarp();
       }
-      if (!ok) {  // wait until this thread's MMAs have finished with TMEM and shared memory
-        mma_commit(&sm.drain[issuer]);
+      if (!ok) {  // wait until this warp's MMAs have finished with TMEM and shared memory
+        if (elect_one()) mma_commit(&sm.drain[issuer]);
+        __syncwarp();
         volatile int never = 0;
         wait_bounded(&sm.drain[issuer], 0, &never, nullptr, 0);
       }

@@ -140,6 +140,7 @@ struct WideSmem {
   uint64_t sc_full[kScaleRing];
   uint64_t sc_empty[kScaleRing];
   uint64_t drain;
+  uint64_t part_bar[8];  // consumer warps: a stream-K partial copied into the idle operand ring
   uint32_t tmem_base;
   int abort;
   long long sk_pos[8];  // consumer warps: position in the stream-K range (kept out of registers)
@@ -229,9 +230,10 @@ __device__ __forceinline__ void promote32(float* acc, float s, const uint32_t (&
   }
 }
 
+template <bool CLUSTER = false>
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort, uint32_t* err,
                                           uint32_t code) {
-  const bool ok = wait_bounded(bar, parity, abort, err, code);
+  const bool ok = wait_bounded<CLUSTER>(bar, parity, abort, err, code);
   return __all_sync(0xffffffffu, ok);
 }
 
@@ -304,6 +306,7 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(&sm.sc_empty[i], MX ? 1 : CONSUMER_WARPS);
     }
     mbar_init(&sm.drain, 1);
+    for (int i = 0; i < CONSUMER_WARPS; ++i) mbar_init(&sm.part_bar[i], 1);
     sm.abort = 0;
     fence_mbar_init();
   }
@@ -389,7 +392,10 @@ __global__ void __launch_bounds__(384, 1)
       __syncwarp();
     } else if (warp == 1) {
       // ---------------------------------------------------------- MMA issuer (leader CTA)
-      if (lane == 0 && leader) {
+      // The whole warp runs the loop, so its waits, fences and descriptor
+      // arithmetic are warp-uniform; one elected lane (always the same) issues
+      // the copies, MMAs and the commits that track them.
+      if (leader) {
         int stage = 0, buf = 0;
         uint32_t phase = 0, bphase = 0;
         uint32_t sfc = 0;  // kFp8Mx: scale-factor slots consumed (ring position)
@@ -402,19 +408,19 @@ __global__ void __launch_bounds__(384, 1)
             // FP8: every K block starts a fresh partial in the next buffer;
             // INT8: the work item's accumulator is claimed once, at its first K block
             if (!FULL_K || first) {
-              if (!wait_bounded(&sm.acc_empty[buf], bphase ^ 1u, abort, p.err, kErrTimeout | kRoleMma | kWaitAccEmpty)) {
+              if (!warp_wait(&sm.acc_empty[buf], bphase ^ 1u, abort, p.err, kErrTimeout | kRoleMma | kWaitAccEmpty)) {
                 ok = false;
                 break;
               }
               // kFp8Mx: the previous tile, in the other buffer, has also read
               // the columns the two buffers share
-              if (MX && !wait_bounded(&sm.ovl_empty[buf ^ 1], buf == 1 ? bphase : (bphase ^ 1u), abort, p.err,
-                                      kErrTimeout | kRoleMma | kWaitAccEmpty)) {
+              if (MX && !warp_wait(&sm.ovl_empty[buf ^ 1], buf == 1 ? bphase : (bphase ^ 1u), abort, p.err,
+                                   kErrTimeout | kRoleMma | kWaitAccEmpty)) {
                 ok = false;
                 break;
               }
             }
-            if (!wait_bounded(&sm.full[stage], phase, abort, p.err, kErrTimeout | kRoleMma | kWaitStageFull)) {
+            if (!warp_wait(&sm.full[stage], phase, abort, p.err, kErrTimeout | kRoleMma | kWaitStageFull)) {
               ok = false;
               break;
             }
@@ -422,8 +428,8 @@ __global__ void __launch_bounds__(384, 1)
             // kFp8Mx: this K block's byte in its slot (slots start at the item's first K block)
             const uint32_t sf_id = static_cast<uint32_t>((kb - w.kb0) & 3);
             if constexpr (MX) {  // both CTAs' scale factors of K blocks kb..kb+3 are in shared memory
-              if (sf_id == 0 && !wait_bounded<true>(&sm.sc_full[sslot], (sfc / kSfRing) & 1u, abort, p.err,
-                                                    kErrTimeout | kRoleMma | kWaitScaleFull)) {
+              if (sf_id == 0 && !warp_wait<true>(&sm.sc_full[sslot], (sfc / kSfRing) & 1u, abort, p.err,
+                                                 kErrTimeout | kRoleMma | kWaitScaleFull)) {
                 ok = false;
                 break;
               }
@@ -432,6 +438,8 @@ __global__ void __launch_bounds__(384, 1)
             const uint32_t d = tmem + acc_col(buf);
             const uint64_t ad = sdesc_k_sw128(smem_u32(sm.a[stage]));
             const uint64_t bd = sdesc_k_sw128(smem_u32(sm.b[stage]));
+            const bool slot_done = MX && (sf_id == 3 || last);  // kFp8Mx: the slot's last K block
+            if (elect_one()) {
             if constexpr (MX) {
               if (sf_id == 0) {
                 // scale factors of four K blocks to TMEM; issued by this
@@ -468,17 +476,15 @@ __global__ void __launch_bounds__(384, 1)
             // tile's last K block also commits the accumulator barrier.
             if constexpr (CG == 2) {
               mma_commit_pair_mc(&sm.empty[stage], 0x3);
-              if constexpr (MX) {  // after the slot's last K block: free it in both CTAs
-                if (sf_id == 3 || last) {
-                  mma_commit_pair_mc(&sm.sc_empty[sslot], 0x3);
-                  ++sfc;
-                }
-              }
+              if (slot_done) mma_commit_pair_mc(&sm.sc_empty[sslot], 0x3);  // free it in both CTAs
               if (FULL_K && last) mma_commit_pair_mc(&sm.acc_full[buf], 0x3);
             } else {
               mma_commit(&sm.empty[stage]);
               if (FULL_K && last) mma_commit(&sm.acc_full[buf]);
             }
+            }
+            __syncwarp();
+            if (slot_done) ++sfc;
             if (!FULL_K || last) {
               if (++buf == NACC) {
                 buf = 0;
@@ -492,11 +498,14 @@ __global__ void __launch_bounds__(384, 1)
           }
         }
         if (!ok) {  // wait until every MMA already issued has finished with TMEM and smem
-          if constexpr (CG == 2) {
-            mma_commit_pair(&sm.drain);
-          } else {
-            mma_commit(&sm.drain);
+          if (elect_one()) {
+            if constexpr (CG == 2) {
+              mma_commit_pair(&sm.drain);
+            } else {
+              mma_commit(&sm.drain);
+            }
           }
+          __syncwarp();
           volatile int never = 0;
           wait_bounded(&sm.drain, 0, &never, nullptr, 0);
         }
@@ -634,6 +643,21 @@ __global__ void __launch_bounds__(384, 1)
     auto has_range = [&](int u) {
       return sk_range_begin(p.sk_iters, u, units) != sk_range_begin(p.sk_iters, u + 1, units);
     };
+    // The head's copy of giver u's partial (this warp's 16 KB piece of the
+    // slot) into this warp's share of the operand ring -- idle once the head
+    // item, the unit's last, has finished its MMAs -- with one bulk copy; the
+    // use-th copy of this warp waits for mbarrier phase use & 1.
+    uint4* const part_smem =
+        reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(&sm.a[0][0]) + cw * (STAGES * (A_BYTES + B_BYTES) / 8));
+    auto fetch_partial = [&](int u, uint32_t use) -> bool {
+      if (lane == 0) {
+        fence_proxy_async_smem();    // this warp's reads of the previous piece before the copy overwrites it
+        fence_proxy_async_global();  // the giver's stores, seen through its flag, before the async-proxy copy
+        mbar_arrive_expect_tx(&sm.part_bar[cw], 128 * 32 * 4);
+        bulk_load_g2s(part_smem, slot_piece(u), 128 * 32 * 4, &sm.part_bar[cw]);
+      }
+      return warp_wait(&sm.part_bar[cw], use & 1u, abort, p.err, kErrTimeout | kRoleConsumer | kWaitPartial);
+    };
     // The item's stream-K role: a whole tile; a later part of a split tile (a
     // giver: its partial goes to this unit's slot); or the head of a split
     // tile, which adds the partials of units c_lo..c_hi, in that order, to its
@@ -711,20 +735,22 @@ __global__ void __launch_bounds__(384, 1)
         }
         int c_lo = 0, c_hi = -1;
         if (!whole) givers_of(w, c_lo, c_hi);
+        uint32_t uses = 0;
         for (int u = c_lo; u <= c_hi; ++u) {
           if (!has_range(u)) continue;
-          if (!wait_flag_bounded(slot_flag(u), abort, p.err, kErrTimeout | kRoleConsumer | kWaitPartial)) {
+          if (!wait_flag_bounded(slot_flag(u), abort, p.err, kErrTimeout | kRoleConsumer | kWaitPartial) ||
+              !fetch_partial(u, uses++)) {
             ok = false;
             break;
           }
-          const uint4* src = slot_piece(u);
-          // four 16-byte pieces in flight at a time: the 128 accumulators
-          // leave no registers for more
+          const uint4* src = part_smem;
+          // four 16-byte pieces at a time: the 128 accumulators leave no
+          // registers for more
 #pragma unroll
           for (int q0 = 0; q0 < 32; q0 += 4) {
             uint4 v[4];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) v[q] = __ldcg(src + (q0 + q) * 32 + lane);
+            for (int q = 0; q < 4; ++q) v[q] = src[(q0 + q) * 32 + lane];
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
               acc[4 * (q0 + q)] += __uint_as_float(v[q].x);
@@ -734,7 +760,7 @@ __global__ void __launch_bounds__(384, 1)
             }
             asm volatile("" ::: "memory");  // keep the next group's loads after these adds
           }
-          __syncwarp();
+          __syncwarp();  // every lane has read the piece before the next copy overwrites it
           if (lane == 0) *slot_flag(u) = 0u;  // zero again for the next launch
         }
         if (!ok) return false;
@@ -768,12 +794,38 @@ __global__ void __launch_bounds__(384, 1)
         if (!warp_wait(&sm.acc_full[buf], bphase, abort, p.err, kErrTimeout | kRoleConsumer | kWaitAccFull))
           return false;
         tc_fence_after();
-        // the head waits for every giver's partial before it reads any
-        for (int u = c_lo; u <= c_hi; ++u) {
-          if (has_range(u) &&
-              !wait_flag_bounded(slot_flag(u), abort, p.err, kErrTimeout | kRoleConsumer | kWaitPartial)) {
-            ok = false;
-            break;
+        // the head adds every giver's partial to its accumulator in TMEM, in
+        // unit order, before the normal epilogue reads it
+        {
+          const uint32_t tb_add = tmem + t_lane + acc_col(buf) + static_cast<uint32_t>(half * 128);
+          uint32_t uses = 0;
+          for (int u = c_lo; u <= c_hi; ++u) {
+            if (!has_range(u)) continue;
+            if (!wait_flag_bounded(slot_flag(u), abort, p.err, kErrTimeout | kRoleConsumer | kWaitPartial) ||
+                !fetch_partial(u, uses++)) {
+              ok = false;
+              break;
+            }
+#pragma unroll 1
+            for (int ch = 0; ch < 4; ++ch) {
+              uint32_t r[32];
+              tmem_ld32(tb_add + 32 * ch, r);
+#pragma unroll
+              for (int q = 0; q < 8; ++q) {
+                const uint4 g4 = part_smem[(8 * ch + q) * 32 + lane];
+                const uint32_t gv[4] = {g4.x, g4.y, g4.z, g4.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  if constexpr (IS_INT8) {
+                    r[4 * q + e] += gv[e];  // exact int32 sum (two's complement)
+                  } else {
+                    r[4 * q + e] = __float_as_uint(__uint_as_float(r[4 * q + e]) + __uint_as_float(gv[e]));
+                  }
+                }
+              }
+              tmem_st32(tb_add + 32 * ch, r);
+            }
+            __syncwarp();  // every lane has read the piece before the next copy overwrites it
           }
         }
         if (!ok) return false;
@@ -818,23 +870,6 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
             for (int q = 0; q < CPC / 4; ++q) dst[q * 32] = make_uint4(r[4 * q], r[4 * q + 1], r[4 * q + 2], r[4 * q + 3]);
             continue;
-          }
-          for (int u = c_lo; u <= c_hi; ++u) {  // the head adds the givers' partials in unit order
-            if (!has_range(u)) continue;
-            const uint4* src = slot_piece(u) + (c0 / 4) * 32 + lane;
-#pragma unroll
-            for (int q = 0; q < CPC / 4; ++q) {
-              const uint4 g = __ldcg(src + q * 32);
-              const uint32_t gv[4] = {g.x, g.y, g.z, g.w};
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                if constexpr (IS_INT8) {
-                  r[4 * q + e] += gv[e];  // exact int32 sum (two's complement)
-                } else {
-                  r[4 * q + e] = __float_as_uint(__uint_as_float(r[4 * q + e]) + __uint_as_float(gv[e]));
-                }
-              }
-            }
           }
           float v[CPC];
           if constexpr (sizeof(OutT) == 4 && !std::is_same<OutT, float>::value) {

@@ -93,25 +93,57 @@ def test_plan_large_fp8_is_persistent_wide_on_cta_pairs():
     # fewer tiles than CTA pairs and too few K blocks to spread: one pair per tile
     p = bs.plan_for(bs.OP_FP8_BLOCKWISE, 300, 1, 512, 1024, 148)
     assert p["ctas"] == 2 * 2 * 2 and p["cluster"] == 2 and p["sk_tiles"] == 0
-    # a badly filled last round with enough K blocks: split over every pair
+    # a badly filled last round: whole tiles by default; with stream-K enabled, split over every pair
     p = bs.plan_for(bs.OP_FP8_BLOCKWISE, 1000, 1, 7168, 2048, 148)
-    assert p["ctas"] == 148 and p["sk_tiles"] == 112 - 74
-    prev = bs.set_stream_k(False)
+    assert p["ctas"] == 148 and p["sk_tiles"] == 0
+    prev = bs.set_stream_k(True)
     try:
-        assert bs.plan_for(bs.OP_FP8_BLOCKWISE, 1000, 1, 7168, 2048, 148)["sk_tiles"] == 0
+        p = bs.plan_for(bs.OP_FP8_BLOCKWISE, 1000, 1, 7168, 2048, 148)
+        assert p["ctas"] == 148 and p["sk_tiles"] == 112 - 74
     finally:
         bs.set_stream_k(prev)
 
 
 @pytest.mark.parametrize("M", [1, 8, 16, 17, 32, 127, 128, 129, 255, 256])
 def test_plan_skinny_split_k(M):
-    p = bs.plan_for(bs.OP_FP8_BLOCKWISE, M, 1, 7168, 2048, 148)
+    prev = bs.set_path_override(bs.PATH_SKINNY if M <= 16 else bs.PATH_AUTO)  # M <= 16 runs the small-M kernel
+    try:
+        p = bs.plan_for(bs.OP_FP8_BLOCKWISE, M, 1, 7168, 2048, 148)
+    finally:
+        bs.set_path_override(prev)
     assert p["kernel"] == 2 and p["launches"] == 1
     assert p["tile_m"] in (16, 32, 64, 128) and p["tile_m"] >= min(M, 128)
     assert p["splits"] in (1, 2, 4, 8) and p["splits"] <= 2048 // 128
     assert p["cluster"] == p["splits"]
     m_tiles = -(-M // p["tile_m"])
     assert p["ctas"] == m_tiles * (7168 // 128) * p["splits"]
+
+
+@pytest.mark.parametrize("M", [1, 5, 8])
+def test_plan_small_m_weight_stream(M):
+    # M <= 8: the warp-MMA weight stream, 16 output columns per CTA, one CTA per (16 columns, batch)
+    p = bs.plan_for(bs.OP_FP8_BLOCKWISE, M, 1, 7168, 2048, 148)
+    assert (p["kernel"], p["tile_m"], p["tile_n"], p["ctas"], p["cluster"]) == (4, 8, 16, 448, 1)
+    b = bs.plan_for(bs.OP_BMM, M, 8, 1000, 4096, 148)
+    assert b["kernel"] == 4 and b["ctas"] == 63 * 8
+    assert bs.plan_for(bs.OP_INT_SCALED_MM, M, 1, 7168, 2048, 148)["kernel"] == 1  # no small-M INT8 kernel
+    prev = bs.set_path_override(bs.PATH_GEMV)
+    try:
+        assert bs.plan_for(bs.OP_FP8_BLOCKWISE, M, 1, 256, 128, 148)["kernel"] == 4
+    finally:
+        bs.set_path_override(prev)
+
+
+@pytest.mark.parametrize("M", [9, 16, 17])
+def test_plan_small_m_beyond_weight_stream(M):
+    # 9 to 16 rows: the tcgen05 skinny kernel (faster there), also under the small-M override
+    assert bs.plan_for(bs.OP_FP8_BLOCKWISE, M, 1, 7168, 2048, 148)["kernel"] == 2
+    assert bs.plan_for(bs.OP_BMM, M, 8, 1000, 4096, 148)["kernel"] == 2
+    prev = bs.set_path_override(bs.PATH_GEMV)
+    try:
+        assert bs.plan_for(bs.OP_FP8_BLOCKWISE, M, 1, 256, 128, 148)["kernel"] != 4  # beyond its M limit
+    finally:
+        bs.set_path_override(prev)
 
 
 def test_plan_skinny_long_k_prefers_two_ctas_per_sm():
@@ -137,6 +169,8 @@ def test_plan_int8_and_edges():
     b = bs.plan_for(bs.OP_BMM, 16384, 8, 1024, 4096, 148)
     assert b["kernel"] == 1 and b["ctas"] == 148 and b["tile_m"] == 256
     b = bs.plan_for(bs.OP_BMM, 1, 8, 1024, 4096, 148)
+    assert b["kernel"] == 4 and b["ctas"] == (1024 // 16) * 8
+    b = bs.plan_for(bs.OP_BMM, 17, 8, 1024, 4096, 148)
     assert b["kernel"] == 2 and b["ctas"] == 8 * 8 * b["splits"]
 
 
@@ -150,7 +184,8 @@ def test_path_override_forces_kernels():
         assert bs.plan_for(bs.OP_INT_SCALED_MM, 1, 1, 4096, 4096, 148)["kernel"] == 1
     finally:
         bs.set_path_override(prev)
-    assert bs.plan_for(bs.OP_FP8_BLOCKWISE, 1, 1, 7168, 2048, 148)["kernel"] == 2
+    assert bs.plan_for(bs.OP_FP8_BLOCKWISE, 1, 1, 7168, 2048, 148)["kernel"] == 4
+    assert bs.plan_for(bs.OP_FP8_BLOCKWISE, 32, 1, 7168, 2048, 148)["kernel"] == 2
 
 
 # ---------------------------------------------------------------------------
@@ -360,11 +395,18 @@ def test_quantize_128x128_validation_codes():
             assert _qb(**kw) == bs.BS_ERR_DEVICE, kw
 
 
+@pytest.fixture
+def stream_k_on():
+    prev = bs.set_stream_k(True)
+    yield
+    bs.set_stream_k(prev)
+
+
 @pytest.mark.parametrize("M,N,K,G,op", [(4096, 4096, 4096, 1, 2), (1000, 7168, 2048, 1, 1), (1024, 1024, 4096, 2, 3),
                                         (1024, 1024, 4096, 8, 3), (300, 1024, 2048, 1, 1), (1024, 1024, 4096, 1, 2),
                                         (16640, 5120, 8192, 1, 1)])
 @pytest.mark.parametrize("sms", [148, 132])
-def test_stream_k_split_covers_every_k_block_once(M, N, K, G, op, sms):
+def test_stream_k_split_covers_every_k_block_once(M, N, K, G, op, sms, stream_k_on):
     """The host copy of the wide kernel's decomposition: every (tile, K block) is computed by exactly one
     unit; each split tile has one head (the unit holding its first block, where that block is the last
     item of the unit); the other pieces are the first split item of their units, so each unit hands over

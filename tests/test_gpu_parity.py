@@ -551,6 +551,47 @@ def test_forward_gemm_through_the_weight_quantiser():
 
 
 # ---------------------------------------------------------------------------
+# small-M weight stream (M <= 8): warp-level e4m3 MMA, 16 output columns per CTA
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("M", [1, 2, 5, 8])
+@pytest.mark.parametrize("N,K", [(7, 128), (130, 640), (1000, 2048), (300, 4224), (4800, 640)])
+def test_fp8_small_m_weight_stream(M, N, K, path):
+    path(bs.PATH_GEMV)
+    d = wl.fp8_blockwise_inputs(M, N, K, seed=1100 + M + N + K)
+    y, S = oracle_fp8(d)
+    for out_dtype in (torch.bfloat16, torch.float32):
+        out = fp8_run(d, out_dtype)
+        fp8_check(out, y, S, out_dtype, f"small-M {M}x{N}x{K}")
+        assert torch.equal(out, fp8_run(d, out_dtype))
+
+
+@pytest.mark.parametrize("M,G,N,K", [(1, 8, 1024, 4096), (3, 3, 100, 512), (8, 2, 1030, 4096), (7, 1, 260, 1024),
+                                     (4, 8, 1000, 1152)])
+@pytest.mark.parametrize("batch_first", [False, True])
+def test_bmm_small_m_weight_stream(M, G, N, K, batch_first, path):
+    path(bs.PATH_GEMV)
+    d = wl.bmm_inputs(M, G, N, K, seed=1200 + M + G + N, batch_first=batch_first)
+    y, S = oracle.bmm_blockscale(d["x"], d["w"], d["x_scale"], d["w_scale"])
+    for out_dtype in (torch.bfloat16, torch.float32):
+        fp8_check(bmm_run(d, out_dtype), y, S, out_dtype, f"bmm small-M {M}x{G}x{N}x{K} bf={batch_first}")
+
+
+def test_small_m_weight_stream_extreme_scales(path):
+    """The edge-of-domain inputs on the small-M kernel: extreme e8m0 bytes (8 rows, two halves) and zero
+    or subnormal fp32 block scales (rows 2..9 of the blockwise case, which hold all of its planted rows)."""
+    path(bs.PATH_GEMV)
+    d = _bmm_edge_inputs(8, 384, 1024, seed=1300)
+    y, S = oracle.bmm_blockscale(d["x"], d["w"], d["x_scale"], d["w_scale"])
+    for out_dtype in (torch.bfloat16, torch.float32):
+        fp8_check(bmm_run(d, out_dtype), y, S, out_dtype, "small-M extreme e8m0")
+    d = _blockwise_zero_and_subnormal_scales(256, 384, 1024, seed=910)
+    d8 = {"A": d["A"][2:10].contiguous(), "B_t": d["B_t"], "scale_a": d["scale_a"][2:10].contiguous(),
+          "scale_b": d["scale_b"]}
+    y, S = oracle_fp8(d8)
+    fp8_check(fp8_run(d8, torch.bfloat16), y, S, torch.bfloat16, "small-M zero/subnormal scales bf16")
+
+
+# ---------------------------------------------------------------------------
 # stream-K: the last, badly filled round of tiles split over every CTA pair
 # ---------------------------------------------------------------------------
 def _sk_tiles(op, M, G, N, K):
@@ -558,16 +599,19 @@ def _sk_tiles(op, M, G, N, K):
 
 
 @pytest.fixture
-def no_stream_k():
+def stream_k():
+    """Enables the split (off by default) for one test; calling the fixture's value turns it off again."""
+    prev = bs.set_stream_k(True)
+
     def off():
         bs.set_stream_k(False)
     yield off
-    bs.set_stream_k(True)
+    bs.set_stream_k(prev)
 
 
 @pytest.mark.parametrize("M,N,K", [(1024, 1024, 4096), (1000, 1800, 2080), (300, 1040, 8192)])
 @pytest.mark.parametrize("kernel", [bs.PATH_WIDE, bs.PATH_WIDE_SINGLE])
-def test_int8_stream_k_bit_exact(M, N, K, kernel, path):
+def test_int8_stream_k_bit_exact(M, N, K, kernel, path, stream_k):
     path(kernel)
     assert _sk_tiles(bs.OP_INT_SCALED_MM, M, 1, N, K) > 0
     _int8_assert(wl.int8_inputs(M, N, K, seed=950 + M), rows=None)
@@ -575,7 +619,7 @@ def test_int8_stream_k_bit_exact(M, N, K, kernel, path):
 
 @pytest.mark.parametrize("M,N,K", [(1024, 1024, 4096), (700, 1800, 2048), (300, 1040, 8192)])
 @pytest.mark.parametrize("kernel", [bs.PATH_WIDE, bs.PATH_WIDE_SINGLE])
-def test_fp8_stream_k_matches_the_oracle_and_is_deterministic(M, N, K, kernel, path, no_stream_k):
+def test_fp8_stream_k_matches_the_oracle_and_is_deterministic(M, N, K, kernel, path, stream_k):
     path(kernel)
     assert _sk_tiles(bs.OP_FP8_BLOCKWISE, M, 1, N, K) > 0
     d = wl.fp8_blockwise_inputs(M, N, K, seed=960 + M)
@@ -584,12 +628,12 @@ def test_fp8_stream_k_matches_the_oracle_and_is_deterministic(M, N, K, kernel, p
         first = fp8_run(d, out_dtype)
         fp8_check(first, y, S, out_dtype, f"fp8 stream-K {M}x{N}x{K} kernel={kernel}")
         assert torch.equal(first, fp8_run(d, out_dtype)), "split tiles are summed in a fixed order"
-    no_stream_k()
+    stream_k()
     fp8_check(fp8_run(d, torch.float32), y, S, torch.float32, "fp8 without the split")
 
 
 @pytest.mark.parametrize("M,N,K", [(1024, 1024, 4096), (300, 1040, 8192)])
-def test_fp8_rowwise_stream_k(M, N, K):
+def test_fp8_rowwise_stream_k(M, N, K, stream_k):
     assert _sk_tiles(bs.OP_FP8_ROWWISE, M, 1, N, K) > 0
     d = wl.fp8_rowwise_inputs(M, N, K, seed=970 + M)
     for out_dtype in (torch.bfloat16, torch.float32):
@@ -602,7 +646,7 @@ def test_fp8_rowwise_stream_k(M, N, K):
 
 @pytest.mark.parametrize("M,G,N,K", [(1024, 2, 1024, 4096), (300, 3, 520, 4096)])
 @pytest.mark.parametrize("kernel", [bs.PATH_WIDE, bs.PATH_WIDE_PROMOTE])
-def test_bmm_stream_k(M, G, N, K, kernel, path):
+def test_bmm_stream_k(M, G, N, K, kernel, path, stream_k):
     path(kernel)
     assert _sk_tiles(bs.OP_BMM, M, G, N, K) > 0
     d = wl.bmm_inputs(M, G, N, K, seed=980 + M + G)
@@ -612,11 +656,11 @@ def test_bmm_stream_k(M, G, N, K, kernel, path):
     assert torch.equal(out, bmm_run(d, torch.float32))
 
 
-def test_int8_stream_k_equals_the_unsplit_plan(no_stream_k):
+def test_int8_stream_k_equals_the_unsplit_plan(stream_k):
     d = wl.int8_inputs(4096, 4096, 4096, seed=990)
     assert _sk_tiles(bs.OP_INT_SCALED_MM, 4096, 1, 4096, 4096) > 0
     a = int8_run(d, torch.int32)
-    no_stream_k()
+    stream_k()
     assert torch.equal(a, int8_run(d, torch.int32))
 
 
