@@ -48,7 +48,8 @@ typedef enum {
   BS_ERR_DEVICE = 6,    /* current device is not an sm_100 (B200-class) GPU */
   BS_ERR_CUDA = 7,      /* a CUDA runtime call failed (launch, encode, ...) */
   BS_ERR_TIMEOUT = 8,   /* a kernel gave up on a bounded wait (bs_get_device_error) */
-  BS_ERR_WORKSPACE = 9  /* workspace smaller than bs_workspace_size() */
+  BS_ERR_WORKSPACE = 9  /* workspace smaller than bs_workspace_size(), or a device with more
+                           SMs than bs_int_scaled_mm_noalloc's built-in scratch holds */
 } bs_status;
 
 typedef enum {
@@ -156,6 +157,40 @@ bs_status int_scaled_mm(const int8_t* A, int64_t lda, const int8_t* B, int64_t l
                         const float* s_a, const float* s_b,
                         void* out, int64_t ldo, bs_out_dtype out_dtype,
                         int64_t M, int64_t N, int64_t K, void* stream);
+
+/*
+ * int_scaled_mm that allocates nothing, for callers that cannot allocate
+ * device memory: a serving loop that reserves all of HBM up front (a cache
+ * or a pool holding the rest), code running inside a custom allocator's own
+ * callbacks (which must not re-enter it), or a C host with no device
+ * allocator of its own.  cudaMalloc and cudaFree also synchronise the
+ * device, which such callers cannot afford between launches.
+ *
+ * Arguments, layouts, results (bit-exact) and error codes are those of
+ * int_scaled_mm.  The difference: the stream-K split of the wide kernel's
+ * last round of tiles always applies where the planner's rule calls for it
+ * (whether or not bs_set_stream_k is on), and its partial sums and flag
+ * words live in a fixed array built into the library -- 20 MB, enough for
+ * devices of up to 160 SMs -- not in a registered workspace.  Neither this
+ * call nor the library allocates device memory for it.
+ *
+ * The first call on a device does the set-up, with that device current: it
+ * looks up the array's address (cudaGetSymbolAddress, which loads the
+ * array's module).  Make that first call before any stream capture.  Every
+ * call that splits clears the array's flag words on `stream` (an
+ * asynchronous memset) before its kernel, so they start at zero.  Calls
+ * whose work overlaps on the GPU -- on different streams or from different
+ * threads -- share the array and race: order them on one stream or
+ * synchronise between them.
+ *
+ * Returns BS_ERR_WORKSPACE on a device with more than 160 SMs, BS_ERR_CUDA if
+ * the set-up fails.  The published method has no counterpart of this entry
+ * point: it is a deployment variant of int_scaled_mm.
+ */
+bs_status bs_int_scaled_mm_noalloc(const int8_t* A, int64_t lda, const int8_t* B, int64_t ldb,
+                                   const float* s_a, const float* s_b,
+                                   void* out, int64_t ldo, bs_out_dtype out_dtype,
+                                   int64_t M, int64_t N, int64_t K, void* stream);
 
 /*
  * Operation 3 -- batched FP8 GEMM with e8m0 (power-of-two) block scales.

@@ -69,6 +69,7 @@ def lib() -> ctypes.CDLL:
             h.bs_gemm_fp8_blockwise.argtypes = [p, i64, p, i64, p, i64, i64, p, i64, i64, p, i64, ctypes.c_int,
                                                 i64, i64, i64, p]
             h.int_scaled_mm.argtypes = [p, i64, p, i64, p, p, p, i64, ctypes.c_int, i64, i64, i64, p]
+            h.bs_int_scaled_mm_noalloc.argtypes = h.int_scaled_mm.argtypes
             h.bs_gemm_fp8_rowwise.argtypes = [p, i64, p, i64, p, i64, p, i64, p, p, p, i64, ctypes.c_int,
                                               i64, i64, i64, p]
             h.bmm_a8w8_blockscale.argtypes = [p, i64, i64, p, i64, i64, p, p, p, i64, i64, ctypes.c_int,
@@ -78,8 +79,9 @@ def lib() -> ctypes.CDLL:
                                             i64, p]
             h.bs_quantize_fp8_128x128.argtypes = [p, ctypes.c_int, i64, i64, i64, p, i64, p, ctypes.c_int, i64, i64,
                                                   p]
-            for f in (h.bs_gemm_fp8_blockwise, h.int_scaled_mm, h.bmm_a8w8_blockscale, h.bs_gemm_fp8_rowwise,
-                      h.bs_quantize_fp8_1x128, h.bs_quantize_fp8_t, h.bs_quantize_fp8_128x128):
+            for f in (h.bs_gemm_fp8_blockwise, h.int_scaled_mm, h.bs_int_scaled_mm_noalloc, h.bmm_a8w8_blockscale,
+                      h.bs_gemm_fp8_rowwise, h.bs_quantize_fp8_1x128, h.bs_quantize_fp8_t,
+                      h.bs_quantize_fp8_128x128):
                 f.restype = ctypes.c_int
             h.bs_status_string.argtypes = [ctypes.c_int]
             h.bs_status_string.restype = ctypes.c_char_p
@@ -314,6 +316,40 @@ def int_scaled_mm(A: torch.Tensor, B: torch.Tensor, s_a: torch.Tensor | None, s_
     with torch.cuda.device(A.device):
         _check(lib().int_scaled_mm(_ptr(A), A.stride(0), _ptr(B), B.stride(1), _ptr(sa), _ptr(sb), _ptr(out),
                                    out.stride(0), _OUT_CODE[out_dtype], M, N, K, _stream(A.device)))
+    return out
+
+
+def bs_int_scaled_mm_noalloc(A: torch.Tensor, B: torch.Tensor, s_a: torch.Tensor | None, s_b: torch.Tensor | None,
+                             out: torch.Tensor) -> torch.Tensor:
+    """int_scaled_mm through the entry point that allocates nothing (for callers that cannot allocate device
+    memory): the wide kernel's stream-K split with the library's built-in scratch.  Results equal
+    int_scaled_mm's.  Nothing is allocated here either: `out` (row-major [M, N], float32, bfloat16 or int32)
+    must be given, and s_a / s_b must be contiguous float32 vectors or None.  The first call on a device sets
+    up the scratch and belongs before any stream capture; calls that overlap on the GPU race on the scratch.
+    """
+    for t, name in ((A, "A"), (B, "B"), (out, "out")):
+        _cuda(t, name)
+    if A.dtype != torch.int8 or B.dtype != torch.int8:
+        raise BsgemmError(BS_ERR_DTYPE, "A and B must be int8")
+    if A.dim() != 2 or B.dim() != 2 or A.shape[1] != B.shape[0]:
+        raise BsgemmError(BS_ERR_SHAPE, f"A [M,K] and B [K,N] expected, got {tuple(A.shape)} and {tuple(B.shape)}")
+    M, K = A.shape
+    N = B.shape[1]
+    for s, n, name in ((s_a, M, "s_a"), (s_b, N, "s_b")):
+        if s is not None:
+            _cuda(s, name)
+            if s.dtype != torch.float32 or s.numel() != n or not s.is_contiguous():
+                raise BsgemmError(BS_ERR_SHAPE, f"{name} must be a contiguous float32 tensor of {n} elements")
+    if A.stride(1) != 1 and M > 1:
+        raise BsgemmError(BS_ERR_LAYOUT, f"A must be row-major, got strides {A.stride()}")
+    if B.stride(0) != 1 and N > 1:
+        raise BsgemmError(BS_ERR_LAYOUT, f"B must be column-major, got strides {B.stride()}")
+    if out.dtype not in _OUT_CODE or tuple(out.shape) != (M, N) or out.stride(1) != 1:
+        raise BsgemmError(BS_ERR_LAYOUT, "out must be a row-major [M, N] float32, bfloat16 or int32 tensor")
+    with torch.cuda.device(A.device):
+        _check(lib().bs_int_scaled_mm_noalloc(_ptr(A), A.stride(0), _ptr(B), B.stride(1), _ptr(s_a), _ptr(s_b),
+                                              _ptr(out), out.stride(0), _OUT_CODE[out.dtype], M, N, K,
+                                              _stream(A.device)))
     return out
 
 

@@ -22,7 +22,7 @@ INCLUDE = os.path.join(ROOT, "include")
 OBJDIR = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libbsgemm.so")
 SOURCES = ["api.cu", "kernels_wide.cu", "kernels_skinny.cu", "kernels_quantize.cu", "kernels_quantize_t.cu",
-           "kernels_quantize_blocks.cu", "kernels_gemv.cu"]
+           "kernels_quantize_blocks.cu", "kernels_gemv.cu", "static_scratch.cu"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2", "-I" + INCLUDE, "-I" + CSRC]

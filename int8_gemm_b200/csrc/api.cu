@@ -69,6 +69,8 @@ struct DeviceCtx {
   // stream-K workspace registered with bs_set_workspace (caller-owned)
   std::atomic<void*> ws{nullptr};
   std::atomic<size_t> ws_bytes{0};
+  // built-in scratch of bs_int_scaled_mm_noalloc, looked up on its first call
+  std::atomic<void*> scratch{nullptr};
 };
 
 constexpr int kMaxDevices = 64;
@@ -171,7 +173,10 @@ void plan_stream_k(Plan& x, long long tiles, long long units, int KB) {
   x.pub.sk_tiles = static_cast<int32_t>(tiles - dp);
 }
 
-Plan make_plan(int op, int64_t M, int64_t G, int64_t N, int64_t K, int sms, bool stream_k_ok) {
+// stream_k_ok: a workspace for the split is at hand; force_split: apply the
+// split rule even while bs_set_stream_k is off.
+Plan make_plan(int op, int64_t M, int64_t G, int64_t N, int64_t K, int sms, bool stream_k_ok,
+               bool force_split = false) {
   Plan x;
   std::memset(&x.pub, 0, sizeof(x.pub));
   if (M == 0 || N == 0 || G == 0) return x;  // kernel 0: nothing to do
@@ -245,7 +250,7 @@ Plan make_plan(int op, int64_t M, int64_t G, int64_t N, int64_t K, int sms, bool
     const long long units = (sms > 0 ? sms : 148) / x.cg;  // persistent CTAs (or CTA pairs)
     x.num_tiles = static_cast<int>(tiles);
     x.dp_tiles = x.num_tiles;
-    if (stream_k_ok && g_stream_k.load() != 0) plan_stream_k(x, tiles, units, KB);
+    if (stream_k_ok && (force_split || g_stream_k.load() != 0)) plan_stream_k(x, tiles, units, KB);
     x.pub.kernel = 1;
     x.pub.tile_m = tile_m;
     x.pub.tile_n = kWideBN;
@@ -772,9 +777,41 @@ bs_status bs_quantize_fp8_128x128(const void* x, bs_in_dtype x_dtype, int64_t R,
                       "block quantise launch");
 }
 
-bs_status int_scaled_mm(const int8_t* A, int64_t lda, const int8_t* B, int64_t ldb, const float* s_a,
-                        const float* s_b, void* out, int64_t ldo, bs_out_dtype out_dtype, int64_t M, int64_t N,
-                        int64_t K, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// The address of the built-in scratch of bs_int_scaled_mm_noalloc on the
+// current device, looked up once per device (this loads the scratch's module).
+bs_status split_scratch(DeviceCtx* dc, void** out) {
+  if (workspace_bytes_for(dc->sms) > kStaticScratchBytes)
+    return fail(BS_ERR_WORKSPACE,
+                "this device has %d SMs; the built-in scratch of bs_int_scaled_mm_noalloc holds the stream-K "
+                "split of at most %d (%zu bytes)",
+                dc->sms, kStaticScratchMaxSms, kStaticScratchBytes);
+  void* p = dc->scratch.load(std::memory_order_acquire);
+  if (!p) {
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    p = dc->scratch.load(std::memory_order_relaxed);
+    if (!p) {
+      const cudaError_t e = static_scratch_address(&p);
+      if (e != cudaSuccess || !p)
+        return fail(BS_ERR_CUDA, "address of the built-in scratch: %s", cudaGetErrorString(e));
+      dc->scratch.store(p, std::memory_order_release);
+    }
+  }
+  *out = p;
+  return BS_OK;
+}
+
+// int_scaled_mm on the wide kernel.  noalloc = false: the plan and workspace
+// of int_scaled_mm (a split only while bs_set_stream_k is on and a workspace
+// is registered); true: the split rule always applies, with the partials and
+// flags in the built-in scratch, whose flag words are cleared on `stream`
+// before the kernel.
+bs_status int8_gemm(const int8_t* A, int64_t lda, const int8_t* B, int64_t ldb, const float* s_a, const float* s_b,
+                    void* out, int64_t ldo, bs_out_dtype out_dtype, int64_t M, int64_t N, int64_t K, void* stream,
+                    bool noalloc) {
   clear_msg();
   if (M < 0 || N < 0 || K < 0) return fail(BS_ERR_SHAPE, "negative size");
   if (M > kMaxDim || N > kMaxDim) return fail(BS_ERR_SHAPE, "size exceeds 2^31-1");
@@ -798,7 +835,10 @@ bs_status int_scaled_mm(const int8_t* A, int64_t lda, const int8_t* B, int64_t l
   bs_status st = device_ctx(&dc);
   if (st != BS_OK) return st;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  const Plan pl = make_plan(2, M, 1, N, K, dc->sms, workspace_ok(dc));
+  void* scratch = nullptr;
+  if (noalloc && (st = split_scratch(dc, &scratch)) != BS_OK) return st;
+  const Plan pl = noalloc ? make_plan(2, M, 1, N, K, dc->sms, true, true)
+                          : make_plan(2, M, 1, N, K, dc->sms, workspace_ok(dc));
   if (pl.pub.kernel == 3)
     return check_launch(launch_fill_zero(out, out_size(out_dtype), M, N, ldo, 1, 0, cs), "zero-fill launch");
 
@@ -820,7 +860,20 @@ bs_status int_scaled_mm(const int8_t* A, int64_t lda, const int8_t* B, int64_t l
   args.group_m = kGroupM;
   args.splits = 1;
   args.err = dc->err;
-  set_work_split(args, pl, dc);
+  if (!noalloc) {
+    set_work_split(args, pl, dc);
+  } else {
+    args.dp_tiles = pl.dp_tiles;
+    args.sk_iters = pl.sk_iters;
+    if (pl.sk_iters > 0) {
+      uint8_t* base = static_cast<uint8_t*>(scratch);
+      args.sk_ws = reinterpret_cast<uint32_t*>(base);
+      args.sk_flags = reinterpret_cast<uint32_t*>(base + workspace_slots_bytes(dc->sms));
+      const size_t flag_bytes = static_cast<size_t>(dc->sms) * kWsFlagsPerSlot * sizeof(uint32_t);
+      const cudaError_t e = cudaMemsetAsync(args.sk_flags, 0, flag_bytes, cs);
+      if (e != cudaSuccess) return fail(BS_ERR_CUDA, "clear the scratch flags: %s", cudaGetErrorString(e));
+    }
+  }
   CUtensorMap ta, tb, td;
   if ((st = encode_3d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, A, K, M, 1, lda, lda * M, 128, 128, "A"))) return st;
   if ((st = encode_3d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, B, K, N, 1, ldb, ldb * N, 128, wide_b_box_rows(pl.cg),
@@ -832,6 +885,22 @@ bs_status int_scaled_mm(const int8_t* A, int64_t lda, const int8_t* B, int64_t l
     return st;
   return check_launch(launch_wide(Mode::kInt8, out_kind(out_dtype), pl.cg, ta, tb, td, args, pl.pub.ctas, cs),
                       "int8 kernel launch");
+}
+
+}  // namespace
+
+extern "C" {
+
+bs_status int_scaled_mm(const int8_t* A, int64_t lda, const int8_t* B, int64_t ldb, const float* s_a,
+                        const float* s_b, void* out, int64_t ldo, bs_out_dtype out_dtype, int64_t M, int64_t N,
+                        int64_t K, void* stream) {
+  return int8_gemm(A, lda, B, ldb, s_a, s_b, out, ldo, out_dtype, M, N, K, stream, false);
+}
+
+bs_status bs_int_scaled_mm_noalloc(const int8_t* A, int64_t lda, const int8_t* B, int64_t ldb, const float* s_a,
+                                   const float* s_b, void* out, int64_t ldo, bs_out_dtype out_dtype, int64_t M,
+                                   int64_t N, int64_t K, void* stream) {
+  return int8_gemm(A, lda, B, ldb, s_a, s_b, out, ldo, out_dtype, M, N, K, stream, true);
 }
 
 }  // extern "C"

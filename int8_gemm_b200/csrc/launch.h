@@ -43,6 +43,16 @@ struct GemvProblem {
 };
 cudaError_t launch_gemv(Mode mode, OutKind out, const GemvProblem& q, const GemmArgs& args, cudaStream_t stream);
 
+// Built-in scratch of bs_int_scaled_mm_noalloc (static_scratch.cu): the
+// stream-K slots and flag words of a device with at most kStaticScratchMaxSms
+// SMs, in the layout of a registered workspace (20 MB in all).
+constexpr int kStaticScratchMaxSms = 160;
+constexpr size_t kStaticScratchBytes =
+    static_cast<size_t>(kStaticScratchMaxSms) * kWsSlotWords * sizeof(uint32_t) +
+    ((static_cast<size_t>(kStaticScratchMaxSms) * kWsFlagsPerSlot * sizeof(uint32_t) + 255) / 256) * 256;
+// Device address of that array (cudaGetSymbolAddress; the current device).
+cudaError_t static_scratch_address(void** ptr);
+
 // Fill of `batches` matrices [rows, cols] (row stride ld, batch stride
 // bstride, elements of `elem_size` bytes: bf16, fp32, or 1 = e4m3) with zero,
 // or with bias[col] (fp32 [cols]) when bias is given; e4m3 elements take the

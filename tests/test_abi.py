@@ -278,17 +278,22 @@ def test_plan_fp8_rowwise_is_the_wide_kernel_for_every_m():
     assert bs.plan_for(bs.OP_FP8_ROWWISE, 16, 1, 512, 0, 148)["kernel"] == 3  # K = 0: bias (or zero) fill
 
 
-def test_int8_and_bmm_validation_codes():
+@pytest.mark.parametrize("entry", ["int_scaled_mm", "bs_int_scaled_mm_noalloc"])
+def test_int8_and_bmm_validation_codes(entry):
     h, v = bs.lib(), ctypes.c_void_p
-    call = lambda **k: h.int_scaled_mm(v(k.get("A", P16)), k.get("lda", 128), v(k.get("B", P16)), k.get("ldb", 128),
-                                       v(P16), v(P16), v(k.get("out", P16)), k.get("ldo", 64), k.get("dt", bs.BS_OUT_F32),
-                                       k.get("M", 8), 64, k.get("K", 128), None)
+    fn = getattr(h, entry)
+    call = lambda **k: fn(v(k.get("A", P16)), k.get("lda", 128), v(k.get("B", P16)), k.get("ldb", 128),
+                          v(P16), v(P16), v(k.get("out", P16)), k.get("ldo", 64), k.get("dt", bs.BS_OUT_F32),
+                          k.get("M", 8), 64, k.get("K", 128), None)
     assert call(K=131072) == bs.BS_ERR_SHAPE
     assert call(dt=7) == bs.BS_ERR_DTYPE
+    assert call(dt=bs.BS_OUT_E4M3) == bs.BS_ERR_DTYPE
     assert call(B=0) == bs.BS_ERR_NULL
     assert call(ldb=64) == bs.BS_ERR_LAYOUT
     assert call(lda=136) == bs.BS_ERR_ALIGNMENT
     assert call(M=0) == bs.BS_OK
+    if not HAS_GPU:
+        assert call() == bs.BS_ERR_DEVICE
     bmm = lambda **k: h.bmm_a8w8_blockscale(v(P16), k.get("x_sm", 1024), 128, v(P16), 128 * 256, 128, v(P16), v(P16),
                                             v(P16), 2048, 256, bs.BS_OUT_BF16, 4, 8, 256, k.get("K", 128), None)
     assert bmm(K=64) == bs.BS_ERR_SHAPE
