@@ -112,9 +112,7 @@ __global__ void __launch_bounds__(kQuantThreads)
       float y[16];
       if constexpr (FMT == 0) {
         const float s = group_scale_f32(amax);
-        const double rinv = __drcp_rn(static_cast<double>(s));
-#pragma unroll
-        for (int i = 0; i < 16; ++i) y[i] = over_scale(v[ps][i], rinv);
+        code_quotients<16>(v[ps], s, y);
         if (j == 0 && g < KB) static_cast<float*>(scale)[static_cast<long long>(m) * lds + g] = s;
       } else {
         const int byte = group_e8m0(amax);

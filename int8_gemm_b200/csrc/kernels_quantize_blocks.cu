@@ -91,11 +91,9 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll
     for (int w = 1; w < kThreads / 32; ++w) amax = fmaxf(amax, wmax[parity][w]);
     float s = 1.f;
-    double rinv = 1.0;
     int byte = 127;
     if constexpr (FMT == 0) {
       s = group_scale_f32(amax);
-      rinv = __drcp_rn(static_cast<double>(s));
     } else {
       byte = group_e8m0(amax);
     }
@@ -112,17 +110,19 @@ __global__ void __launch_bounds__(kThreads)
     for (int k = 0; k < P::kPasses; ++k) {
       const long long r = rb * kTile + row0 + k * P::kRowsPerPass;
       if (r >= R) continue;
+      float e[P::kElems], y[P::kElems];
+#pragma unroll
+      for (int j = 0; j < P::kElems; ++j) e[j] = piece_elem<InT>(v[k], j);
+      if constexpr (FMT == 0) {
+        code_quotients<P::kElems>(e, s, y);
+      } else {
+#pragma unroll
+        for (int j = 0; j < P::kElems; ++j) y[j] = e[j] * mul;
+      }
       uint32_t w[P::kElems / 4];
 #pragma unroll
-      for (int i = 0; i < P::kElems / 4; ++i) {
-        float y[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const float e = piece_elem<InT>(v[k], 4 * i + j);
-          y[j] = FMT == 0 ? over_scale(e, rinv) : e * mul;
-        }
-        w[i] = e4m3x2(y[0], y[1]) | (e4m3x2(y[2], y[3]) << 16);
-      }
+      for (int i = 0; i < P::kElems / 4; ++i)
+        w[i] = e4m3x2(y[4 * i], y[4 * i + 1]) | (e4m3x2(y[4 * i + 2], y[4 * i + 3]) << 16);
       uint8_t* dst = q + r * ldq + c;
       if (vec_q && c + P::kElems <= C) {
         if constexpr (P::kElems == 8) {

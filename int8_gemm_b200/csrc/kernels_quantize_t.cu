@@ -119,11 +119,9 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks<InT>)
     }
     const long long c = c0 + col;
     float s = 1.f;
-    double rinv = 1.0;
     int byte = 127;
     if constexpr (FMT == 0) {
       s = group_scale_f32(amax);
-      rinv = __drcp_rn(static_cast<double>(s));
     } else {
       byte = group_e8m0(amax);
     }
@@ -141,11 +139,14 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks<InT>)
     uint8_t* dst = q + c * ldq + r0 + 64 * half;
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-      float y[16];
+      float e[16], y[16];
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const float e = to_f32(colp[(16 * k + j) * kTile]);
-        y[j] = FMT == 0 ? over_scale(e, rinv) : e * mul;
+      for (int j = 0; j < 16; ++j) e[j] = to_f32(colp[(16 * k + j) * kTile]);
+      if constexpr (FMT == 0) {
+        code_quotients<16>(e, s, y);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) y[j] = e[j] * mul;
       }
       uint4 codes;
       codes.x = e4m3x2(y[0], y[1]) | (e4m3x2(y[2], y[3]) << 16);

@@ -39,3 +39,71 @@ def test_fp64_reciprocal_product_near_fp32_midpoints():
     ref = (x / s).astype(np.float32)
     got = (x.astype(np.float64) * (1.0 / s.astype(np.float64))).astype(np.float32)
     assert np.array_equal(ref.view(np.uint32), got.view(np.uint32))
+
+
+# ---------------------------------------------------------------------------
+# The quantisers' fp32 division: q1 = RN(x * r), r = RN(1 / s); rem = RN(x - q1 * s) (one fma, exact);
+# q = RN(q1 + rem * r) (one fma), with copysign for a zero x.  Markstein's correction step makes q the
+# correctly rounded quotient when the residual does not underflow, which the kernels guarantee by taking
+# this path only for group scales s >= 2^-90.  The fma's single rounding is emulated exactly with
+# rational arithmetic.
+# ---------------------------------------------------------------------------
+from fractions import Fraction
+
+
+def _rn32(x: Fraction) -> np.float32:
+    """Round a rational to the nearest fp32, ties to even (normal and subnormal range)."""
+    if x == 0:
+        return np.float32(0.0)
+    sign = -1 if x < 0 else 1
+    a = abs(x)
+    e = a.numerator.bit_length() - a.denominator.bit_length()
+    if Fraction(2) ** e > a:
+        e -= 1
+    ulp = Fraction(2) ** (max(e, -126) - 23)
+    n, rem = divmod(a, ulp)
+    if rem * 2 > ulp or (rem * 2 == ulp and n % 2 == 1):
+        n += 1
+    return np.float32(sign * float(n * ulp))
+
+
+def _fma32(a, b, c) -> np.float32:
+    return _rn32(Fraction(float(a)) * Fraction(float(b)) + Fraction(float(c)))
+
+
+def _quotient_rn(x: np.float32, s: np.float32) -> np.float32:
+    r = np.float32(np.float32(1.0) / s)
+    q1 = np.float32(x * r)
+    rem = _fma32(-q1, s, x)
+    q = _fma32(rem, r, q1)
+    return np.copysign(q, x).astype(np.float32)
+
+
+def test_fp32_corrected_quotient_is_the_correctly_rounded_quotient():
+    rng = np.random.default_rng(21)
+    n = 20_000
+    amax = np.ldexp(1.0 + rng.random(n), rng.integers(-80, 120, n)).astype(np.float32)
+    s = (amax / np.float32(448.0)).astype(np.float32)
+    x = (amax * rng.uniform(-1, 1, n)).astype(np.float32)
+    # a third of the quotients steered next to fp32 rounding midpoints, a few exact multiples and zeros
+    k = np.arange(n) % 3 == 1
+    m = rng.uniform(2.0 ** -11, 448, n)
+    mid = (m.astype(np.float32).astype(np.float64) + np.spacing(m.astype(np.float32)).astype(np.float64) / 2)
+    x[k] = (mid[k] * s[k].astype(np.float64)).astype(np.float32)
+    x[::97] = (s[::97] * np.float32(7.0)).astype(np.float32)
+    x[::89] = np.float32(-0.0)
+    assert float(s.min()) >= 2.0 ** -90
+    for xi, si in zip(x, s):
+        ref = np.float32(xi / si)
+        got = _quotient_rn(xi, si)
+        assert ref.view(np.uint32) == got.view(np.uint32), (float(xi), float(si), float(ref), float(got))
+
+
+def test_fp32_corrected_quotient_needs_the_correction():
+    # the plain reciprocal product alone is not the correctly rounded quotient for some of the same pairs,
+    # so the test above would catch a kernel that dropped the correction step
+    rng = np.random.default_rng(22)
+    s = np.ldexp(1.0 + rng.random(5000), rng.integers(-40, 40, 5000)).astype(np.float32)
+    x = (s.astype(np.float64) * rng.uniform(1, 448, 5000)).astype(np.float32)
+    r = (np.float32(1.0) / s).astype(np.float32)
+    assert np.any((x * r).astype(np.float32) != (x / s).astype(np.float32))

@@ -492,6 +492,42 @@ def test_backward_gemms_through_the_transposed_quantiser():
 # ---------------------------------------------------------------------------
 # forward-orientation 128x128 weight quantiser (B_t [N, K] and scale_b) -- bit-exact
 # ---------------------------------------------------------------------------
+def _near_midpoint_blocks(R, C, bh, bw, seed):
+    """fp32 [R, C] whose bh x bw groups have quotients x / (amax / 448) within 3 fp32 ulps of e4m3
+    rounding midpoints (normal and subnormal e4m3 range), with group amax from 2^-115 to 2^120 (so
+    scales on both sides of 2^-90, the bound of the kernels' fp32 division path).  Element (0, 0) of
+    each group holds its amax.  A quotient with too few correct bits rounds to a different code here."""
+    rng = np.random.default_rng(seed)
+    gr, gc = -(-R // bh), -(-C // bw)
+    e = rng.integers(-115, 121, size=(gr, gc))
+    amax = np.ldexp(1.0 + rng.random((gr, gc)), e).astype(np.float32)
+    s = (amax / np.float32(448.0)).astype(np.float32).astype(np.float64)
+    s_full = np.repeat(np.repeat(s, bh, 0), bw, 1)[:R, :C]
+    a_full = np.repeat(np.repeat(amax, bh, 0), bw, 1)[:R, :C]
+    k = rng.integers(0, 8, (R, C))
+    ex = rng.integers(-9, 9, (R, C))
+    mids = (8 + k + 0.5) / 8.0 * np.exp2(ex)                       # midpoints between e4m3 normals
+    subn = (2 * rng.integers(0, 8, (R, C)) + 1) * 2.0 ** -10          # midpoints in the subnormal range
+    mids = np.where(ex < -6, subn, mids)
+    v = (mids * s_full).astype(np.float32)
+    v = (v.view(np.int32) + rng.integers(-3, 4, (R, C)).astype(np.int32)).view(np.float32)
+    v = np.minimum(np.abs(v), a_full) * rng.choice(np.array([-1.0, 1.0], np.float32), (R, C))
+    v[::bh, ::bw] = amax[: -(-R // bh), : -(-C // bw)]
+    return torch.from_numpy(v.astype(np.float32))
+
+
+def test_quantizers_quotients_next_to_rounding_midpoints():
+    """All three quantisers, fp32 scales, on groups built so that each code sits on a knife edge:
+    bit-exact against the oracle (the kernels divide with an fp32 correction step, not in fp64)."""
+    x = _near_midpoint_blocks(256, 1024, 1, 128, 9900)
+    _quant_check(x.to(DEV), 0)
+    xt = _near_midpoint_blocks(1024, 256, 128, 1, 9901)
+    _quant_t_check(xt.to(DEV), "128x1", 0)
+    xb = _near_midpoint_blocks(512, 640, 128, 128, 9902)
+    _quant_t_check(xb.to(DEV), "128x128", 0)
+    _quant_b_check(xb.to(DEV), 0)
+
+
 def _quant_b_check(x_dev, fmt, **kw):
     q, s = bs.bs_quantize_fp8_128x128(x_dev, "f32" if fmt == 0 else "e8m0", **kw)
     rq, rs = oracle.quantize_128x128(x_dev.float().cpu(), fmt)
