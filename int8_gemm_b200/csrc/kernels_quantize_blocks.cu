@@ -50,8 +50,13 @@ __device__ __forceinline__ float piece_elem(const uint4& v, int j) {
 // FMT 0: fp32 scales; 1: e8m0 bytes.  vec_x: x and its row stride allow
 // 16-byte loads; vec_q: q and its row stride allow the 8-byte (bf16) or
 // 4-byte (fp32) code stores.
+// Three bf16 CTAs (two fp32) per SM: a register budget that keeps one CTA's
+// tile loads in flight while the others reduce and store.
+template <typename InT>
+constexpr int kBlocksMinCtas = sizeof(InT) == 2 ? 3 : 2;
+
 template <typename InT, int FMT>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, kBlocksMinCtas<InT>)
     quantize_blocks_kernel(const InT* __restrict__ x, long long R, long long C, long long ldx,
                            uint8_t* __restrict__ q, long long ldq, void* __restrict__ scale, long long s_rb,
                            long long s_cb, long long ctiles, long long ntiles, bool vec_x, bool vec_q) {

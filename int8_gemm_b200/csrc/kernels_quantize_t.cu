@@ -16,13 +16,15 @@
 //
 // One CTA quantises a 128 x 128 tile at a time (persistent over tiles).  The
 // tile is read row by row with 16-byte loads and kept in shared memory in the
-// input type; thread t then owns column t % 128, rows 64 (t / 128) .. + 63,
-// reading them down the column (a warp reads 32 consecutive elements of one
-// row per step, no bank conflicts) once for the amax and once to quantise, so
-// few registers are live and several CTAs share an SM: while one quantises,
-// the others' loads are in flight.  The column halves' amaxes meet in shared
-// memory (128x1), or the whole tile's in a block reduction (128x128).  Each
-// thread writes its 64 codes, contiguous in q_t, as four 16-byte stores.
+// input type; thread t then owns the column pair 2 (t % 64), 2 (t % 64) + 1
+// and rows 32 (t / 64) .. + 31, reading both columns with one 4-byte (bf16)
+// or 8-byte (fp32) shared load per row (a warp reads 64 consecutive elements
+// of one row per step, no bank conflicts), once for the amax and once to
+// quantise, so few registers are live and several CTAs share an SM: while one
+// quantises, the others' loads are in flight.  The four row quarters' column
+// amaxes meet in shared memory (128x1), or the whole tile's in a block
+// reduction (128x128).  Each thread writes its 2 x 32 codes, contiguous in two
+// rows of q_t, as 16-byte stores.
 #include <cuda_bf16.h>
 
 #include <cstring>
@@ -41,15 +43,46 @@ constexpr int kThreads = 256;
 template <typename InT>
 constexpr int kMinBlocks = sizeof(InT) == 2 ? 4 : 3;
 
+constexpr int kQuarters = kThreads / (kTile / 2);  // row quarters: threads per column pair
+constexpr int kRowsPerThread = kTile / kQuarters;
+
 template <typename InT>
 struct TileSmem {
-  InT v[kTile][kTile];   // the tile, [row][column]
-  float part[2][kTile];  // per-column amax of the two row halves
+  InT v[kTile][kTile];          // the tile, [row][column]
+  float part[kQuarters][kTile];  // per-column amax of the row quarters
   float wmax[kThreads / 32];
 };
 
-__device__ __forceinline__ float to_f32(float v) { return v; }
-__device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
+// Elements (row, 2p) and (row, 2p + 1) of the shared tile, widened to fp32
+// (exact for bf16), with one shared load.
+__device__ __forceinline__ void pair_at(const TileSmem<__nv_bfloat16>& sm, int row, int p, float& a, float& b) {
+  const uint32_t w = *reinterpret_cast<const uint32_t*>(&sm.v[row][2 * p]);
+  a = __uint_as_float(w << 16);
+  b = __uint_as_float(w & 0xFFFF0000u);
+}
+__device__ __forceinline__ void pair_at(const TileSmem<float>& sm, int row, int p, float& a, float& b) {
+  const float2 w = *reinterpret_cast<const float2*>(&sm.v[row][2 * p]);
+  a = w.x;
+  b = w.y;
+}
+
+// 16 codes of one column to q_t row `dst` (rows r .. r + 15 of x), a 16-byte
+// store where alignment and the row count allow.
+__device__ __forceinline__ void store16(uint8_t* dst, const float (&y)[16], long long r, long long R, bool vec_q) {
+  uint4 codes;
+  codes.x = e4m3x2(y[0], y[1]) | (e4m3x2(y[2], y[3]) << 16);
+  codes.y = e4m3x2(y[4], y[5]) | (e4m3x2(y[6], y[7]) << 16);
+  codes.z = e4m3x2(y[8], y[9]) | (e4m3x2(y[10], y[11]) << 16);
+  codes.w = e4m3x2(y[12], y[13]) | (e4m3x2(y[14], y[15]) << 16);
+  if (vec_q && r + 16 <= R) {
+    *reinterpret_cast<uint4*>(dst) = codes;
+  } else {
+    const uint32_t w[4] = {codes.x, codes.y, codes.z, codes.w};
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      if (r + j < R) dst[j] = static_cast<uint8_t>(w[j / 4] >> (8 * (j % 4)));
+  }
+}
 
 // Tile rows are read as 16-byte vectors: 8 bf16 or 4 fp32 elements.
 template <typename InT>
@@ -71,8 +104,8 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks<InT>)
   TileSmem<InT>& sm = *reinterpret_cast<TileSmem<InT>*>(smem_raw);
   using V = Vec<InT>;
   const int t = threadIdx.x;
-  const int col = t % kTile;   // this thread's column in the compute phase
-  const int half = t / kTile;  // and its half of the rows
+  const int cp = t % (kTile / 2);  // this thread's column pair in the compute phase
+  const int qr = t / (kTile / 2);  // and its quarter of the rows
   for (long long tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
     const long long rb = tile / ctiles, cb = tile - rb * ctiles;
     const long long r0 = rb * kTile, c0 = cb * kTile;
@@ -99,16 +132,27 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks<InT>)
       *reinterpret_cast<uint4*>(&sm.v[i / V::kPerRow][(i % V::kPerRow) * V::kElems]) = raw[k];
     }
     __syncthreads();
-    // the amax of this thread's 64 values, down its column
-    const InT* colp = &sm.v[64 * half][col];
-    float amax = 0.f;
-#pragma unroll 16
-    for (int i = 0; i < 64; ++i) amax = fmaxf(amax, fabsf(to_f32(colp[i * kTile])));
+    // the amaxes of this thread's two columns, down its quarter of the rows
+    const int rq = kRowsPerThread * qr;
+    float amax0 = 0.f, amax1 = 0.f;
+#pragma unroll 8
+    for (int i = 0; i < kRowsPerThread; ++i) {
+      float a, b;
+      pair_at(sm, rq + i, cp, a, b);
+      amax0 = fmaxf(amax0, fabsf(a));
+      amax1 = fmaxf(amax1, fabsf(b));
+    }
     if constexpr (GROUP == 0) {
-      sm.part[half][col] = amax;
+      sm.part[qr][2 * cp] = amax0;
+      sm.part[qr][2 * cp + 1] = amax1;
       __syncthreads();
-      amax = fmaxf(sm.part[0][col], sm.part[1][col]);
+#pragma unroll
+      for (int k = 1; k < kQuarters; ++k) {
+        amax0 = fmaxf(amax0, sm.part[(qr + k) % kQuarters][2 * cp]);
+        amax1 = fmaxf(amax1, sm.part[(qr + k) % kQuarters][2 * cp + 1]);
+      }
     } else {
+      float amax = fmaxf(amax0, amax1);
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
       if ((t & 31) == 0) sm.wmax[t / 32] = amax;
@@ -116,51 +160,61 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks<InT>)
       amax = sm.wmax[0];
 #pragma unroll
       for (int w = 1; w < kThreads / 32; ++w) amax = fmaxf(amax, sm.wmax[w]);
+      amax0 = amax1 = amax;
     }
-    const long long c = c0 + col;
-    float s = 1.f;
-    int byte = 127;
+    const long long ca = c0 + 2 * cp, cbn = ca + 1;  // this thread's two columns of x
+    float s0 = 1.f, s1 = 1.f;
+    int byte0 = 127, byte1 = 127;
     if constexpr (FMT == 0) {
-      s = group_scale_f32(amax);
+      s0 = group_scale_f32(amax0);
+      s1 = group_scale_f32(amax1);
     } else {
-      byte = group_e8m0(amax);
+      byte0 = group_e8m0(amax0);
+      byte1 = group_e8m0(amax1);
     }
-    const float mul = ldexpf(1.f, 127 - byte);  // exact power of two (e8m0)
-    const bool owner = GROUP == 0 ? (half == 0 && c < C) : t == 0;
-    if (owner) {
-      const long long si = GROUP == 0 ? c * lds + rb : rb * lds + cb;
+    const float mul0 = ldexpf(1.f, 127 - byte0), mul1 = ldexpf(1.f, 127 - byte1);  // exact powers of two
+    if constexpr (GROUP == 0) {
+      if (qr == 0) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const long long c = ca + h;
+          if (c >= C) continue;
+          if constexpr (FMT == 0) {
+            static_cast<float*>(scale)[c * lds + rb] = h ? s1 : s0;
+          } else {
+            static_cast<uint8_t*>(scale)[c * lds + rb] = static_cast<uint8_t>(h ? byte1 : byte0);
+          }
+        }
+      }
+    } else if (t == 0) {
       if constexpr (FMT == 0) {
-        static_cast<float*>(scale)[si] = s;
+        static_cast<float*>(scale)[rb * lds + cb] = s0;
       } else {
-        static_cast<uint8_t*>(scale)[si] = static_cast<uint8_t>(byte);
+        static_cast<uint8_t*>(scale)[rb * lds + cb] = static_cast<uint8_t>(byte0);
       }
     }
-    if (c >= C) continue;  // a column past the matrix: nothing to store
-    uint8_t* dst = q + c * ldq + r0 + 64 * half;
+    if (ca >= C) continue;  // both columns past the matrix: nothing to store
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      float e[16], y[16];
+    for (int k = 0; k < kRowsPerThread / 16; ++k) {
+      const long long r = r0 + rq + 16 * k;
+      float e0[16], e1[16], y[16];
 #pragma unroll
-      for (int j = 0; j < 16; ++j) e[j] = to_f32(colp[(16 * k + j) * kTile]);
+      for (int j = 0; j < 16; ++j) pair_at(sm, rq + 16 * k + j, cp, e0[j], e1[j]);
       if constexpr (FMT == 0) {
-        code_quotients<16>(e, s, y);
+        code_quotients<16>(e0, s0, y);
       } else {
 #pragma unroll
-        for (int j = 0; j < 16; ++j) y[j] = e[j] * mul;
+        for (int j = 0; j < 16; ++j) y[j] = e0[j] * mul0;
       }
-      uint4 codes;
-      codes.x = e4m3x2(y[0], y[1]) | (e4m3x2(y[2], y[3]) << 16);
-      codes.y = e4m3x2(y[4], y[5]) | (e4m3x2(y[6], y[7]) << 16);
-      codes.z = e4m3x2(y[8], y[9]) | (e4m3x2(y[10], y[11]) << 16);
-      codes.w = e4m3x2(y[12], y[13]) | (e4m3x2(y[14], y[15]) << 16);
-      const long long r = r0 + 64 * half + 16 * k;
-      if (vec_q && r + 16 <= R) {
-        *reinterpret_cast<uint4*>(dst + 16 * k) = codes;
-      } else {
-        const uint32_t w[4] = {codes.x, codes.y, codes.z, codes.w};
+      store16(q + ca * ldq + r, y, r, R, vec_q);
+      if (cbn < C) {
+        if constexpr (FMT == 0) {
+          code_quotients<16>(e1, s1, y);
+        } else {
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
-          if (r + j < R) dst[16 * k + j] = static_cast<uint8_t>(w[j / 4] >> (8 * (j % 4)));
+          for (int j = 0; j < 16; ++j) y[j] = e1[j] * mul1;
+        }
+        store16(q + cbn * ldq + r, y, r, R, vec_q);
       }
     }
   }
