@@ -19,7 +19,8 @@
 // of a row per pass, reading and writing them contiguously.  The per-group
 // work (amax, scale, reciprocal) is shared by four groups per instruction.  A
 // warp takes chunks of eight groups (two passes) and keeps all their loads in
-// flight before it reduces any of them.
+// flight before it reduces any of them, then asks L2 for its next chunk while
+// it quantises this one.
 #include <cuda_bf16.h>
 
 #include "group_quant.cuh"
@@ -75,7 +76,7 @@ __device__ __forceinline__ void load16(const InT* row, long long k, long long K,
 }
 
 template <typename InT, int FMT>
-__global__ void __launch_bounds__(kQuantThreads)
+__global__ void __launch_bounds__(kQuantThreads, 4)
     quantize_1x128_kernel(const InT* __restrict__ x, int M, long long K, long long ldx, uint8_t* __restrict__ q,
                           long long ldq, void* __restrict__ scale, long long lds) {
   const int lane = threadIdx.x & 31;
@@ -99,6 +100,20 @@ __global__ void __launch_bounds__(kQuantThreads)
       const long long k0 = static_cast<long long>(g) * 128;
       const bool vec = k0 + 128 <= K && (reinterpret_cast<uintptr_t>(row + k0) & 15u) == 0;
       load16<InT>(row, k0 + 16 * j, g < KB ? K : 0, vec, v[ps]);  // groups past the row read zeros
+    }
+    {  // the next chunk of this warp into L2 while this one is quantised
+      const unsigned cn = c + nwarps;
+      if (cn < chunks) {
+        const unsigned mn = cn / cpr;
+        const int gn0 = static_cast<int>(cn - mn * cpr) * kGroupsPerChunk;
+#pragma unroll
+        for (int ps = 0; ps < kPasses; ++ps) {
+          const int g = gn0 + ps * kGroupsPerPass + sub;
+          const long long k = static_cast<long long>(g) * 128 + 16 * j;
+          if (g < KB && k < K)
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(x + static_cast<long long>(mn) * ldx + k));
+        }
+      }
     }
 #pragma unroll
     for (int ps = 0; ps < kPasses; ++ps) {
