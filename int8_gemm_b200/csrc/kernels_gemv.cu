@@ -10,9 +10,9 @@
 //
 // A CTA of 8 warps owns 16 weight rows (output columns n0 .. n0+15) of one
 // batch; its warps split the K blocks into 8 contiguous ranges, and each warp
-// has the loads of one K block (KBS = 1, grids of more than two CTAs per SM)
-// or two (KBS = 2, small grids, which need more bytes in flight per CTA) in
-// flight before its MMAs.  Per 64-deep
+// has the loads of KBS K blocks in flight before its MMAs: one for grids of
+// more than two CTAs per SM, two for grids of up to two, four for grids of at
+// most one CTA per SM (small grids need more bytes in flight per CTA).  Per 64-deep
 // K group a thread loads 16 contiguous bytes of weight rows g and g+8
 // (g = lane / 4) and 16 bytes of activation row lane / 4 at the same K
 // offset (lane % 4) * 16, and issues two MMAs: the dot product does not care
@@ -49,9 +49,9 @@ __device__ __forceinline__ void mma_e4m3_16x8x32(float (&d)[4], const uint32_t (
 // Output element (m, g, n) at out[m * o_sm + g * o_sg + n].  KBS = 1 keeps a
 // thread at 64 registers, so four CTAs share an SM and the grid of a 7168-row
 // weight (448 CTAs) or of eight 1024-row batches (512) runs in one wave;
-// KBS = 2 (two CTAs per SM) serves grids of at most two CTAs per SM.
+// KBS = 2 (two CTAs per SM) and KBS = 4 (one) serve the smaller grids.
 template <Mode MODE, int KBS, typename OutT>
-__global__ void __launch_bounds__(kGemvWarps * 32, KBS == 1 ? 4 : 2)
+__global__ void __launch_bounds__(kGemvWarps * 32, KBS == 1 ? 4 : (KBS == 2 ? 2 : 1))
     gemv_kernel(const uint8_t* __restrict__ A, long long a_sm, long long a_sg, const uint8_t* __restrict__ B,
                 long long b_sn, long long b_sg, const GemmArgs p, void* out, long long o_sm, long long o_sg) {
   constexpr int NT = 1;  // one 8-wide activation tile: M <= 8
@@ -202,6 +202,7 @@ cudaError_t launch_kbs(const GemvProblem& q, const GemmArgs& args, cudaStream_t 
 template <Mode MODE, typename OutT>
 cudaError_t launch_mode(const GemvProblem& q, const GemmArgs& args, cudaStream_t stream) {
   const long long ctas = static_cast<long long>((args.N + kGemvRows - 1) / kGemvRows) * args.G;
+  if (ctas <= q.sms) return launch_kbs<MODE, 4, OutT>(q, args, stream);
   return ctas <= 2LL * q.sms ? launch_kbs<MODE, 2, OutT>(q, args, stream) : launch_kbs<MODE, 1, OutT>(q, args, stream);
 }
 

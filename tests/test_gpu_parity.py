@@ -590,7 +590,9 @@ def test_forward_gemm_through_the_weight_quantiser():
 # small-M weight stream (M <= 8): warp-level e4m3 MMA, 16 output columns per CTA
 # ---------------------------------------------------------------------------
 @pytest.mark.parametrize("M", [1, 2, 5, 8])
-@pytest.mark.parametrize("N,K", [(7, 128), (130, 640), (1000, 2048), (300, 4224), (4800, 640)])
+# grids of at most one CTA per SM (N <= 16 * 148), of up to two (N = 3000) and more (N = 4800): the
+# kernel keeps four, two or one K blocks per warp in flight accordingly
+@pytest.mark.parametrize("N,K", [(7, 128), (130, 640), (1000, 2048), (300, 4224), (3000, 1152), (4800, 640)])
 def test_fp8_small_m_weight_stream(M, N, K, path):
     path(bs.PATH_GEMV)
     d = wl.fp8_blockwise_inputs(M, N, K, seed=1100 + M + N + K)
