@@ -25,8 +25,8 @@
 //   work with torch.compile" (1x128 / 128x128 scale shapes); ROCm/aiter PR
 //   "Add opus fp8 mxscale BMM kernels for gfx950" (batched m-major layout,
 //   e8m0 scales, m = 1 .. 16 among its test sizes).  From 9 to 16 rows the
-//   tcgen05 skinny kernel measured faster (16 rows of eight 1024 x 7168
-//   batches: 11.4 against 20.3 us), so this kernel stops at 8.
+//   tcgen05 skinny kernel measured faster (16 activation rows, eight batches
+//   of a 1024 x 4096 weight: 11.4 against 20.3 us), so this kernel stops at 8.
 #include <cuda_bf16.h>
 
 #include "launch.h"

@@ -106,7 +106,7 @@ def test_plan_large_fp8_is_persistent_wide_on_cta_pairs():
 
 @pytest.mark.parametrize("M", [1, 8, 16, 17, 32, 127, 128, 129, 255, 256])
 def test_plan_skinny_split_k(M):
-    prev = bs.set_path_override(bs.PATH_SKINNY if M <= 16 else bs.PATH_AUTO)  # M <= 16 runs the small-M kernel
+    prev = bs.set_path_override(bs.PATH_SKINNY if M <= 8 else bs.PATH_AUTO)  # M <= 8 runs the small-M kernel
     try:
         p = bs.plan_for(bs.OP_FP8_BLOCKWISE, M, 1, 7168, 2048, 148)
     finally:
