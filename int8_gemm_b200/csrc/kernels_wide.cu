@@ -13,9 +13,9 @@ constexpr int kMaxDevices = 64;
 template <Mode MODE, int CG, typename OutT, bool SPLIT>
 cudaError_t launch_split(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& d, const GemmArgs& args,
                          int grid, cudaStream_t stream) {
-  constexpr int STAGES = CG == 2 ? kWideStagesPair : kWideStages;
+  constexpr int STAGES = wide_stages<MODE, CG>();
   auto kernel = wide_gemm_kernel<MODE, CG, STAGES, OutT, SPLIT>;
-  constexpr size_t smem = sizeof(WideSmem<kWideBN / CG, STAGES>) + 1024;
+  constexpr size_t smem = sizeof(WideSmem<kWideBN / CG, STAGES, wide_stage_bufs<MODE, CG>()>) + 1024;
   static std::atomic<uint64_t> configured{0};  // one bit per device
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);

@@ -13,8 +13,6 @@ namespace bsg {
 enum class OutKind : int { kBF16 = 0, kF32 = 1, kI32 = 2, kE4M3 = 3 };
 
 constexpr int kWideBN = 256;
-constexpr int kWideStages = 4;      // single-CTA tiles: 48 KB per stage
-constexpr int kWideStagesPair = 6;  // CTA-pair tiles: 32 KB per stage and CTA
 constexpr int kWideThreads = 384;
 
 // Persistent wide kernel over `grid` CTAs; cta_group 2 launches clusters of two

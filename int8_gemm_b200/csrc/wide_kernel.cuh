@@ -40,7 +40,8 @@
 //   Sources: pytorch/ao PR "Remove int_scaled_mm's dependency on triton for
 //   cpu" (int_scaled_matmul_cpu); pytorch/ao issue "Unify scaled INT8 matmul"
 //   (cast acc_i32 to f32, then multiply by the fp32 scales).
-// Epilogue: registers -> 64B-swizzled shared staging (2 KB per consumer warp)
+// Epilogue: registers -> 64B-swizzled shared staging (2 KB per consumer warp,
+// two such buffers for INT8 on CTA pairs)
 // -> TMA store, which clips rows >= M and columns >= N (the masked store of
 // mm_template in pytorch/torch/_inductor/kernel/mm.py).  Rows >= M of A are
 // zero-filled by the TMA loads, so ragged M needs no padding copies.
@@ -117,11 +118,29 @@ constexpr int kSfRing = 5;      // kFp8Mx: scale-factor slots (four K blocks eac
 // 256-column buffers share 32 columns and the scale factors fit behind them.
 constexpr uint32_t kAcc1Col = 224, kSfaCol = 480, kSfbCol = 484;
 
-template <int BNL, int STAGES>
+// Output staging buffers per consumer warp: two for INT8 on CTA pairs (a
+// chunk is staged while the previous chunk's TMA store still reads the
+// other), with one operand stage fewer to make room.  Its epilogue has to
+// hide behind the next tile's MMAs, and its fp32 and int32 outputs take eight
+// chunks per warp; measured on 4096^3 with fp32 out, 62.3 -> 60.0 us.  The
+// FP8 modes keep one buffer and the deeper ring (rowwise and the block-scaled
+// MMA measured about 1 % slower with two), and so do single-CTA tiles, whose
+// 48 KB stages leave no room for a second buffer.
+template <Mode MODE, int CG>
+__host__ __device__ constexpr int wide_stage_bufs() {
+  return CG == 2 && MODE == Mode::kInt8 ? 2 : 1;
+}
+template <Mode MODE, int CG>
+__host__ __device__ constexpr int wide_stages() {
+  return CG == 2 ? (wide_stage_bufs<MODE, CG>() == 2 ? 5 : 6) : 4;
+}
+
+template <int BNL, int STAGES, int SBUFS>
 struct WideSmem {
+  static constexpr int kStageBufs = SBUFS;
   uint8_t a[STAGES][128 * 128];  // this CTA's 128 A rows of one K block
   uint8_t b[STAGES][BNL * 128];  // this CTA's BNL B rows (output columns) of one K block
-  uint8_t stage_out[8][32 * 64];  // per consumer warp: 32 rows x 64 bytes, 64-byte swizzle
+  uint8_t stage_out[kStageBufs][8][32 * 64];  // per consumer warp: 32 rows x 64 bytes, 64-byte swizzle
   union {
     float sa[kScaleRing][128];  // scale_a of this CTA's rows, per K block
     // kFp8Mx, per four K blocks: three 512-byte scale-factor chunks (this
@@ -272,7 +291,7 @@ __global__ void __launch_bounds__(384, 1)
   static_assert(!MX || CG == 2, "hardware block scaling is built for CTA pairs");
   constexpr int CPC = 64 / sizeof(OutT);  // output columns per 64-byte staging row
   static_assert(CG == 1 || CG == 2, "CTA group is 1 or 2");
-  using Smem = WideSmem<BNL, STAGES>;
+  using Smem = WideSmem<BNL, STAGES, wide_stage_bufs<MODE, CG>()>;
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
@@ -622,7 +641,13 @@ __global__ void __launch_bounds__(384, 1)
     const int half = cw >> 2;
     const uint32_t t_lane = static_cast<uint32_t>(lg * 32) << 16;
     const int row = lg * 32 + lane;
-    uint8_t* stg = sm.stage_out[cw];
+    uint8_t* const stg0 = sm.stage_out[0][cw];  // this warp's (first) output staging buffer
+    // With two staging buffers (INT8 on CTA pairs) a warp's output chunks
+    // alternate between them, and every chunk commits exactly one bulk group
+    // (empty when its box lies outside the output), so "at most one group
+    // still reading" before a chunk means the buffer it is about to fill --
+    // used two chunks earlier -- is free.
+    int sbuf = 0;
     // release target of the accumulator buffers: the leader's barrier
     // release target of this warpgroup's accumulator half: the leader's barrier
     const uint32_t acc_empty0 =
@@ -774,11 +799,11 @@ __global__ void __launch_bounds__(384, 1)
           float v[CPC];
 #pragma unroll
           for (int j = 0; j < CPC; ++j) v[j] = acc[ch * CPC + j];
-          stage_row64<OutT, CPC>(stg, lane, v);
+          stage_row64<OutT, CPC>(stg0, lane, v);
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0 && m0 + lg * 32 < p.M && ncol0 + ch * CPC < p.N) {  // skip boxes wholly outside
-            tma_store_3d(&tmD, stg, ncol0 + ch * CPC, m0 + lg * 32, tc.g);
+            tma_store_3d(&tmD, stg0, ncol0 + ch * CPC, m0 + lg * 32, tc.g);
             bulk_commit();
           }
         }
@@ -846,7 +871,13 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int ch = 0; ch < NCH; ++ch) {
           if (!giver) {
-            if (lane == 0) bulk_wait_read_all();
+            if (lane == 0) {
+              if constexpr (Smem::kStageBufs == 2) {
+                bulk_wait_read1();
+              } else {
+                bulk_wait_read_all();
+              }
+            }
             __syncwarp();
           }
           const int c0 = (MX ? (ch + rot) % NCH : ch) * CPC;
@@ -904,13 +935,15 @@ __global__ void __launch_bounds__(384, 1)
               v[j] = f;
             }
           }
+          uint8_t* stg = stg0 + sbuf * static_cast<int>(sizeof(sm.stage_out[0]));
           stage_row64<OutT, CPC>(stg, lane, v);
           fence_proxy_async_smem();
           __syncwarp();
-          if (lane == 0 && m0 + lg * 32 < p.M && ncol0 + c0 < p.N) {
-            tma_store_3d(&tmD, stg, ncol0 + c0, m0 + lg * 32, tc.g);
+          if (lane == 0) {
+            if (m0 + lg * 32 < p.M && ncol0 + c0 < p.N) tma_store_3d(&tmD, stg, ncol0 + c0, m0 + lg * 32, tc.g);
             bulk_commit();
           }
+          if constexpr (Smem::kStageBufs == 2) sbuf ^= 1;
         }
         if (giver) {
           __threadfence();
