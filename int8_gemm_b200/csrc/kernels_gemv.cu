@@ -88,20 +88,43 @@ __global__ void __launch_bounds__(kGemvWarps * 32, KBS == 1 ? 4 : (KBS == 2 ? 2 
 #pragma unroll
     for (int i = 0; i < 4; ++i) acc[j][i] = 0.f;
 
-  // KBS K blocks per step, all of their loads in flight before the MMAs
+  // KBS K blocks per step: their operand and block-scale loads all in flight
+  // before the MMAs (a scale loaded after the MMAs would add its latency to
+  // every step)
   for (int kb0 = kb_lo; kb0 < kb_hi; kb0 += KBS) {
     uint4 wa[KBS][2], wb[KBS][2], xv[KBS][2][NT];
+    float sbk[KBS], sam[KBS][2];  // the block's weight scale; activation rows 2t, 2t + 1
 #pragma unroll
     for (int u = 0; u < KBS; ++u) {
-      const bool in = kb0 + u < kb_hi;
+      const int kb = kb0 + u;
+      const bool in = kb < kb_hi;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        const long long k = static_cast<long long>(kb0 + u) * 128 + 64 * h;
+        const long long k = static_cast<long long>(kb) * 128 + 64 * h;
         wa[u][h] = in && ok0 ? __ldg(reinterpret_cast<const uint4*>(w0 + k)) : make_uint4(0, 0, 0, 0);
         wb[u][h] = in && ok1 ? __ldg(reinterpret_cast<const uint4*>(w1 + k)) : make_uint4(0, 0, 0, 0);
 #pragma unroll
         for (int j = 0; j < NT; ++j)
           xv[u][h][j] = in && oka[j] ? __ldg(reinterpret_cast<const uint4*>(xa[j] + k)) : make_uint4(0, 0, 0, 0);
+      }
+      if constexpr (MODE == Mode::kFp8F32Scale) {
+        sbk[u] = in && nb < p.NB ? __ldg(p.sb + static_cast<long long>(kb) * p.sb_sk + static_cast<long long>(nb) * p.sb_sn)
+                                 : 0.f;
+      } else {
+        sbk[u] = in && nb < p.NB ? e8m0_to_f32(__ldg(p.ws + (static_cast<long long>(g) * p.NB + nb) * p.KB + kb)) : 0.f;
+      }
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const int m = 2 * t + c;
+        float v = 0.f;
+        if (in && m < p.M) {
+          if constexpr (MODE == Mode::kFp8F32Scale) {
+            v = __ldg(p.sa + static_cast<long long>(m) * p.sa_sm + static_cast<long long>(kb) * p.sa_sk);
+          } else {
+            v = e8m0_to_f32(__ldg(p.xs + (static_cast<long long>(m) * p.G + g) * p.KB + kb));
+          }
+        }
+        sam[u][c] = v;
       }
     }
 #pragma unroll
@@ -126,32 +149,13 @@ __global__ void __launch_bounds__(kGemvWarps * 32, KBS == 1 ? 4 : (KBS == 2 ? 2 
           mma_e4m3_16x8x32(part[j], hi, xv[u][h][j].z, xv[u][h][j].w);
         }
       }
-      // promotion: part[j][i] is row (gr or gr + 8) x activation row
-      // m = 8 j + 2 t + (i & 1) of this block's partial
-      float sbk;
-      if constexpr (MODE == Mode::kFp8F32Scale) {
-        sbk = nb < p.NB ? __ldg(p.sb + static_cast<long long>(kb) * p.sb_sk + static_cast<long long>(nb) * p.sb_sn)
-                        : 0.f;
-      } else {
-        sbk = nb < p.NB ? e8m0_to_f32(__ldg(p.ws + (static_cast<long long>(g) * p.NB + nb) * p.KB + kb)) : 0.f;
-      }
+      // promotion: part[0][i] is row (gr or gr + 8) x activation row
+      // m = 2 t + (i & 1) of this block's partial
 #pragma unroll
-      for (int j = 0; j < NT; ++j) {
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          const int m = 8 * j + 2 * t + c;
-          float sam = 0.f;
-          if (m < p.M) {
-            if constexpr (MODE == Mode::kFp8F32Scale) {
-              sam = __ldg(p.sa + static_cast<long long>(m) * p.sa_sm + static_cast<long long>(kb) * p.sa_sk);
-            } else {
-              sam = e8m0_to_f32(__ldg(p.xs + (static_cast<long long>(m) * p.G + g) * p.KB + kb));
-            }
-          }
-          const float s = sam * sbk;
-          acc[j][c] = fmaf(s, part[j][c], acc[j][c]);
-          acc[j][2 + c] = fmaf(s, part[j][2 + c], acc[j][2 + c]);
-        }
+      for (int c = 0; c < 2; ++c) {
+        const float s = sam[u][c] * sbk[u];
+        acc[0][c] = fmaf(s, part[0][c], acc[0][c]);
+        acc[0][2 + c] = fmaf(s, part[0][2 + c], acc[0][2 + c]);
       }
     }
   }
