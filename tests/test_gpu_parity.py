@@ -176,7 +176,7 @@ def oracle_rowwise(d, bias=True, rows=None):
 
 
 @pytest.mark.parametrize("M,N,K", [(256, 256, 512), (300, 520, 640), (1, 256, 128), (129, 384, 176), (640, 1280, 1024),
-                                   (5, 259, 48)])
+                                   (5, 259, 48), (2300, 2100, 256)])
 @pytest.mark.parametrize("tensorwise", [False, True])
 @pytest.mark.parametrize("kernel", [bs.PATH_AUTO, bs.PATH_WIDE_SINGLE])
 def test_fp8_rowwise_and_tensorwise(M, N, K, tensorwise, kernel, path):
@@ -274,8 +274,10 @@ def _int8_assert(d, rows, s_b=True):
     np.testing.assert_array_equal(bf16_bits(sel(int8_run(d, torch.bfloat16, s_b))), bf)
 
 
+# (2300, 2100, 512): 81 ragged tiles, so some CTA pairs run two tiles and reuse their staging buffers and
+# staged column scales across tiles
 @pytest.mark.parametrize("M,N,K", [(128, 256, 128), (300, 520, 1040), (1, 256, 4096), (257, 264, 48),
-                                   (600, 1024, 2048)])
+                                   (600, 1024, 2048), (2300, 2100, 512)])
 @pytest.mark.parametrize("kernel", [bs.PATH_WIDE, bs.PATH_WIDE_SINGLE])
 def test_int8_bit_exact_small(M, N, K, kernel, path):
     path(kernel)
