@@ -73,7 +73,7 @@ KERNEL_SOURCES = {
     "skinny": ["sm100.cuh", "tile_order.h", "wide_kernel.cuh", "skinny_kernel.cuh", "kernels_skinny.cu", "launch.h"],
     "gemv": ["sm100.cuh", "tile_order.h", "wide_kernel.cuh", "skinny_kernel.cuh", "kernels_gemv.cu", "launch.h"],
     "quantize": ["group_quant.cuh", "quantize.h", "kernels_quantize.cu"],
-    "quantize_t": ["group_quant.cuh", "quantize.h", "kernels_quantize_t.cu"],
+    "quantize_t": ["sm100.cuh", "group_quant.cuh", "quantize.h", "kernels_quantize_t.cu"],
     "quantize_blocks": ["group_quant.cuh", "quantize.h", "kernels_quantize_blocks.cu"],
 }
 

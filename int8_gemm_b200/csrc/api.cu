@@ -744,8 +744,26 @@ bs_status bs_quantize_fp8_t(const void* x, bs_in_dtype x_dtype, int64_t R, int64
   DeviceCtx* dc = nullptr;
   bs_status st = device_ctx(&dc);
   if (st != BS_OK) return st;
+  // The TMA-fed kernel where x and q_t allow tensor copies: 16-byte bases and row strides, and rows whose
+  // used bytes (C elements of x, R codes of q_t) end on a 16-byte boundary.  (A tensor store of a last row
+  // tile that ended inside a 16-byte piece, R = 260, wrote bytes past R.)
+  CUtensorMap tmx, tmq;
+  const bool tma = aligned16(x) && (ldx * static_cast<int64_t>(es)) % 16 == 0 && (C * static_cast<int64_t>(es)) % 16 == 0 &&
+                   aligned16(q_t) && ldq % 16 == 0 && R % 16 == 0;
+  if (tma) {
+    st = encode_3d(&tmx, x_dtype == BS_IN_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                   static_cast<int>(es), x, static_cast<uint64_t>(C), static_cast<uint64_t>(R), 1,
+                   static_cast<uint64_t>(ldx), static_cast<uint64_t>(ldx) * static_cast<uint64_t>(R), 128, 128, "x",
+                   CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (st != BS_OK) return st;
+    st = encode_3d(&tmq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, q_t, static_cast<uint64_t>(R), static_cast<uint64_t>(C), 1,
+                   static_cast<uint64_t>(ldq), static_cast<uint64_t>(ldq) * static_cast<uint64_t>(C), 128, 128, "q_t",
+                   CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != BS_OK) return st;
+  }
   return check_launch(launch_quantize_t(x, x_dtype == BS_IN_BF16, R, C, ldx, static_cast<uint8_t*>(q_t), ldq, scale,
                                         scale_fmt == BS_SCALE_E8M0, group == BS_GROUP_128x128, ld_scale, dc->sms,
+                                        tma ? &tmx : nullptr, tma ? &tmq : nullptr, dc->err,
                                         static_cast<cudaStream_t>(stream)),
                       "transposed quantise launch");
 }

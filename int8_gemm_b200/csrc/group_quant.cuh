@@ -74,6 +74,31 @@ __device__ __forceinline__ void code_quotients(const float (&v)[N], float s, flo
   }
 }
 
+// y[i] = (fp32(v[i].x / s0), fp32(v[i].y / s1)) for N elements of two groups
+// side by side (two columns, scales s0 and s1): quotient_rn on both lanes of
+// the packed two-wide fp32 operations, under code_quotients' warp-uniform
+// range test.  (-q1 * s and q1 * -s are the same exact product, so the
+// residual is quotient_rn's.)
+template <int N>
+__device__ __forceinline__ void code_quotients2(const float2 (&v)[N], float s0, float s1, float2 (&y)[N]) {
+  const bool fast = s0 >= 0x1p-90f && s0 <= 3.40282347e38f && s1 >= 0x1p-90f && s1 <= 3.40282347e38f;
+  if (__all_sync(__activemask(), fast)) {
+    const float2 r = make_float2(__frcp_rn(s0), __frcp_rn(s1));
+    const float2 ns = make_float2(-s0, -s1);
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+      const float2 q1 = __fmul2_rn(v[i], r);
+      const float2 rem = __ffma2_rn(q1, ns, v[i]);
+      const float2 q = __ffma2_rn(rem, r, q1);
+      y[i] = make_float2(copysignf(q.x, v[i].x), copysignf(q.y, v[i].y));
+    }
+  } else {
+    const double r0 = __drcp_rn(static_cast<double>(s0)), r1 = __drcp_rn(static_cast<double>(s1));
+#pragma unroll
+    for (int i = 0; i < N; ++i) y[i] = make_float2(over_scale(v[i].x, r0), over_scale(v[i].y, r1));
+  }
+}
+
 // The e8m0 byte: ceil(log2(amax / 448)) from amax = f * 2^ex, f in [0.5, 1):
 // with 448 = 0.875 * 2^9 it is ex - 9, plus one when f > 0.875.
 __device__ __forceinline__ int group_e8m0(float amax) {

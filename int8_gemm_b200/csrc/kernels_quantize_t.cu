@@ -31,6 +31,7 @@
 
 #include "group_quant.cuh"
 #include "quantize.h"
+#include "sm100.cuh"
 
 namespace bsg {
 
@@ -252,11 +253,259 @@ cudaError_t launch_t_fmt(const void* x, long long R, long long C, long long ldx,
               : launch_t<InT, 0, 0>(x, R, C, ldx, q, ldq, scale, lds, sms, stream);
 }
 
+// ---------------------------------------------------------------------------
+// TMA-fed form (x and q_t both 16-byte aligned with 16-byte row strides)
+// ---------------------------------------------------------------------------
+// One CTA of 512 threads per SM, persistent over 128 x 128 tiles.  One thread
+// keeps a ring of kTmaStages tiles in flight with 2-D tensor copies (rows and
+// columns past the matrix arrive as zeros), so no thread spends instructions
+// or registers on loads.  Thread t owns the column pair 2 (t % 64), + 1 and
+// the 16 rows 16 (t / 64) .. + 15: it reads its 16 pairs from the tile once
+// (one 4- or 8-byte shared load each, a warp reading 128 or 256 contiguous
+// bytes), takes their amax in registers (bf16: one packed max of magnitudes
+// per pair), and after the amaxes meet in shared memory quantises the values
+// it still holds.  Its 2 x 16 codes go as two 16-byte pieces into a shared
+// [column][row] code tile laid out in the 128-byte swizzle, which one thread
+// then writes to q_t with a tensor store that clips at R and C.
+constexpr int kTmaThreads = 512;
+constexpr int kTmaParts = kTmaThreads / (kTile / 2);  // row groups per column pair
+constexpr int kTmaRows = kTile / kTmaParts;           // rows per thread
+static_assert(kTmaRows == 16, "a thread's codes of one column are one 16-byte piece");
+
+template <typename InT>
+struct TmaRing {
+  static constexpr int kStages = sizeof(InT) == 2 ? 4 : 3;  // input tiles (32 or 64 KB each)
+  static constexpr int kCodeBufs = sizeof(InT) == 2 ? 2 : 1;  // code tiles (16 KB each)
+};
+
+template <typename InT>
+struct TmaSmem {
+  alignas(1024) InT v[TmaRing<InT>::kStages][kTile][kTile];       // input tiles, [row][column]
+  alignas(1024) uint8_t codes[TmaRing<InT>::kCodeBufs][kTile][kTile];  // [column][row], 128-byte swizzle
+  float2 part[kTmaParts][kTile / 2];  // amaxes of each row group's column pairs
+  float wmax[kTmaThreads / 32];
+  uint64_t full[TmaRing<InT>::kStages];
+  int abort;
+};
+
+// Magnitude-wise max of two bf16 pairs; the result's sign bits are not
+// meaningful (callers clear them).
+__device__ __forceinline__ uint32_t max_abs_bf16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+// This thread's 16 pairs of the tile in stage `st`, widened to fp32, and
+// their two column amaxes.
+__device__ __forceinline__ void load_pairs(const TmaSmem<__nv_bfloat16>& sm, int st, int r0, int p, float2 (&e)[kTmaRows],
+                                           float& amax0, float& amax1) {
+  uint32_t w[kTmaRows];
+#pragma unroll
+  for (int i = 0; i < kTmaRows; ++i) w[i] = *reinterpret_cast<const uint32_t*>(&sm.v[st][r0 + i][2 * p]);
+  uint32_t m = 0;
+#pragma unroll
+  for (int i = 0; i < kTmaRows; ++i) m = max_abs_bf16x2(m, w[i]);
+  amax0 = __uint_as_float((m << 16) & 0x7FFFFFFFu);
+  amax1 = __uint_as_float(m & 0x7FFF0000u);
+#pragma unroll
+  for (int i = 0; i < kTmaRows; ++i) e[i] = make_float2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
+}
+__device__ __forceinline__ void load_pairs(const TmaSmem<float>& sm, int st, int r0, int p, float2 (&e)[kTmaRows],
+                                           float& amax0, float& amax1) {
+#pragma unroll
+  for (int i = 0; i < kTmaRows; ++i) e[i] = *reinterpret_cast<const float2*>(&sm.v[st][r0 + i][2 * p]);
+  amax0 = amax1 = 0.f;
+#pragma unroll
+  for (int i = 0; i < kTmaRows; ++i) {
+    amax0 = fmaxf(amax0, fabsf(e[i].x));
+    amax1 = fmaxf(amax1, fabsf(e[i].y));
+  }
+}
+
+// 16 codes of one column (lane h of y) as a 16-byte piece.
+__device__ __forceinline__ uint4 pack_column(const float2 (&y)[kTmaRows], int h) {
+  uint32_t w[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float a = h ? y[4 * j].y : y[4 * j].x, b = h ? y[4 * j + 1].y : y[4 * j + 1].x;
+    const float c = h ? y[4 * j + 2].y : y[4 * j + 2].x, d = h ? y[4 * j + 3].y : y[4 * j + 3].x;
+    w[j] = e4m3x2(a, b) | (e4m3x2(c, d) << 16);
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+template <typename InT, int FMT, int GROUP>
+__global__ void __launch_bounds__(kTmaThreads, 1)
+    quantize_t_tma_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmq, long long R,
+                          long long C, void* __restrict__ scale, long long lds, long long ctiles, long long ntiles,
+                          uint32_t* err) {
+  using S = TmaSmem<InT>;
+  constexpr int kStages = TmaRing<InT>::kStages, kCodeBufs = TmaRing<InT>::kCodeBufs;
+  constexpr uint32_t kTileBytes = kTile * kTile * sizeof(InT);
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+  if (pad + sizeof(S) > dynamic_smem_bytes()) {  // never touch memory the launch did not provide
+    if (threadIdx.x == 0) record_error(err, kErrSmemTooSmall);
+    return;
+  }
+  S& sm = *reinterpret_cast<S*>(smem_raw + pad);
+  const int t = threadIdx.x;
+  const int cp = t % (kTile / 2);  // column pair
+  const int qr = t / (kTile / 2);  // row group: rows kTmaRows * qr ..
+  if (t == 0) {
+    for (int s = 0; s < kStages; ++s) mbar_init(&sm.full[s], 1);
+    sm.abort = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmx);
+    tma_prefetch_desc(&tmq);
+  }
+  __syncthreads();
+  auto issue = [&](long long tile, int s) {
+    const long long rb = tile / ctiles, cb = tile - rb * ctiles;
+    mbar_arrive_expect_tx(&sm.full[s], kTileBytes);
+    tma_load_3d(&sm.v[s][0][0], &tmx, &sm.full[s], static_cast<int>(cb * kTile), static_cast<int>(rb * kTile), 0);
+  };
+  if (t == 0)
+    for (int s = 0; s < kStages; ++s) {
+      const long long tile = blockIdx.x + static_cast<long long>(s) * gridDim.x;
+      if (tile < ntiles) issue(tile, s);
+    }
+  int it = 0;
+  bool ok = true;
+  for (long long tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
+    const int st = it % kStages, cbuf = it % kCodeBufs;
+    const long long rb = tile / ctiles, cb = tile - rb * ctiles;
+    const bool got = wait_bounded(&sm.full[st], static_cast<uint32_t>(it / kStages) & 1u, &sm.abort, err,
+                                  kErrTimeout | kRoleConsumer | kWaitStageFull);
+    float2 e[kTmaRows];
+    float amax0, amax1;
+    load_pairs(sm, st, kTmaRows * qr, cp, e, amax0, amax1);
+    if constexpr (GROUP == 0) {
+      sm.part[qr][cp] = make_float2(amax0, amax1);
+    } else {
+      float a = fmaxf(amax0, amax1);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
+      if ((t & 31) == 0) sm.wmax[t / 32] = a;
+    }
+    // the code tile written kCodeBufs tiles ago has been read by its store
+    if (t == 0) {
+      if constexpr (kCodeBufs == 2) {
+        bulk_wait_read1();
+      } else {
+        bulk_wait_read_all();
+      }
+    }
+    // every thread holds its values: the stage can be refilled
+    ok = __syncthreads_and(got) != 0;
+    if (!ok) break;
+    if (t == 0) {
+      const long long next = tile + static_cast<long long>(kStages) * gridDim.x;
+      if (next < ntiles) {
+        fence_proxy_async_smem();
+        issue(next, st);
+      }
+    }
+    if constexpr (GROUP == 0) {
+#pragma unroll
+      for (int k = 0; k < kTmaParts; ++k) {
+        const float2 pk = sm.part[k][cp];
+        amax0 = fmaxf(amax0, pk.x);
+        amax1 = fmaxf(amax1, pk.y);
+      }
+    } else {
+      float a = sm.wmax[0];
+#pragma unroll
+      for (int w = 1; w < kTmaThreads / 32; ++w) a = fmaxf(a, sm.wmax[w]);
+      amax0 = amax1 = a;
+    }
+    const long long ca = cb * kTile + 2 * cp;  // this thread's first column of x
+    float2 y[kTmaRows];
+    if constexpr (FMT == 0) {
+      const float s0 = group_scale_f32(amax0), s1 = group_scale_f32(amax1);
+      if constexpr (GROUP == 0) {
+        if (qr == 0) {
+          if (ca < C) static_cast<float*>(scale)[ca * lds + rb] = s0;
+          if (ca + 1 < C) static_cast<float*>(scale)[(ca + 1) * lds + rb] = s1;
+        }
+      } else if (t == 0) {
+        static_cast<float*>(scale)[rb * lds + cb] = s0;
+      }
+      code_quotients2<kTmaRows>(e, s0, s1, y);
+    } else {
+      const int byte0 = group_e8m0(amax0), byte1 = group_e8m0(amax1);
+      if constexpr (GROUP == 0) {
+        if (qr == 0) {
+          if (ca < C) static_cast<uint8_t*>(scale)[ca * lds + rb] = static_cast<uint8_t>(byte0);
+          if (ca + 1 < C) static_cast<uint8_t*>(scale)[(ca + 1) * lds + rb] = static_cast<uint8_t>(byte1);
+        }
+      } else if (t == 0) {
+        static_cast<uint8_t*>(scale)[rb * lds + cb] = static_cast<uint8_t>(byte0);
+      }
+      const float2 mul = make_float2(ldexpf(1.f, 127 - byte0), ldexpf(1.f, 127 - byte1));  // exact powers of two
+#pragma unroll
+      for (int i = 0; i < kTmaRows; ++i) y[i] = __fmul2_rn(e[i], mul);
+    }
+    // code tile rows 2 cp and 2 cp + 1, 16-byte piece qr (swizzled by the row)
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int c = 2 * cp + h;
+      *reinterpret_cast<uint4*>(&sm.codes[cbuf][c][(qr ^ (c & 7)) * 16]) = pack_column(y, h);
+    }
+    fence_proxy_async_smem();  // the code tile, before the tensor store reads it
+    __syncthreads();
+    if (t == 0) {
+      tma_store_3d(&tmq, &sm.codes[cbuf][0][0], static_cast<int>(rb * kTile), static_cast<int>(cb * kTile), 0);
+      bulk_commit();
+    }
+  }
+  if (t == 0) {
+    bulk_wait_all();
+    if (!ok) {  // a wait gave up: let the copies still in flight land before the CTA retires
+      volatile int never = 0;
+      for (int j = it; j < it + kStages; ++j) {
+        const long long tile = blockIdx.x + static_cast<long long>(j) * gridDim.x;
+        if (tile < ntiles) wait_bounded(&sm.full[j % kStages], static_cast<uint32_t>(j / kStages) & 1u, &never, nullptr, 0);
+      }
+    }
+  }
+}
+
+template <typename InT, int FMT, int GROUP>
+cudaError_t launch_t_tma(const CUtensorMap& tmx, const CUtensorMap& tmq, long long R, long long C, void* scale,
+                         long long lds, int sms, uint32_t* err, cudaStream_t stream) {
+  const long long ctiles = (C + kTile - 1) / kTile;
+  const long long ntiles = ((R + kTile - 1) / kTile) * ctiles;
+  const size_t smem = sizeof(TmaSmem<InT>) + 1024;
+  cudaError_t e = cudaFuncSetAttribute(quantize_t_tma_kernel<InT, FMT, GROUP>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  long long blocks = sms > 0 ? sms : 148;
+  if (blocks > ntiles) blocks = ntiles;
+  quantize_t_tma_kernel<InT, FMT, GROUP><<<static_cast<unsigned>(blocks), kTmaThreads, smem, stream>>>(
+      tmx, tmq, R, C, scale, lds, ctiles, ntiles, err);
+  return cudaGetLastError();
+}
+
+template <typename InT>
+cudaError_t launch_t_tma_fmt(const CUtensorMap& tmx, const CUtensorMap& tmq, long long R, long long C, void* scale,
+                             bool e8m0, bool block, long long lds, int sms, uint32_t* err, cudaStream_t stream) {
+  if (block)
+    return e8m0 ? launch_t_tma<InT, 1, 1>(tmx, tmq, R, C, scale, lds, sms, err, stream)
+                : launch_t_tma<InT, 0, 1>(tmx, tmq, R, C, scale, lds, sms, err, stream);
+  return e8m0 ? launch_t_tma<InT, 1, 0>(tmx, tmq, R, C, scale, lds, sms, err, stream)
+              : launch_t_tma<InT, 0, 0>(tmx, tmq, R, C, scale, lds, sms, err, stream);
+}
+
 }  // namespace
 
 cudaError_t launch_quantize_t(const void* x, bool x_bf16, long long R, long long C, long long ldx, uint8_t* q_t,
                               long long ldq, void* scale, bool e8m0, bool block128, long long lds, int sms,
-                              cudaStream_t stream) {
+                              const CUtensorMap* tmx, const CUtensorMap* tmq, uint32_t* err, cudaStream_t stream) {
+  if (tmx && tmq)
+    return x_bf16 ? launch_t_tma_fmt<__nv_bfloat16>(*tmx, *tmq, R, C, scale, e8m0, block128, lds, sms, err, stream)
+                  : launch_t_tma_fmt<float>(*tmx, *tmq, R, C, scale, e8m0, block128, lds, sms, err, stream);
   return x_bf16 ? launch_t_fmt<__nv_bfloat16>(x, R, C, ldx, q_t, ldq, scale, e8m0, block128, lds, sms, stream)
                 : launch_t_fmt<float>(x, R, C, ldx, q_t, ldq, scale, e8m0, block128, lds, sms, stream);
 }

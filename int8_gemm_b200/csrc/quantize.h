@@ -3,6 +3,7 @@
 // Not part of the public header.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -20,9 +21,13 @@ cudaError_t launch_quantize_1x128(const void* x, bool x_bf16, long long M, long 
 // code of x[r][c].  block128 = false: 128x1 groups (rows 128rb.. of one
 // column), scale [C, ceil(R/128)]; true: 128x128 blocks, scale
 // [ceil(R/128), ceil(C/128)]; scale row stride lds, fp32 or e8m0 bytes.
+// tmx / tmq: tensor maps of x (box 128 x 128, no swizzle) and q_t (box 128 x
+// 128 bytes, 128-byte swizzle), or null where x or q_t is not 16-byte aligned
+// with a 16-byte row stride; with both given the TMA-fed kernel runs, whose
+// bounded waits record a timeout in the device error word `err`.
 cudaError_t launch_quantize_t(const void* x, bool x_bf16, long long R, long long C, long long ldx, uint8_t* q_t,
                               long long ldq, void* scale, bool e8m0, bool block128, long long lds, int sms,
-                              cudaStream_t stream);
+                              const CUtensorMap* tmx, const CUtensorMap* tmq, uint32_t* err, cudaStream_t stream);
 
 // 128x128 block quantisation of x [R, C] (bf16 or fp32, row stride ldx
 // elements) in its own orientation: codes q [R, C] (row stride ldq bytes),

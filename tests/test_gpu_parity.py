@@ -430,7 +430,10 @@ def _quant_t_check(x_dev, group, fmt, **kw):
     return qt, s
 
 
-@pytest.mark.parametrize("R,C", [(1, 1), (128, 128), (300, 5), (5, 300), (130, 260), (1000, 384), (4096, 640)])
+# (128, 128), (4096, 640), (1040, 264), (272, 8) and (16, 1000) have 16-byte row strides in x and q_t, so the
+# TMA-fed kernel runs them (the last three with ragged tiles); the others take the kernel with plain loads
+@pytest.mark.parametrize("R,C", [(1, 1), (128, 128), (300, 5), (5, 300), (130, 260), (1000, 384), (4096, 640),
+                                 (1040, 264), (272, 8), (16, 1000)])
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
 @pytest.mark.parametrize("group", ["128x1", "128x128"])
 @pytest.mark.parametrize("fmt", [0, 1])
@@ -441,8 +444,11 @@ def test_quantize_t_bit_exact(R, C, dtype, group, fmt):
 
 @pytest.mark.parametrize("group", ["128x1", "128x128"])
 @pytest.mark.parametrize("fmt", [0, 1])
-def test_quantize_t_special_blocks_strides_and_canaries(group, fmt):
-    R, C = 260, 136
+# (144, 272): 16-byte rows and R a multiple of 16, the TMA-fed kernel (its tensor store must stop at R inside the
+# 288-byte rows); (141, 260) and (144, 260) take the kernel with plain loads and stores
+@pytest.mark.parametrize("x_stride,R", [(141, 260), (144, 260), (144, 272)])
+def test_quantize_t_special_blocks_strides_and_canaries(group, fmt, x_stride, R):
+    C = 136
     x = wl.normal_with_outliers((R, C), 7500)
     x[:128, :128] = 0.0                                  # an all-zero block / columns
     x[128:256, 0] = 448.0 * 2.0 ** 5                     # amax exactly 448 * 2^5
@@ -450,16 +456,27 @@ def test_quantize_t_special_blocks_strides_and_canaries(group, fmt):
     x[256:, 5] = 1e-30                                   # tiny values
     x[3, 130] = 3e20                                     # one huge value
     x[:128, 133] = 3e-44 * torch.linspace(-1.0, 1.0, 128)  # a 128x1 group whose amax / 448 underflows
-    base = torch.zeros(R, 141)                           # row stride 141: no 16-byte loads
+    base = torch.zeros(R, x_stride)                      # row stride 141: no 16-byte loads
     base[:, :C] = x
     xv = base.to(DEV)[:, :C]
-    q = torch.full((C, 288), 0x55, dtype=torch.uint8, device=DEV)[:, :R]  # rows of 288 bytes, R = 260 used
+    q = torch.full((C, 288), 0x55, dtype=torch.uint8, device=DEV)[:, :R]  # rows of 288 bytes, R used
     sshape = (C, 3) if group == "128x1" else (3, 2)
     s = torch.zeros((sshape[0], sshape[1] + 3), dtype=torch.float32 if fmt == 0 else torch.uint8,
                     device=DEV)[:, :sshape[1]]
     _quant_t_check(xv, group, fmt, q_t=q, scale=s)
     full = torch.as_strided(q, (C, 288), (288, 1))
     assert torch.all(full[:, R:] == 0x55), "wrote past R"
+
+
+@pytest.mark.parametrize("group", ["128x1", "128x128"])
+def test_quantize_t_reads_no_column_past_c(group):
+    """x rows of 16-byte strides whose C columns end inside a 16-byte piece: the columns between C and the
+    stride hold huge values, which must not reach a 128x128 block's amax."""
+    R, C, ld = 256, 132, 136
+    base = torch.full((R, ld), 1e30)
+    base[:, :C] = wl.normal_with_outliers((R, C), 7550)
+    xv = base.to(torch.bfloat16).to(DEV)[:, :C]
+    _quant_t_check(xv, group, 0)
 
 
 def test_quantize_t_full_size_output_gradient():
