@@ -74,7 +74,7 @@ KERNEL_SOURCES = {
     "gemv": ["sm100.cuh", "tile_order.h", "wide_kernel.cuh", "skinny_kernel.cuh", "kernels_gemv.cu", "launch.h"],
     "quantize": ["group_quant.cuh", "quantize.h", "kernels_quantize.cu"],
     "quantize_t": ["sm100.cuh", "group_quant.cuh", "quantize.h", "kernels_quantize_t.cu"],
-    "quantize_blocks": ["group_quant.cuh", "quantize.h", "kernels_quantize_blocks.cu"],
+    "quantize_blocks": ["sm100.cuh", "group_quant.cuh", "quantize.h", "kernels_quantize_blocks.cu"],
 }
 
 

@@ -789,9 +789,24 @@ bs_status bs_quantize_fp8_128x128(const void* x, bs_in_dtype x_dtype, int64_t R,
   DeviceCtx* dc = nullptr;
   bs_status st = device_ctx(&dc);
   if (st != BS_OK) return st;
+  // the TMA-fed kernel where x and q allow tensor copies whose rows end on 16-byte boundaries
+  CUtensorMap tmx, tmq;
+  const bool tma = aligned16(x) && (ldx * static_cast<int64_t>(es)) % 16 == 0 && C % 16 == 0 && aligned16(q) &&
+                   ldq % 16 == 0;
+  if (tma) {
+    st = encode_3d(&tmx, x_dtype == BS_IN_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                   static_cast<int>(es), x, static_cast<uint64_t>(C), static_cast<uint64_t>(R), 1,
+                   static_cast<uint64_t>(ldx), static_cast<uint64_t>(ldx) * static_cast<uint64_t>(R), 128, 128, "x",
+                   CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (st != BS_OK) return st;
+    st = encode_3d(&tmq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, q, static_cast<uint64_t>(C), static_cast<uint64_t>(R), 1,
+                   static_cast<uint64_t>(ldq), static_cast<uint64_t>(ldq) * static_cast<uint64_t>(R), 128, 128, "q",
+                   CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (st != BS_OK) return st;
+  }
   return check_launch(launch_quantize_blocks(x, x_dtype == BS_IN_BF16, R, C, ldx, static_cast<uint8_t*>(q), ldq, scale,
-                                             scale_fmt == BS_SCALE_E8M0, s_rb, s_cb, dc->sms,
-                                             static_cast<cudaStream_t>(stream)),
+                                             scale_fmt == BS_SCALE_E8M0, s_rb, s_cb, dc->sms, tma ? &tmx : nullptr,
+                                             tma ? &tmq : nullptr, dc->err, static_cast<cudaStream_t>(stream)),
                       "block quantise launch");
 }
 

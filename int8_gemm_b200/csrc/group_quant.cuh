@@ -99,6 +99,15 @@ __device__ __forceinline__ void code_quotients2(const float2 (&v)[N], float s0, 
   }
 }
 
+// Lane-wise magnitude max of two bf16 pairs (exact: the result is one of the
+// inputs' magnitudes); the result's sign bits are not meaningful, callers
+// clear them.
+__device__ __forceinline__ uint32_t max_abs_bf16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
 // The e8m0 byte: ceil(log2(amax / 448)) from amax = f * 2^ex, f in [0.5, 1):
 // with 448 = 0.875 * 2^9 it is ex - 9, plus one when f > 0.875.
 __device__ __forceinline__ int group_e8m0(float amax) {

@@ -288,14 +288,6 @@ struct TmaSmem {
   int abort;
 };
 
-// Magnitude-wise max of two bf16 pairs; the result's sign bits are not
-// meaningful (callers clear them).
-__device__ __forceinline__ uint32_t max_abs_bf16x2(uint32_t a, uint32_t b) {
-  uint32_t d;
-  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-  return d;
-}
-
 // This thread's 16 pairs of the tile in stage `st`, widened to fp32, and
 // their two column amaxes.
 __device__ __forceinline__ void load_pairs(const TmaSmem<__nv_bfloat16>& sm, int st, int r0, int p, float2 (&e)[kTmaRows],

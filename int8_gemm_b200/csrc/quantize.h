@@ -33,8 +33,13 @@ cudaError_t launch_quantize_t(const void* x, bool x_bf16, long long R, long long
 // elements) in its own orientation: codes q [R, C] (row stride ldq bytes),
 // q[r][c] the code of x[r][c], one scale per block (rb, cb) at
 // scale[rb * s_rb + cb * s_cb] (element strides), fp32 or e8m0 bytes.
+// tmx / tmq: tensor maps of x and q (box 128 x 128, no swizzle), or null where
+// x or q is not 16-byte aligned with 16-byte row strides or C is not a
+// multiple of 16; with both given the TMA-fed kernel runs, whose bounded
+// waits record a timeout in the device error word `err`.
 cudaError_t launch_quantize_blocks(const void* x, bool x_bf16, long long R, long long C, long long ldx, uint8_t* q,
                                    long long ldq, void* scale, bool e8m0, long long s_rb, long long s_cb, int sms,
+                                   const CUtensorMap* tmx, const CUtensorMap* tmq, uint32_t* err,
                                    cudaStream_t stream);
 
 }  // namespace bsg

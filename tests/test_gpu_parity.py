@@ -554,7 +554,10 @@ def _quant_b_check(x_dev, fmt, **kw):
     return q, s
 
 
-@pytest.mark.parametrize("R,C", [(1, 1), (128, 128), (300, 5), (5, 300), (130, 260), (1000, 384), (384, 4104)])
+# (128, 128), (1000, 384), (1040, 272) and (16, 1008) have 16-byte row strides and C a multiple of 16, so the
+# TMA-fed kernel runs them (the last three with ragged tiles); the others take the kernel with plain loads
+@pytest.mark.parametrize("R,C", [(1, 1), (128, 128), (300, 5), (5, 300), (130, 260), (1000, 384), (384, 4104),
+                                 (1040, 272), (16, 1008)])
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
 @pytest.mark.parametrize("fmt", [0, 1])
 def test_quantize_128x128_bit_exact(R, C, dtype, fmt):
@@ -563,15 +566,19 @@ def test_quantize_128x128_bit_exact(R, C, dtype, fmt):
 
 
 @pytest.mark.parametrize("fmt", [0, 1])
-def test_quantize_128x128_special_blocks_strides_and_canaries(fmt):
-    R, C = 260, 300
+# (320, 304): 16-byte rows and C a multiple of 16, the TMA-fed kernel (its tensor store must stop at C inside the
+# 320-byte rows of q); (303, 300) takes the kernel with plain loads and stores.  The columns of x past C hold
+# huge values, which must not reach a block's amax.
+@pytest.mark.parametrize("x_stride,C", [(303, 300), (320, 304)])
+def test_quantize_128x128_special_blocks_strides_and_canaries(fmt, x_stride, C):
+    R = 260
     x = wl.normal_with_outliers((R, C), 9500)
     x[:128, :128] = 0.0                                   # an all-zero block
     x[:128, 128:256] = 3e-44 * torch.linspace(-1.0, 1.0, 128)[None, :]  # amax / 448 underflows: scale 1
     x[128:256, :128] = torch.linspace(-1.0, 1.0, 128)[:, None] * 448.0 * 2.0 ** 5  # amax exactly 448 * 2^5
     x[256:, 7] = 1e-30                                    # tiny values
     x[200, 290] = 3e20                                    # one huge value
-    base = torch.zeros(R, 303)                            # row stride 303: no 16-byte loads
+    base = torch.full((R, x_stride), 1e30)                # row stride 303: no 16-byte loads
     base[:, :C] = x
     xv = base.to(DEV)[:, :C]
     q = torch.full((R, 320), 0x55, dtype=torch.uint8, device=DEV)[:, :C]
