@@ -299,6 +299,28 @@ bs_status encode_3d(CUtensorMap* map, CUtensorMapDataType dt, int esize, const v
   return BS_OK;
 }
 
+// Tensor maps of a quantiser's input x and codes q, both [R, C] in their own
+// orientation (128 x 128 boxes; x without swizzle, q with the 128-byte
+// swizzle of the kernels' code tiles), for the TMA-fed kernels; `tma`
+// is false (and nothing is encoded) unless x and q have 16-byte bases and row
+// strides and C is a multiple of 16, so that no row ends inside a 16-byte
+// piece.
+bs_status encode_quant_maps(const void* x, bs_in_dtype x_dtype, int64_t R, int64_t C, int64_t ldx, const void* q,
+                            int64_t ldq, CUtensorMap* tmx, CUtensorMap* tmq, bool* tma) {
+  const int es = x_dtype == BS_IN_BF16 ? 2 : 4;
+  *tma = (reinterpret_cast<uintptr_t>(x) & 15u) == 0 && (ldx * es) % 16 == 0 && C % 16 == 0 &&
+         (reinterpret_cast<uintptr_t>(q) & 15u) == 0 && ldq % 16 == 0;
+  if (!*tma) return BS_OK;
+  bs_status st = encode_3d(tmx, x_dtype == BS_IN_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                           es, x, static_cast<uint64_t>(C), static_cast<uint64_t>(R), 1, static_cast<uint64_t>(ldx),
+                           static_cast<uint64_t>(ldx) * static_cast<uint64_t>(R), 128, 128, "x",
+                           CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (st != BS_OK) return st;
+  return encode_3d(tmq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, q, static_cast<uint64_t>(C), static_cast<uint64_t>(R), 1,
+                   static_cast<uint64_t>(ldq), static_cast<uint64_t>(ldq) * static_cast<uint64_t>(R), 128, 128, "q",
+                   CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
 // Rows of one B box of the wide kernel: single CTAs load all 256 tile columns,
 // each CTA of a pair its 128.
 uint32_t wide_b_box_rows(int cg) { return static_cast<uint32_t>(kWideBN / cg); }
@@ -716,9 +738,12 @@ bs_status bs_quantize_fp8_1x128(const void* x, bs_in_dtype x_dtype, int64_t M, i
   DeviceCtx* dc = nullptr;
   bs_status st = device_ctx(&dc);
   if (st != BS_OK) return st;
+  CUtensorMap tmx, tmq;
+  bool tma = false;
+  if ((st = encode_quant_maps(x, x_dtype, M, K, ldx, q, ldq, &tmx, &tmq, &tma))) return st;
   return check_launch(launch_quantize_1x128(x, x_dtype == BS_IN_BF16, M, K, ldx, static_cast<uint8_t*>(q), ldq, scale,
-                                            scale_fmt == BS_SCALE_E8M0, ld_scale, dc->sms,
-                                            static_cast<cudaStream_t>(stream)),
+                                            scale_fmt == BS_SCALE_E8M0, ld_scale, dc->sms, tma ? &tmx : nullptr,
+                                            tma ? &tmq : nullptr, dc->err, static_cast<cudaStream_t>(stream)),
                       "quantise launch");
 }
 
@@ -789,21 +814,9 @@ bs_status bs_quantize_fp8_128x128(const void* x, bs_in_dtype x_dtype, int64_t R,
   DeviceCtx* dc = nullptr;
   bs_status st = device_ctx(&dc);
   if (st != BS_OK) return st;
-  // the TMA-fed kernel where x and q allow tensor copies whose rows end on 16-byte boundaries
   CUtensorMap tmx, tmq;
-  const bool tma = aligned16(x) && (ldx * static_cast<int64_t>(es)) % 16 == 0 && C % 16 == 0 && aligned16(q) &&
-                   ldq % 16 == 0;
-  if (tma) {
-    st = encode_3d(&tmx, x_dtype == BS_IN_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
-                   static_cast<int>(es), x, static_cast<uint64_t>(C), static_cast<uint64_t>(R), 1,
-                   static_cast<uint64_t>(ldx), static_cast<uint64_t>(ldx) * static_cast<uint64_t>(R), 128, 128, "x",
-                   CU_TENSOR_MAP_SWIZZLE_NONE);
-    if (st != BS_OK) return st;
-    st = encode_3d(&tmq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, q, static_cast<uint64_t>(C), static_cast<uint64_t>(R), 1,
-                   static_cast<uint64_t>(ldq), static_cast<uint64_t>(ldq) * static_cast<uint64_t>(R), 128, 128, "q",
-                   CU_TENSOR_MAP_SWIZZLE_NONE);
-    if (st != BS_OK) return st;
-  }
+  bool tma = false;
+  if ((st = encode_quant_maps(x, x_dtype, R, C, ldx, q, ldq, &tmx, &tmq, &tma))) return st;
   return check_launch(launch_quantize_blocks(x, x_dtype == BS_IN_BF16, R, C, ldx, static_cast<uint8_t*>(q), ldq, scale,
                                              scale_fmt == BS_SCALE_E8M0, s_rb, s_cb, dc->sms, tma ? &tmx : nullptr,
                                              tma ? &tmq : nullptr, dc->err, static_cast<cudaStream_t>(stream)),

@@ -22,8 +22,20 @@ __device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
 
 // amax / 448, or 1 where that fp32 quotient is zero: an all-zero group, or a
 // group whose amax is below 448 * 2^-150 so that the quotient underflows.
+// The correctly rounded quotient comes from Markstein's correction step (see
+// quotient_rn) with r = RN(1/448) = 0x1.24924ap-9 for every amax in
+// [2^-116, FLT_MAX] -- an exhaustive check of those 2.05e9 fp32 values against
+// the exactly rounded quotient found no difference -- and from an IEEE
+// division below that range (and for inf or NaN).
 __device__ __forceinline__ float group_scale_f32(float amax) {
-  const float s = __fdiv_rn(amax, 448.f);
+  float s;
+  if (amax >= 0x1p-116f && amax <= 3.40282347e38f) {
+    constexpr float r = 0x1.24924ap-9f;
+    const float q1 = __fmul_rn(amax, r);
+    s = __fmaf_rn(__fmaf_rn(-q1, 448.f, amax), r, q1);
+  } else {
+    s = __fdiv_rn(amax, 448.f);
+  }
   return s == 0.f ? 1.f : s;
 }
 
@@ -56,14 +68,16 @@ __device__ __forceinline__ float quotient_rn(float v, float s, float r) {
   return copysignf(__fmaf_rn(rem, r, q1), v);
 }
 
+// Whether a group scale lies in quotient_rn's range.
+__device__ __forceinline__ bool quotient_fast_range(float s) { return s >= 0x1p-90f && s <= 3.40282347e38f; }
+
 // y[i] = fp32(v[i] / s) for the N elements of one group held by this thread.
 // The fp32 path runs when every active lane of the warp has a scale in its
 // range (a branch the warp takes together, so the fp64 conversions are not
 // issued); otherwise the lanes take the fp64 path.
 template <int N>
 __device__ __forceinline__ void code_quotients(const float (&v)[N], float s, float (&y)[N]) {
-  const bool fast = s >= 0x1p-90f && s <= 3.40282347e38f;
-  if (__all_sync(__activemask(), fast)) {
+  if (__all_sync(__activemask(), quotient_fast_range(s))) {
     const float r = __frcp_rn(s);
 #pragma unroll
     for (int i = 0; i < N; ++i) y[i] = quotient_rn(v[i], s, r);
@@ -74,17 +88,17 @@ __device__ __forceinline__ void code_quotients(const float (&v)[N], float s, flo
   }
 }
 
-// y[i] = (fp32(v[i].x / s0), fp32(v[i].y / s1)) for N elements of two groups
-// side by side (two columns, scales s0 and s1): quotient_rn on both lanes of
-// the packed two-wide fp32 operations, under code_quotients' warp-uniform
-// range test.  (-q1 * s and q1 * -s are the same exact product, so the
-// residual is quotient_rn's.)
+// y[i] = (fp32(v[i].x / s.x), fp32(v[i].y / s.y)) for N elements of two groups
+// side by side (scales s.x and s.y): quotient_rn on both lanes of the packed
+// two-wide fp32 operations when `fast` -- true on every lane of the warp or on
+// none, and then r = (RN(1 / s.x), RN(1 / s.y)) -- else the fp64 path.  (-q1 * s
+// and q1 * -s are the same exact product, so the residual is quotient_rn's.)
+// Callers that code several runs of elements with one pair of scales compute
+// `fast` and r once.
 template <int N>
-__device__ __forceinline__ void code_quotients2(const float2 (&v)[N], float s0, float s1, float2 (&y)[N]) {
-  const bool fast = s0 >= 0x1p-90f && s0 <= 3.40282347e38f && s1 >= 0x1p-90f && s1 <= 3.40282347e38f;
-  if (__all_sync(__activemask(), fast)) {
-    const float2 r = make_float2(__frcp_rn(s0), __frcp_rn(s1));
-    const float2 ns = make_float2(-s0, -s1);
+__device__ __forceinline__ void code_quotients2(const float2 (&v)[N], float2 s, float2 r, bool fast, float2 (&y)[N]) {
+  if (fast) {
+    const float2 ns = make_float2(-s.x, -s.y);
 #pragma unroll
     for (int i = 0; i < N; ++i) {
       const float2 q1 = __fmul2_rn(v[i], r);
@@ -93,10 +107,18 @@ __device__ __forceinline__ void code_quotients2(const float2 (&v)[N], float s0, 
       y[i] = make_float2(copysignf(q.x, v[i].x), copysignf(q.y, v[i].y));
     }
   } else {
-    const double r0 = __drcp_rn(static_cast<double>(s0)), r1 = __drcp_rn(static_cast<double>(s1));
+    const double r0 = __drcp_rn(static_cast<double>(s.x)), r1 = __drcp_rn(static_cast<double>(s.y));
 #pragma unroll
     for (int i = 0; i < N; ++i) y[i] = make_float2(over_scale(v[i].x, r0), over_scale(v[i].y, r1));
   }
+}
+
+// The same with the range test (warp-uniform, over the active lanes) and the
+// reciprocals worked out here.
+template <int N>
+__device__ __forceinline__ void code_quotients2(const float2 (&v)[N], float s0, float s1, float2 (&y)[N]) {
+  const bool fast = __all_sync(__activemask(), quotient_fast_range(s0) && quotient_fast_range(s1));
+  code_quotients2<N>(v, make_float2(s0, s1), make_float2(__frcp_rn(s0), __frcp_rn(s1)), fast, y);
 }
 
 // Lane-wise magnitude max of two bf16 pairs (exact: the result is one of the

@@ -20,10 +20,13 @@
 // work (amax, scale, reciprocal) is shared by four groups per instruction.  A
 // warp takes chunks of eight groups (two passes) and keeps all their loads in
 // flight before it reduces any of them, then asks L2 for its next chunk while
-// it quantises this one.
+// it quantises this one.  This kernel serves layouts the tensor copies cannot
+// take; where x and q have 16-byte bases and row strides and K is a multiple of
+// 16, the TMA-fed kernel of quant_ring.cuh runs instead.
 #include <cuda_bf16.h>
 
 #include "group_quant.cuh"
+#include "quant_ring.cuh"
 #include "quantize.h"
 
 namespace bsg {
@@ -173,7 +176,15 @@ cudaError_t launch_q(const void* x, long long M, long long K, long long ldx, uin
 
 cudaError_t launch_quantize_1x128(const void* x, bool x_bf16, long long M, long long K, long long ldx, uint8_t* q,
                                   long long ldq, void* scale, bool e8m0, long long lds, int sms,
+                                  const CUtensorMap* tmx, const CUtensorMap* tmq, uint32_t* err,
                                   cudaStream_t stream) {
+  if (tmx && tmq) {
+    if (x_bf16)
+      return e8m0 ? ring::launch_ring<__nv_bfloat16, 1, true>(*tmx, *tmq, M, K, scale, lds, 1, sms, err, stream)
+                  : ring::launch_ring<__nv_bfloat16, 0, true>(*tmx, *tmq, M, K, scale, lds, 1, sms, err, stream);
+    return e8m0 ? ring::launch_ring<float, 1, true>(*tmx, *tmq, M, K, scale, lds, 1, sms, err, stream)
+                : ring::launch_ring<float, 0, true>(*tmx, *tmq, M, K, scale, lds, 1, sms, err, stream);
+  }
   if (x_bf16)
     return e8m0 ? launch_q<__nv_bfloat16, 1>(x, M, K, ldx, q, ldq, scale, lds, sms, stream)
                 : launch_q<__nv_bfloat16, 0>(x, M, K, ldx, q, ldq, scale, lds, sms, stream);

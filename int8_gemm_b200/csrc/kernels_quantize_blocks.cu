@@ -14,13 +14,16 @@
 // tile amax comes from a warp then block reduction, and each piece is written
 // back as its 8 (bf16) or 4 (fp32) codes at the same place in q.  Several
 // CTAs share an SM, so one CTA's loads are in flight while another reduces.
+// This kernel serves layouts the tensor copies cannot take; where x and q have
+// 16-byte bases and row strides and C is a multiple of 16, the TMA-fed kernel
+// of quant_ring.cuh runs instead.
 #include <cuda_bf16.h>
 
 #include <cstring>
 
 #include "group_quant.cuh"
+#include "quant_ring.cuh"
 #include "quantize.h"
-#include "sm100.cuh"
 
 namespace bsg {
 
@@ -164,205 +167,6 @@ cudaError_t launch_blocks(const void* x, long long R, long long C, long long ldx
   return cudaGetLastError();
 }
 
-// ---------------------------------------------------------------------------
-// TMA-fed form (x and q with 16-byte bases and row strides, C a multiple of 16)
-// ---------------------------------------------------------------------------
-// One CTA of 512 threads per SM, persistent over tiles.  One thread keeps a
-// ring of kRingStages input tiles in flight with 2-D tensor copies (rows past
-// R arrive as zeros) and writes each tile's codes back with one tensor store
-// that clips at R; no thread spends instructions or registers on global loads
-// or stores.  Consecutive threads take consecutive 16-byte pieces of a tile
-// row from shared memory (a warp reads 512 contiguous bytes), the tile amax
-// comes from a warp then block reduction (bf16: one packed magnitude max per
-// element pair), and each piece's 8 (bf16) or 4 (fp32) codes go to the same
-// place of a shared code tile.
-constexpr int kRingThreads = 512;
-
-template <typename InT>
-struct Ring {
-  static constexpr int kStages = sizeof(InT) == 2 ? 4 : 3;    // input tiles (32 or 64 KB each)
-  static constexpr int kCodeBufs = sizeof(InT) == 2 ? 2 : 1;  // code tiles (16 KB each)
-  static constexpr int kElems = 16 / sizeof(InT);             // elements per 16-byte piece
-  static constexpr int kPerRow = kTile / kElems;              // pieces per tile row
-  static constexpr int kRowsPerPass = kRingThreads / kPerRow;
-  static constexpr int kPasses = kTile / kRowsPerPass;        // pieces per thread
-};
-
-template <typename InT>
-struct RingSmem {
-  alignas(1024) InT v[Ring<InT>::kStages][kTile][kTile];          // input tiles, [row][column]
-  alignas(1024) uint8_t codes[Ring<InT>::kCodeBufs][kTile][kTile];  // code tiles, [row][column]
-  float wmax[kRingThreads / 32];
-  uint64_t full[Ring<InT>::kStages];
-  int abort;
-};
-
-// The amax of a piece's elements.
-__device__ __forceinline__ float piece_amax(const uint4& v, __nv_bfloat16) {
-  const uint32_t m = max_abs_bf16x2(max_abs_bf16x2(v.x, v.y), max_abs_bf16x2(v.z, v.w));
-  return fmaxf(__uint_as_float((m << 16) & 0x7FFFFFFFu), __uint_as_float(m & 0x7FFF0000u));
-}
-__device__ __forceinline__ float piece_amax(const uint4& v, float) {
-  return fmaxf(fmaxf(fabsf(__uint_as_float(v.x)), fabsf(__uint_as_float(v.y))),
-               fmaxf(fabsf(__uint_as_float(v.z)), fabsf(__uint_as_float(v.w))));
-}
-
-// A piece's elements as fp32 pairs (exact widening for bf16).
-__device__ __forceinline__ void piece_pairs(const uint4& v, float2 (&e)[4]) {  // bf16: 8 elements
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) e[i] = make_float2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
-}
-__device__ __forceinline__ void piece_pairs(const uint4& v, float2 (&e)[2]) {  // fp32: 4 elements
-  e[0] = make_float2(__uint_as_float(v.x), __uint_as_float(v.y));
-  e[1] = make_float2(__uint_as_float(v.z), __uint_as_float(v.w));
-}
-
-template <typename InT, int FMT>
-__global__ void __launch_bounds__(kRingThreads, 1)
-    quantize_blocks_tma_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmq,
-                               void* __restrict__ scale, long long s_rb, long long s_cb, long long ctiles,
-                               long long ntiles, uint32_t* err) {
-  using G = Ring<InT>;
-  using S = RingSmem<InT>;
-  constexpr uint32_t kTileBytes = kTile * kTile * sizeof(InT);
-  constexpr int kPairs = G::kElems / 2;
-  extern __shared__ uint8_t smem_raw[];
-  const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
-  if (pad + sizeof(S) > dynamic_smem_bytes()) {  // never touch memory the launch did not provide
-    if (threadIdx.x == 0) record_error(err, kErrSmemTooSmall);
-    return;
-  }
-  S& sm = *reinterpret_cast<S*>(smem_raw + pad);
-  const int t = threadIdx.x;
-  const int piece = t % G::kPerRow;  // this thread's piece within a row
-  const int row0 = t / G::kPerRow;   // and its first row within the tile
-  if (t == 0) {
-    for (int s = 0; s < G::kStages; ++s) mbar_init(&sm.full[s], 1);
-    sm.abort = 0;
-    fence_mbar_init();
-    tma_prefetch_desc(&tmx);
-    tma_prefetch_desc(&tmq);
-  }
-  __syncthreads();
-  auto issue = [&](long long tile, int s) {
-    const long long rb = tile / ctiles, cb = tile - rb * ctiles;
-    mbar_arrive_expect_tx(&sm.full[s], kTileBytes);
-    tma_load_3d(&sm.v[s][0][0], &tmx, &sm.full[s], static_cast<int>(cb * kTile), static_cast<int>(rb * kTile), 0);
-  };
-  if (t == 0)
-    for (int s = 0; s < G::kStages; ++s) {
-      const long long tile = blockIdx.x + static_cast<long long>(s) * gridDim.x;
-      if (tile < ntiles) issue(tile, s);
-    }
-  int it = 0;
-  bool ok = true;
-  for (long long tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
-    const int st = it % G::kStages, cbuf = it % G::kCodeBufs;
-    const long long rb = tile / ctiles, cb = tile - rb * ctiles;
-    const bool got = wait_bounded(&sm.full[st], static_cast<uint32_t>(it / G::kStages) & 1u, &sm.abort, err,
-                                  kErrTimeout | kRoleConsumer | kWaitStageFull);
-    uint4 v[G::kPasses];
-#pragma unroll
-    for (int k = 0; k < G::kPasses; ++k)
-      v[k] = *reinterpret_cast<const uint4*>(&sm.v[st][row0 + k * G::kRowsPerPass][piece * G::kElems]);
-    float amax = 0.f;
-#pragma unroll
-    for (int k = 0; k < G::kPasses; ++k) amax = fmaxf(amax, piece_amax(v[k], InT()));
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-    if ((t & 31) == 0) sm.wmax[t / 32] = amax;
-    // the code tile written kCodeBufs tiles ago has been read by its store
-    if (t == 0) {
-      if constexpr (G::kCodeBufs == 2) {
-        bulk_wait_read1();
-      } else {
-        bulk_wait_read_all();
-      }
-    }
-    // every thread holds its pieces: the stage can be refilled
-    ok = __syncthreads_and(got) != 0;
-    if (!ok) break;
-    if (t == 0) {
-      const long long next = tile + static_cast<long long>(G::kStages) * gridDim.x;
-      if (next < ntiles) {
-        fence_proxy_async_smem();
-        issue(next, st);
-      }
-    }
-    amax = sm.wmax[0];
-#pragma unroll
-    for (int w = 1; w < kRingThreads / 32; ++w) amax = fmaxf(amax, sm.wmax[w]);
-    float s = 1.f;
-    int byte = 127;
-    if constexpr (FMT == 0) {
-      s = group_scale_f32(amax);
-    } else {
-      byte = group_e8m0(amax);
-    }
-    if (t == 0) {
-      const long long si = rb * s_rb + cb * s_cb;
-      if constexpr (FMT == 0) {
-        static_cast<float*>(scale)[si] = s;
-      } else {
-        static_cast<uint8_t*>(scale)[si] = static_cast<uint8_t>(byte);
-      }
-    }
-    const float mul = ldexpf(1.f, 127 - byte);  // exact power of two (e8m0)
-#pragma unroll
-    for (int k = 0; k < G::kPasses; ++k) {
-      float2 e[kPairs], y[kPairs];
-      piece_pairs(v[k], e);
-      if constexpr (FMT == 0) {
-        code_quotients2<kPairs>(e, s, s, y);
-      } else {
-#pragma unroll
-        for (int i = 0; i < kPairs; ++i) y[i] = __fmul2_rn(e[i], make_float2(mul, mul));
-      }
-      uint8_t* dst = &sm.codes[cbuf][row0 + k * G::kRowsPerPass][piece * G::kElems];
-      if constexpr (kPairs == 4) {
-        *reinterpret_cast<uint2*>(dst) = make_uint2(e4m3x2(y[0].x, y[0].y) | (e4m3x2(y[1].x, y[1].y) << 16),
-                                                    e4m3x2(y[2].x, y[2].y) | (e4m3x2(y[3].x, y[3].y) << 16));
-      } else {
-        *reinterpret_cast<uint32_t*>(dst) = e4m3x2(y[0].x, y[0].y) | (e4m3x2(y[1].x, y[1].y) << 16);
-      }
-    }
-    fence_proxy_async_smem();  // the code tile, before the tensor store reads it
-    __syncthreads();
-    if (t == 0) {
-      tma_store_3d(&tmq, &sm.codes[cbuf][0][0], static_cast<int>(cb * kTile), static_cast<int>(rb * kTile), 0);
-      bulk_commit();
-    }
-  }
-  if (t == 0) {
-    bulk_wait_all();
-    if (!ok) {  // a wait gave up: let the copies still in flight land before the CTA retires
-      volatile int never = 0;
-      for (int j = it; j < it + G::kStages; ++j) {
-        const long long tile = blockIdx.x + static_cast<long long>(j) * gridDim.x;
-        if (tile < ntiles)
-          wait_bounded(&sm.full[j % G::kStages], static_cast<uint32_t>(j / G::kStages) & 1u, &never, nullptr, 0);
-      }
-    }
-  }
-}
-
-template <typename InT, int FMT>
-cudaError_t launch_blocks_tma(const CUtensorMap& tmx, const CUtensorMap& tmq, long long R, long long C, void* scale,
-                              long long s_rb, long long s_cb, int sms, uint32_t* err, cudaStream_t stream) {
-  const long long ctiles = (C + kTile - 1) / kTile;
-  const long long ntiles = ((R + kTile - 1) / kTile) * ctiles;
-  const size_t smem = sizeof(RingSmem<InT>) + 1024;
-  cudaError_t e = cudaFuncSetAttribute(quantize_blocks_tma_kernel<InT, FMT>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
-  long long blocks = sms > 0 ? sms : 148;
-  if (blocks > ntiles) blocks = ntiles;
-  quantize_blocks_tma_kernel<InT, FMT><<<static_cast<unsigned>(blocks), kRingThreads, smem, stream>>>(
-      tmx, tmq, scale, s_rb, s_cb, ctiles, ntiles, err);
-  return cudaGetLastError();
-}
-
 }  // namespace
 
 cudaError_t launch_quantize_blocks(const void* x, bool x_bf16, long long R, long long C, long long ldx, uint8_t* q,
@@ -371,10 +175,10 @@ cudaError_t launch_quantize_blocks(const void* x, bool x_bf16, long long R, long
                                    cudaStream_t stream) {
   if (tmx && tmq) {
     if (x_bf16)
-      return e8m0 ? launch_blocks_tma<__nv_bfloat16, 1>(*tmx, *tmq, R, C, scale, s_rb, s_cb, sms, err, stream)
-                  : launch_blocks_tma<__nv_bfloat16, 0>(*tmx, *tmq, R, C, scale, s_rb, s_cb, sms, err, stream);
-    return e8m0 ? launch_blocks_tma<float, 1>(*tmx, *tmq, R, C, scale, s_rb, s_cb, sms, err, stream)
-                : launch_blocks_tma<float, 0>(*tmx, *tmq, R, C, scale, s_rb, s_cb, sms, err, stream);
+      return e8m0 ? ring::launch_ring<__nv_bfloat16, 1, false>(*tmx, *tmq, R, C, scale, s_rb, s_cb, sms, err, stream)
+                  : ring::launch_ring<__nv_bfloat16, 0, false>(*tmx, *tmq, R, C, scale, s_rb, s_cb, sms, err, stream);
+    return e8m0 ? ring::launch_ring<float, 1, false>(*tmx, *tmq, R, C, scale, s_rb, s_cb, sms, err, stream)
+                : ring::launch_ring<float, 0, false>(*tmx, *tmq, R, C, scale, s_rb, s_cb, sms, err, stream);
   }
   if (x_bf16)
     return e8m0 ? launch_blocks<__nv_bfloat16, 1>(x, R, C, ldx, q, ldq, scale, s_rb, s_cb, sms, stream)

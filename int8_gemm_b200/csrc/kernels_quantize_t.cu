@@ -28,6 +28,7 @@
 #include <cuda_bf16.h>
 
 #include <cstring>
+#include <type_traits>
 
 #include "group_quant.cuh"
 #include "quantize.h"
@@ -254,69 +255,54 @@ cudaError_t launch_t_fmt(const void* x, long long R, long long C, long long ldx,
 }
 
 // ---------------------------------------------------------------------------
-// TMA-fed form (x and q_t both 16-byte aligned with 16-byte row strides)
+// TMA-fed form (x and q_t with 16-byte bases and row strides, rows ending on
+// 16-byte boundaries)
 // ---------------------------------------------------------------------------
-// One CTA of 512 threads per SM, persistent over 128 x 128 tiles.  One thread
-// keeps a ring of kTmaStages tiles in flight with 2-D tensor copies (rows and
-// columns past the matrix arrive as zeros), so no thread spends instructions
-// or registers on loads.  Thread t owns the column pair 2 (t % 64), + 1 and
-// the 16 rows 16 (t / 64) .. + 15: it reads its 16 pairs from the tile once
-// (one 4- or 8-byte shared load each, a warp reading 128 or 256 contiguous
-// bytes), takes their amax in registers (bf16: one packed max of magnitudes
-// per pair), and after the amaxes meet in shared memory quantises the values
-// it still holds.  Its 2 x 16 codes go as two 16-byte pieces into a shared
+// Persistent CTAs (two of 256 threads per SM for bf16 input, each with two
+// input and two code tiles, so that one CTA's reductions and barriers overlap
+// the other's work; one of 512 threads for fp32, with three input tiles and one
+// code tile).  One thread keeps the ring of input tiles in flight with 2-D
+// tensor copies (rows and columns past the matrix arrive as zeros), so no
+// thread spends instructions or registers on loads.  Thread t owns the column
+// pair 2 (t % 64), + 1 and kRows consecutive rows (32 for bf16, 16 for fp32):
+// it reads its pairs from the tile once (one 4- or 8-byte shared load each, a
+// warp reading 128 or 256 contiguous bytes), takes their amax in registers
+// (bf16: one packed max of magnitudes per pair), and after the amaxes meet in
+// shared memory quantises the values it still holds, 16 rows at a time.  Each
+// run of 16 codes of a column goes as one 16-byte piece into a shared
 // [column][row] code tile laid out in the 128-byte swizzle, which one thread
 // then writes to q_t with a tensor store that clips at R and C.
-constexpr int kTmaThreads = 512;
-constexpr int kTmaParts = kTmaThreads / (kTile / 2);  // row groups per column pair
-constexpr int kTmaRows = kTile / kTmaParts;           // rows per thread
-static_assert(kTmaRows == 16, "a thread's codes of one column are one 16-byte piece");
-
 template <typename InT>
-struct TmaRing {
-  static constexpr int kStages = sizeof(InT) == 2 ? 4 : 3;  // input tiles (32 or 64 KB each)
-  static constexpr int kCodeBufs = sizeof(InT) == 2 ? 2 : 1;  // code tiles (16 KB each)
+struct TRing {
+  static constexpr bool kPair = sizeof(InT) == 2;
+  static constexpr int kThreads = kPair ? 256 : 512;
+  static constexpr int kCtasPerSm = kPair ? 2 : 1;
+  static constexpr int kStages = kPair ? 2 : 3;    // input tiles (32 or 64 KB each)
+  static constexpr int kCodeBufs = kPair ? 2 : 1;  // code tiles (16 KB each)
+  static constexpr int kParts = kThreads / (kTile / 2);  // row groups per column pair
+  static constexpr int kRows = kTile / kParts;           // rows per thread
+  static constexpr int kRuns = kRows / 16;               // 16-row runs: one 16-byte code piece per column each
+  using Held = typename std::conditional<kPair, uint32_t, float2>::type;  // one row of the column pair
 };
 
 template <typename InT>
 struct TmaSmem {
-  alignas(1024) InT v[TmaRing<InT>::kStages][kTile][kTile];       // input tiles, [row][column]
-  alignas(1024) uint8_t codes[TmaRing<InT>::kCodeBufs][kTile][kTile];  // [column][row], 128-byte swizzle
-  float2 part[kTmaParts][kTile / 2];  // amaxes of each row group's column pairs
-  float wmax[kTmaThreads / 32];
-  uint64_t full[TmaRing<InT>::kStages];
+  alignas(1024) InT v[TRing<InT>::kStages][kTile][kTile];          // input tiles, [row][column]
+  alignas(1024) uint8_t codes[TRing<InT>::kCodeBufs][kTile][kTile];  // [column][row], 128-byte swizzle
+  float2 part[TRing<InT>::kParts][kTile / 2];  // amaxes of each row group's column pairs
+  float wmax[TRing<InT>::kThreads / 32];
+  uint64_t full[TRing<InT>::kStages];
   int abort;
 };
 
-// This thread's 16 pairs of the tile in stage `st`, widened to fp32, and
-// their two column amaxes.
-__device__ __forceinline__ void load_pairs(const TmaSmem<__nv_bfloat16>& sm, int st, int r0, int p, float2 (&e)[kTmaRows],
-                                           float& amax0, float& amax1) {
-  uint32_t w[kTmaRows];
-#pragma unroll
-  for (int i = 0; i < kTmaRows; ++i) w[i] = *reinterpret_cast<const uint32_t*>(&sm.v[st][r0 + i][2 * p]);
-  uint32_t m = 0;
-#pragma unroll
-  for (int i = 0; i < kTmaRows; ++i) m = max_abs_bf16x2(m, w[i]);
-  amax0 = __uint_as_float((m << 16) & 0x7FFFFFFFu);
-  amax1 = __uint_as_float(m & 0x7FFF0000u);
-#pragma unroll
-  for (int i = 0; i < kTmaRows; ++i) e[i] = make_float2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
+// One held row of a column pair as fp32 (exact widening for bf16).
+__device__ __forceinline__ float2 widen(uint32_t w) {
+  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
 }
-__device__ __forceinline__ void load_pairs(const TmaSmem<float>& sm, int st, int r0, int p, float2 (&e)[kTmaRows],
-                                           float& amax0, float& amax1) {
-#pragma unroll
-  for (int i = 0; i < kTmaRows; ++i) e[i] = *reinterpret_cast<const float2*>(&sm.v[st][r0 + i][2 * p]);
-  amax0 = amax1 = 0.f;
-#pragma unroll
-  for (int i = 0; i < kTmaRows; ++i) {
-    amax0 = fmaxf(amax0, fabsf(e[i].x));
-    amax1 = fmaxf(amax1, fabsf(e[i].y));
-  }
-}
+__device__ __forceinline__ float2 widen(float2 v) { return v; }
 
 // 16 codes of one column (lane h of y) as a 16-byte piece.
-__device__ __forceinline__ uint4 pack_column(const float2 (&y)[kTmaRows], int h) {
+__device__ __forceinline__ uint4 pack_column(const float2 (&y)[16], int h) {
   uint32_t w[4];
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
@@ -328,12 +314,13 @@ __device__ __forceinline__ uint4 pack_column(const float2 (&y)[kTmaRows], int h)
 }
 
 template <typename InT, int FMT, int GROUP>
-__global__ void __launch_bounds__(kTmaThreads, 1)
+__global__ void __launch_bounds__(TRing<InT>::kThreads, TRing<InT>::kCtasPerSm)
     quantize_t_tma_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmq, long long R,
                           long long C, void* __restrict__ scale, long long lds, long long ctiles, long long ntiles,
                           uint32_t* err) {
+  using G = TRing<InT>;
   using S = TmaSmem<InT>;
-  constexpr int kStages = TmaRing<InT>::kStages, kCodeBufs = TmaRing<InT>::kCodeBufs;
+  using Held = typename G::Held;
   constexpr uint32_t kTileBytes = kTile * kTile * sizeof(InT);
   extern __shared__ uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
@@ -344,9 +331,9 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
   S& sm = *reinterpret_cast<S*>(smem_raw + pad);
   const int t = threadIdx.x;
   const int cp = t % (kTile / 2);  // column pair
-  const int qr = t / (kTile / 2);  // row group: rows kTmaRows * qr ..
+  const int qr = t / (kTile / 2);  // row group: rows kRows * qr ..
   if (t == 0) {
-    for (int s = 0; s < kStages; ++s) mbar_init(&sm.full[s], 1);
+    for (int s = 0; s < G::kStages; ++s) mbar_init(&sm.full[s], 1);
     sm.abort = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmx);
@@ -359,20 +346,35 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
     tma_load_3d(&sm.v[s][0][0], &tmx, &sm.full[s], static_cast<int>(cb * kTile), static_cast<int>(rb * kTile), 0);
   };
   if (t == 0)
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < G::kStages; ++s) {
       const long long tile = blockIdx.x + static_cast<long long>(s) * gridDim.x;
       if (tile < ntiles) issue(tile, s);
     }
   int it = 0;
   bool ok = true;
   for (long long tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
-    const int st = it % kStages, cbuf = it % kCodeBufs;
+    const int st = it % G::kStages, cbuf = it % G::kCodeBufs;
     const long long rb = tile / ctiles, cb = tile - rb * ctiles;
-    const bool got = wait_bounded(&sm.full[st], static_cast<uint32_t>(it / kStages) & 1u, &sm.abort, err,
+    const bool got = wait_bounded(&sm.full[st], static_cast<uint32_t>(it / G::kStages) & 1u, &sm.abort, err,
                                   kErrTimeout | kRoleConsumer | kWaitStageFull);
-    float2 e[kTmaRows];
+    Held h[G::kRows];
+#pragma unroll
+    for (int i = 0; i < G::kRows; ++i) h[i] = *reinterpret_cast<const Held*>(&sm.v[st][G::kRows * qr + i][2 * cp]);
     float amax0, amax1;
-    load_pairs(sm, st, kTmaRows * qr, cp, e, amax0, amax1);
+    if constexpr (G::kPair) {
+      uint32_t m = 0;
+#pragma unroll
+      for (int i = 0; i < G::kRows; ++i) m = max_abs_bf16x2(m, h[i]);
+      amax0 = __uint_as_float((m << 16) & 0x7FFFFFFFu);
+      amax1 = __uint_as_float(m & 0x7FFF0000u);
+    } else {
+      amax0 = amax1 = 0.f;
+#pragma unroll
+      for (int i = 0; i < G::kRows; ++i) {
+        amax0 = fmaxf(amax0, fabsf(widen(h[i]).x));
+        amax1 = fmaxf(amax1, fabsf(widen(h[i]).y));
+      }
+    }
     if constexpr (GROUP == 0) {
       sm.part[qr][cp] = make_float2(amax0, amax1);
     } else {
@@ -383,7 +385,7 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
     }
     // the code tile written kCodeBufs tiles ago has been read by its store
     if (t == 0) {
-      if constexpr (kCodeBufs == 2) {
+      if constexpr (G::kCodeBufs == 2) {
         bulk_wait_read1();
       } else {
         bulk_wait_read_all();
@@ -393,7 +395,7 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
     ok = __syncthreads_and(got) != 0;
     if (!ok) break;
     if (t == 0) {
-      const long long next = tile + static_cast<long long>(kStages) * gridDim.x;
+      const long long next = tile + static_cast<long long>(G::kStages) * gridDim.x;
       if (next < ntiles) {
         fence_proxy_async_smem();
         issue(next, st);
@@ -401,7 +403,7 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
     }
     if constexpr (GROUP == 0) {
 #pragma unroll
-      for (int k = 0; k < kTmaParts; ++k) {
+      for (int k = 0; k < G::kParts; ++k) {
         const float2 pk = sm.part[k][cp];
         amax0 = fmaxf(amax0, pk.x);
         amax1 = fmaxf(amax1, pk.y);
@@ -409,22 +411,24 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
     } else {
       float a = sm.wmax[0];
 #pragma unroll
-      for (int w = 1; w < kTmaThreads / 32; ++w) a = fmaxf(a, sm.wmax[w]);
+      for (int w = 1; w < G::kThreads / 32; ++w) a = fmaxf(a, sm.wmax[w]);
       amax0 = amax1 = a;
     }
     const long long ca = cb * kTile + 2 * cp;  // this thread's first column of x
-    float2 y[kTmaRows];
+    float2 sc = make_float2(1.f, 1.f), rc = sc, mul = sc;
+    bool fast = true;
     if constexpr (FMT == 0) {
-      const float s0 = group_scale_f32(amax0), s1 = group_scale_f32(amax1);
+      sc = make_float2(group_scale_f32(amax0), group_scale_f32(amax1));
       if constexpr (GROUP == 0) {
         if (qr == 0) {
-          if (ca < C) static_cast<float*>(scale)[ca * lds + rb] = s0;
-          if (ca + 1 < C) static_cast<float*>(scale)[(ca + 1) * lds + rb] = s1;
+          if (ca < C) static_cast<float*>(scale)[ca * lds + rb] = sc.x;
+          if (ca + 1 < C) static_cast<float*>(scale)[(ca + 1) * lds + rb] = sc.y;
         }
       } else if (t == 0) {
-        static_cast<float*>(scale)[rb * lds + cb] = s0;
+        static_cast<float*>(scale)[rb * lds + cb] = sc.x;
       }
-      code_quotients2<kTmaRows>(e, s0, s1, y);
+      fast = __all_sync(0xffffffffu, quotient_fast_range(sc.x) && quotient_fast_range(sc.y));
+      rc = make_float2(__frcp_rn(sc.x), __frcp_rn(sc.y));
     } else {
       const int byte0 = group_e8m0(amax0), byte1 = group_e8m0(amax1);
       if constexpr (GROUP == 0) {
@@ -435,15 +439,26 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
       } else if (t == 0) {
         static_cast<uint8_t*>(scale)[rb * lds + cb] = static_cast<uint8_t>(byte0);
       }
-      const float2 mul = make_float2(ldexpf(1.f, 127 - byte0), ldexpf(1.f, 127 - byte1));  // exact powers of two
-#pragma unroll
-      for (int i = 0; i < kTmaRows; ++i) y[i] = __fmul2_rn(e[i], mul);
+      mul = make_float2(ldexpf(1.f, 127 - byte0), ldexpf(1.f, 127 - byte1));  // exact powers of two
     }
-    // code tile rows 2 cp and 2 cp + 1, 16-byte piece qr (swizzled by the row)
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int c = 2 * cp + h;
-      *reinterpret_cast<uint4*>(&sm.codes[cbuf][c][(qr ^ (c & 7)) * 16]) = pack_column(y, h);
+    for (int run = 0; run < G::kRuns; ++run) {
+      float2 e[16], y[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) e[i] = widen(h[16 * run + i]);
+      if constexpr (FMT == 0) {
+        code_quotients2<16>(e, sc, rc, fast, y);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) y[i] = __fmul2_rn(e[i], mul);
+      }
+      // code tile rows 2 cp and 2 cp + 1, 16-byte piece kRuns qr + run (swizzled by the row)
+      const int piece = G::kRuns * qr + run;
+#pragma unroll
+      for (int hc = 0; hc < 2; ++hc) {
+        const int c = 2 * cp + hc;
+        *reinterpret_cast<uint4*>(&sm.codes[cbuf][c][(piece ^ (c & 7)) * 16]) = pack_column(y, hc);
+      }
     }
     fence_proxy_async_smem();  // the code tile, before the tensor store reads it
     __syncthreads();
@@ -456,9 +471,10 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
     bulk_wait_all();
     if (!ok) {  // a wait gave up: let the copies still in flight land before the CTA retires
       volatile int never = 0;
-      for (int j = it; j < it + kStages; ++j) {
+      for (int j = it; j < it + G::kStages; ++j) {
         const long long tile = blockIdx.x + static_cast<long long>(j) * gridDim.x;
-        if (tile < ntiles) wait_bounded(&sm.full[j % kStages], static_cast<uint32_t>(j / kStages) & 1u, &never, nullptr, 0);
+        if (tile < ntiles)
+          wait_bounded(&sm.full[j % G::kStages], static_cast<uint32_t>(j / G::kStages) & 1u, &never, nullptr, 0);
       }
     }
   }
@@ -473,9 +489,9 @@ cudaError_t launch_t_tma(const CUtensorMap& tmx, const CUtensorMap& tmq, long lo
   cudaError_t e = cudaFuncSetAttribute(quantize_t_tma_kernel<InT, FMT, GROUP>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  long long blocks = sms > 0 ? sms : 148;
+  long long blocks = static_cast<long long>(sms > 0 ? sms : 148) * TRing<InT>::kCtasPerSm;
   if (blocks > ntiles) blocks = ntiles;
-  quantize_t_tma_kernel<InT, FMT, GROUP><<<static_cast<unsigned>(blocks), kTmaThreads, smem, stream>>>(
+  quantize_t_tma_kernel<InT, FMT, GROUP><<<static_cast<unsigned>(blocks), TRing<InT>::kThreads, smem, stream>>>(
       tmx, tmq, R, C, scale, lds, ctiles, ntiles, err);
   return cudaGetLastError();
 }

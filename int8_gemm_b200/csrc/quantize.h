@@ -12,8 +12,14 @@ namespace bsg {
 // 1x128 group quantisation of x [M, K] (bf16 or fp32, row stride ldx
 // elements) to e4m3 codes q (row stride ldq bytes) and one scale per group:
 // fp32 amax / 448, or an e8m0 byte (e8m0 = true); scale row stride lds.
+// tmx / tmq: tensor maps of x and q (box 128 x 128; q with the 128-byte
+// swizzle), or null where x or q is not 16-byte aligned with 16-byte row
+// strides or K is not a multiple of 16; with both given the TMA-fed kernel of
+// quant_ring.cuh runs, whose bounded waits record a timeout in the device
+// error word `err`.
 cudaError_t launch_quantize_1x128(const void* x, bool x_bf16, long long M, long long K, long long ldx, uint8_t* q,
                                   long long ldq, void* scale, bool e8m0, long long lds, int sms,
+                                  const CUtensorMap* tmx, const CUtensorMap* tmq, uint32_t* err,
                                   cudaStream_t stream);
 
 // Transposed-output quantisation of x [R, C] (bf16 or fp32, row stride ldx
@@ -22,9 +28,10 @@ cudaError_t launch_quantize_1x128(const void* x, bool x_bf16, long long M, long 
 // column), scale [C, ceil(R/128)]; true: 128x128 blocks, scale
 // [ceil(R/128), ceil(C/128)]; scale row stride lds, fp32 or e8m0 bytes.
 // tmx / tmq: tensor maps of x (box 128 x 128, no swizzle) and q_t (box 128 x
-// 128 bytes, 128-byte swizzle), or null where x or q_t is not 16-byte aligned
-// with a 16-byte row stride; with both given the TMA-fed kernel runs, whose
-// bounded waits record a timeout in the device error word `err`.
+// 128 bytes, 128-byte swizzle), or null unless x and q_t have 16-byte bases and
+// row strides and their rows' used bytes (C elements, R codes) end on 16-byte
+// boundaries; with both given the TMA-fed kernel runs, whose bounded waits
+// record a timeout in the device error word `err`.
 cudaError_t launch_quantize_t(const void* x, bool x_bf16, long long R, long long C, long long ldx, uint8_t* q_t,
                               long long ldq, void* scale, bool e8m0, bool block128, long long lds, int sms,
                               const CUtensorMap* tmx, const CUtensorMap* tmq, uint32_t* err, cudaStream_t stream);
@@ -33,10 +40,11 @@ cudaError_t launch_quantize_t(const void* x, bool x_bf16, long long R, long long
 // elements) in its own orientation: codes q [R, C] (row stride ldq bytes),
 // q[r][c] the code of x[r][c], one scale per block (rb, cb) at
 // scale[rb * s_rb + cb * s_cb] (element strides), fp32 or e8m0 bytes.
-// tmx / tmq: tensor maps of x and q (box 128 x 128, no swizzle), or null where
-// x or q is not 16-byte aligned with 16-byte row strides or C is not a
-// multiple of 16; with both given the TMA-fed kernel runs, whose bounded
-// waits record a timeout in the device error word `err`.
+// tmx / tmq: tensor maps of x and q (box 128 x 128; q with the 128-byte
+// swizzle), or null where x or q is not 16-byte aligned with 16-byte row
+// strides or C is not a multiple of 16; with both given the TMA-fed kernel of
+// quant_ring.cuh runs, whose bounded waits record a timeout in the device
+// error word `err`.
 cudaError_t launch_quantize_blocks(const void* x, bool x_bf16, long long R, long long C, long long ldx, uint8_t* q,
                                    long long ldq, void* scale, bool e8m0, long long s_rb, long long s_cb, int sms,
                                    const CUtensorMap* tmx, const CUtensorMap* tmq, uint32_t* err,

@@ -107,3 +107,77 @@ def test_fp32_corrected_quotient_needs_the_correction():
     x = (s.astype(np.float64) * rng.uniform(1, 448, 5000)).astype(np.float32)
     r = (np.float32(1.0) / s).astype(np.float32)
     assert np.any((x * r).astype(np.float32) != (x / s).astype(np.float32))
+
+
+# ---------------------------------------------------------------------------
+# The fp32 group scale amax / 448: Markstein's correction step with the fixed reciprocal r = RN(1/448) for
+# every amax in [2^-116, FLT_MAX], an IEEE division below.
+# ---------------------------------------------------------------------------
+_R448 = np.float32(float.fromhex("0x1.24924ap-9"))
+
+
+def _scale_markstein(a: np.float32) -> np.float32:
+    q1 = np.float32(a * _R448)
+    return _fma32(_fma32(-q1, np.float32(448.0), a), _R448, q1)
+
+
+def test_reciprocal_of_448_is_the_rounded_reciprocal():
+    assert _R448 == _rn32(Fraction(1, 448))
+
+
+def test_group_scale_division_by_448_sampled():
+    rng = np.random.default_rng(31)
+    lo, hi = np.float32(2.0 ** -116), np.finfo(np.float32).max
+    a = np.ldexp(1.0 + rng.random(6000), rng.integers(-116, 128, 6000)).astype(np.float32)
+    edges = [lo, np.nextafter(lo, np.float32(np.inf)), hi, np.nextafter(hi, np.float32(0)), np.float32(448.0),
+             np.float32(448.0 * 2.0 ** 5), np.float32(1.0), np.float32(7.0)]
+    # quotients steered next to fp32 rounding midpoints
+    m = np.ldexp(1.0 + rng.random(3000), rng.integers(-100, 100, 3000)).astype(np.float32)
+    mid = (m.astype(np.float64) + np.spacing(m).astype(np.float64) / 2) * 448.0
+    near = mid.astype(np.float32)
+    for ai in list(a) + edges + list(near[np.isfinite(near) & (near >= lo)]):
+        ref = _rn32(Fraction(float(ai)) / 448)
+        got = _scale_markstein(np.float32(ai))
+        assert ref.view(np.uint32) == got.view(np.uint32), (float(ai), float(ref), float(got))
+
+
+_DIV448_C = r"""
+#include <math.h>
+#include <stdint.h>
+#include <stdio.h>
+#include <string.h>
+static float f_of(uint32_t u) { float f; memcpy(&f, &u, 4); return f; }
+static uint32_t u_of(float f) { uint32_t u; memcpy(&u, &f, 4); return u; }
+static int check(uint32_t u, float r) {
+  const float a = f_of(u), q1 = a * r, q = fmaf(fmaf(-q1, 448.0f, a), r, q1);
+  return u_of(q) != u_of((float)((double)a / 448.0));  /* double quotient rounded once more: exact here */
+}
+int main(int argc, char** argv) {
+  const uint32_t step = (uint32_t)atoi(argv[1]);
+  const float r = 0x1.24924ap-9f;
+  const uint32_t lo = u_of(0x1p-116f), hi = u_of(3.40282347e38f);
+  unsigned long long bad = 0;
+  for (uint32_t u = lo; u < lo + (1u << 20); ++u) bad += check(u, r);
+  for (uint32_t u = hi - (1u << 20); u <= hi; ++u) bad += check(u, r);
+  for (uint32_t u = lo; u <= hi - step; u += step) bad += check(u, r);
+  printf("%llu\n", bad);
+  return 0;
+}
+"""
+
+
+def test_group_scale_division_by_448_strided_sweep(tmp_path):
+    """Every fp32 amax at the two ends of [2^-116, FLT_MAX] (2^20 values each) and every 61st in between, in
+    C with hardware fp32 arithmetic (no contraction); the full range was also swept once with step 1."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        import pytest
+        pytest.skip("no C compiler")
+    src = tmp_path / "div448.c"
+    src.write_text(_DIV448_C.replace("#include <math.h>", "#include <math.h>\n#include <stdlib.h>"))
+    exe = tmp_path / "div448"
+    subprocess.run([gcc, "-O2", "-ffp-contract=off", str(src), "-o", str(exe), "-lm"], check=True)
+    out = subprocess.run([str(exe), "61"], check=True, capture_output=True, text=True).stdout
+    assert int(out.strip()) == 0

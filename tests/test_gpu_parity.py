@@ -371,7 +371,9 @@ def _quant_check(x_dev, fmt, rows=None, **kw):
     assert_quantised(q.cpu().numpy(), s.cpu().numpy(), rq, rs, fmt)
 
 
-@pytest.mark.parametrize("M,K", [(1, 128), (7, 300), (64, 1000), (256, 4096), (33, 8200)])
+# (1, 128), (256, 4096), (130, 1040) and (16, 272) have 16-byte row strides and K a multiple of 16, so the
+# TMA-fed kernel runs them (the last two with ragged tiles); the others take the kernel with plain loads
+@pytest.mark.parametrize("M,K", [(1, 128), (7, 300), (64, 1000), (256, 4096), (33, 8200), (130, 1040), (16, 272)])
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
 @pytest.mark.parametrize("fmt", [0, 1])
 def test_quantize_1x128_bit_exact(M, K, dtype, fmt):
@@ -380,25 +382,29 @@ def test_quantize_1x128_bit_exact(M, K, dtype, fmt):
 
 
 @pytest.mark.parametrize("fmt", [0, 1])
-def test_quantize_special_groups_and_strides(fmt):
-    x = torch.zeros(7, 520)
-    x[1] = wl.normal_with_outliers((1, 520), 7100)[0] * 1e-30     # tiny values
-    x[6] = wl.normal_with_outliers((1, 520), 7102)[0] * 1e-44     # amax / 448 underflows fp32: scale 1
+# K = 528 (a multiple of 16) takes the TMA-fed kernel, whose tensor store must stop at K inside the 544-byte rows
+# of q; K = 520 the kernel with plain loads.  The columns of x past K hold huge values, which must not reach a
+# group's amax.
+@pytest.mark.parametrize("K", [520, 528])
+def test_quantize_special_groups_and_strides(fmt, K):
+    x = torch.zeros(7, K)
+    x[1] = wl.normal_with_outliers((1, K), 7100)[0] * 1e-30       # tiny values
+    x[6] = wl.normal_with_outliers((1, K), 7102)[0] * 1e-44       # amax / 448 underflows fp32: scale 1
     x[2, :128] = 448.0 * 2.0 ** 5                                   # amax exactly 448 * 2^5, constant group
     x[2, 128:256] = torch.linspace(-1.0, 1.0, 128)                  # a tie-rich ramp
     x[3] = -0.0
-    x[4] = wl.normal_with_outliers((1, 520), 7101)[0] * 1e20       # huge values
+    x[4] = wl.normal_with_outliers((1, K), 7101)[0] * 1e20         # huge values
     x[5, 7] = 1.0                                                   # one non-zero element per group
-    base = torch.zeros(7, 640)
-    base[:, :520] = x
-    xv = base.to(DEV)[:, :520]                                      # row stride 640 > K
-    q = torch.full((7, 544), 0x55, dtype=torch.uint8, device=DEV)[:, :520]
+    base = torch.full((7, 640), 1e30)
+    base[:, :K] = x
+    xv = base.to(DEV)[:, :K]                                        # row stride 640 > K
+    q = torch.full((7, 544), 0x55, dtype=torch.uint8, device=DEV)[:, :K]
     s = torch.zeros((7, 8), dtype=torch.float32 if fmt == 0 else torch.uint8, device=DEV)[:, :5]
     _quant_check(xv, fmt, q=q, scale=s)
     if fmt == 0:
         assert torch.all(s[6] == 1.0)
     full = torch.as_strided(q, (7, 544), (544, 1))
-    assert torch.all(full[:, 520:] == 0x55), "wrote past K"
+    assert torch.all(full[:, K:] == 0x55), "wrote past K"
 
 
 def test_quantize_full_size_activations_sampled_rows():
