@@ -117,6 +117,10 @@ __global__ void __launch_bounds__(Ring<InT>::kThreads, Ring<InT>::kCtasPerSm)
     tma_prefetch_desc(&tmq);
   }
   __syncthreads();
+  // x may come from the previous kernel in the stream, which may also still read
+  // q and the scales: every global access comes after this wait
+  grid_dependency_wait();
+  grid_launch_dependents();
   auto issue = [&](long long tile, int s) {
     const long long rb = tile / ctiles, cb = tile - rb * ctiles;
     mbar_arrive_expect_tx(&sm.full[s], kTileBytes);
@@ -259,9 +263,19 @@ cudaError_t launch_ring(const CUtensorMap& tmx, const CUtensorMap& tmq, long lon
   if (e != cudaSuccess) return e;
   long long blocks = static_cast<long long>(sms > 0 ? sms : 148) * Ring<InT>::kCtasPerSm;
   if (blocks > ntiles) blocks = ntiles;
-  quantize_ring_kernel<InT, FMT, ROWS><<<static_cast<unsigned>(blocks), Ring<InT>::kThreads, smem, stream>>>(
-      tmx, tmq, R, scale, s_r, s_c, ctiles, ntiles, err);
-  return cudaGetLastError();
+  cudaLaunchAttribute attr[1];
+  // programmatic dependent launch: the set-up may overlap the previous kernel in the stream
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(blocks), 1, 1);
+  cfg.blockDim = dim3(Ring<InT>::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, quantize_ring_kernel<InT, FMT, ROWS>, tmx, tmq, R, scale, s_r, s_c, ctiles, ntiles,
+                            err);
 }
 
 }  // namespace ring
