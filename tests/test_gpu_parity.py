@@ -485,6 +485,64 @@ def test_quantize_t_reads_no_column_past_c(group):
     _quant_t_check(xv, group, 0)
 
 
+def test_quantise_gemm_chains_reuse_buffers_back_to_back():
+    """Quantisers and GEMMs launched back to back on one stream with programmatic dependent launch, reusing the
+    same code, scale and output buffers: each quantiser must wait for the GEMM before it to finish reading the
+    codes it overwrites, and each GEMM and the quantiser that reads a GEMM's output must see the whole of the
+    kernel before it.  Every result equals the same computation run one call at a time."""
+    M, N, K = 1024, 1024, 2048
+    xs = [wl.normal_with_outliers((M, K), 7700 + i).to(torch.bfloat16).to(DEV) for i in range(4)]
+    ws = [wl.normal_with_outliers((N, K), 7710 + i).to(torch.bfloat16).to(DEV) for i in range(4)]
+    a, sa = torch.empty(M, K, dtype=torch.uint8, device=DEV), torch.empty(M, K // 128, device=DEV)
+    b, sb = bs.bs_quantize_fp8_128x128(ws[0], "f32")
+    ys = [torch.empty(M, N, dtype=torch.bfloat16, device=DEV) for _ in range(4)]
+    qy = [torch.empty(M, N, dtype=torch.uint8, device=DEV) for _ in range(4)]
+    sy = [torch.empty(M, N // 128, device=DEV) for _ in range(4)]
+    torch.cuda.synchronize()
+    for i in range(4):  # no synchronisation inside the chain
+        bs.quantize_fp8_1x128(xs[i], "f32", q=a, scale=sa)
+        bs.bs_quantize_fp8_128x128(ws[i], "f32", q=b, scale=sb)
+        bs.bs_gemm_fp8_blockwise(a, b.t(), sa, sb, out=ys[i])
+        bs.quantize_fp8_1x128(ys[i], "f32", q=qy[i], scale=sy[i])
+    torch.cuda.synchronize()
+    assert bs.device_error() == 0
+    for i in range(4):
+        ra, rsa = bs.quantize_fp8_1x128(xs[i], "f32")
+        rb, rsb = bs.bs_quantize_fp8_128x128(ws[i], "f32")
+        torch.cuda.synchronize()
+        ry = bs.bs_gemm_fp8_blockwise(ra, rb.t(), rsa, rsb)
+        torch.cuda.synchronize()
+        rq, rs = bs.quantize_fp8_1x128(ry, "f32")
+        torch.cuda.synchronize()
+        assert torch.equal(ys[i], ry), f"GEMM {i}"
+        assert torch.equal(qy[i], rq) and torch.equal(sy[i], rs), f"quantised output {i}"
+
+
+def test_transposed_quantiser_chain_reuses_buffers_back_to_back():
+    """The backward operands of several steps quantised into the same buffers, each followed by its weight-
+    gradient GEMM, with no synchronisation in between; equal to the same steps run one call at a time."""
+    M, N, K = 1024, 512, 768  # tokens, output features, input features
+    dys = [wl.normal_with_outliers((M, N), 7720 + i).to(torch.bfloat16).to(DEV) for i in range(3)]
+    xs = [wl.normal_with_outliers((M, K), 7730 + i).to(torch.bfloat16).to(DEV) for i in range(3)]
+    a, sa = bs.quantize_fp8_t(dys[0], "128x1", "f32")
+    b, sb = bs.quantize_fp8_t(xs[0], "128x128", "f32")
+    outs = [torch.empty(N, K, dtype=torch.bfloat16, device=DEV) for _ in range(3)]
+    torch.cuda.synchronize()
+    for i in range(3):
+        bs.quantize_fp8_t(dys[i], "128x1", "f32", q_t=a, scale=sa)
+        bs.quantize_fp8_t(xs[i], "128x128", "f32", q_t=b, scale=sb)
+        bs.bs_gemm_fp8_blockwise(a, b.t(), sa, sb, out=outs[i])
+    torch.cuda.synchronize()
+    assert bs.device_error() == 0
+    for i in range(3):
+        ra, rsa = bs.quantize_fp8_t(dys[i], "128x1", "f32")
+        rb, rsb = bs.quantize_fp8_t(xs[i], "128x128", "f32")
+        torch.cuda.synchronize()
+        ref = bs.bs_gemm_fp8_blockwise(ra, rb.t(), rsa, rsb)
+        torch.cuda.synchronize()
+        assert torch.equal(outs[i], ref), f"weight gradient {i}"
+
+
 def test_quantize_t_full_size_output_gradient():
     dy = wl.normal_with_outliers((16640, 5120), 7600).to(torch.bfloat16).to(DEV)
     _quant_t_check(dy, "128x1", 0)
