@@ -311,10 +311,11 @@ bs_status encode_quant_maps(const void* x, bs_in_dtype x_dtype, int64_t R, int64
   *tma = (reinterpret_cast<uintptr_t>(x) & 15u) == 0 && (ldx * es) % 16 == 0 && C % 16 == 0 &&
          (reinterpret_cast<uintptr_t>(q) & 15u) == 0 && ldq % 16 == 0;
   if (!*tma) return BS_OK;
-  bs_status st = encode_3d(tmx, x_dtype == BS_IN_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
-                           es, x, static_cast<uint64_t>(C), static_cast<uint64_t>(R), 1, static_cast<uint64_t>(ldx),
-                           static_cast<uint64_t>(ldx) * static_cast<uint64_t>(R), 128, 128, "x",
-                           CU_TENSOR_MAP_SWIZZLE_NONE);
+  const CUtensorMapDataType xt =
+      x_dtype == BS_IN_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  bs_status st = encode_3d(tmx, xt, es, x, static_cast<uint64_t>(C), static_cast<uint64_t>(R), 1,
+                           static_cast<uint64_t>(ldx), static_cast<uint64_t>(ldx) * static_cast<uint64_t>(R), 128, 128,
+                           "x", CU_TENSOR_MAP_SWIZZLE_NONE);
   if (st != BS_OK) return st;
   return encode_3d(tmq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, q, static_cast<uint64_t>(C), static_cast<uint64_t>(R), 1,
                    static_cast<uint64_t>(ldq), static_cast<uint64_t>(ldq) * static_cast<uint64_t>(R), 128, 128, "q",

@@ -153,10 +153,10 @@ cudaError_t launch_blocks(const void* x, long long R, long long C, long long ldx
                           void* scale, long long s_rb, long long s_cb, int sms, cudaStream_t stream) {
   const long long ctiles = (C + kTile - 1) / kTile;
   const long long ntiles = ((R + kTile - 1) / kTile) * ctiles;
-  int per_sm = 0;  // resident CTAs per SM: one wave of persistent CTAs
-  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quantize_blocks_kernel<InT, FMT>, kThreads, 0);
+  int per_sm = 1;  // resident CTAs per SM: one wave of persistent CTAs
+  const cudaError_t e = ctas_per_sm_once<quantize_blocks_kernel<InT, FMT>>(kThreads, 0, &per_sm);
   if (e != cudaSuccess) return e;
-  long long blocks = static_cast<long long>(sms > 0 ? sms : 148) * (per_sm > 0 ? per_sm : 1);
+  long long blocks = static_cast<long long>(sms > 0 ? sms : 148) * per_sm;
   if (blocks > ntiles) blocks = ntiles;
   if (blocks < 1) blocks = 1;
   constexpr long long kStoreBytes = 16 / static_cast<long long>(sizeof(InT));  // codes per piece

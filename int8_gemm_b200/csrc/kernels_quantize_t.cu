@@ -228,13 +228,10 @@ cudaError_t launch_t(const void* x, long long R, long long C, long long ldx, uin
   const long long ctiles = (C + kTile - 1) / kTile;
   const long long ntiles = ((R + kTile - 1) / kTile) * ctiles;
   const size_t smem = sizeof(TileSmem<InT>);
-  cudaError_t e = cudaFuncSetAttribute(quantize_t_kernel<InT, FMT, GROUP>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  int per_sm = 1;  // resident CTAs per SM (shared memory and registers): one wave, no stragglers
+  const cudaError_t e = ctas_per_sm_once<quantize_t_kernel<InT, FMT, GROUP>>(kThreads, smem, &per_sm);
   if (e != cudaSuccess) return e;
-  int per_sm = 0;  // resident CTAs per SM (shared memory and registers): one wave, no stragglers
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quantize_t_kernel<InT, FMT, GROUP>, kThreads, smem);
-  if (e != cudaSuccess) return e;
-  long long blocks = static_cast<long long>(sms > 0 ? sms : 148) * (per_sm > 0 ? per_sm : 1);
+  long long blocks = static_cast<long long>(sms > 0 ? sms : 148) * per_sm;
   if (blocks > ntiles) blocks = ntiles;
   if (blocks < 1) blocks = 1;
   const bool vec_x = (reinterpret_cast<uintptr_t>(x) & 15u) == 0 && (ldx * static_cast<long long>(sizeof(InT))) % 16 == 0;
@@ -486,10 +483,11 @@ cudaError_t launch_t_tma(const CUtensorMap& tmx, const CUtensorMap& tmq, long lo
   const long long ctiles = (C + kTile - 1) / kTile;
   const long long ntiles = ((R + kTile - 1) / kTile) * ctiles;
   const size_t smem = sizeof(TmaSmem<InT>) + 1024;
-  cudaError_t e = cudaFuncSetAttribute(quantize_t_tma_kernel<InT, FMT, GROUP>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  int per_sm = 1;
+  const cudaError_t e = ctas_per_sm_once<quantize_t_tma_kernel<InT, FMT, GROUP>>(TRing<InT>::kThreads, smem, &per_sm);
   if (e != cudaSuccess) return e;
-  long long blocks = static_cast<long long>(sms > 0 ? sms : 148) * TRing<InT>::kCtasPerSm;
+  if (per_sm > TRing<InT>::kCtasPerSm) per_sm = TRing<InT>::kCtasPerSm;
+  long long blocks = static_cast<long long>(sms > 0 ? sms : 148) * per_sm;
   if (blocks > ntiles) blocks = ntiles;
   quantize_t_tma_kernel<InT, FMT, GROUP><<<static_cast<unsigned>(blocks), TRing<InT>::kThreads, smem, stream>>>(
       tmx, tmq, R, C, scale, lds, ctiles, ntiles, err);

@@ -27,6 +27,7 @@
 #include <stdint.h>
 
 #include "group_quant.cuh"
+#include "quantize.h"
 #include "sm100.cuh"
 
 namespace bsg {
@@ -258,10 +259,11 @@ cudaError_t launch_ring(const CUtensorMap& tmx, const CUtensorMap& tmq, long lon
   const long long ctiles = (C + kTile - 1) / kTile;
   const long long ntiles = ((R + kTile - 1) / kTile) * ctiles;
   const size_t smem = sizeof(Smem<InT>) + 1024;
-  cudaError_t e = cudaFuncSetAttribute(quantize_ring_kernel<InT, FMT, ROWS>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  int per_sm = 1;
+  const cudaError_t e = ctas_per_sm_once<quantize_ring_kernel<InT, FMT, ROWS>>(Ring<InT>::kThreads, smem, &per_sm);
   if (e != cudaSuccess) return e;
-  long long blocks = static_cast<long long>(sms > 0 ? sms : 148) * Ring<InT>::kCtasPerSm;
+  if (per_sm > Ring<InT>::kCtasPerSm) per_sm = Ring<InT>::kCtasPerSm;
+  long long blocks = static_cast<long long>(sms > 0 ? sms : 148) * per_sm;
   if (blocks > ntiles) blocks = ntiles;
   cudaLaunchAttribute attr[1];
   // programmatic dependent launch: the set-up may overlap the previous kernel in the stream

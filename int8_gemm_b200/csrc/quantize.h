@@ -7,7 +7,36 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 namespace bsg {
+
+// Launch facts of a kernel that hold for the whole process, worked out on a
+// device's first launch only (as the GEMM launchers do): the dynamic
+// shared-memory limit is raised to `smem` bytes and the number of CTAs of
+// `threads` threads that fit on one SM is queried.  Devices are told apart by
+// their index modulo 64.
+template <auto KERNEL>
+cudaError_t ctas_per_sm_once(int threads, size_t smem, int* per_sm) {
+  static std::atomic<int> known[64];  // 0: not yet worked out on that device
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::atomic<int>& slot = known[dev % 64];
+  int v = slot.load(std::memory_order_acquire);
+  if (v == 0) {
+    if (smem > 0) {
+      e = cudaFuncSetAttribute(KERNEL, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+      if (e != cudaSuccess) return e;
+    }
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, KERNEL, threads, smem);
+    if (e != cudaSuccess) return e;
+    if (v < 1) v = 1;
+    slot.store(v, std::memory_order_release);
+  }
+  *per_sm = v;
+  return cudaSuccess;
+}
 
 // 1x128 group quantisation of x [M, K] (bf16 or fp32, row stride ldx
 // elements) to e4m3 codes q (row stride ldq bytes) and one scale per group:
