@@ -72,9 +72,10 @@ KERNEL_SOURCES = {
     "wide": ["sm100.cuh", "tile_order.h", "wide_kernel.cuh", "skinny_kernel.cuh", "kernels_wide.cu", "launch.h"],
     "skinny": ["sm100.cuh", "tile_order.h", "wide_kernel.cuh", "skinny_kernel.cuh", "kernels_skinny.cu", "launch.h"],
     "gemv": ["sm100.cuh", "tile_order.h", "wide_kernel.cuh", "skinny_kernel.cuh", "kernels_gemv.cu", "launch.h"],
-    "quantize": ["sm100.cuh", "group_quant.cuh", "quant_ring.cuh", "quantize.h", "kernels_quantize.cu"],
-    "quantize_t": ["sm100.cuh", "group_quant.cuh", "quantize.h", "kernels_quantize_t.cu"],
-    "quantize_blocks": ["sm100.cuh", "group_quant.cuh", "quant_ring.cuh", "quantize.h", "kernels_quantize_blocks.cu"],
+    "quantize": ["sm100.cuh", "group_quant.cuh", "tile_ring.cuh", "quant_ring.cuh", "quantize.h", "kernels_quantize.cu"],
+    "quantize_t": ["sm100.cuh", "group_quant.cuh", "tile_ring.cuh", "quantize.h", "kernels_quantize_t.cu"],
+    "quantize_blocks": ["sm100.cuh", "group_quant.cuh", "tile_ring.cuh", "quant_ring.cuh", "quantize.h",
+                        "kernels_quantize_blocks.cu"],
 }
 
 

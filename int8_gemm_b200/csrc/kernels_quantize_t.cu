@@ -33,6 +33,7 @@
 #include "group_quant.cuh"
 #include "quantize.h"
 #include "sm100.cuh"
+#include "tile_ring.cuh"
 
 namespace bsg {
 
@@ -259,8 +260,9 @@ cudaError_t launch_t_fmt(const void* x, long long R, long long C, long long ldx,
 // input and two code tiles, so that one CTA's reductions and barriers overlap
 // the other's work; one of 512 threads for fp32, with three input tiles and one
 // code tile).  One thread keeps the ring of input tiles in flight with 2-D
-// tensor copies (rows and columns past the matrix arrive as zeros), so no
-// thread spends instructions or registers on loads.  Thread t owns the column
+// tensor copies and writes the code tiles back with tensor stores (TileRing,
+// tile_ring.cuh), so no thread spends instructions or registers on loads.
+// Thread t owns the column
 // pair 2 (t % 64), + 1 and kRows consecutive rows (32 for bf16, 16 for fp32):
 // it reads its pairs from the tile once (one 4- or 8-byte shared load each, a
 // warp reading 128 or 256 contiguous bytes), takes their amax in registers
@@ -329,31 +331,19 @@ __global__ void __launch_bounds__(TRing<InT>::kThreads, TRing<InT>::kCtasPerSm)
   const int t = threadIdx.x;
   const int cp = t % (kTile / 2);  // column pair
   const int qr = t / (kTile / 2);  // row group: rows kRows * qr ..
+  const TileRing<G::kStages, G::kCodeBufs> ring{sm.full, &sm.abort, &tmx, reinterpret_cast<uint8_t*>(&sm.v[0][0][0]),
+                                                kTileBytes, ctiles, ntiles};
   if (t == 0) {
-    for (int s = 0; s < G::kStages; ++s) mbar_init(&sm.full[s], 1);
-    sm.abort = 0;
-    fence_mbar_init();
-    tma_prefetch_desc(&tmx);
-    tma_prefetch_desc(&tmq);
+    ring.init(&tmq);
+    ring.start();
   }
-  __syncthreads();
-  auto issue = [&](long long tile, int s) {
-    const long long rb = tile / ctiles, cb = tile - rb * ctiles;
-    mbar_arrive_expect_tx(&sm.full[s], kTileBytes);
-    tma_load_3d(&sm.v[s][0][0], &tmx, &sm.full[s], static_cast<int>(cb * kTile), static_cast<int>(rb * kTile), 0);
-  };
-  if (t == 0)
-    for (int s = 0; s < G::kStages; ++s) {
-      const long long tile = blockIdx.x + static_cast<long long>(s) * gridDim.x;
-      if (tile < ntiles) issue(tile, s);
-    }
   int it = 0;
   bool ok = true;
+  __syncthreads();  // the mbarriers are initialised
   for (long long tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
     const int st = it % G::kStages, cbuf = it % G::kCodeBufs;
     const long long rb = tile / ctiles, cb = tile - rb * ctiles;
-    const bool got = wait_bounded(&sm.full[st], static_cast<uint32_t>(it / G::kStages) & 1u, &sm.abort, err,
-                                  kErrTimeout | kRoleConsumer | kWaitStageFull);
+    const bool got = ring.wait(it, err);
     Held h[G::kRows];
 #pragma unroll
     for (int i = 0; i < G::kRows; ++i) h[i] = *reinterpret_cast<const Held*>(&sm.v[st][G::kRows * qr + i][2 * cp]);
@@ -380,24 +370,11 @@ __global__ void __launch_bounds__(TRing<InT>::kThreads, TRing<InT>::kCtasPerSm)
       for (int off = 16; off > 0; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
       if ((t & 31) == 0) sm.wmax[t / 32] = a;
     }
-    // the code tile written kCodeBufs tiles ago has been read by its store
-    if (t == 0) {
-      if constexpr (G::kCodeBufs == 2) {
-        bulk_wait_read1();
-      } else {
-        bulk_wait_read_all();
-      }
-    }
+    if (t == 0) ring.code_tile_free();
     // every thread holds its values: the stage can be refilled
     ok = __syncthreads_and(got) != 0;
     if (!ok) break;
-    if (t == 0) {
-      const long long next = tile + static_cast<long long>(G::kStages) * gridDim.x;
-      if (next < ntiles) {
-        fence_proxy_async_smem();
-        issue(next, st);
-      }
-    }
+    if (t == 0) ring.refill(tile, it);
     if constexpr (GROUP == 0) {
 #pragma unroll
       for (int k = 0; k < G::kParts; ++k) {
@@ -459,22 +436,9 @@ __global__ void __launch_bounds__(TRing<InT>::kThreads, TRing<InT>::kCtasPerSm)
     }
     fence_proxy_async_smem();  // the code tile, before the tensor store reads it
     __syncthreads();
-    if (t == 0) {
-      tma_store_3d(&tmq, &sm.codes[cbuf][0][0], static_cast<int>(rb * kTile), static_cast<int>(cb * kTile), 0);
-      bulk_commit();
-    }
+    if (t == 0) ring.store(&tmq, &sm.codes[cbuf][0][0], rb * kTile, cb * kTile);
   }
-  if (t == 0) {
-    bulk_wait_all();
-    if (!ok) {  // a wait gave up: let the copies still in flight land before the CTA retires
-      volatile int never = 0;
-      for (int j = it; j < it + G::kStages; ++j) {
-        const long long tile = blockIdx.x + static_cast<long long>(j) * gridDim.x;
-        if (tile < ntiles)
-          wait_bounded(&sm.full[j % G::kStages], static_cast<uint32_t>(j / G::kStages) & 1u, &never, nullptr, 0);
-      }
-    }
-  }
+  if (t == 0) ring.finish(ok, it);
 }
 
 template <typename InT, int FMT, int GROUP>

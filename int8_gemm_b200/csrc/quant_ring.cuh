@@ -29,6 +29,7 @@
 #include "group_quant.cuh"
 #include "quantize.h"
 #include "sm100.cuh"
+#include "tile_ring.cuh"
 
 namespace bsg {
 namespace ring {
@@ -110,35 +111,21 @@ __global__ void __launch_bounds__(Ring<InT>::kThreads, Ring<InT>::kCtasPerSm)
   const int j8 = t % G::kRowThreads;
   const int w = t / 32, slot = (t % 32) / G::kRowThreads;
   const int row0 = (w / 4) * 16 + (w % 4) + 4 * slot;
-  if (t == 0) {
-    for (int s = 0; s < G::kStages; ++s) mbar_init(&sm.full[s], 1);
-    sm.abort = 0;
-    fence_mbar_init();
-    tma_prefetch_desc(&tmx);
-    tma_prefetch_desc(&tmq);
-  }
+  const TileRing<G::kStages, G::kCodeBufs> ring{sm.full, &sm.abort, &tmx, reinterpret_cast<uint8_t*>(&sm.v[0][0][0]),
+                                                kTileBytes, ctiles, ntiles};
+  if (t == 0) ring.init(&tmq);
   __syncthreads();
   // x may come from the previous kernel in the stream, which may also still read
   // q and the scales: every global access comes after this wait
   grid_dependency_wait();
   grid_launch_dependents();
-  auto issue = [&](long long tile, int s) {
-    const long long rb = tile / ctiles, cb = tile - rb * ctiles;
-    mbar_arrive_expect_tx(&sm.full[s], kTileBytes);
-    tma_load_3d(&sm.v[s][0][0], &tmx, &sm.full[s], static_cast<int>(cb * kTile), static_cast<int>(rb * kTile), 0);
-  };
-  if (t == 0)
-    for (int s = 0; s < G::kStages; ++s) {
-      const long long tile = blockIdx.x + static_cast<long long>(s) * gridDim.x;
-      if (tile < ntiles) issue(tile, s);
-    }
+  if (t == 0) ring.start();
   int it = 0;
   bool ok = true;
   for (long long tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
     const int st = it % G::kStages, cbuf = it % G::kCodeBufs;
     const long long rb = tile / ctiles, cb = tile - rb * ctiles;
-    const bool got = wait_bounded(&sm.full[st], static_cast<uint32_t>(it / G::kStages) & 1u, &sm.abort, err,
-                                  kErrTimeout | kRoleConsumer | kWaitStageFull);
+    const bool got = ring.wait(it, err);
     uint4 v[G::kPasses][G::kPieces];
 #pragma unroll
     for (int k = 0; k < G::kPasses; ++k)
@@ -167,24 +154,11 @@ __global__ void __launch_bounds__(Ring<InT>::kThreads, Ring<InT>::kCtasPerSm)
       for (int off = 16; off > 0; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
       if ((t & 31) == 0) sm.wmax[t / 32] = a;
     }
-    // the code tile written kCodeBufs tiles ago has been read by its store
-    if (t == 0) {
-      if constexpr (G::kCodeBufs == 2) {
-        bulk_wait_read1();
-      } else {
-        bulk_wait_read_all();
-      }
-    }
+    if (t == 0) ring.code_tile_free();
     // every thread holds its pieces: the stage can be refilled
     ok = __syncthreads_and(got) != 0;
     if (!ok) break;
-    if (t == 0) {
-      const long long next = tile + static_cast<long long>(G::kStages) * gridDim.x;
-      if (next < ntiles) {
-        fence_proxy_async_smem();
-        issue(next, st);
-      }
-    }
+    if (t == 0) ring.refill(tile, it);
     if constexpr (!ROWS) {
       float a = sm.wmax[0];
 #pragma unroll
@@ -233,22 +207,9 @@ __global__ void __launch_bounds__(Ring<InT>::kThreads, Ring<InT>::kCtasPerSm)
     }
     fence_proxy_async_smem();  // the code tile, before the tensor store reads it
     __syncthreads();
-    if (t == 0) {
-      tma_store_3d(&tmq, &sm.codes[cbuf][0][0], static_cast<int>(cb * kTile), static_cast<int>(rb * kTile), 0);
-      bulk_commit();
-    }
+    if (t == 0) ring.store(&tmq, &sm.codes[cbuf][0][0], cb * kTile, rb * kTile);
   }
-  if (t == 0) {
-    bulk_wait_all();
-    if (!ok) {  // a wait gave up: let the copies still in flight land before the CTA retires
-      volatile int never = 0;
-      for (int j = it; j < it + G::kStages; ++j) {
-        const long long tile = blockIdx.x + static_cast<long long>(j) * gridDim.x;
-        if (tile < ntiles)
-          wait_bounded(&sm.full[j % G::kStages], static_cast<uint32_t>(j / G::kStages) & 1u, &never, nullptr, 0);
-      }
-    }
-  }
+  if (t == 0) ring.finish(ok, it);
 }
 
 // tmx / tmq: x and q [R, C] as tensors of 128 x 128 boxes, x without swizzle,
