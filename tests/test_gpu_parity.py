@@ -518,6 +518,49 @@ def test_quantise_gemm_chains_reuse_buffers_back_to_back():
         assert torch.equal(qy[i], rq) and torch.equal(sy[i], rs), f"quantised output {i}"
 
 
+def test_quantise_gemm_chain_replays_in_a_cuda_graph():
+    """The forward and backward operand quantisers and the blockwise GEMM captured once in a CUDA graph (the
+    kernels launch on the capturing stream, with programmatic dependent launch between them) and replayed on
+    new inputs copied into the captured buffers: every replay equals the same calls run eagerly."""
+    M, N, K = 640, 768, 1024
+    x = torch.empty(M, K, dtype=torch.bfloat16, device=DEV)
+    w = torch.empty(N, K, dtype=torch.bfloat16, device=DEV)
+    a, sa = torch.empty(M, K, dtype=torch.uint8, device=DEV), torch.empty(M, K // 128, device=DEV)
+    b, sb = torch.empty(N, K, dtype=torch.uint8, device=DEV), torch.empty(K // 128, N // 128, device=DEV)
+    xt, sxt = torch.empty(K, M, dtype=torch.uint8, device=DEV), torch.empty(M // 128, K // 128, device=DEV)
+    y = torch.empty(M, N, dtype=torch.bfloat16, device=DEV)
+
+    def step():
+        bs.quantize_fp8_1x128(x, "f32", q=a, scale=sa)
+        bs.bs_quantize_fp8_128x128(w, "f32", q=b, scale=sb)
+        bs.bs_gemm_fp8_blockwise(a, b.t(), sa, sb, out=y)
+        bs.quantize_fp8_t(x, "128x128", "f32", q_t=xt, scale=sxt)
+
+    x.copy_(wl.normal_with_outliers((M, K), 7740).to(torch.bfloat16))
+    w.copy_(wl.normal_with_outliers((N, K), 7741).to(torch.bfloat16))
+    side = torch.cuda.Stream(DEV)
+    side.wait_stream(torch.cuda.current_stream(DEV))
+    with torch.cuda.stream(side):
+        step()  # warm-up on the capturing stream (one-time launch set-up outside the capture)
+    torch.cuda.current_stream(DEV).wait_stream(side)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=side):
+        step()
+    for i in range(3):
+        x.copy_(wl.normal_with_outliers((M, K), 7750 + i).to(torch.bfloat16))
+        w.copy_(wl.normal_with_outliers((N, K), 7760 + i).to(torch.bfloat16))
+        graph.replay()
+        torch.cuda.synchronize()
+        got = [t.clone() for t in (a, sa, b, sb, y, xt, sxt)]
+        step()
+        torch.cuda.synchronize()
+        for name, g, e in zip(("a", "scale_a", "b", "scale_b", "y", "x_t", "scale_x_t"), got, (a, sa, b, sb, y, xt, sxt)):
+            assert torch.equal(g, e), f"replay {i}: {name}"
+    del graph
+    assert bs.device_error() == 0
+
+
 def test_transposed_quantiser_chain_reuses_buffers_back_to_back():
     """The backward operands of several steps quantised into the same buffers, each followed by its weight-
     gradient GEMM, with no synchronisation in between; equal to the same steps run one call at a time."""
