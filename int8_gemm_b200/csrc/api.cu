@@ -735,7 +735,8 @@ bs_status bs_quantize_fp8_1x128(const void* x, bs_in_dtype x_dtype, int64_t M, i
   if (M * ((KB + 3) / 4) > kMaxDim) return fail(BS_ERR_SHAPE, "M * ceil(K/512) exceeds 2^31-1");
   const uintptr_t es = x_dtype == BS_IN_BF16 ? 2 : 4;
   if (reinterpret_cast<uintptr_t>(x) % es != 0) return fail(BS_ERR_ALIGNMENT, "x must be aligned to its element size");
-  if (scale_fmt == BS_SCALE_F32 && !aligned4(scale)) return fail(BS_ERR_ALIGNMENT, "fp32 scales must be 4-byte aligned");
+  if (scale_fmt == BS_SCALE_F32 && !aligned4(scale))
+    return fail(BS_ERR_ALIGNMENT, "fp32 scales must be 4-byte aligned");
   DeviceCtx* dc = nullptr;
   bs_status st = device_ctx(&dc);
   if (st != BS_OK) return st;
@@ -766,7 +767,8 @@ bs_status bs_quantize_fp8_t(const void* x, bs_in_dtype x_dtype, int64_t R, int64
   if (RB * CB > kMaxDim) return fail(BS_ERR_SHAPE, "more than 2^31-1 tiles of 128 x 128");
   const uintptr_t es = x_dtype == BS_IN_BF16 ? 2 : 4;
   if (reinterpret_cast<uintptr_t>(x) % es != 0) return fail(BS_ERR_ALIGNMENT, "x must be aligned to its element size");
-  if (scale_fmt == BS_SCALE_F32 && !aligned4(scale)) return fail(BS_ERR_ALIGNMENT, "fp32 scales must be 4-byte aligned");
+  if (scale_fmt == BS_SCALE_F32 && !aligned4(scale))
+    return fail(BS_ERR_ALIGNMENT, "fp32 scales must be 4-byte aligned");
   DeviceCtx* dc = nullptr;
   bs_status st = device_ctx(&dc);
   if (st != BS_OK) return st;
@@ -774,8 +776,9 @@ bs_status bs_quantize_fp8_t(const void* x, bs_in_dtype x_dtype, int64_t R, int64
   // used bytes (C elements of x, R codes of q_t) end on a 16-byte boundary.  (A tensor store of a last row
   // tile that ended inside a 16-byte piece, R = 260, wrote bytes past R.)
   CUtensorMap tmx, tmq;
-  const bool tma = aligned16(x) && (ldx * static_cast<int64_t>(es)) % 16 == 0 && (C * static_cast<int64_t>(es)) % 16 == 0 &&
-                   aligned16(q_t) && ldq % 16 == 0 && R % 16 == 0;
+  const int64_t esz = static_cast<int64_t>(es);
+  const bool tma = aligned16(x) && (ldx * esz) % 16 == 0 && (C * esz) % 16 == 0 && aligned16(q_t) && ldq % 16 == 0 &&
+                   R % 16 == 0;
   if (tma) {
     st = encode_3d(&tmx, x_dtype == BS_IN_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
                    static_cast<int>(es), x, static_cast<uint64_t>(C), static_cast<uint64_t>(R), 1,
@@ -811,7 +814,8 @@ bs_status bs_quantize_fp8_128x128(const void* x, bs_in_dtype x_dtype, int64_t R,
   if (RB * CB > kMaxDim) return fail(BS_ERR_SHAPE, "more than 2^31-1 blocks of 128 x 128");
   const uintptr_t es = x_dtype == BS_IN_BF16 ? 2 : 4;
   if (reinterpret_cast<uintptr_t>(x) % es != 0) return fail(BS_ERR_ALIGNMENT, "x must be aligned to its element size");
-  if (scale_fmt == BS_SCALE_F32 && !aligned4(scale)) return fail(BS_ERR_ALIGNMENT, "fp32 scales must be 4-byte aligned");
+  if (scale_fmt == BS_SCALE_F32 && !aligned4(scale))
+    return fail(BS_ERR_ALIGNMENT, "fp32 scales must be 4-byte aligned");
   DeviceCtx* dc = nullptr;
   bs_status st = device_ctx(&dc);
   if (st != BS_OK) return st;
